@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark: decode-stage SwiGLU MLP layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dfk|reference] [--quick]
+
+One step = one pass of the hot path over one decode batch of a
+Llama-3-8B-shaped MLP layer (B = 1, d_model 4096, d_ff 14336, bf16 weights
+~N(0, 0.02), x ~N(0, 1), gamma = 1 + N(0, 0.1), seed 1, row-major weights):
+the fused RMSNorm + gate/up + SiLU * up kernel followed by the separate
+down-projection kernel.  Inputs are synthetic and resident in HBM; two
+weight copies are used in rotation (705 MB, more than 5x the 126 MB L2) so
+no step reads weights the previous step left in L2.
+
+Printed (rank 0, one JSON line): whole-job achieved HBM GB/s over the
+algorithmic bytes of the step (the metric is "fused gate/up us/call &
+achieved HBM GB/s (% of B200 roofline) at batch 1-64"), the gate/up
+kernel's us/call and roofline fraction, the end-to-end figure through the
+host-memory C entry point, the batch sweep B = 1..64 (row- vs column-major,
+scheduler's choice), the fused-vs-unfused speedup and the CPU oracle
+baseline.  ``--impl reference`` times the fp64 CPU oracle on the same
+workload instead.  Under torchrun every rank runs an independent replica on
+its own GPU (the decode MLP does not shard across data-parallel replicas):
+value = bytes of all ranks / max-over-ranks time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused gate/up µs/call & achieved HBM GB/s (% of B200 roofline) at batch 1–64"
+UNIT = "GB/s"
+B1, D, F = 1, 4096, 14336
+SEED = 1
+FALLBACK_HBM_GBS = 6650.0
+
+
+def gate_up_bytes(B, D, F):
+    """Algorithmic bytes of the fused gate/up call: both weight matrices once,
+    x, gamma, and h written once (bf16)."""
+    return 2 * F * D * 2 + B * D * 2 + D * 2 + B * F * 2
+
+
+def down_bytes(B, D, F):
+    return D * F * 2 + B * F * 2 + B * D * 2
+
+
+def step_bytes(B, D, F):
+    return gate_up_bytes(B, D, F) + down_bytes(B, D, F)
+
+
+def config_dict(parallelism):
+    return {"workload": "llama3_8b_mlp_layer_decode", "B": B1, "d_model": D, "d_ff": F,
+            "layout": "row", "rmsnorm": True, "seed": SEED,
+            "step": "fused RMSNorm+gate/up+SiLU*up kernel, then down-projection kernel",
+            "global_batch": B1, "seq_len": 1, "parallelism": parallelism,
+            "l2": "inputs larger than L2: 2 rotating weight copies (705 MB vs 126 MB L2)"}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def engine_source_hash():
+    h = hashlib.sha256()
+    for rel in ("swiglu_mlp_dfk_b200/csrc/cc_engine.cuh", "swiglu_mlp_dfk_b200/csrc/ptx.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per gate/up launch from the committed ncu summary, if it was
+    taken on the kernel source as it is now; else None."""
+    p = os.path.join(ROOT, "profiles", "gate_up_llama3_8b_b1.md")
+    try:
+        text = open(p).read()
+    except OSError:
+        return None
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    m_h = re.search(r"engine_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m_b or not m_h or m_h.group(1) != engine_source_hash():
+        return None
+    return int(m_b.group(1))
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_dev):
+        self.samples = []
+        self.phase = "idle"
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_dev]) if vis and vis.split(",")[0].isdigit() \
+                    else torch_dev
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+
+    def _reasons(self):
+        nv = self.nv
+        for name in ("nvmlDeviceGetCurrentClocksEventReasons",
+                     "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            fn = getattr(nv, name, None)
+            if fn:
+                return fn(self.h)
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((self.phase, mhz, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, phase="timed"):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        sel = [s for s in self.samples if s[0] == phase]
+        note = "sampled during the timed region"
+        if len(sel) < 3:
+            sel = [s for s in self.samples if s[0] in ("warmup", "timed", "extra")]
+            note = "timed region shorter than the sampling period: warm-up, timed and " \
+                   "follow-on measurements pooled"
+        mhz = [s[1] for s in sel]
+        bits = 0
+        for s in sel:
+            bits |= s[2]
+        reasons = sorted(n for b, n in self.REASONS.items() if bits & b)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel), "note": note}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import build as kbuild
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    if rank == 0 or not os.path.exists(kbuild.LIB):
+        kbuild.build()
+    if world > 1:
+        dist.barrier()
+    dfk.lib()
+    dfk.dfk_device_error()
+
+    inp = I.make_inputs(B1, D, F, seed=SEED, w_std=0.02, norm=True, with_down=True,
+                        device="cuda")
+    copies = [(inp.w_gate, inp.w_up, inp.w_down),
+              (inp.w_gate.clone(), inp.w_up.clone(), inp.w_down.clone())]
+    h = torch.empty(B1, F, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(B1, D, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        wg, wu, wd = copies[i % len(copies)]
+        dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu, "row", h=h)
+        dfk.dfk_down_proj(h, wd, y=y)
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    clocks.phase = "warmup"
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events around every gate/up launch
+    K = args.steps
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.phase = "timed"
+    for i in range(K):
+        wg, wu, wd = copies[i % len(copies)]
+        ev_a[i].record(stream)
+        dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu, "row", h=h)
+        ev_b[i].record(stream)
+        dfk.dfk_down_proj(h, wd, y=y)
+    ev_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.phase = "extra"
+    if world > 1:
+        dist.barrier()
+    total_ms = ev_a[0].elapsed_time(ev_end)
+    gu_us = [ev_a[i].elapsed_time(ev_b[i]) * 1000.0 for i in range(K)]
+    t_max = total_ms
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    value = step_bytes(B1, D, F) * K * world / (t_max / 1e3) / 1e9
+    gu_avg = sum(gu_us) / len(gu_us)
+    gu_med = statistics.median(gu_us)
+    peak, peak_src = measured_peaks()
+    achieved = gate_up_bytes(B1, D, F) / (gu_avg * 1e-6) / 1e9
+
+    # ---- end to end through the host-memory C entry point
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(B1, D, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    Ke = max(1, min(K, 500))
+    for i in range(3):
+        wg, wu, wd = copies[i % 2]
+        dfk.dfk_mlp_forward_host(x_host, inp.gamma, inp.eps, wg, wu, "row", wd, y_host, x_dev,
+                                 h, y)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    t0 = time.perf_counter()
+    for i in range(Ke):
+        wg, wu, wd = copies[i % 2]
+        dfk.dfk_mlp_forward_host(x_host, inp.gamma, inp.eps, wg, wu, "row", wd, y_host, x_dev,
+                                 h, y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    e2e_ms = max(e0.elapsed_time(e1), wall * 1e3)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = step_bytes(B1, D, F) * Ke * world / (e2e_ms / 1e3) / 1e9
+
+    extra = {}
+    if rank == 0 and not args.quick:
+        extra = extra_measurements(args, inp, copies, h, y)
+    clocks.stop()
+    err = dfk.dfk_device_error()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t_max / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict("replicas%d" % world if world > 1 else "single-gpu"),
+        "gate_up_us_per_call": round(gu_avg, 2), "gate_up_us_median": round(gu_med, 2),
+        "gate_up_GBps": round(achieved, 1), "step_alg_bytes": step_bytes(B1, D, F),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s",
+                     "traffic": profiled_traffic(),
+                     "kernel": "fused RMSNorm+gate/up (CUDA-core, TMA ring)",
+                     "alg_bytes_per_launch": gate_up_bytes(B1, D, F)},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
+                "h2d_bytes_per_step": B1 * D * 2, "d2h_bytes_per_step": B1 * D * 2,
+                "ms_per_step": round(e2e_ms / Ke, 5), "steps": Ke,
+                "path": "dfk_mlp_forward_host: pinned x -> device, gate/up, down, y -> host"},
+        "gpu_launches": 2 * K,
+        "clocks": clocks.summary("timed"),
+        "device_error_word": err,
+    }
+    line.update(extra)
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    return line
+
+
+def timed_us(fn, reps, flush=None):
+    import torch
+    es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        if flush is not None:
+            flush.add_(1)
+        es[i][0].record()
+        fn(i)
+        es[i][1].record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) * 1000.0 for a, b in es)
+
+
+def extra_measurements(args, inp, copies, h, y):
+    """Interleaved layout, fused vs unfused, and the B = 1..64 sweep (row vs col)."""
+    import torch
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    peak, _ = measured_peaks()
+    reps = 30
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")  # 256 MB > L2
+    out = {}
+    # interleaved layout of the same weights
+    il = I.to_layout(inp.w_gate, inp.w_up, I.LAYOUT_INTERLEAVED)[0]
+    dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, il, None, "interleaved", h=h)
+    t_il = timed_us(lambda i: dfk.dfk_rmsnorm_swiglu_gate_up(
+        inp.x, inp.gamma, inp.eps, il, None, "interleaved", h=h), reps, flush)
+    del il
+    # fused vs unfused (separate RMSNorm, 2 GEMVs, SiLU, multiply; bf16 in HBM)
+    xn = torch.empty_like(inp.x)
+    a = torch.empty_like(h)
+    u = torch.empty_like(h)
+    s = torch.empty_like(h)
+
+    def unfused(i):
+        wg, wu, _ = copies[i % 2]
+        dfk.dfk_rmsnorm(inp.x, inp.gamma, inp.eps, out=xn)
+        dfk.dfk_gemv(xn, wg, out=a)
+        dfk.dfk_gemv(xn, wu, out=u)
+        dfk.dfk_silu(a, out=s)
+        dfk.dfk_mul(s, u, out=h)
+
+    def fused(i):
+        wg, wu, _ = copies[i % 2]
+        dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu, "row", h=h)
+
+    unfused(0)
+    t_unf = timed_us(unfused, reps, flush)
+    t_fus = timed_us(fused, reps, flush)
+    t_down = timed_us(lambda i: dfk.dfk_down_proj(h, copies[i % 2][2], y=y), reps, flush)
+    out["interleaved_gate_up_us"] = round(t_il, 2)
+    out["fused_vs_unfused"] = {"fused_us": round(t_fus, 2), "unfused_us": round(t_unf, 2),
+                               "speedup": round(t_unf / t_fus, 3),
+                               "unfused": "rmsnorm + gemv(Wg) + gemv(Wu) + silu + mul"}
+    out["down_proj_us"] = round(t_down, 2)
+    out["down_proj_GBps"] = round(down_bytes(B1, D, F) / (t_down * 1e-6) / 1e9, 1)
+
+    # batch sweep B = 1..64, row vs column-major, scheduler's choice
+    sweep = []
+    x64 = I.make_inputs(64, D, F, seed=2, with_down=False, device="cuda").x
+    wgc, wuc = I.to_layout(inp.w_gate, inp.w_up, I.LAYOUT_COL)
+    for B in (1, 2, 4, 8, 16, 32, 64):
+        xb = x64[:B].contiguous()
+        hb = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+        row = {"B": B}
+        for name, (wg, wu) in (("row", (inp.w_gate, inp.w_up)), ("col", (wgc, wuc))):
+            dfk.dfk_rmsnorm_swiglu_gate_up(xb, inp.gamma, inp.eps, wg, wu, name, h=hb)  # tunes
+            t = timed_us(lambda i: dfk.dfk_rmsnorm_swiglu_gate_up(
+                xb, inp.gamma, inp.eps, wg, wu, name, h=hb), reps, flush)
+            gbs = gate_up_bytes(B, D, F) / (t * 1e-6) / 1e9
+            row[name] = {"us": round(t, 2), "GBps": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        row["scheduler_pick"] = "row" if row["row"]["us"] <= row["col"]["us"] else "col"
+        sweep.append(row)
+    out["batch_sweep"] = sweep
+    return out
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_layer_inputs():
+    from swiglu_mlp_dfk_b200 import inputs as I
+    inp = I.make_inputs(B1, D, F, seed=SEED, w_std=0.02, norm=True, with_down=True,
+                        device="cpu")
+    return [I.to_bits(t) for t in (inp.x, inp.gamma, inp.w_gate, inp.w_up, inp.w_down)]
+
+
+def cpu_baseline(min_s=10.0, max_reps=400):
+    """The fp64 CPU oracle, as it stands, on the full B = 1 layer, repeated ~10 s."""
+    import oracle
+    x, g, wg, wu, wd = _oracle_layer_inputs()
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        hh = oracle.gate_up(x, wg, wu, gamma=g, eps=1e-5)
+        oracle.down(hh, wd)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or reps >= max_reps:
+            break
+    return {"value": round(step_bytes(B1, D, F) * reps / el / 1e9, 3), "unit": UNIT,
+            "cores": oracle.threads(), "kind": "oracle",
+            "sample": "full Llama-3-8B-shaped layer at B=1 (14336 gate/up columns + 4096 "
+                      "down rows), repeated %d times in %.1f s" % (reps, el)}
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 CPU oracle timed on this arm's workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    x, g, wg, wu, wd = _oracle_layer_inputs()
+    # one step = a bounded sample of the layer: 1/8 of the gate/up columns and
+    # 1/8 of the down rows (the metric counts the sample's algorithmic bytes)
+    rows = np.arange(0, F, 8, dtype=np.int32)
+    drows = np.arange(0, D, 8, dtype=np.int32)
+    sample_bytes = (2 * rows.size * D * 2 + B1 * D * 2 + D * 2 + B1 * rows.size * 2
+                    + drows.size * F * 2 + B1 * F * 2 + B1 * drows.size * 2)
+    hfull = oracle.gate_up(x, wg, wu, gamma=g, eps=1e-5)
+
+    def one():
+        oracle.gate_up(x, wg, wu, gamma=g, eps=1e-5, rows=rows)
+        oracle.down(hfull, wd, rows=drows)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    value = sample_bytes * args.steps / el / 1e9
+    sample = ("1/8 of the Llama-3-8B-shaped layer per step (1792 gate/up columns + 512 "
+              "down rows, B=1)")
+    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el * 1e3 / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": config_dict("cpu"),
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["dfk", "reference"], default="dfk")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the sweep / unfused / interleaved measurements")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * dfk.h -- C ABI of libdfk.so, the B200 (sm_100a) decode-stage SwiGLU MLP.
+ *
+ * The method ("Deep Kernel Fusion for Transformer Decoding", episode
+ * description; "Deep Kernel Fusion for Transformers", abstract): at decode
+ * time the SwiGLU MLP is a weight-streaming, memory-bandwidth-bound
+ * matrix-vector product.  The gate projection, the up projection, the SiLU
+ * activation and the elementwise multiply run as ONE kernel, so the gate
+ * and up activations never reach HBM; the down projection stays a separate
+ * kernel; a profiler-driven runtime scheduler picks among row-major and
+ * column-major kernel variants.  The RMSNorm that precedes the MLP can be
+ * fused in front of the gate/up projection (GPULlama3.java PR #78, the
+ * `rms_ffn_gate_up` task).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE memory (unless a function says host),
+ *     contiguous, bf16 (IEEE binary32 upper halves) unless noted.
+ *   - x is [B][d_model] row-major; h is [B][d_ff]; y is [B][d_model].
+ *   - Every device pointer must be 16-byte aligned; d_model % 8 == 0; for the
+ *     column-major layout also d_ff % 8 == 0.  Violations return
+ *     DFK_ERR_MISALIGNED / DFK_ERR_UNSUPPORTED_SHAPE without launching.
+ *   - 0 <= B <= 64 (decode batch).  B == 0 is a no-op returning DFK_OK.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: the return code covers argument validation and
+ *     launch errors only; a device-side failure (a pipeline wait that gave
+ *     up) is recorded in a device error word read by dfk_device_error().
+ *   - `variant` = 0 lets the scheduler choose (timed on first use for the
+ *     shape, cached; never timed while the stream is being captured);
+ *     a positive id forces that variant (dfk_variant_info lists them).
+ *   - Accumulation is fp32; every output is rounded once to bf16
+ *     (round-to-nearest-even).  CUDA-core variants of one operation give
+ *     bit-identical results for every layout, tile and pipeline choice and
+ *     for every batch size (row b of the output depends on row b of x only).
+ *   - There is no CPU fallback: without an sm_100 device every compute call
+ *     returns DFK_ERR_ARCH (or DFK_ERR_CUDA).
+ *   - Thread-safe: the variant cache and descriptor cache are locked.
+ */
+#ifndef DFK_H
+#define DFK_H
+
+#if defined(__GNUC__)
+#define DFK_API __attribute__((visibility("default")))
+#else
+#define DFK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dfk_status {
+  DFK_OK = 0,
+  DFK_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum, bad variant id */
+  DFK_ERR_UNSUPPORTED_SHAPE = 2,  /* B > 64, d_model % 8, d_ff % 8 (column-major), too large */
+  DFK_ERR_UNSUPPORTED_LAYOUT = 3, /* layout not valid for this entry point */
+  DFK_ERR_MISALIGNED = 4,         /* a device pointer is not 16-byte aligned */
+  DFK_ERR_CUDA = 5,               /* a CUDA runtime call failed; see dfk_last_error() */
+  DFK_ERR_ARCH = 6,               /* no sm_100 device current */
+  DFK_ERR_TIMEOUT = 7,            /* a kernel's pipeline wait gave up (dfk_device_error) */
+  DFK_ERR_NO_VARIANT = 8          /* no variant fits this shape (shared memory / threads) */
+} dfk_status;
+
+/* Storage of W_gate / W_up (as stated in the pages: W_gate, W_up are [d_ff, d_model]). */
+typedef enum dfk_wlayout {
+  DFK_W_ROW_MAJOR = 0,      /* w_gate, w_up: [d_ff][d_model] each                        */
+  DFK_W_COL_MAJOR = 1,      /* w_gate, w_up: [d_model][d_ff] each (the transposes)       */
+  DFK_W_GU_INTERLEAVED = 2, /* w_gate: [d_ff][2][d_model], [j][0] = gate row j,
+                               [j][1] = up row j; w_up must be NULL                      */
+  DFK_W_ANY = -1            /* dfk_select_variant only: time every layout               */
+} dfk_wlayout;
+
+typedef enum dfk_op {
+  DFK_OP_GATE_UP = 0,         /* dfk_swiglu_gate_up          */
+  DFK_OP_RMSNORM_GATE_UP = 1, /* dfk_rmsnorm_swiglu_gate_up  */
+  DFK_OP_DOWN = 2             /* dfk_down_proj               */
+} dfk_op;
+
+typedef enum dfk_family {
+  DFK_FAMILY_CUDA_CORE = 0,   /* TMA-fed shared-memory ring, fp32 FMA on CUDA cores   */
+  DFK_FAMILY_TENSOR_CORE = 1  /* tcgen05 MMA with TMEM accumulators                    */
+} dfk_family;
+
+typedef struct dfk_variant {
+  int variant_id;   /* id accepted by the `variant` arguments                        */
+  int op;           /* dfk_op                                                         */
+  int layout;       /* dfk_wlayout the variant reads                                 */
+  int family;       /* dfk_family                                                    */
+  int j_per_thread; /* output columns per thread (CUDA-core)                         */
+  int token_tile;   /* tokens per pass over the weights                              */
+  int k_split;      /* thread teams splitting the reduction dimension               */
+  int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
+  float measured_us;/* median timed duration; < 0 when chosen without timing        */
+} dfk_variant;
+
+/*
+ * h = SiLU(x . W_gate^T) (*) (x . W_up^T)      -- the fused gate/up kernel
+ * ("Deep Kernel Fusion for Transformer Decoding", episode description: the
+ * up projection, gate projection, SiLU and elementwise multiply fused into
+ * one decode kernel).
+ *   x       [B][d_model] bf16, device
+ *   w_gate  per `layout` (dfk_wlayout), bf16, device
+ *   w_up    per `layout`; NULL for DFK_W_GU_INTERLEAVED
+ *   h       [B][d_ff] bf16, device, written once
+ * SiLU(a) = a / (1 + exp(-a)), applied to the gate branch.
+ */
+DFK_API int dfk_swiglu_gate_up(const void *x, const void *w_gate, const void *w_up, int layout,
+                       void *h, int B, int d_model, int d_ff, int variant, void *stream);
+
+/*
+ * Same, with the RMSNorm fused in front (GPULlama3.java PR #78, the
+ * `rms_ffn_gate_up` task):
+ *   xn[b][k] = bf16( x[b][k] * r_b * gamma[k] ),
+ *   r_b = 1 / sqrt( (1/d_model) * sum_k x[b][k]^2 + eps ),
+ * then h = SiLU(xn . W_gate^T) (*) (xn . W_up^T).  xn lives in shared memory
+ * only.  gamma [d_model] bf16, device.  eps >= 0.
+ */
+DFK_API int dfk_rmsnorm_swiglu_gate_up(const void *x, const void *gamma, float eps,
+                               const void *w_gate, const void *w_up, int layout,
+                               void *h, int B, int d_model, int d_ff, int variant,
+                               void *stream);
+
+/*
+ * y = h . W_down^T, the separate down projection ("Deep Kernel Fusion for
+ * Transformer Decoding", episode description: the down projection is left
+ * out of the fused kernel).
+ *   h       [B][d_ff] bf16, device
+ *   w_down  [d_model][d_ff] bf16 row-major, device
+ *   y       [B][d_model] bf16, device
+ */
+DFK_API int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int d_model,
+                  int d_ff, int variant, void *stream);
+
+/*
+ * Profiler-driven variant choice ("Deep Kernel Fusion for Transformer
+ * Decoding", episode description: runtime scheduling across row-major and
+ * column-major kernel variants; "Deep Kernel Fusion for Transformers",
+ * abstract: the kernel is paired with a kernel scheduler).
+ * Times every feasible variant of `op` for (B, d_model, d_ff, layout) with
+ * CUDA events (L2 flushed before each timed call), caches the fastest and
+ * returns it in *out.  layout == DFK_W_ANY times every layout and reports
+ * the fastest layout in out->layout (gate/up ops only).
+ *   sample_ptrs  NULL, or the caller's buffers in argument order of the op:
+ *                gate_up: {x, w_gate, w_up, h}; rmsnorm_gate_up: {x, gamma,
+ *                w_gate, w_up, h}; down: {h, w_down, y}.  With NULL (or with
+ *                DFK_W_ANY) the function allocates throwaway buffers on
+ *                `stream` and frees them before returning.
+ * Returns DFK_ERR_INVALID_ARG if the stream is being captured.
+ * Environment: DFK_TUNE=0 disables timing (heuristic choice),
+ * DFK_TUNE_REPS (default 7) sets the timed repetitions, DFK_LOG=1 logs
+ * decisions to stderr.
+ */
+DFK_API int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
+                       const void *const *sample_ptrs, void *stream, dfk_variant *out);
+
+/* Number of variant ids (valid ids are 1..count) and their description. */
+DFK_API int dfk_variant_count(void);
+DFK_API int dfk_variant_info(int variant_id, dfk_variant *out);
+
+/* Forget every cached scheduler decision (all devices). */
+DFK_API void dfk_clear_variant_cache(void);
+
+/* ---- building blocks of the unfused baseline and of the decode stack -------
+ * These exist to measure what the fusion saves (separate RMSNorm, GEMV,
+ * SiLU and multiply kernels with bf16 intermediates in HBM) and to run a
+ * multi-layer decode loop; they are not part of the fused path. */
+
+/* xn[b][k] = bf16(x[b][k] * r_b * gamma[k]), r_b as in the fused prologue. */
+DFK_API int dfk_rmsnorm(const void *x, const void *gamma, float eps, void *xn, int B, int d,
+                void *stream);
+
+/* out[b][n] = bf16( sum_k x[b][k] * w[n][k] ), w [N][K] row-major bf16. */
+DFK_API int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int variant,
+             void *stream);
+
+/* out[i] = bf16( SiLU(a[i]) ), n elements. */
+DFK_API int dfk_silu(const void *a, void *out, long long n, void *stream);
+
+/* out[i] = bf16( a[i] * b[i] ), n elements. */
+DFK_API int dfk_mul(const void *a, const void *b, void *out, long long n, void *stream);
+
+/* x_next[b][k] = bf16( y[b][k] / sqrt(mean_k y[b][k]^2 + eps) ). */
+DFK_API int dfk_rms_rescale(const void *y, float eps, void *x_next, int B, int d, void *stream);
+
+/*
+ * One MLP layer end to end from HOST memory: copies x_host (pinned or
+ * pageable, [B][d_model] bf16) to the device, runs the fused RMSNorm+gate/up
+ * kernel (gamma may be NULL: no RMSNorm) and the down projection, and copies
+ * y back to y_host ([B][d_model] bf16).  Weights are device-resident.
+ * x_dev, h_dev, y_dev are caller-owned device work buffers of the sizes of
+ * x, h and y.  Synchronises `stream` before returning.
+ */
+DFK_API int dfk_mlp_forward_host(const void *x_host, const void *gamma, float eps,
+                         const void *w_gate, const void *w_up, int layout,
+                         const void *w_down, void *y_host, void *x_dev, void *h_dev,
+                         void *y_dev, int B, int d_model, int d_ff, void *stream);
+
+/* ---- status --------------------------------------------------------------- */
+
+/* Static text for a dfk_status value. */
+DFK_API const char *dfk_status_string(int status);
+
+/* Text of the last error seen by this thread (CUDA error string or a
+ * description of the rejected argument); "" when none. */
+DFK_API const char *dfk_last_error(void);
+
+/* Reads the current device's error word (0 = none; bit 0 = a pipeline wait
+ * timed out) into *code and clears it.  Synchronises the device. */
+DFK_API int dfk_device_error(int *code);
+
+/* Library version, e.g. "dfk 0.1.0 sm_100a". */
+DFK_API const char *dfk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFK_H */

@@ -1,0 +1,314 @@
+"""swiglu_mlp_dfk_b200 -- B200 (sm_100a) decode-stage SwiGLU MLP.
+
+Thin Python binding over the C ABI of ``libdfk.so`` (declared in
+``include/dfk.h``): the functions below carry the C entry points' names and
+only marshal arguments -- torch tensors become device pointers, the current
+torch stream becomes the ``stream`` argument, output tensors are allocated
+when not given.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU path.  If ``libdfk.so`` is missing or no sm_100
+device is present, every compute call raises ``DfkError``.
+
+The method ("Deep Kernel Fusion for Transformer Decoding", episode
+description): gate projection, up projection, SiLU and elementwise multiply
+fused into one decode kernel, the down projection left separate, and a
+profiler-driven scheduler choosing among row-major and column-major kernel
+variants.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdfk.so")
+
+# dfk_wlayout
+DFK_W_ROW_MAJOR = 0
+DFK_W_COL_MAJOR = 1
+DFK_W_GU_INTERLEAVED = 2
+DFK_W_ANY = -1
+# dfk_op
+DFK_OP_GATE_UP = 0
+DFK_OP_RMSNORM_GATE_UP = 1
+DFK_OP_DOWN = 2
+# dfk_status
+DFK_OK = 0
+DFK_ERR_INVALID_ARG = 1
+DFK_ERR_UNSUPPORTED_SHAPE = 2
+DFK_ERR_UNSUPPORTED_LAYOUT = 3
+DFK_ERR_MISALIGNED = 4
+DFK_ERR_CUDA = 5
+DFK_ERR_ARCH = 6
+DFK_ERR_TIMEOUT = 7
+DFK_ERR_NO_VARIANT = 8
+
+_LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W_GU_INTERLEAVED,
+            "any": DFK_W_ANY}
+
+# Every symbol the header declares (the CPU test checks the library exports them all).
+EXPORTED = (
+    "dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj", "dfk_select_variant",
+    "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
+    "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
+    "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
+)
+
+
+class DfkError(RuntimeError):
+    """A libdfk call returned a non-zero dfk_status."""
+
+    def __init__(self, status, msg):
+        super().__init__("%s (status %d)" % (msg, status))
+        self.status = status
+
+
+class dfk_variant(ctypes.Structure):
+    _fields_ = [("variant_id", ctypes.c_int), ("op", ctypes.c_int), ("layout", ctypes.c_int),
+                ("family", ctypes.c_int), ("j_per_thread", ctypes.c_int),
+                ("token_tile", ctypes.c_int), ("k_split", ctypes.c_int),
+                ("stages", ctypes.c_int), ("measured_us", ctypes.c_float)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded libdfk.so (ctypes.CDLL); raises DfkError if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise DfkError(DFK_ERR_ARCH, "libdfk.so is not built (%s); run "
+                               "`python -m swiglu_mlp_dfk_b200.build`" % LIB_PATH)
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+            sig = {
+                "dfk_swiglu_gate_up": [vp, vp, vp, i, vp, i, i, i, i, vp],
+                "dfk_rmsnorm_swiglu_gate_up": [vp, vp, f, vp, vp, i, vp, i, i, i, i, vp],
+                "dfk_down_proj": [vp, vp, vp, i, i, i, i, vp],
+                "dfk_select_variant": [i, i, i, i, i, ctypes.POINTER(vp), vp,
+                                       ctypes.POINTER(dfk_variant)],
+                "dfk_variant_count": [],
+                "dfk_variant_info": [i, ctypes.POINTER(dfk_variant)],
+                "dfk_rmsnorm": [vp, vp, f, vp, i, i, vp],
+                "dfk_gemv": [vp, vp, vp, i, i, i, i, vp],
+                "dfk_silu": [vp, vp, ll, vp],
+                "dfk_mul": [vp, vp, vp, ll, vp],
+                "dfk_rms_rescale": [vp, f, vp, i, i, vp],
+                "dfk_mlp_forward_host": [vp, vp, f, vp, vp, i, vp, vp, vp, vp, vp, i, i, i, vp],
+                "dfk_device_error": [ctypes.POINTER(i)],
+                "dfk_status_string": [i],
+                "dfk_last_error": [],
+                "dfk_version": [],
+            }
+            for name, args in sig.items():
+                fn = getattr(L, name)
+                fn.argtypes = args
+                fn.restype = i
+            for name in ("dfk_status_string", "dfk_last_error", "dfk_version"):
+                getattr(L, name).restype = ctypes.c_char_p
+            L.dfk_clear_variant_cache.argtypes = []
+            L.dfk_clear_variant_cache.restype = None
+            _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != DFK_OK:
+        L = lib()
+        raise DfkError(status, "%s: %s" % (L.dfk_status_string(status).decode(),
+                                           L.dfk_last_error().decode()))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev_bf16(name, t):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise DfkError(DFK_ERR_INVALID_ARG, "%s must be a bf16 CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise DfkError(DFK_ERR_INVALID_ARG, "%s must be contiguous" % name)
+
+
+def _layout(layout):
+    return _LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+
+
+def _gate_up_shapes(x, w_gate, layout):
+    B, D = x.shape
+    if layout == DFK_W_ROW_MAJOR:
+        F = w_gate.shape[0]
+    elif layout == DFK_W_COL_MAJOR:
+        F = w_gate.shape[-1]
+    else:
+        F = w_gate.numel() // (2 * D)
+    return B, D, F
+
+
+def dfk_swiglu_gate_up(x, w_gate, w_up=None, layout=DFK_W_ROW_MAJOR, h=None, variant=0,
+                       stream=None):
+    """h = SiLU(x W_gate^T) * (x W_up^T) in one kernel; returns h [B, d_ff] bf16."""
+    layout = _layout(layout)
+    for n, t in (("x", x), ("w_gate", w_gate), ("w_up", w_up), ("h", h)):
+        _dev_bf16(n, t)
+    B, D, F = _gate_up_shapes(x, w_gate, layout)
+    if h is None:
+        h = torch.empty((B, F), dtype=torch.bfloat16, device=x.device)
+    _check(lib().dfk_swiglu_gate_up(_ptr(x), _ptr(w_gate), _ptr(w_up), layout, _ptr(h), B, D, F,
+                                    int(variant), _stream(stream)))
+    return h
+
+
+def dfk_rmsnorm_swiglu_gate_up(x, gamma, eps, w_gate, w_up=None, layout=DFK_W_ROW_MAJOR, h=None,
+                               variant=0, stream=None):
+    """RMSNorm(x; gamma, eps) fused in front of the gate/up kernel; returns h."""
+    layout = _layout(layout)
+    for n, t in (("x", x), ("gamma", gamma), ("w_gate", w_gate), ("w_up", w_up), ("h", h)):
+        _dev_bf16(n, t)
+    B, D, F = _gate_up_shapes(x, w_gate, layout)
+    if h is None:
+        h = torch.empty((B, F), dtype=torch.bfloat16, device=x.device)
+    _check(lib().dfk_rmsnorm_swiglu_gate_up(_ptr(x), _ptr(gamma), float(eps), _ptr(w_gate),
+                                            _ptr(w_up), layout, _ptr(h), B, D, F, int(variant),
+                                            _stream(stream)))
+    return h
+
+
+def dfk_down_proj(h, w_down, y=None, variant=0, stream=None):
+    """y = h W_down^T (separate kernel); w_down [d_model, d_ff]; returns y [B, d_model]."""
+    for n, t in (("h", h), ("w_down", w_down), ("y", y)):
+        _dev_bf16(n, t)
+    B, F = h.shape
+    D = w_down.shape[0]
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=h.device)
+    _check(lib().dfk_down_proj(_ptr(h), _ptr(w_down), _ptr(y), B, D, F, int(variant),
+                               _stream(stream)))
+    return y
+
+
+def dfk_gemv(x, w, out=None, variant=0, stream=None):
+    """out = x W^T with W [N, K] row-major (unfused-baseline building block)."""
+    for n, t in (("x", x), ("w", w), ("out", out)):
+        _dev_bf16(n, t)
+    B, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().dfk_gemv(_ptr(x), _ptr(w), _ptr(out), B, K, N, int(variant), _stream(stream)))
+    return out
+
+
+def dfk_rmsnorm(x, gamma, eps, out=None, stream=None):
+    """Standalone RMSNorm (unfused-baseline building block)."""
+    for n, t in (("x", x), ("gamma", gamma), ("out", out)):
+        _dev_bf16(n, t)
+    B, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().dfk_rmsnorm(_ptr(x), _ptr(gamma), float(eps), _ptr(out), B, D, _stream(stream)))
+    return out
+
+
+def dfk_rms_rescale(y, eps=1e-5, out=None, stream=None):
+    """out = y / sqrt(mean(y^2) + eps) per row (decode-stack step input)."""
+    for n, t in (("y", y), ("out", out)):
+        _dev_bf16(n, t)
+    B, D = y.shape
+    if out is None:
+        out = torch.empty_like(y)
+    _check(lib().dfk_rms_rescale(_ptr(y), float(eps), _ptr(out), B, D, _stream(stream)))
+    return out
+
+
+def dfk_silu(a, out=None, stream=None):
+    """out = SiLU(a) elementwise (unfused-baseline building block)."""
+    _dev_bf16("a", a)
+    if out is None:
+        out = torch.empty_like(a)
+    _dev_bf16("out", out)
+    _check(lib().dfk_silu(_ptr(a), _ptr(out), a.numel(), _stream(stream)))
+    return out
+
+
+def dfk_mul(a, b, out=None, stream=None):
+    """out = a * b elementwise (unfused-baseline building block)."""
+    _dev_bf16("a", a)
+    _dev_bf16("b", b)
+    if out is None:
+        out = torch.empty_like(a)
+    _dev_bf16("out", out)
+    _check(lib().dfk_mul(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)))
+    return out
+
+
+def dfk_mlp_forward_host(x_host, gamma, eps, w_gate, w_up, layout, w_down, y_host, x_dev, h_dev,
+                         y_dev, stream=None):
+    """One MLP layer from host memory: x_host -> device -> gate/up -> down -> y_host."""
+    layout = _layout(layout)
+    for n, t in (("gamma", gamma), ("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down),
+                 ("x_dev", x_dev), ("h_dev", h_dev), ("y_dev", y_dev)):
+        _dev_bf16(n, t)
+    B, D = x_host.shape
+    F = h_dev.shape[1]
+    _check(lib().dfk_mlp_forward_host(_ptr(x_host), _ptr(gamma), float(eps), _ptr(w_gate),
+                                      _ptr(w_up), layout, _ptr(w_down), _ptr(y_host),
+                                      _ptr(x_dev), _ptr(h_dev), _ptr(y_dev), B, D, F,
+                                      _stream(stream)))
+    return y_host
+
+
+def dfk_select_variant(op, B, d_model, d_ff, layout=DFK_W_ROW_MAJOR, sample=None, stream=None):
+    """Time the variants of ``op`` for the shape and cache the winner; returns a dict."""
+    layout = _layout(layout)
+    out = dfk_variant()
+    arr = None
+    if sample is not None:
+        arr = (ctypes.c_void_p * len(sample))(*[None if t is None else t.data_ptr()
+                                                for t in sample])
+    _check(lib().dfk_select_variant(int(op), int(B), int(d_model), int(d_ff), layout, arr,
+                                    _stream(stream), ctypes.byref(out)))
+    return out.as_dict()
+
+
+def dfk_variant_count():
+    return lib().dfk_variant_count()
+
+
+def dfk_variant_info(variant_id):
+    out = dfk_variant()
+    _check(lib().dfk_variant_info(int(variant_id), ctypes.byref(out)))
+    return out.as_dict()
+
+
+def dfk_clear_variant_cache():
+    lib().dfk_clear_variant_cache()
+
+
+def dfk_device_error():
+    """Read and clear the device error word; returns the code (0 = none)."""
+    code = ctypes.c_int(0)
+    st = lib().dfk_device_error(ctypes.byref(code))
+    if st not in (DFK_OK, DFK_ERR_TIMEOUT):
+        _check(st)
+    return code.value
+
+
+def dfk_version():
+    return lib().dfk_version().decode()

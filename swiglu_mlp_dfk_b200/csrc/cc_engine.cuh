@@ -1,0 +1,435 @@
+// cc_engine.cuh -- CUDA-core weight-streaming GEMV engine for sm_100a.
+//
+// One kernel template covers
+//   * the fused gate/up kernel (NMAT = 2): h = SiLU(xn . Wg^T) * (xn . Wu^T),
+//     optionally with the RMSNorm prologue (NORM) -- "Deep Kernel Fusion for
+//     Transformer Decoding", episode description (gate, up, SiLU and multiply
+//     in one decode kernel) and GPULlama3.java PR #78 (`rms_ffn_gate_up`);
+//   * a plain GEMV (NMAT = 1): out = x . W^T, used for the separate down
+//     projection and for the unfused baseline.
+//
+// Data flow per CTA (one CTA per SM, persistent over its share of outputs):
+//   - a producer warp streams weight tiles [rows x 64 k] of every matrix
+//     through an S-stage shared-memory ring with TMA (cp.async.bulk.tensor),
+//     each tile read from HBM exactly once for all B tokens and both
+//     projections; mbarriers carry the full/empty hand-off;
+//   - consumer warps hold the (normalised) activations in shared memory,
+//     multiply-accumulate in fp32 registers, reduce across the 8 slots of a
+//     tile row, apply SiLU(a)*u in registers and store h once as bf16.
+//
+// Canonical summation order (shared by every layout and every tile, thread
+// and pipeline choice of the CUDA-core family, so that row-major,
+// column-major and interleaved weights give bit-identical results):
+//   k = 64 t + 8 s + e  (tile t, slot s in [0,8), element e in [0,8));
+//   with KSPLIT teams, team c owns the tiles t = c (mod KSPLIT).
+//   p[c][s] = fp32 chain from +0 over its tiles t ascending, then e
+//             ascending:  p = fma(xn[b][k], W[j][k], p);
+//   q[c]    = ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7));
+//   total   = left fold q[0] + q[1] + ... + q[KSPLIT-1].
+// Products of two bf16 values are exact in fp32, so fma and mul+add agree;
+// only the order above matters.  Tokens never interact, so row b of the
+// output is independent of the batch size.
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace dfk {
+
+constexpr int TILE_K = 64;          // reduction elements per tile row (128 bytes)
+constexpr int NSLOT = 8;            // 16-byte slots per tile row
+constexpr int CC_MAX_THREADS = 512; // consumers + one producer warp
+
+enum : int { LAYOUT_ROW = 0, LAYOUT_COL = 1, LAYOUT_IL = 2 };
+
+struct CcParams {
+  const uint16_t *x;      // [B][K] bf16 activations
+  const uint16_t *gamma;  // [K] bf16 RMSNorm weight (NORM only)
+  uint16_t *out;          // [B][N] bf16
+  unsigned *err;          // device error word
+  int B, K, N;
+  float eps;
+  int nsteps;       // ring steps per pass = ceil(ceil(K/64) / KSPLIT)
+  int kpad;         // nsteps * KSPLIT * 64: activation row pitch in shared memory
+  int granule;      // output rows per partition unit
+  int ubase, uextra;// units per CTA: ubase, +1 for the first uextra CTAs
+  int r_hi;         // largest row count of any CTA (shared-memory slot size)
+  int stages;       // ring depth
+  int stage_bytes;  // KSPLIT * NMAT * r_hi * 128
+  int npass;        // ceil(B / BT)
+  int tpt;          // consumer threads per K team (multiple of 32)
+  int xs_off;       // shared-memory offset of the activation / reduction area
+  int bar_off;      // shared-memory offset of the barrier area
+};
+
+// Tensor maps: index matrix * 2 + (CTA has the short row count ? 1 : 0).
+struct CcMaps {
+  CUtensorMap m[4];
+};
+
+template <int NMAT, int JPT, int BT>
+struct CcAcc {
+  float v[NMAT][JPT][BT];
+};
+
+template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NORM>
+__global__ void __launch_bounds__(CC_MAX_THREADS, 1)
+    cc_gemv_kernel(const __grid_constant__ CcMaps maps, const CcParams p) {
+  static_assert(LAYOUT != LAYOUT_IL || NMAT == 2, "interleaved layout holds both matrices");
+  static_assert(JPT == 2 || JPT == 4, "JPT");
+  extern __shared__ __align__(1024) uint8_t smem[];
+
+  const int tid = threadIdx.x;
+  const int nthr = blockDim.x;
+  const int ncons = nthr - 32;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int S = p.stages;
+
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+  uint64_t *empty = full + S;
+  volatile int *s_abort = reinterpret_cast<volatile int *>(empty + S);
+  int *s_issued = reinterpret_cast<int *>(empty + S) + 1;
+  float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(empty + S) + 16);
+
+  // ---- this CTA's contiguous share of output rows [j0, j0 + r)
+  const int cta = blockIdx.x;
+  const int u0 = cta * p.ubase + min(cta, p.uextra);
+  const int nu = p.ubase + (cta < p.uextra ? 1 : 0);
+  const int j0 = u0 * p.granule;
+  const int r = nu * p.granule;
+  const int mi = (r == p.r_hi) ? 0 : 1;
+  const uint32_t slot_bytes = static_cast<uint32_t>(p.r_hi) * TILE_K * 2;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncons / 32);
+    }
+    *s_abort = 0;
+    *s_issued = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+
+  const int total_steps = p.npass * p.nsteps;
+
+  if (warp == (nthr >> 5) - 1) {
+    // ================= producer warp: one lane issues all TMA traffic
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      const uint32_t tile_bytes = static_cast<uint32_t>(r) * TILE_K * 2;
+      const uint32_t tx = tile_bytes * NMAT * KSPLIT;
+      int issued = 0;
+      for (int i = 0; i < total_steps; ++i) {
+        const int st = i % S;
+        if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
+        const int step = i % p.nsteps;
+        uint8_t *base = smem + static_cast<size_t>(st) * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[st], tx);
+#pragma unroll
+        for (int kt = 0; kt < KSPLIT; ++kt) {
+          const int k0 = (step * KSPLIT + kt) * TILE_K;
+          uint8_t *tb = base + static_cast<size_t>(kt) * NMAT * slot_bytes;
+          if (LAYOUT == LAYOUT_ROW) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+              tma_load_2d(tb + m * slot_bytes, &maps.m[m * 2 + mi], &full[st], k0, j0, pol);
+          } else if (LAYOUT == LAYOUT_COL) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+              tma_load_2d(tb + m * slot_bytes, &maps.m[m * 2 + mi], &full[st], j0, k0, pol);
+          } else {
+            // interleaved rows [2 j0, 2 j0 + 2r) as two boxes of r rows
+            tma_load_2d(tb, &maps.m[mi], &full[st], k0, 2 * j0, pol);
+            tma_load_2d(tb + tile_bytes, &maps.m[mi], &full[st], k0, 2 * j0 + r, pol);
+          }
+        }
+        issued = i + 1;
+      }
+      *s_issued = issued;
+    }
+  } else {
+    // ================= consumer warps
+    const int team = tid / p.tpt;
+    const int lt = tid - team * p.tpt;
+    int s, q;
+    if (LAYOUT == LAYOUT_COL) {
+      s = (lt >> 5) & 7;                  // a warp shares one slot
+      q = (lt >> 8) * 32 + (lt & 31);     // lanes walk consecutive column groups
+    } else {
+      s = lt & 7;                         // 8 lanes cover one 128-byte tile row
+      q = lt >> 3;
+    }
+    const int jl0 = q * JPT;              // first local output row of this thread
+    const bool active = jl0 < r;
+    const int cw = tid >> 5, ncw = ncons >> 5;
+
+    float *xs_f = reinterpret_cast<float *>(smem + p.xs_off);
+    uint16_t *xs_h = reinterpret_cast<uint16_t *>(smem + p.xs_off);
+    float *red = reinterpret_cast<float *>(smem + p.xs_off);  // reused after the K loop
+
+    pdl_wait();  // activations come from the previous kernel in the stream
+
+    for (int pass = 0; pass < p.npass; ++pass) {
+      const int b0 = pass * BT;
+
+      // ---- prologue: RMS statistics (one warp per token, fixed order)
+      if (NORM) {
+        for (int bb = cw; bb < BT; bb += ncw) {
+          float ss = 0.f;
+          if (b0 + bb < p.B) {
+            const uint16_t *xr = p.x + static_cast<size_t>(b0 + bb) * p.K;
+            for (int k = 8 * lane; k < p.K; k += 256) {
+              const uint4 v = ld_nc_v4(xr + k);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float f0 = bf16_lo(w[i]), f1 = bf16_hi(w[i]);
+                ss = fmaf(f0, f0, ss);
+                ss = fmaf(f1, f1, ss);
+              }
+            }
+          }
+#pragma unroll
+          for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+          if (lane == 0) s_rinv[bb] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+        }
+        named_barrier(1, ncons);
+      }
+
+      // ---- prologue: activations into shared memory (fp32, or bf16 bits)
+      {
+        const int c8n = p.kpad >> 3;
+        for (int idx = tid; idx < BT * c8n; idx += ncons) {
+          const int bb = idx / c8n;
+          const int k = (idx - bb * c8n) * 8;
+          float f[8];
+          if (b0 + bb < p.B && k < p.K) {
+            const uint4 v = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              f[2 * i] = bf16_lo(w[i]);
+              f[2 * i + 1] = bf16_hi(w[i]);
+            }
+            if (NORM) {
+              const uint4 gv = ld_nc_v4(p.gamma + k);
+              const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
+              const float rr = s_rinv[bb];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                f[2 * i] = round_bf16((f[2 * i] * rr) * bf16_lo(g[i]));
+                f[2 * i + 1] = round_bf16((f[2 * i + 1] * rr) * bf16_hi(g[i]));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+          }
+          if (XF32) {
+            // within a 64-wide tile, element 8s + 4h + i sits at 32h + 4s + i
+            float *row = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63);
+            const int s8 = (k >> 3) & 7;
+            *reinterpret_cast<float4 *>(row + 4 * s8) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4 *>(row + 32 + 4 * s8) = make_float4(f[4], f[5], f[6], f[7]);
+          } else {
+            uint4 o;
+            o.x = __float_as_uint(f[0]) >> 16 | (__float_as_uint(f[1]) & 0xffff0000u);
+            o.y = __float_as_uint(f[2]) >> 16 | (__float_as_uint(f[3]) & 0xffff0000u);
+            o.z = __float_as_uint(f[4]) >> 16 | (__float_as_uint(f[5]) & 0xffff0000u);
+            o.w = __float_as_uint(f[6]) >> 16 | (__float_as_uint(f[7]) & 0xffff0000u);
+            *reinterpret_cast<uint4 *>(xs_h + static_cast<size_t>(bb) * p.kpad + k) = o;
+          }
+        }
+        named_barrier(1, ncons);
+      }
+
+      // ---- main loop over the weight stream
+      CcAcc<NMAT, JPT, BT> acc;
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+        for (int jj = 0; jj < JPT; ++jj)
+#pragma unroll
+          for (int bb = 0; bb < BT; ++bb) acc.v[m][jj][bb] = 0.f;
+
+      for (int step = 0; step < p.nsteps; ++step) {
+        const int i = pass * p.nsteps + step;
+        const int st = i % S;
+        const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
+        if (ok && active) {
+          const int t = step * KSPLIT + team;
+          const uint8_t *tb = smem + static_cast<size_t>(st) * p.stage_bytes +
+                              static_cast<size_t>(team) * NMAT * slot_bytes;
+          float xv[BT][8];
+#pragma unroll
+          for (int bb = 0; bb < BT; ++bb) {
+            if (XF32) {
+              const float *row = xs_f + static_cast<size_t>(bb) * p.kpad + t * TILE_K;
+              const float4 lo = *reinterpret_cast<const float4 *>(row + 4 * s);
+              const float4 hi = *reinterpret_cast<const float4 *>(row + 32 + 4 * s);
+              xv[bb][0] = lo.x; xv[bb][1] = lo.y; xv[bb][2] = lo.z; xv[bb][3] = lo.w;
+              xv[bb][4] = hi.x; xv[bb][5] = hi.y; xv[bb][6] = hi.z; xv[bb][7] = hi.w;
+            } else {
+              const uint4 v = *reinterpret_cast<const uint4 *>(
+                  xs_h + static_cast<size_t>(bb) * p.kpad + t * TILE_K + 8 * s);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int ii = 0; ii < 4; ++ii) {
+                xv[bb][2 * ii] = bf16_lo(w[ii]);
+                xv[bb][2 * ii + 1] = bf16_hi(w[ii]);
+              }
+            }
+          }
+          if (LAYOUT != LAYOUT_COL) {
+            // thread reads 8 consecutive k of each of its rows (one 16-byte slot)
+            uint32_t wv[NMAT][JPT][4];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+              for (int jj = 0; jj < JPT; ++jj) {
+                const int row = (LAYOUT == LAYOUT_IL) ? 2 * (jl0 + jj) + m : jl0 + jj;
+                const uint8_t *bse = (LAYOUT == LAYOUT_IL) ? tb : tb + m * slot_bytes;
+                const uint4 v = *reinterpret_cast<const uint4 *>(bse + row * (TILE_K * 2) + s * 16);
+                wv[m][jj][0] = v.x; wv[m][jj][1] = v.y; wv[m][jj][2] = v.z; wv[m][jj][3] = v.w;
+              }
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                for (int jj = 0; jj < JPT; ++jj) {
+                  const uint32_t w = wv[m][jj][e >> 1];
+                  const float wf = (e & 1) ? bf16_hi(w) : bf16_lo(w);
+#pragma unroll
+                  for (int bb = 0; bb < BT; ++bb)
+                    acc.v[m][jj][bb] = fmaf(xv[bb][e], wf, acc.v[m][jj][bb]);
+                }
+          } else {
+            // column-major tile [64 k][r j]: thread reads JPT consecutive j per k row
+            const int pitch = r * 2;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int krow = 8 * s + e;
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m) {
+                const uint8_t *src = tb + m * slot_bytes + krow * pitch + jl0 * 2;
+                uint32_t w[JPT / 2];
+                if constexpr (JPT == 4) {
+                  const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                  w[0] = v.x;
+                  w[1] = v.y;
+                } else {
+                  w[0] = *reinterpret_cast<const uint32_t *>(src);
+                }
+#pragma unroll
+                for (int jj = 0; jj < JPT; ++jj) {
+                  const float wf = (jj & 1) ? bf16_hi(w[jj >> 1]) : bf16_lo(w[jj >> 1]);
+#pragma unroll
+                  for (int bb = 0; bb < BT; ++bb)
+                    acc.v[m][jj][bb] = fmaf(xv[bb][e], wf, acc.v[m][jj][bb]);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
+
+      // ---- reduce over the 8 slots, fold the K teams, SwiGLU epilogue
+      if (LAYOUT != LAYOUT_COL) {
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+          for (int jj = 0; jj < JPT; ++jj)
+#pragma unroll
+            for (int bb = 0; bb < BT; ++bb) {
+              float v = acc.v[m][jj][bb];
+              v += __shfl_xor_sync(0xffffffffu, v, 4);
+              v += __shfl_xor_sync(0xffffffffu, v, 2);
+              v += __shfl_xor_sync(0xffffffffu, v, 1);
+              acc.v[m][jj][bb] = v;
+            }
+      }
+      named_barrier(1, ncons);  // activation reads done: `red` aliases them
+      const int rh = p.r_hi;
+      if (active) {
+        if (LAYOUT != LAYOUT_COL) {
+          if (s == 0) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+              for (int jj = 0; jj < JPT; ++jj)
+#pragma unroll
+                for (int bb = 0; bb < BT; ++bb)
+                  red[((team * NMAT + m) * BT + bb) * rh + jl0 + jj] = acc.v[m][jj][bb];
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+            for (int jj = 0; jj < JPT; ++jj)
+#pragma unroll
+              for (int bb = 0; bb < BT; ++bb)
+                red[(((team * NSLOT + s) * NMAT + m) * BT + bb) * rh + jl0 + jj] =
+                    acc.v[m][jj][bb];
+        }
+      }
+      named_barrier(1, ncons);
+      const bool aborted = *s_abort != 0;
+      for (int o = tid; o < BT * r; o += ncons) {
+        const int bb = o / r;
+        const int jl = o - bb * r;
+        const int b = b0 + bb, j = j0 + jl;
+        float v[NMAT];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          float tot = 0.f;
+#pragma unroll
+          for (int kt = 0; kt < KSPLIT; ++kt) {
+            float tk;
+            if (LAYOUT == LAYOUT_COL) {
+              const float *pp = red + ((kt * NSLOT * NMAT + m) * BT + bb) * rh + jl;
+              const int ss = NMAT * BT * rh;  // slot stride
+              tk = ((pp[0] + pp[4 * ss]) + (pp[2 * ss] + pp[6 * ss])) +
+                   ((pp[1 * ss] + pp[5 * ss]) + (pp[3 * ss] + pp[7 * ss]));
+            } else {
+              tk = red[((kt * NMAT + m) * BT + bb) * rh + jl];
+            }
+            tot = (kt == 0) ? tk : tot + tk;
+          }
+          v[m] = tot;
+        }
+        if (!aborted && b < p.B && j < p.N) {
+          float res;
+          if (NMAT == 2) {
+            const float a = v[0];
+            res = (a / (1.0f + expf(-a))) * v[NMAT - 1];
+          } else {
+            res = v[0];
+          }
+          p.out[static_cast<size_t>(b) * p.N + j] = f32_to_bf16_bits(res);
+        }
+      }
+      named_barrier(1, ncons);  // `red` / activations are rewritten by the next pass
+    }
+  }
+
+  __syncthreads();
+  // After an aborted pipeline, wait (bounded) for this CTA's copies still in
+  // flight before shared memory is released.
+  if (tid == nthr - 32 && *s_abort) {
+    const int issued = *s_issued;
+    for (int st = 0; st < S; ++st) {
+      int last = -1;
+      for (int i = issued - 1; i >= 0 && i >= issued - S; --i)
+        if (i % S == st) { last = i; break; }
+      if (last >= 0) mbar_wait_bounded(&full[st], (last / S) & 1, nullptr, p.err);
+    }
+  }
+}
+
+}  // namespace dfk

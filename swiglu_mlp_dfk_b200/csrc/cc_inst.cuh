@@ -1,0 +1,18 @@
+// cc_inst.cuh -- instantiation helpers for the CUDA-core engine.  Each
+// cc_inst_*.cu file instantiates a slice of the template space (so the
+// slices compile in parallel) and exposes a lookup by key.
+#pragma once
+#include "cc_engine.cuh"
+#include "cc_key.h"
+
+#define DFK_CC_CASE(L, NM, J, BT, KS, XF, NO)                    \
+  case DFK_CC_KEY(L, NM, J, BT, KS, XF, NO):                     \
+    return reinterpret_cast<const void *>(                       \
+        &dfk::cc_gemv_kernel<L, NM, J, BT, KS, (XF) != 0, (NO) != 0>);
+
+// every (j_per_thread, token_tile) pair compiled
+#define DFK_CC_JB(L, NM, KS, XF, NO)                                                 \
+  DFK_CC_CASE(L, NM, 4, 1, KS, XF, NO) DFK_CC_CASE(L, NM, 4, 2, KS, XF, NO)          \
+  DFK_CC_CASE(L, NM, 4, 4, KS, XF, NO) DFK_CC_CASE(L, NM, 2, 1, KS, XF, NO)          \
+  DFK_CC_CASE(L, NM, 2, 2, KS, XF, NO) DFK_CC_CASE(L, NM, 2, 4, KS, XF, NO)          \
+  DFK_CC_CASE(L, NM, 2, 8, KS, XF, NO)

@@ -1,0 +1,13 @@
+// Fused gate/up, column-major weights [D][F] x2.
+#include "cc_inst.cuh"
+namespace dfk {
+const void *cc_lookup_col(int key) {
+  switch (key) {
+    DFK_CC_JB(1, 2, 1, 1, 0)
+    DFK_CC_JB(1, 2, 1, 1, 1)
+    DFK_CC_JB(1, 2, 1, 0, 0)
+    DFK_CC_JB(1, 2, 1, 0, 1)
+    default: return nullptr;
+  }
+}
+}  // namespace dfk

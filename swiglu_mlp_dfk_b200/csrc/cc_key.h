@@ -1,0 +1,18 @@
+// cc_key.h -- key of one compiled CUDA-core engine instantiation.
+#pragma once
+
+// layout (2 bits) | matrices (2) | j per thread (4) | token tile (4) |
+// k split (4) | fp32 activations (1) | RMSNorm prologue (1)
+#define DFK_CC_KEY(L, NM, J, BT, KS, XF, NO)                                     \
+  ((L) | ((NM) << 2) | ((J) << 4) | ((BT) << 8) | ((KS) << 12) | ((XF) << 16) | \
+   ((NO) << 17))
+
+namespace dfk {
+// Pointer to the __global__ function for a key, or nullptr if not compiled.
+const void *cc_find_kernel(int key);
+const void *cc_lookup_row(int key);
+const void *cc_lookup_col(int key);
+const void *cc_lookup_il(int key);
+const void *cc_lookup_gemv_a(int key);
+const void *cc_lookup_gemv_b(int key);
+}  // namespace dfk

@@ -1,0 +1,938 @@
+// dfk_api.cu -- the C ABI of libdfk.so: argument validation, work
+// partitioning, TMA descriptor cache, the profiler-driven variant scheduler
+// and the launches.  Declarations and argument contracts: include/dfk.h.
+//
+// Scheduler ("Deep Kernel Fusion for Transformer Decoding", episode
+// description: profiler-driven runtime scheduling across row-major and
+// column-major kernel variants; "Deep Kernel Fusion for Transformers",
+// abstract: the fused kernel is paired with a kernel scheduler): on the
+// first call for a (device, op, B, d_model, d_ff, layout) the candidate
+// variants are timed with CUDA events on the caller's stream, L2 flushed
+// before every timed call, and the fastest is cached.  During stream capture
+// nothing is timed: a cached winner or the heuristic default is used.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "cc_engine.cuh"
+#include "cc_key.h"
+#include "dfk.h"
+#include "launch_util.h"
+
+// Device error word: bit 0 = a pipeline wait in some kernel gave up.
+__device__ unsigned g_dfk_err;
+
+namespace dfk {
+
+// ---------------------------------------------------------------- errors
+
+static thread_local std::string t_last_error;
+
+static int fail(int status, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return status;
+}
+
+static int cuda_fail(cudaError_t e, const char *what) {
+  return fail(DFK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool env_flag(const char *name, bool dflt) {
+  const char *v = getenv(name);
+  if (!v || !*v) return dflt;
+  return !(v[0] == '0' || v[0] == 'n' || v[0] == 'N' || v[0] == 'f' || v[0] == 'F');
+}
+
+static int env_int(const char *name, int dflt) {
+  const char *v = getenv(name);
+  if (!v || !*v) return dflt;
+  return atoi(v);
+}
+
+static void log_msg(const char *fmt, ...) {
+  if (!env_flag("DFK_LOG", false)) return;
+  va_list ap;
+  va_start(ap, fmt);
+  fprintf(stderr, "[dfk] ");
+  vfprintf(stderr, fmt, ap);
+  fprintf(stderr, "\n");
+  va_end(ap);
+}
+
+// ---------------------------------------------------------------- kernels table
+
+const void *cc_find_kernel(int key) {
+  const void *f = nullptr;
+  if ((f = cc_lookup_row(key))) return f;
+  if ((f = cc_lookup_col(key))) return f;
+  if ((f = cc_lookup_il(key))) return f;
+  if ((f = cc_lookup_gemv_a(key))) return f;
+  if ((f = cc_lookup_gemv_b(key))) return f;
+  return nullptr;
+}
+
+// ---------------------------------------------------------------- devices
+
+struct DeviceState {
+  bool init = false;
+  int sms = 0;
+  int major = 0, minor = 0;
+  int smem_optin = 0;
+  int l2_bytes = 0;
+  unsigned *err = nullptr;
+};
+
+static std::mutex g_mu;
+static std::map<int, DeviceState> g_dev;
+
+static int current_device(DeviceState **out, int *dev_out = nullptr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(DFK_ERR_ARCH, "no CUDA device: %s", cudaGetErrorString(e));
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState &st = g_dev[dev];
+  if (!st.init) {
+    if ((e = cudaDeviceGetAttribute(&st.major, cudaDevAttrComputeCapabilityMajor, dev)) ||
+        (e = cudaDeviceGetAttribute(&st.minor, cudaDevAttrComputeCapabilityMinor, dev)) ||
+        (e = cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev)) ||
+        (e = cudaDeviceGetAttribute(&st.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                    dev)) ||
+        (e = cudaDeviceGetAttribute(&st.l2_bytes, cudaDevAttrL2CacheSize, dev))) {
+      cudaGetLastError();
+      return fail(DFK_ERR_ARCH, "device query failed: %s", cudaGetErrorString(e));
+    }
+    if (st.major != 10)
+      return fail(DFK_ERR_ARCH, "device %d is sm_%d%d; this library runs on sm_100 only", dev,
+                  st.major, st.minor);
+    if ((e = cudaGetSymbolAddress(reinterpret_cast<void **>(&st.err), g_dfk_err))) {
+      cudaGetLastError();
+      return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    }
+    st.init = true;
+  }
+  *out = &st;
+  if (dev_out) *dev_out = dev;
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn g_encode = nullptr;
+
+static int get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return DFK_OK;
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+    cudaGetLastError();
+    return fail(DFK_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  }
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return DFK_OK;
+}
+
+using MapKey = std::tuple<uintptr_t, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t>;
+static std::map<MapKey, CUtensorMap> g_maps;
+
+// 2-D bf16 tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
+// between rows, box of box_inner x box_outer, no swizzle, zero fill outside.
+static int tensor_map_2d(const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
+                         uint32_t box_inner, uint32_t box_outer, CUtensorMap *out) {
+  int rc = get_encoder();
+  if (rc) return rc;
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), inner, outer, pitch, box_inner, box_outer};
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return DFK_OK;
+    }
+  }
+  CUtensorMap m;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DFK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llux%llu box %ux%u",
+                static_cast<int>(r), static_cast<unsigned long long>(inner),
+                static_cast<unsigned long long>(outer), box_inner, box_outer);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps[key] = m;
+  *out = m;
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- variants
+
+enum { CLS_GATE_UP = 0, CLS_GEMV = 1 };
+
+struct VDef {
+  int id;
+  int cls;
+  int family;
+  int jpt, bt, ksplit;
+};
+
+static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
+
+static const std::vector<VDef> &variants() {
+  static std::vector<VDef> v = [] {
+    std::vector<VDef> t;
+    int id = 1;
+    for (auto &jb : kJB) t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1});
+    for (int ks : {1, 2, 4, 8})
+      for (auto &jb : kJB) t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks});
+    return t;
+  }();
+  return v;
+}
+
+static const VDef *find_variant(int id) {
+  for (const VDef &d : variants())
+    if (d.id == id) return &d;
+  return nullptr;
+}
+
+static int next_pow2(int b) {
+  int p = 1;
+  while (p < b) p <<= 1;
+  return p;
+}
+
+// Token tile a variant family uses for batch B (largest compiled tile for
+// its j-per-thread: 4 tokens with 4 rows per thread, 8 with 2).
+static int bt_for(int B, int jpt) { return std::min(next_pow2(std::max(B, 1)), jpt == 4 ? 4 : 8); }
+
+// ---------------------------------------------------------------- CUDA-core plan
+
+struct CcPlan {
+  const void *fn = nullptr;
+  int grid = 0, block = 0;
+  size_t smem = 0;
+  int r_lo = 0;
+  bool xf32 = true;
+  CcParams p{};
+};
+
+static int ceil_div(int a, int b) { return (a + b - 1) / b; }
+static int round_up(int a, int b) { return ceil_div(a, b) * b; }
+
+// Partition N output rows over the SMs and size the shared-memory ring.
+static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
+                    const DeviceState &ds, CcPlan *pl, std::string *why) {
+  const int g = (layout == LAYOUT_COL) ? 8 : 4;
+  const int U = ceil_div(N, g);
+  const int smem_cap = std::min(ds.smem_optin, 232448);
+  for (int mult = 1; mult <= 16; mult *= 2) {
+    const int P = std::min(U, ds.sms * mult);
+    const int ubase = U / P, uextra = U % P;
+    const int r_hi = (ubase + (uextra ? 1 : 0)) * g;
+    const int r_lo = ubase * g;
+    if (r_hi > 256) continue;  // TMA box limit
+    const int nq = r_hi / v.jpt;
+    const int tpt = (layout == LAYOUT_COL) ? 256 * ceil_div(nq, 32) : round_up(8 * nq, 32);
+    const int ncons = v.ksplit * tpt;
+    if (ncons + 32 > CC_MAX_THREADS) continue;
+    const int nT = ceil_div(K, TILE_K);
+    const int nsteps = ceil_div(nT, v.ksplit);
+    const int kpad = nsteps * v.ksplit * TILE_K;
+    const int stage_bytes = v.ksplit * nmat * r_hi * TILE_K * 2;
+    const int red_bytes = v.ksplit * (layout == LAYOUT_COL ? NSLOT : 1) * nmat * v.bt * r_hi * 4;
+    const int bar_bytes = 256;
+    int best_s = 0, best_region = 0;
+    bool best_xf32 = true;
+    for (int xf = 1; xf >= 0; --xf) {
+      const int xs_bytes = v.bt * kpad * (xf ? 4 : 2);
+      const int region = round_up(std::max(xs_bytes, red_bytes), 128);
+      const int avail = smem_cap - region - bar_bytes;
+      const int S = avail > 0 ? std::min(8, avail / stage_bytes) : 0;
+      if (xf && S >= 4) { best_s = S; best_region = region; best_xf32 = true; break; }
+      if (S > best_s) { best_s = S; best_region = region; best_xf32 = xf != 0; }
+    }
+    if (best_s < 2) {
+      if (why) *why = "shared memory too small for two ring stages";
+      continue;
+    }
+    const int key = DFK_CC_KEY(layout, nmat, v.jpt, v.bt, v.ksplit, best_xf32 ? 1 : 0,
+                               norm ? 1 : 0);
+    const void *fn = cc_find_kernel(key);
+    if (!fn) {
+      if (why) *why = "variant not compiled for this layout";
+      return false;
+    }
+    pl->fn = fn;
+    pl->grid = P;
+    pl->block = ncons + 32;
+    pl->r_lo = r_lo;
+    pl->xf32 = best_xf32;
+    CcParams &p = pl->p;
+    p = CcParams{};
+    p.K = K;
+    p.N = N;
+    p.B = B;
+    p.nsteps = nsteps;
+    p.kpad = kpad;
+    p.granule = g;
+    p.ubase = ubase;
+    p.uextra = uextra;
+    p.r_hi = r_hi;
+    p.stages = best_s;
+    p.stage_bytes = stage_bytes;
+    p.npass = ceil_div(B, v.bt);
+    p.tpt = tpt;
+    p.xs_off = best_s * stage_bytes;
+    p.bar_off = p.xs_off + best_region;
+    pl->smem = static_cast<size_t>(p.bar_off) + bar_bytes;
+    return true;
+  }
+  if (why && why->empty()) *why = "no partition fits the thread / TMA-box limits";
+  return false;
+}
+
+static std::mutex g_attr_mu;
+static std::map<std::pair<int, const void *>, bool> g_attr_done;
+
+static int ensure_smem_attr(int dev, const void *fn) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  auto k = std::make_pair(dev, fn);
+  if (g_attr_done.count(k)) return DFK_OK;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaFuncSetAttribute");
+  }
+  g_attr_done[k] = true;
+  return DFK_OK;
+}
+
+struct CcCall {
+  int layout;      // LAYOUT_ROW / COL / IL
+  int nmat;        // 2 fused gate/up, 1 plain GEMV
+  bool norm;
+  const void *x, *gamma;
+  float eps;
+  const void *w0, *w1;
+  void *out;
+  int B, K, N;
+};
+
+static bool pdl_enabled() { return env_flag("DFK_PDL", true); }
+
+static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  CcPlan pl;
+  std::string why;
+  if (!plan_cc(c.layout, c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
+    return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit B=%d K=%d N=%d: %s", v.id, c.B,
+                c.K, c.N, why.c_str());
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  CcMaps maps;
+  memset(&maps, 0, sizeof maps);
+  const int r_hi = pl.p.r_hi, r_lo = pl.r_lo > 0 ? pl.r_lo : pl.p.r_hi;
+  const void *w[2] = {c.w0, c.w1};
+  for (int m = 0; m < (c.layout == LAYOUT_IL ? 1 : c.nmat); ++m) {
+    for (int lo = 0; lo < 2; ++lo) {
+      const uint32_t r = lo ? r_lo : r_hi;
+      if (c.layout == LAYOUT_ROW)
+        rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K) * 2, TILE_K, r,
+                           &maps.m[m * 2 + lo]);
+      else if (c.layout == LAYOUT_COL)
+        rc = tensor_map_2d(w[m], c.N, c.K, static_cast<uint64_t>(c.N) * 2, r, TILE_K,
+                           &maps.m[m * 2 + lo]);
+      else
+        rc = tensor_map_2d(w[m], c.K, 2ull * c.N, static_cast<uint64_t>(c.K) * 2, TILE_K, r,
+                           &maps.m[m * 2 + lo]);
+      if (rc) return rc;
+    }
+  }
+  CcParams p = pl.p;
+  p.x = static_cast<const uint16_t *>(c.x);
+  p.gamma = static_cast<const uint16_t *>(c.gamma);
+  p.out = static_cast<uint16_t *>(c.out);
+  p.err = ds->err;
+  p.eps = c.eps;
+  void *args[] = {&maps, &p};
+  cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(pl.block), pl.smem, s, pdl_enabled(),
+                                args);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "kernel launch");
+  }
+  if (stages_used) *stages_used = p.stages;
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- scheduler
+
+struct TuneKey {
+  int dev, op, B, D, F, layout;
+  bool operator<(const TuneKey &o) const {
+    return std::tie(dev, op, B, D, F, layout) < std::tie(o.dev, o.op, o.B, o.D, o.F, o.layout);
+  }
+};
+
+static std::mutex g_tune_mu;
+static std::map<TuneKey, dfk_variant> g_tuned;
+
+static int op_class(int op) { return op == DFK_OP_DOWN ? CLS_GEMV : CLS_GATE_UP; }
+
+static void fill_variant(const VDef &d, int op, int layout, int stages, float us,
+                         dfk_variant *out) {
+  out->variant_id = d.id;
+  out->op = op;
+  out->layout = layout;
+  out->family = d.family;
+  out->j_per_thread = d.jpt;
+  out->token_tile = d.bt;
+  out->k_split = d.ksplit;
+  out->stages = stages;
+  out->measured_us = us;
+}
+
+// Candidates worth timing for (op, B): every j-per-thread choice at its
+// largest useful token tile; every k split for the plain GEMV.
+static std::vector<const VDef *> candidates(int op, int B) {
+  std::vector<const VDef *> c;
+  for (const VDef &d : variants()) {
+    if (d.cls != op_class(op)) continue;
+    if (d.bt != bt_for(B, d.jpt)) continue;
+    c.push_back(&d);
+  }
+  return c;
+}
+
+// Heuristic default (no timing): 4 rows per thread up to B = 4, then 2;
+// for the GEMV the largest k split whose CTA fits.  If that family does not
+// fit (shared memory), the feasible variant with the fewest passes wins.
+static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
+  const int jpt = B <= 4 ? 4 : 2;
+  const VDef *best = nullptr;
+  for (const VDef &d : variants()) {
+    if (d.cls != op_class(op) || d.jpt != jpt || d.bt != bt_for(B, jpt)) continue;
+    CcPlan pl;
+    if (!plan_cc(c.layout, c.nmat, c.norm, d, B, c.K, c.N, ds, &pl, nullptr)) continue;
+    if (!best || d.ksplit > best->ksplit) best = &d;
+  }
+  if (best) return best;
+  int best_pass = 1 << 30;
+  for (const VDef &d : variants()) {
+    if (d.cls != op_class(op)) continue;
+    CcPlan pl;
+    if (!plan_cc(c.layout, c.nmat, c.norm, d, B, c.K, c.N, ds, &pl, nullptr)) continue;
+    const int passes = ceil_div(B, d.bt);
+    if (passes < best_pass || (passes == best_pass && d.ksplit > best->ksplit)) {
+      best = &d;
+      best_pass = passes;
+    }
+  }
+  return best;
+}
+
+static bool stream_capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return true;  // be conservative: do not time
+  }
+  return cs != cudaStreamCaptureStatusNone;
+}
+
+// Time `cands` for call `c` on stream s; returns the winner (or nullptr).
+static const VDef *time_candidates(int op, const CcCall &c, const std::vector<const VDef *> &cands,
+                                   cudaStream_t s, const DeviceState &ds, float *best_us,
+                                   int *best_stages) {
+  const char *fault = getenv("DFK_FAULT");
+  if (fault && strcmp(fault, "tune") == 0) {
+    log_msg("tuning disabled by DFK_FAULT=tune; using the heuristic");
+    return nullptr;
+  }
+  const int reps = std::max(1, env_int("DFK_TUNE_REPS", 7));
+  size_t flush_bytes = static_cast<size_t>(std::max(ds.l2_bytes, 1 << 20)) * 2;
+  void *flush = nullptr;
+  cudaError_t e = cudaMallocAsync(&flush, flush_bytes, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    flush = nullptr;
+  }
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  cudaEventCreate(&e0);
+  cudaEventCreate(&e1);
+  const VDef *best = nullptr;
+  float best_t = 1e30f;
+  for (const VDef *d : cands) {
+    int st = 0;
+    if (launch_cc(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible variants
+    std::vector<float> ts;
+    bool ok = true;
+    for (int r = 0; r < reps && ok; ++r) {
+      if (flush) cudaMemsetAsync(flush, r & 0xff, flush_bytes, s);
+      cudaEventRecord(e0, s);
+      ok = launch_cc(c, *d, s, nullptr) == DFK_OK;
+      cudaEventRecord(e1, s);
+      if (cudaEventSynchronize(e1) != cudaSuccess) ok = false;
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, e0, e1);
+      ts.push_back(ms * 1000.f);
+    }
+    if (!ok || ts.empty()) continue;
+    std::sort(ts.begin(), ts.end());
+    const float med = ts[ts.size() / 2];
+    log_msg("op %d B=%d K=%d N=%d layout %d: variant %d (jpt %d bt %d ks %d, %d stages) %.2f us",
+            op, c.B, c.K, c.N, c.layout, d->id, d->jpt, d->bt, d->ksplit, st, med);
+    if (med < best_t) {
+      best_t = med;
+      best = d;
+      *best_stages = st;
+    }
+  }
+  if (flush) cudaFreeAsync(flush, s);
+  cudaStreamSynchronize(s);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  cudaGetLastError();
+  *best_us = best_t;
+  return best;
+}
+
+// Pick the variant for call `c` (variant 0 = scheduler's choice).
+static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const VDef **out) {
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  if (variant > 0) {
+    const VDef *d = find_variant(variant);
+    if (!d || d->cls != op_class(op))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a variant of op %d", variant, op);
+    *out = d;
+    return DFK_OK;
+  }
+  TuneKey key{dev, op, c.B, op == DFK_OP_DOWN ? c.N : c.K, op == DFK_OP_DOWN ? c.K : c.N,
+              c.layout};
+  {
+    std::lock_guard<std::mutex> lk(g_tune_mu);
+    auto it = g_tuned.find(key);
+    if (it != g_tuned.end()) {
+      *out = find_variant(it->second.variant_id);
+      return DFK_OK;
+    }
+  }
+  const VDef *h = heuristic(op, c.B, c, *ds);
+  if (!h) return fail(DFK_ERR_NO_VARIANT, "no variant fits B=%d K=%d N=%d", c.B, c.K, c.N);
+  const bool tune = env_flag("DFK_TUNE", true) && !stream_capturing(s);
+  const VDef *win = h;
+  float us = -1.f;
+  int stages = 0;
+  if (tune) {
+    const VDef *t = time_candidates(op, c, candidates(op, c.B), s, *ds, &us, &stages);
+    if (t) win = t;
+    else us = -1.f;
+  }
+  if (tune || !env_flag("DFK_TUNE", true)) {
+    dfk_variant rec;
+    fill_variant(*win, op, c.layout, stages, us, &rec);
+    std::lock_guard<std::mutex> lk(g_tune_mu);
+    g_tuned[key] = rec;
+  }
+  log_msg("op %d B=%d D=%d F=%d layout %d -> variant %d (%s)", op, c.B, key.D, key.F, c.layout,
+          win->id, us >= 0 ? "timed" : "heuristic");
+  *out = win;
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- validation
+
+static bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+static int check_gate_up(const void *x, const void *gamma, bool norm, float eps, const void *wg,
+                         const void *wu, int layout, const void *h, int B, int D, int F,
+                         int variant) {
+  if (layout != DFK_W_ROW_MAJOR && layout != DFK_W_COL_MAJOR && layout != DFK_W_GU_INTERLEAVED)
+    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "layout %d is not a weight layout", layout);
+  if (B < 0 || D <= 0 || F <= 0) return fail(DFK_ERR_INVALID_ARG, "negative or zero size");
+  if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
+  if (variant > 0) {
+    const VDef *d = find_variant(variant);
+    if (!d || d->cls != CLS_GATE_UP)
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a gate/up variant", variant);
+  }
+  if (norm && !(eps >= 0.f && std::isfinite(eps)))
+    return fail(DFK_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (B > 64) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "B=%d > 64 (decode batches only)", B);
+  if (D % 8) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "d_model %% 8 != 0 (d_model=%d)", D);
+  if (layout == DFK_W_COL_MAJOR && F % 8)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "column-major needs d_ff %% 8 == 0 (d_ff=%d)", F);
+  if (static_cast<long long>(F) * 2 > (1ll << 31))
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "d_ff too large");
+  if (layout == DFK_W_GU_INTERLEAVED && wu)
+    return fail(DFK_ERR_INVALID_ARG, "interleaved layout: w_up must be NULL");
+  if (B == 0) return DFK_OK;
+  if (!x || !wg || !h || (norm && !gamma) || (layout != DFK_W_GU_INTERLEAVED && !wu))
+    return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if (misaligned(x) || misaligned(wg) || misaligned(h) || (wu && misaligned(wu)) ||
+      (norm && misaligned(gamma)))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  return DFK_OK;
+}
+
+static int check_gemv(const void *x, const void *w, const void *out, int B, int K, int N,
+                      int variant) {
+  if (B < 0 || K <= 0 || N <= 0) return fail(DFK_ERR_INVALID_ARG, "negative or zero size");
+  if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
+  if (variant > 0) {
+    const VDef *d = find_variant(variant);
+    if (!d || d->cls != CLS_GEMV)
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a GEMV variant", variant);
+  }
+  if (B > 64) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "B=%d > 64 (decode batches only)", B);
+  if (K % 8) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "reduction length %% 8 != 0 (K=%d)", K);
+  if (B == 0) return DFK_OK;
+  if (!x || !w || !out) return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if (misaligned(x) || misaligned(w) || misaligned(out))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  return DFK_OK;
+}
+
+static int to_engine_layout(int layout) {
+  return layout == DFK_W_COL_MAJOR ? LAYOUT_COL
+                                   : (layout == DFK_W_GU_INTERLEAVED ? LAYOUT_IL : LAYOUT_ROW);
+}
+
+static int gate_up_impl(int op, const void *x, const void *gamma, float eps, const void *wg,
+                        const void *wu, int layout, void *h, int B, int D, int F, int variant,
+                        cudaStream_t s) {
+  const bool norm = op == DFK_OP_RMSNORM_GATE_UP;
+  int rc = check_gate_up(x, gamma, norm, eps, wg, wu, layout, h, B, D, F, variant);
+  if (rc || B == 0) return rc;
+  CcCall c{to_engine_layout(layout), 2, norm, x, gamma, eps, wg, wu, h, B, D, F};
+  const VDef *v = nullptr;
+  if ((rc = resolve(op, variant, c, s, &v))) return rc;
+  return launch_cc(c, *v, s, nullptr);
+}
+
+static int gemv_impl(int op, const void *x, const void *w, void *out, int B, int K, int N,
+                     int variant, cudaStream_t s) {
+  int rc = check_gemv(x, w, out, B, K, N, variant);
+  if (rc || B == 0) return rc;
+  CcCall c{LAYOUT_ROW, 1, false, x, nullptr, 0.f, w, nullptr, out, B, K, N};
+  const VDef *v = nullptr;
+  if ((rc = resolve(op, variant, c, s, &v))) return rc;
+  return launch_cc(c, *v, s, nullptr);
+}
+
+}  // namespace dfk
+
+using namespace dfk;
+
+// ================================================================ C ABI
+
+extern "C" {
+
+int dfk_swiglu_gate_up(const void *x, const void *w_gate, const void *w_up, int layout, void *h,
+                       int B, int d_model, int d_ff, int variant, void *stream) {
+  return gate_up_impl(DFK_OP_GATE_UP, x, nullptr, 0.f, w_gate, w_up, layout, h, B, d_model,
+                      d_ff, variant, static_cast<cudaStream_t>(stream));
+}
+
+int dfk_rmsnorm_swiglu_gate_up(const void *x, const void *gamma, float eps, const void *w_gate,
+                               const void *w_up, int layout, void *h, int B, int d_model,
+                               int d_ff, int variant, void *stream) {
+  return gate_up_impl(DFK_OP_RMSNORM_GATE_UP, x, gamma, eps, w_gate, w_up, layout, h, B,
+                      d_model, d_ff, variant, static_cast<cudaStream_t>(stream));
+}
+
+int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int d_model, int d_ff,
+                  int variant, void *stream) {
+  return gemv_impl(DFK_OP_DOWN, h, w_down, y, B, d_ff, d_model, variant,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int variant,
+             void *stream) {
+  return gemv_impl(DFK_OP_DOWN, x, w, out, B, K, N, variant, static_cast<cudaStream_t>(stream));
+}
+
+int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
+                       const void *const *sample_ptrs, void *stream, dfk_variant *out) {
+  if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
+  if (op != DFK_OP_GATE_UP && op != DFK_OP_RMSNORM_GATE_UP && op != DFK_OP_DOWN)
+    return fail(DFK_ERR_INVALID_ARG, "unknown op %d", op);
+  if (B <= 0 || B > 64 || d_model <= 0 || d_ff <= 0)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "bad shape B=%d d_model=%d d_ff=%d", B, d_model, d_ff);
+  if (op == DFK_OP_DOWN && layout != DFK_W_ROW_MAJOR && layout != DFK_W_ANY)
+    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "the down projection reads row-major W_down");
+  if (layout != DFK_W_ANY && layout != DFK_W_ROW_MAJOR && layout != DFK_W_COL_MAJOR &&
+      layout != DFK_W_GU_INTERLEAVED)
+    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "layout %d", layout);
+  if (d_model % 8 || (op == DFK_OP_DOWN && d_ff % 8))
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "sizes must be multiples of 8");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  if (stream_capturing(s))
+    return fail(DFK_ERR_INVALID_ARG, "dfk_select_variant cannot time inside stream capture");
+
+  std::vector<int> layouts;
+  if (op == DFK_OP_DOWN) layouts = {DFK_W_ROW_MAJOR};
+  else if (layout == DFK_W_ANY) layouts = {DFK_W_ROW_MAJOR, DFK_W_COL_MAJOR, DFK_W_GU_INTERLEAVED};
+  else layouts = {layout};
+
+  const size_t xb = static_cast<size_t>(B) * (op == DFK_OP_DOWN ? d_ff : d_model) * 2;
+  const size_t wb = static_cast<size_t>(d_model) * d_ff * 2;
+  const size_t ob = static_cast<size_t>(B) * (op == DFK_OP_DOWN ? d_model : d_ff) * 2;
+  bool best_set = false;
+  dfk_variant best{};
+  for (int L : layouts) {
+    if (L == DFK_W_COL_MAJOR && d_ff % 8) continue;
+    const bool own = !sample_ptrs || layout == DFK_W_ANY;
+    void *bx = nullptr, *bg = nullptr, *bw0 = nullptr, *bw1 = nullptr, *bo = nullptr;
+    const void *px, *pg = nullptr, *pw0, *pw1 = nullptr;
+    void *po;
+    if (own) {
+      cudaError_t e = cudaMallocAsync(&bx, xb, s);
+      if (!e) e = cudaMallocAsync(&bo, ob, s);
+      if (!e && op == DFK_OP_RMSNORM_GATE_UP) e = cudaMallocAsync(&bg, d_model * 2, s);
+      if (!e) e = cudaMallocAsync(&bw0, op == DFK_OP_DOWN ? wb : 2 * wb, s);
+      if (e) {
+        cudaGetLastError();
+        if (bx) cudaFreeAsync(bx, s);
+        if (bo) cudaFreeAsync(bo, s);
+        if (bg) cudaFreeAsync(bg, s);
+        if (bw0) cudaFreeAsync(bw0, s);
+        return cuda_fail(e, "cudaMallocAsync (tuning buffers)");
+      }
+      cudaMemsetAsync(bx, 0, xb, s);
+      if (bg) cudaMemsetAsync(bg, 0, d_model * 2, s);
+      cudaMemsetAsync(bw0, 0, op == DFK_OP_DOWN ? wb : 2 * wb, s);
+      bw1 = (op == DFK_OP_DOWN || L == DFK_W_GU_INTERLEAVED) ? nullptr
+                                                              : static_cast<char *>(bw0) + wb;
+      px = bx; pg = bg; pw0 = bw0; pw1 = bw1; po = bo;
+    } else if (op == DFK_OP_DOWN) {
+      px = sample_ptrs[0]; pw0 = sample_ptrs[1]; po = const_cast<void *>(sample_ptrs[2]);
+    } else if (op == DFK_OP_GATE_UP) {
+      px = sample_ptrs[0]; pw0 = sample_ptrs[1]; pw1 = sample_ptrs[2];
+      po = const_cast<void *>(sample_ptrs[3]);
+    } else {
+      px = sample_ptrs[0]; pg = sample_ptrs[1]; pw0 = sample_ptrs[2]; pw1 = sample_ptrs[3];
+      po = const_cast<void *>(sample_ptrs[4]);
+    }
+    CcCall c;
+    if (op == DFK_OP_DOWN) c = CcCall{LAYOUT_ROW, 1, false, px, nullptr, 0.f, pw0, nullptr, po,
+                                      B, d_ff, d_model};
+    else c = CcCall{to_engine_layout(L), 2, op == DFK_OP_RMSNORM_GATE_UP, px, pg, 1e-5f, pw0,
+                    L == DFK_W_GU_INTERLEAVED ? nullptr : pw1, po, B, d_model, d_ff};
+    float us = -1.f;
+    int stages = 0;
+    const VDef *win = time_candidates(op, c, candidates(op, B), s, *ds, &us, &stages);
+    if (!win) {
+      win = heuristic(op, B, c, *ds);
+      us = -1.f;
+    }
+    if (own) {
+      cudaFreeAsync(bx, s);
+      cudaFreeAsync(bo, s);
+      if (bg) cudaFreeAsync(bg, s);
+      cudaFreeAsync(bw0, s);
+      cudaStreamSynchronize(s);
+    }
+    if (!win) continue;
+    dfk_variant rec;
+    fill_variant(*win, op, L, stages, us, &rec);
+    {
+      TuneKey key{dev, op, B, d_model, d_ff, L};
+      std::lock_guard<std::mutex> lk(g_tune_mu);
+      g_tuned[key] = rec;
+    }
+    if (!best_set || (us >= 0 && (best.measured_us < 0 || us < best.measured_us))) {
+      best = rec;
+      best_set = true;
+    }
+  }
+  if (!best_set) return fail(DFK_ERR_NO_VARIANT, "no variant fits this shape");
+  *out = best;
+  return DFK_OK;
+}
+
+int dfk_variant_count(void) { return static_cast<int>(variants().size()); }
+
+int dfk_variant_info(int variant_id, dfk_variant *out) {
+  if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
+  const VDef *d = find_variant(variant_id);
+  if (!d) return fail(DFK_ERR_INVALID_ARG, "no variant %d", variant_id);
+  fill_variant(*d, d->cls == CLS_GEMV ? DFK_OP_DOWN : DFK_OP_GATE_UP, -1, 0, -1.f, out);
+  return DFK_OK;
+}
+
+void dfk_clear_variant_cache(void) {
+  std::lock_guard<std::mutex> lk(g_tune_mu);
+  g_tuned.clear();
+}
+
+int dfk_rmsnorm(const void *x, const void *gamma, float eps, void *xn, int B, int d,
+                void *stream) {
+  if (B < 0 || d <= 0) return fail(DFK_ERR_INVALID_ARG, "negative or zero size");
+  if (!(eps >= 0.f && std::isfinite(eps))) return fail(DFK_ERR_INVALID_ARG, "bad eps");
+  if (d % 8) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "d %% 8 != 0");
+  if (B == 0) return DFK_OK;
+  if (!x || !xn) return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if (misaligned(x) || misaligned(xn) || (gamma && misaligned(gamma)))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  DeviceState *ds;
+  int rc = current_device(&ds);
+  if (rc) return rc;
+  cudaError_t e = launch_rmsnorm_rows(x, gamma, eps, xn, B, d, static_cast<cudaStream_t>(stream),
+                                      pdl_enabled());
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "rmsnorm launch");
+  }
+  return DFK_OK;
+}
+
+int dfk_rms_rescale(const void *y, float eps, void *x_next, int B, int d, void *stream) {
+  return dfk_rmsnorm(y, nullptr, eps, x_next, B, d, stream);
+}
+
+static int ew_check(const void *a, const void *b, const void *out, long long n, bool two) {
+  if (n < 0) return fail(DFK_ERR_INVALID_ARG, "negative size");
+  if (n == 0) return DFK_OK;
+  if (!a || !out || (two && !b)) return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(out) |
+       reinterpret_cast<uintptr_t>(b)) & 1u)
+    return fail(DFK_ERR_MISALIGNED, "bf16 pointers must be 2-byte aligned");
+  return DFK_OK;
+}
+
+int dfk_silu(const void *a, void *out, long long n, void *stream) {
+  int rc = ew_check(a, nullptr, out, n, false);
+  if (rc || n == 0) return rc;
+  DeviceState *ds;
+  if ((rc = current_device(&ds))) return rc;
+  cudaError_t e = launch_silu(a, out, n, static_cast<cudaStream_t>(stream), pdl_enabled());
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "silu launch");
+  }
+  return DFK_OK;
+}
+
+int dfk_mul(const void *a, const void *b, void *out, long long n, void *stream) {
+  int rc = ew_check(a, b, out, n, true);
+  if (rc || n == 0) return rc;
+  DeviceState *ds;
+  if ((rc = current_device(&ds))) return rc;
+  cudaError_t e = launch_mul(a, b, out, n, static_cast<cudaStream_t>(stream), pdl_enabled());
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "mul launch");
+  }
+  return DFK_OK;
+}
+
+int dfk_mlp_forward_host(const void *x_host, const void *gamma, float eps, const void *w_gate,
+                         const void *w_up, int layout, const void *w_down, void *y_host,
+                         void *x_dev, void *h_dev, void *y_dev, int B, int d_model, int d_ff,
+                         void *stream) {
+  if (B < 0) return fail(DFK_ERR_INVALID_ARG, "negative batch");
+  if (B == 0) return DFK_OK;
+  if (!x_host || !y_host || !x_dev || !h_dev || !y_dev || !w_down)
+    return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(B) * d_model * 2;
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "copy x to device");
+  }
+  int rc = gamma ? dfk_rmsnorm_swiglu_gate_up(x_dev, gamma, eps, w_gate, w_up, layout, h_dev, B,
+                                              d_model, d_ff, 0, stream)
+                 : dfk_swiglu_gate_up(x_dev, w_gate, w_up, layout, h_dev, B, d_model, d_ff, 0,
+                                      stream);
+  if (rc) return rc;
+  if ((rc = dfk_down_proj(h_dev, w_down, y_dev, B, d_model, d_ff, 0, stream))) return rc;
+  e = cudaMemcpyAsync(y_host, y_dev, xb, cudaMemcpyDeviceToHost, s);
+  if (!e) e = cudaStreamSynchronize(s);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "copy y to host");
+  }
+  return DFK_OK;
+}
+
+const char *dfk_status_string(int status) {
+  switch (status) {
+    case DFK_OK: return "ok";
+    case DFK_ERR_INVALID_ARG: return "invalid argument";
+    case DFK_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DFK_ERR_UNSUPPORTED_LAYOUT: return "unsupported layout";
+    case DFK_ERR_MISALIGNED: return "misaligned pointer";
+    case DFK_ERR_CUDA: return "CUDA error";
+    case DFK_ERR_ARCH: return "no sm_100 device";
+    case DFK_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case DFK_ERR_NO_VARIANT: return "no variant fits this shape";
+    default: return "unknown status";
+  }
+}
+
+const char *dfk_last_error(void) { return t_last_error.c_str(); }
+
+int dfk_device_error(int *code) {
+  if (!code) return fail(DFK_ERR_INVALID_ARG, "code is NULL");
+  DeviceState *ds;
+  int rc = current_device(&ds);
+  if (rc) return rc;
+  cudaError_t e = cudaDeviceSynchronize();
+  unsigned v = 0;
+  if (!e) e = cudaMemcpyFromSymbol(&v, g_dfk_err, sizeof v);
+  const unsigned zero = 0;
+  if (!e) e = cudaMemcpyToSymbol(g_dfk_err, &zero, sizeof zero);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "reading the device error word");
+  }
+  *code = static_cast<int>(v);
+  return v ? DFK_ERR_TIMEOUT : DFK_OK;
+}
+
+const char *dfk_version(void) { return "dfk 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every function ``include/dfk.h`` declares;
+argument validation must reject bad calls with the documented status codes
+before touching the device; without a device every compute call fails
+loudly (there is no CPU fallback).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import swiglu_mlp_dfk_b200 as dfk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from swiglu_mlp_dfk_b200 import build
+    build.build()
+    return dfk.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "dfk.h")).read()
+    return sorted(set(re.findall(r"DFK_API\s+[\w\s\*]*?\b(dfk_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for n in ("dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj",
+              "dfk_select_variant"):
+        assert n in names
+    assert set(names) == set(dfk.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in header_functions():
+        assert hasattr(L, n), n
+    assert dfk.dfk_version().startswith("dfk ")
+
+
+def test_status_strings(L):
+    for s in range(9):
+        assert L.dfk_status_string(s).decode()
+    assert L.dfk_status_string(99).decode() == "unknown status"
+
+
+def test_variant_table(L):
+    n = dfk.dfk_variant_count()
+    assert n >= 8
+    ids = set()
+    for i in range(1, n + 1):
+        v = dfk.dfk_variant_info(i)
+        assert v["variant_id"] == i
+        assert v["j_per_thread"] in (2, 4)
+        assert v["token_tile"] in (1, 2, 4, 8, 16, 32, 64)
+        ids.add(i)
+    with pytest.raises(dfk.DfkError) as e:
+        dfk.dfk_variant_info(n + 1)
+    assert e.value.status == dfk.DFK_ERR_INVALID_ARG
+
+
+# Fake, 16-byte aligned "device" addresses: validation rejects the calls below
+# before any CUDA call, so the pointers are never dereferenced.
+P = ctypes.c_void_p(0x10000)
+P2 = ctypes.c_void_p(0x20000)
+P3 = ctypes.c_void_p(0x30000)
+MIS = ctypes.c_void_p(0x10008)
+
+
+@pytest.mark.parametrize("call,status", [
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 7, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_LAYOUT),
+    (lambda L: L.dfk_swiglu_gate_up(None, P2, P3, 0, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, None, 0, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 2, P, 1, 64, 64, 0, None),   # interleaved + w_up
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 0, P, 65, 64, 64, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 0, P, 1, 60, 64, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 1, P, 1, 64, 60, 0, None),   # col needs F%8
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_swiglu_gate_up(MIS, P2, P3, 0, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 0, P, -1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_swiglu_gate_up(P, P2, P3, 0, P, 1, 64, 64, 9999, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_swiglu_gate_up(P, None, 1e-5, P2, P3, 0, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_swiglu_gate_up(P, P, -1.0, P2, P3, 0, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_down_proj(P, P2, P3, 1, 64, 60, 0, None), dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_down_proj(P, None, P3, 1, 64, 64, 0, None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_down_proj(P, P2, MIS, 1, 64, 64, 0, None), dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_down_proj(P, P2, P3, 1, 64, 64, 1, None),   # id 1 is a gate/up variant
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_silu(P, P2, -5, None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_select_variant(9, 1, 64, 64, 0, None, None, None), dfk.DFK_ERR_INVALID_ARG),
+])
+def test_validation_rejects_without_launch(L, call, status):
+    assert call(L) == status
+    assert L.dfk_last_error().decode() != ""
+
+
+def test_empty_batch_is_a_no_op(L):
+    assert L.dfk_swiglu_gate_up(None, P2, P3, 0, None, 0, 64, 64, 0, None) == dfk.DFK_OK
+    assert L.dfk_down_proj(None, P2, None, 0, 64, 64, 0, None) == dfk.DFK_OK
+    assert L.dfk_silu(None, None, 0, None) == dfk.DFK_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device behaviour")
+def test_no_device_means_no_compute(L):
+    # valid-looking arguments, but no CUDA device: the library refuses (no CPU fallback)
+    assert L.dfk_swiglu_gate_up(P, P2, P3, 0, P, 1, 64, 64, 0, None) == dfk.DFK_ERR_ARCH
+    assert L.dfk_down_proj(P, P2, P3, 1, 64, 64, 0, None) == dfk.DFK_ERR_ARCH
+    code = ctypes.c_int(0)
+    assert L.dfk_device_error(ctypes.byref(code)) == dfk.DFK_ERR_ARCH
+    with pytest.raises(dfk.DfkError):
+        dfk.dfk_device_error()
+
+
+def test_python_binding_rejects_host_tensors():
+    x = torch.zeros(1, 64, dtype=torch.bfloat16)
+    with pytest.raises(dfk.DfkError):
+        dfk.dfk_swiglu_gate_up(x, torch.zeros(64, 64, dtype=torch.bfloat16),
+                               torch.zeros(64, 64, dtype=torch.bfloat16))
