@@ -475,6 +475,37 @@ def reference_arm(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def profile_arm(args):
+    """--profile KERNEL: run one kernel of the workload inside an NVTX range
+    named dfk_profile (for ncu --nvtx-include dfk_profile/), nothing else."""
+    import torch
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    torch.cuda.set_device(0)
+    B = args.batch
+    inp = I.make_inputs(B, D, F, seed=SEED, w_std=0.02, norm=True,
+                        with_down=args.profile == "down", device="cuda")
+    h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+    if args.profile == "gate_up":
+        fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate,
+                                                    inp.w_up, args.layout, h=h)
+    else:
+        fn = lambda: dfk.dfk_down_proj(h, inp.w_down, y=y)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("dfk_profile")
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    print(json.dumps({"profile": args.profile, "B": B, "layout": args.layout,
+                      "calls": args.steps, "device_error_word": dfk.dfk_device_error()}))
+    return None
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,9 +514,15 @@ def main():
     ap.add_argument("--impl", choices=["dfk", "reference"], default="dfk")
     ap.add_argument("--quick", action="store_true",
                     help="skip the sweep / unfused / interleaved measurements")
+    ap.add_argument("--profile", choices=["gate_up", "down"], default=None,
+                    help="run only this kernel (inside an NVTX range) for ncu")
+    ap.add_argument("--batch", type=int, default=1, help="batch for --profile")
+    ap.add_argument("--layout", default="row", help="weight layout for --profile")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile:
+        return profile_arm(args)
     line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
     if line is not None:
         print(json.dumps(line), flush=True)

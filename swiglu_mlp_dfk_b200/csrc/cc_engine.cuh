@@ -26,8 +26,10 @@
 //             ascending:  p = fma(xn[b][k], W[j][k], p);
 //   q[c]    = ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7));
 //   total   = left fold q[0] + q[1] + ... + q[KSPLIT-1].
-// Products of two bf16 values are exact in fp32, so fma and mul+add agree;
-// only the order above matters.  Tokens never interact, so row b of the
+// With the RMSNorm prologue, xn = (x * r) * gamma stays in fp32 (it is not
+// rounded to bf16), so the products are fused multiply-adds of an fp32 and a
+// bf16 value; without it, x is bf16 and every product is exact in fp32.
+// Either way the result is fixed by the order above.  Tokens never interact, so row b of the
 // output is independent of the batch size.
 #pragma once
 #include <cuda.h>
@@ -77,6 +79,7 @@ template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NOR
 __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     cc_gemv_kernel(const __grid_constant__ CcMaps maps, const CcParams p) {
   static_assert(LAYOUT != LAYOUT_IL || NMAT == 2, "interleaved layout holds both matrices");
+  static_assert(XF32 || !NORM, "normalised activations are kept in fp32");
   static_assert(JPT == 2 || JPT == 4, "JPT");
   extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -215,13 +218,14 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
               f[2 * i + 1] = bf16_hi(w[i]);
             }
             if (NORM) {
+              // xn = (x * r) * gamma, kept in fp32 (never rounded to bf16)
               const uint4 gv = ld_nc_v4(p.gamma + k);
               const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
               const float rr = s_rinv[bb];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                f[2 * i] = round_bf16((f[2 * i] * rr) * bf16_lo(g[i]));
-                f[2 * i + 1] = round_bf16((f[2 * i + 1] * rr) * bf16_hi(g[i]));
+                f[2 * i] = (f[2 * i] * rr) * bf16_lo(g[i]);
+                f[2 * i + 1] = (f[2 * i + 1] * rr) * bf16_hi(g[i]);
               }
             }
           } else {

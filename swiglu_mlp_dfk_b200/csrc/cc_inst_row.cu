@@ -6,7 +6,6 @@ const void *cc_lookup_row(int key) {
     DFK_CC_JB(0, 2, 1, 1, 0)
     DFK_CC_JB(0, 2, 1, 1, 1)
     DFK_CC_JB(0, 2, 1, 0, 0)
-    DFK_CC_JB(0, 2, 1, 0, 1)
     default: return nullptr;
   }
 }

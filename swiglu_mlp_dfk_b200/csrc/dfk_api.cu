@@ -275,7 +275,8 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     const int bar_bytes = 256;
     int best_s = 0, best_region = 0;
     bool best_xf32 = true;
-    for (int xf = 1; xf >= 0; --xf) {
+    // normalised activations are kept in fp32: only the fp32 store is allowed then
+    for (int xf = 1; xf >= (norm ? 1 : 0); --xf) {
       const int xs_bytes = v.bt * kpad * (xf ? 4 : 2);
       const int region = round_up(std::max(xs_bytes, red_bytes), 128);
       const int avail = smem_cap - region - bar_bytes;

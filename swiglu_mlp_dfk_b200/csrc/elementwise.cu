@@ -14,8 +14,9 @@ namespace dfk {
 
 // One warp per row.  The sum of squares uses the same fixed order as the
 // fused gate/up prologue: lane l accumulates k = 8 l + e + 256 c (c, then e
-// ascending), then a xor butterfly over the 32 lanes -- so the standalone
-// RMSNorm produces the same bf16 xn bits as the fused prologue.
+// ascending), then a xor butterfly over the 32 lanes -- so r_b is the same
+// fp32 value.  Unlike the fused prologue (which keeps xn in fp32), this
+// kernel stores xn in HBM and therefore rounds it to bf16.
 __global__ void rmsnorm_rows_kernel(const uint16_t *__restrict__ x,
                                     const uint16_t *__restrict__ gamma, float eps,
                                     uint16_t *__restrict__ out, int B, int D) {

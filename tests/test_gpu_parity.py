@@ -154,19 +154,30 @@ def test_batch_independence_and_row_permutation():
     assert bits_equal(hp, full[perm])
 
 
-def test_fused_prologue_equals_standalone_rmsnorm():
-    # the standalone RMSNorm kernel and the fused prologue produce the same xn bits,
-    # so gate/up on the standalone xn equals the fused kernel bit for bit
+def test_standalone_rmsnorm_and_fused_prologue():
+    # the standalone RMSNorm kernel stores xn in bf16 (it feeds HBM); the fused
+    # prologue keeps xn in fp32.  Both are held to the oracle.
     inp = I.make_inputs(4, 1024, 1200, seed=5, w_std=0.05, with_down=False, device="cuda")
     fused = run_gate_up(inp, I.LAYOUT_ROW, True)
     xn = dfk.dfk_rmsnorm(inp.x, inp.gamma, inp.eps)
-    plain = dfk.dfk_swiglu_gate_up(xn, inp.w_gate, inp.w_up, I.LAYOUT_ROW)
-    assert bits_equal(fused, plain)
     torch.cuda.synchronize()
     assert_close(xn, oracle.rmsnorm(I.to_bits(inp.x), I.to_bits(inp.gamma), inp.eps), "rmsnorm")
+    # bf16 rounding of the standalone output, mirrored by the oracle, is exact RNE
+    mirror = oracle.rmsnorm(I.to_bits(inp.x), I.to_bits(inp.gamma), inp.eps, mirror=True)
+    assert np.max(np.abs(values(xn) - mirror)) <= 2.0 ** -7 * np.max(np.abs(mirror))
+    assert_close(fused, oracle_gate_up(inp, True), "fused prologue")
+    # the fused kernel without the prologue, fed x itself, is the plain gate/up
+    plain = dfk.dfk_swiglu_gate_up(inp.x, inp.w_gate, inp.w_up, I.LAYOUT_ROW)
+    torch.cuda.synchronize()
+    assert_close(plain, oracle_gate_up(inp, False), "plain gate/up")
 
 
 def test_unfused_chain_matches_oracle():
+    # The unfused baseline (measurement only) stores xn, a, u and SiLU(a) in HBM
+    # as bf16: five roundings to bf16 (unit roundoff 2^-8) on the way to h, so
+    # its bound is 1e-2 + 2.5e-2 |oracle| (5 x 2^-8 ~ 2.0e-2, plus the spread of
+    # the xn rounding through the dot products).  The fused kernel keeps those
+    # values in fp32 and is held to the contract bound 1e-2 + 1e-2 |oracle|.
     B, D, F = 4, 1024, 2048
     inp = I.make_inputs(B, D, F, seed=9, w_std=0.03, device="cuda")
     xn = dfk.dfk_rmsnorm(inp.x, inp.gamma, inp.eps)
@@ -176,10 +187,18 @@ def test_unfused_chain_matches_oracle():
     h = dfk.dfk_mul(s, u)
     torch.cuda.synchronize()
     ref = oracle_gate_up(inp, True)
-    assert_close(h, ref, "unfused chain")
+    err = np.abs(values(h) - ref)
+    assert np.all(err <= 1e-2 + 2.5e-2 * np.abs(ref)), float(np.max(err - 2.5e-2 * np.abs(ref)))
+    # each stage of the chain on its own, against the oracle on the GPU's own inputs
+    xnv = I.to_bits(xn)
+    a_ref = oracle.gate_up(xnv, I.to_bits(inp.w_gate), I.to_bits(inp.w_gate), return_au=True)[1]
+    assert_close(a, a_ref, "unfused gemv")
+    s_ref = np.vectorize(oracle.silu)(values(a))
+    assert_close(s, s_ref, "unfused silu")
+    assert_close(h, values(s) * values(u), "unfused mul")
     fused = run_gate_up(inp, I.LAYOUT_ROW, True)
     torch.cuda.synchronize()
-    assert_close(fused, values(h), "fused vs unfused")
+    assert_close(fused, ref, "fused")
 
 
 @pytest.mark.parametrize("B,D,F", [(1, 256, 688), (3, 512, 1032), (8, 1024, 4096),
