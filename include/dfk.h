@@ -88,6 +88,7 @@ typedef struct dfk_variant {
   int j_per_thread; /* output columns per thread (CUDA-core)                         */
   int token_tile;   /* tokens per pass over the weights                              */
   int k_split;      /* thread teams splitting the reduction dimension               */
+  int k_tiles_per_stage; /* consecutive 64-wide reduction tiles per ring stage       */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
 } dfk_variant;
@@ -136,7 +137,8 @@ DFK_API int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int
  * column-major kernel variants; "Deep Kernel Fusion for Transformers",
  * abstract: the kernel is paired with a kernel scheduler).
  * Times every feasible variant of `op` for (B, d_model, d_ff, layout) with
- * CUDA events (L2 flushed before each timed call), caches the fastest and
+ * CUDA events (each sample: L2 flushed, then a burst of 4 back-to-back
+ * launches; median of DFK_TUNE_REPS samples), caches the fastest and
  * returns it in *out.  layout == DFK_W_ANY times every layout and reports
  * the fastest layout in out->layout (gate/up ops only).
  *   sample_ptrs  NULL, or the caller's buffers in argument order of the op:

@@ -21,7 +21,8 @@
 // and pipeline choice of the CUDA-core family, so that row-major,
 // column-major and interleaved weights give bit-identical results):
 //   k = 64 t + 8 s + e  (tile t, slot s in [0,8), element e in [0,8));
-//   with KSPLIT teams, team c owns the tiles t = c (mod KSPLIT).
+//   with KSPLIT teams, team c owns the tiles t with floor(t / nt) = c
+//   (mod KSPLIT), nt = tiles per ring stage (KSPLIT = 1: one team, all tiles).
 //   p[c][s] = fp32 chain from +0 over its tiles t ascending, then e
 //             ascending:  p = fma(xn[b][k], W[j][k], p);
 //   q[c]    = ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7));
@@ -52,16 +53,18 @@ struct CcParams {
   unsigned *err;          // device error word
   int B, K, N;
   float eps;
-  int nsteps;       // ring steps per pass = ceil(ceil(K/64) / KSPLIT)
-  int kpad;         // nsteps * KSPLIT * 64: activation row pitch in shared memory
+  int nt;           // consecutive 64-wide tiles per team per ring stage (1, 2 or 4)
+  int nsteps;       // ring steps per pass = ceil(ceil(K/64) / (KSPLIT * nt))
+  int kpad;         // nsteps * KSPLIT * nt * 64: activation row pitch in shared memory
   int granule;      // output rows per partition unit
   int ubase, uextra;// units per CTA: ubase, +1 for the first uextra CTAs
   int r_hi;         // largest row count of any CTA (shared-memory slot size)
   int stages;       // ring depth
-  int stage_bytes;  // KSPLIT * NMAT * r_hi * 128
+  int stage_bytes;  // KSPLIT * NMAT * r_hi * 128 * nt
   int npass;        // ceil(B / BT)
   int tpt;          // consumer threads per K team (multiple of 32)
   int xs_off;       // shared-memory offset of the activation / reduction area
+  int g_off;        // shared-memory offset of gamma (bf16 bits, NORM only)
   int bar_off;      // shared-memory offset of the barrier area
 };
 
@@ -102,7 +105,9 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
   const int j0 = u0 * p.granule;
   const int r = nu * p.granule;
   const int mi = (r == p.r_hi) ? 0 : 1;
-  const uint32_t slot_bytes = static_cast<uint32_t>(p.r_hi) * TILE_K * 2;
+  const int nt = p.nt;
+  const uint32_t slot_bytes = static_cast<uint32_t>(p.r_hi) * TILE_K * 2 * nt;
+  const int rowb = TILE_K * 2 * nt;  // bytes per row of a row-major / interleaved tile
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     // ================= producer warp: one lane issues all TMA traffic
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      const uint32_t tile_bytes = static_cast<uint32_t>(r) * TILE_K * 2;
+      const uint32_t tile_bytes = static_cast<uint32_t>(r) * TILE_K * 2 * nt;
       const uint32_t tx = tile_bytes * NMAT * KSPLIT;
       int issued = 0;
       for (int i = 0; i < total_steps; ++i) {
@@ -133,7 +138,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
         mbar_arrive_expect_tx(&full[st], tx);
 #pragma unroll
         for (int kt = 0; kt < KSPLIT; ++kt) {
-          const int k0 = (step * KSPLIT + kt) * TILE_K;
+          const int k0 = (step * KSPLIT + kt) * nt * TILE_K;
           uint8_t *tb = base + static_cast<size_t>(kt) * NMAT * slot_bytes;
           if (LAYOUT == LAYOUT_ROW) {
 #pragma unroll
@@ -172,80 +177,97 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     float *xs_f = reinterpret_cast<float *>(smem + p.xs_off);
     uint16_t *xs_h = reinterpret_cast<uint16_t *>(smem + p.xs_off);
     float *red = reinterpret_cast<float *>(smem + p.xs_off);  // reused after the K loop
+    uint16_t *gs = reinterpret_cast<uint16_t *>(smem + p.g_off);  // gamma (NORM only)
 
     pdl_wait();  // activations come from the previous kernel in the stream
 
     for (int pass = 0; pass < p.npass; ++pass) {
       const int b0 = pass * BT;
 
-      // ---- prologue: RMS statistics (one warp per token, fixed order)
-      if (NORM) {
-        for (int bb = cw; bb < BT; bb += ncw) {
-          float ss = 0.f;
-          if (b0 + bb < p.B) {
-            const uint16_t *xr = p.x + static_cast<size_t>(b0 + bb) * p.K;
-            for (int k = 8 * lane; k < p.K; k += 256) {
-              const uint4 v = ld_nc_v4(xr + k);
-              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      // ---- prologue 1: raw activations (and gamma) into shared memory.  Every
+      // consumer thread issues its 16-byte loads back to back, so the whole
+      // prologue costs one L2 round trip; x is read only after pdl_wait().
+      {
+        const int c8n = p.kpad >> 3;               // 8-element chunks per activation row
+        const int nx = BT * c8n;                   // activation chunks
+        const int ntot = nx + (NORM ? c8n : 0);    // + gamma chunks
+        for (int base = tid; base < ntot; base += 4 * ncons) {
+          uint4 v[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float f0 = bf16_lo(w[i]), f1 = bf16_hi(w[i]);
-                ss = fmaf(f0, f0, ss);
-                ss = fmaf(f1, f1, ss);
-              }
+          for (int u = 0; u < 4; ++u) {
+            const int idx = base + u * ncons;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (idx < nx) {
+              const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
+              if (b0 + bb < p.B && k < p.K)
+                v[u] = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
+            } else if (idx < ntot) {
+              const int k = (idx - nx) * 8;
+              if (k < p.K) v[u] = ld_nc_v4(p.gamma + k);
             }
           }
 #pragma unroll
-          for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-          if (lane == 0) s_rinv[bb] = 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+          for (int u = 0; u < 4; ++u) {
+            const int idx = base + u * ncons;
+            if (idx >= ntot) continue;
+            if (idx >= nx) {  // gamma, kept as bf16 bits
+              *reinterpret_cast<uint4 *>(gs + (idx - nx) * 8) = v[u];
+              continue;
+            }
+            const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
+            if (XF32) {
+              // within a 64-wide tile, element 8s + 4h + i sits at 32h + 4s + i
+              float *row = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63);
+              const int s8 = (k >> 3) & 7;
+              *reinterpret_cast<float4 *>(row + 4 * s8) =
+                  make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y));
+              *reinterpret_cast<float4 *>(row + 32 + 4 * s8) =
+                  make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w));
+            } else {
+              *reinterpret_cast<uint4 *>(xs_h + static_cast<size_t>(bb) * p.kpad + k) = v[u];
+            }
+          }
         }
         named_barrier(1, ncons);
       }
 
-      // ---- prologue: activations into shared memory (fp32, or bf16 bits)
-      {
+      if (NORM) {
+        // ---- prologue 2: r_b = 1/sqrt(mean(x^2) + eps), one warp per token.  Fixed
+        // order: lane l chains k = 8 l + e + 256 c (c, then e ascending), then a xor
+        // butterfly over the 32 lanes (the same order as the standalone RMSNorm).
+        for (int bb = cw; bb < BT; bb += ncw) {
+          float ss = 0.f;
+          const float *row = xs_f + static_cast<size_t>(bb) * p.kpad;
+          for (int k = 8 * lane; k < p.K; k += 256) {
+            const float *tp = row + (k & ~63) + 4 * ((k >> 3) & 7);
+            const float4 lo = *reinterpret_cast<const float4 *>(tp);
+            const float4 hi = *reinterpret_cast<const float4 *>(tp + 32);
+            ss = fmaf(lo.x, lo.x, ss); ss = fmaf(lo.y, lo.y, ss);
+            ss = fmaf(lo.z, lo.z, ss); ss = fmaf(lo.w, lo.w, ss);
+            ss = fmaf(hi.x, hi.x, ss); ss = fmaf(hi.y, hi.y, ss);
+            ss = fmaf(hi.z, hi.z, ss); ss = fmaf(hi.w, hi.w, ss);
+          }
+#pragma unroll
+          for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+          if (lane == 0)
+            s_rinv[bb] = (b0 + bb < p.B) ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 0.f;
+        }
+        named_barrier(1, ncons);
+        // ---- prologue 3: xn = (x * r) * gamma in place, kept in fp32
         const int c8n = p.kpad >> 3;
         for (int idx = tid; idx < BT * c8n; idx += ncons) {
-          const int bb = idx / c8n;
-          const int k = (idx - bb * c8n) * 8;
-          float f[8];
-          if (b0 + bb < p.B && k < p.K) {
-            const uint4 v = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              f[2 * i] = bf16_lo(w[i]);
-              f[2 * i + 1] = bf16_hi(w[i]);
-            }
-            if (NORM) {
-              // xn = (x * r) * gamma, kept in fp32 (never rounded to bf16)
-              const uint4 gv = ld_nc_v4(p.gamma + k);
-              const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
-              const float rr = s_rinv[bb];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                f[2 * i] = (f[2 * i] * rr) * bf16_lo(g[i]);
-                f[2 * i + 1] = (f[2 * i + 1] * rr) * bf16_hi(g[i]);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0.f;
-          }
-          if (XF32) {
-            // within a 64-wide tile, element 8s + 4h + i sits at 32h + 4s + i
-            float *row = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63);
-            const int s8 = (k >> 3) & 7;
-            *reinterpret_cast<float4 *>(row + 4 * s8) = make_float4(f[0], f[1], f[2], f[3]);
-            *reinterpret_cast<float4 *>(row + 32 + 4 * s8) = make_float4(f[4], f[5], f[6], f[7]);
-          } else {
-            uint4 o;
-            o.x = __float_as_uint(f[0]) >> 16 | (__float_as_uint(f[1]) & 0xffff0000u);
-            o.y = __float_as_uint(f[2]) >> 16 | (__float_as_uint(f[3]) & 0xffff0000u);
-            o.z = __float_as_uint(f[4]) >> 16 | (__float_as_uint(f[5]) & 0xffff0000u);
-            o.w = __float_as_uint(f[6]) >> 16 | (__float_as_uint(f[7]) & 0xffff0000u);
-            *reinterpret_cast<uint4 *>(xs_h + static_cast<size_t>(bb) * p.kpad + k) = o;
-          }
+          const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
+          float *tp = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63) + 4 * ((k >> 3) & 7);
+          const uint4 g = *reinterpret_cast<const uint4 *>(gs + k);
+          const float rr = s_rinv[bb];
+          float4 lo = *reinterpret_cast<float4 *>(tp);
+          float4 hi = *reinterpret_cast<float4 *>(tp + 32);
+          lo.x = (lo.x * rr) * bf16_lo(g.x); lo.y = (lo.y * rr) * bf16_hi(g.x);
+          lo.z = (lo.z * rr) * bf16_lo(g.y); lo.w = (lo.w * rr) * bf16_hi(g.y);
+          hi.x = (hi.x * rr) * bf16_lo(g.z); hi.y = (hi.y * rr) * bf16_hi(g.z);
+          hi.z = (hi.z * rr) * bf16_lo(g.w); hi.w = (hi.w * rr) * bf16_hi(g.w);
+          *reinterpret_cast<float4 *>(tp) = lo;
+          *reinterpret_cast<float4 *>(tp + 32) = hi;
         }
         named_barrier(1, ncons);
       }
@@ -263,8 +285,8 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
         const int i = pass * p.nsteps + step;
         const int st = i % S;
         const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
-        if (ok && active) {
-          const int t = step * KSPLIT + team;
+        for (int tt = 0; ok && active && tt < nt; ++tt) {
+          const int t = (step * KSPLIT + team) * nt + tt;
           const uint8_t *tb = smem + static_cast<size_t>(st) * p.stage_bytes +
                               static_cast<size_t>(team) * NMAT * slot_bytes;
           float xv[BT][8];
@@ -296,7 +318,8 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
               for (int jj = 0; jj < JPT; ++jj) {
                 const int row = (LAYOUT == LAYOUT_IL) ? 2 * (jl0 + jj) + m : jl0 + jj;
                 const uint8_t *bse = (LAYOUT == LAYOUT_IL) ? tb : tb + m * slot_bytes;
-                const uint4 v = *reinterpret_cast<const uint4 *>(bse + row * (TILE_K * 2) + s * 16);
+                const uint4 v =
+                    *reinterpret_cast<const uint4 *>(bse + row * rowb + tt * (TILE_K * 2) + s * 16);
                 wv[m][jj][0] = v.x; wv[m][jj][1] = v.y; wv[m][jj][2] = v.z; wv[m][jj][3] = v.w;
               }
 #pragma unroll
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
             const int pitch = r * 2;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const int krow = 8 * s + e;
+              const int krow = tt * TILE_K + 8 * s + e;
 #pragma unroll
               for (int m = 0; m < NMAT; ++m) {
                 const uint8_t *src = tb + m * slot_bytes + krow * pitch + jl0 * 2;

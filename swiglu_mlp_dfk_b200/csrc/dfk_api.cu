@@ -7,8 +7,9 @@
 // column-major kernel variants; "Deep Kernel Fusion for Transformers",
 // abstract: the fused kernel is paired with a kernel scheduler): on the
 // first call for a (device, op, B, d_model, d_ff, layout) the candidate
-// variants are timed with CUDA events on the caller's stream, L2 flushed
-// before every timed call, and the fastest is cached.  During stream capture
+// variants are timed with CUDA events on the caller's stream (L2 flushed,
+// then a short burst of back-to-back launches per sample), and the fastest
+// is cached.  During stream capture
 // nothing is timed: a cached winner or the heuristic default is used.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -204,7 +205,7 @@ struct VDef {
   int id;
   int cls;
   int family;
-  int jpt, bt, ksplit;
+  int jpt, bt, ksplit, nt;
 };
 
 static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
@@ -213,9 +214,13 @@ static const std::vector<VDef> &variants() {
   static std::vector<VDef> v = [] {
     std::vector<VDef> t;
     int id = 1;
-    for (auto &jb : kJB) t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1});
-    for (int ks : {1, 2, 4, 8})
-      for (auto &jb : kJB) t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks});
+    for (int nt : {1, 2, 4})
+      for (auto &jb : kJB)
+        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt});
+    for (int nt : {1, 2, 4})
+      for (int ks : {1, 2, 4, 8})
+        for (auto &jb : kJB)
+          t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt});
     return t;
   }();
   return v;
@@ -268,9 +273,9 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     const int ncons = v.ksplit * tpt;
     if (ncons + 32 > CC_MAX_THREADS) continue;
     const int nT = ceil_div(K, TILE_K);
-    const int nsteps = ceil_div(nT, v.ksplit);
-    const int kpad = nsteps * v.ksplit * TILE_K;
-    const int stage_bytes = v.ksplit * nmat * r_hi * TILE_K * 2;
+    const int nsteps = ceil_div(nT, v.ksplit * v.nt);
+    const int kpad = nsteps * v.ksplit * v.nt * TILE_K;
+    const int stage_bytes = v.ksplit * nmat * r_hi * TILE_K * 2 * v.nt;
     const int red_bytes = v.ksplit * (layout == LAYOUT_COL ? NSLOT : 1) * nmat * v.bt * r_hi * 4;
     const int bar_bytes = 256;
     int best_s = 0, best_region = 0;
@@ -278,7 +283,8 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     // normalised activations are kept in fp32: only the fp32 store is allowed then
     for (int xf = 1; xf >= (norm ? 1 : 0); --xf) {
       const int xs_bytes = v.bt * kpad * (xf ? 4 : 2);
-      const int region = round_up(std::max(xs_bytes, red_bytes), 128);
+      const int g_bytes = norm ? kpad * 2 : 0;  // gamma, prologue only (aliases `red`)
+      const int region = round_up(std::max(xs_bytes + g_bytes, red_bytes), 128);
       const int avail = smem_cap - region - bar_bytes;
       const int S = avail > 0 ? std::min(8, avail / stage_bytes) : 0;
       if (xf && S >= 4) { best_s = S; best_region = region; best_xf32 = true; break; }
@@ -305,6 +311,7 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     p.K = K;
     p.N = N;
     p.B = B;
+    p.nt = v.nt;
     p.nsteps = nsteps;
     p.kpad = kpad;
     p.granule = g;
@@ -316,6 +323,7 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     p.npass = ceil_div(B, v.bt);
     p.tpt = tpt;
     p.xs_off = best_s * stage_bytes;
+    p.g_off = p.xs_off + v.bt * kpad * (best_xf32 ? 4 : 2);
     p.bar_off = p.xs_off + best_region;
     pl->smem = static_cast<size_t>(p.bar_off) + bar_bytes;
     return true;
@@ -368,17 +376,18 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   memset(&maps, 0, sizeof maps);
   const int r_hi = pl.p.r_hi, r_lo = pl.r_lo > 0 ? pl.r_lo : pl.p.r_hi;
   const void *w[2] = {c.w0, c.w1};
+  const uint32_t kbox = TILE_K * v.nt;
   for (int m = 0; m < (c.layout == LAYOUT_IL ? 1 : c.nmat); ++m) {
     for (int lo = 0; lo < 2; ++lo) {
       const uint32_t r = lo ? r_lo : r_hi;
       if (c.layout == LAYOUT_ROW)
-        rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K) * 2, TILE_K, r,
+        rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K) * 2, kbox, r,
                            &maps.m[m * 2 + lo]);
       else if (c.layout == LAYOUT_COL)
-        rc = tensor_map_2d(w[m], c.N, c.K, static_cast<uint64_t>(c.N) * 2, r, TILE_K,
+        rc = tensor_map_2d(w[m], c.N, c.K, static_cast<uint64_t>(c.N) * 2, r, kbox,
                            &maps.m[m * 2 + lo]);
       else
-        rc = tensor_map_2d(w[m], c.K, 2ull * c.N, static_cast<uint64_t>(c.K) * 2, TILE_K, r,
+        rc = tensor_map_2d(w[m], c.K, 2ull * c.N, static_cast<uint64_t>(c.K) * 2, kbox, r,
                            &maps.m[m * 2 + lo]);
       if (rc) return rc;
     }
@@ -423,6 +432,7 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->j_per_thread = d.jpt;
   out->token_tile = d.bt;
   out->k_split = d.ksplit;
+  out->k_tiles_per_stage = d.nt;
   out->stages = stages;
   out->measured_us = us;
 }
@@ -500,23 +510,28 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
   for (const VDef *d : cands) {
     int st = 0;
     if (launch_cc(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible variants
+    // Each repetition: flush L2, then a burst of back-to-back launches (the
+    // way a decode loop issues them, neighbours overlapping through
+    // programmatic dependent launch); the sample is the burst's mean.
+    const int burst = 4;
     std::vector<float> ts;
     bool ok = true;
     for (int r = 0; r < reps && ok; ++r) {
       if (flush) cudaMemsetAsync(flush, r & 0xff, flush_bytes, s);
       cudaEventRecord(e0, s);
-      ok = launch_cc(c, *d, s, nullptr) == DFK_OK;
+      for (int b = 0; b < burst && ok; ++b) ok = launch_cc(c, *d, s, nullptr) == DFK_OK;
       cudaEventRecord(e1, s);
       if (cudaEventSynchronize(e1) != cudaSuccess) ok = false;
       float ms = 0.f;
       cudaEventElapsedTime(&ms, e0, e1);
-      ts.push_back(ms * 1000.f);
+      ts.push_back(ms * 1000.f / burst);
     }
     if (!ok || ts.empty()) continue;
     std::sort(ts.begin(), ts.end());
     const float med = ts[ts.size() / 2];
-    log_msg("op %d B=%d K=%d N=%d layout %d: variant %d (jpt %d bt %d ks %d, %d stages) %.2f us",
-            op, c.B, c.K, c.N, c.layout, d->id, d->jpt, d->bt, d->ksplit, st, med);
+    log_msg("op %d B=%d K=%d N=%d layout %d: variant %d (jpt %d bt %d ks %d nt %d, %d stages) "
+            "%.2f us", op, c.B, c.K, c.N, c.layout, d->id, d->jpt, d->bt, d->ksplit, d->nt, st,
+            med);
     if (med < best_t) {
       best_t = med;
       best = d;
