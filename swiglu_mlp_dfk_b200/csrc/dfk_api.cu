@@ -31,6 +31,8 @@
 #include "cc_key.h"
 #include "dfk.h"
 #include "launch_util.h"
+#include "tc_engine.cuh"
+#include "tc_key.h"
 
 // Device error word: bit 0 = a pipeline wait in some kernel gave up.
 __device__ unsigned g_dfk_err;
@@ -159,16 +161,21 @@ static int get_encoder() {
   return DFK_OK;
 }
 
-using MapKey = std::tuple<uintptr_t, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t>;
+// key: pointer, rank, dims[3], strides[2], box[3], swizzle
+using MapKey = std::tuple<uintptr_t, int, uint64_t, uint64_t, uint64_t, uint64_t, uint64_t,
+                          uint32_t, uint32_t, uint32_t, int>;
 static std::map<MapKey, CUtensorMap> g_maps;
 
-// 2-D bf16 tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
-// between rows, box of box_inner x box_outer, no swizzle, zero fill outside.
-static int tensor_map_2d(const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
-                         uint32_t box_inner, uint32_t box_outer, CUtensorMap *out) {
+// bf16 tensor map of rank 2 or 3: dims[0] contiguous elements, strides in
+// bytes for dims 1.., box extents, 128-byte swizzle or none, zero fill
+// outside the tensor.
+static int tensor_map(const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
+                      const uint32_t *box, bool sw128, CUtensorMap *out) {
   int rc = get_encoder();
   if (rc) return rc;
-  MapKey key{reinterpret_cast<uintptr_t>(ptr), inner, outer, pitch, box_inner, box_outer};
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), rank, dims[0], dims[1], rank > 2 ? dims[2] : 0,
+             strides[0], rank > 2 ? strides[1] : 0, box[0], box[1], rank > 2 ? box[2] : 0,
+             sw128 ? 1 : 0};
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_maps.find(key);
@@ -178,23 +185,34 @@ static int tensor_map_2d(const void *ptr, uint64_t inner, uint64_t outer, uint64
     }
   }
   CUtensorMap m;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {pitch};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t d[3] = {dims[0], dims[1], rank > 2 ? dims[2] : 1};
+  cuuint64_t st[2] = {strides[0], rank > 2 ? strides[1] : 0};
+  cuuint32_t bx[3] = {box[0], box[1], rank > 2 ? box[2] : 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                        const_cast<void *>(ptr), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
-    return fail(DFK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llux%llu box %ux%u",
-                static_cast<int>(r), static_cast<unsigned long long>(inner),
-                static_cast<unsigned long long>(outer), box_inner, box_outer);
+    return fail(DFK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d), rank %d dims %llu x %llu "
+                "box %u x %u", static_cast<int>(r), rank, static_cast<unsigned long long>(d[0]),
+                static_cast<unsigned long long>(d[1]), bx[0], bx[1]);
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_maps.size() > 4096) g_maps.clear();
   g_maps[key] = m;
   *out = m;
   return DFK_OK;
+}
+
+// 2-D bf16 tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
+// between rows, box of box_inner x box_outer.
+static int tensor_map_2d(const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
+                         uint32_t box_inner, uint32_t box_outer, CUtensorMap *out,
+                         bool sw128 = false) {
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {pitch};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return tensor_map(ptr, 2, dims, strides, box, sw128, out);
 }
 
 // ---------------------------------------------------------------- variants
@@ -221,6 +239,11 @@ static const std::vector<VDef> &variants() {
       for (int ks : {1, 2, 4, 8})
         for (auto &jb : kJB)
           t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt});
+    // tensor-core family: token tile chosen from B at launch (16 / 32 / 64)
+    for (int nt : {1, 2})
+      t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt});
+    for (int nt : {1, 2, 4, 8})
+      t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt});
     return t;
   }();
   return v;
@@ -409,6 +432,149 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   return DFK_OK;
 }
 
+// ---------------------------------------------------------------- tensor-core plan
+
+struct TcPlan {
+  const void *fn = nullptr;
+  int grid = 0;
+  size_t smem = 0;
+  int mt = 1;
+  TcParams p{};
+};
+
+static int pow2_ceil(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// One CTA per SM over rows [j0, j0 + r) for the whole reduction; each
+// 128-row MMA tile reads 128 rows from shared memory starting at its A
+// tile, so the space behind the last A tile of the ring is kept readable.
+static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
+                    const DeviceState &ds, TcPlan *pl, std::string *why) {
+  if (layout == LAYOUT_COL) {
+    if (why) *why = "the tensor-core family reads K-major (row-major / interleaved) weights";
+    return false;
+  }
+  if (B < 1 || B > 64) {
+    if (why) *why = "tensor-core family needs 1 <= B <= 64";
+    return false;
+  }
+  const int bn = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
+  const int cap = std::min(ds.smem_optin, 232448);
+  const int nt = v.nt;
+  for (int mult = 1; mult <= 8; mult *= 2) {
+    const int P = std::min(N, ds.sms * mult);
+    const int rbase = N / P, rextra = N % P;
+    const int r_hi = rbase + (rextra ? 1 : 0);
+    for (int mt = 1; mt <= 2; ++mt) {
+      if (r_hi > 128 * mt) continue;
+      if (mt == 2 && rbase < 2) continue;
+      const int hmax = (r_hi + mt - 1) / mt;
+      const int rc = round_up(hmax, 8);
+      const int a_bytes = nt * mt * nmat * rc * 128;
+      const int x_bytes = nt * bn * 128 * (norm ? 2 : 1);
+      const int stage = a_bytes + x_bytes;
+      const int slack = std::max(0, 16384 - rc * 128 - x_bytes);
+      const int nsteps = ceil_div(K, TC_TILE_K * nt);
+      const int kpad = nsteps * nt * TC_TILE_K;
+      const int g_bytes = norm ? round_up(kpad * 2, 1024) : 0;
+      const int fixed = 1024 /* alignment */ + slack + g_bytes + 1024 /* barriers */;
+      const int S = std::min(8, (cap - fixed) / stage);
+      if (S < 2) continue;
+      const int cols = pow2_ceil(std::max(32, mt * nmat * bn));
+      if (cols > 512) continue;
+      const void *fn = tc_find_kernel(nmat, norm ? 1 : 0, layout == LAYOUT_IL ? 1 : 0, mt);
+      if (!fn) {
+        if (why) *why = "tensor-core kernel not compiled for this case";
+        return false;
+      }
+      pl->fn = fn;
+      pl->grid = P;
+      pl->mt = mt;
+      TcParams &p = pl->p;
+      p = TcParams{};
+      p.B = B;
+      p.K = K;
+      p.N = N;
+      p.nsteps = nsteps;
+      p.nt = nt;
+      p.rbase = rbase;
+      p.rextra = rextra;
+      p.hmax = hmax;
+      p.rc = rc;
+      p.bn = bn;
+      p.stages = S;
+      p.stage_bytes = stage;
+      p.a_bytes = a_bytes;
+      p.tmem_cols = cols;
+      p.g_off = S * stage + slack;
+      p.bar_off = p.g_off + g_bytes;
+      pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
+      return true;
+    }
+  }
+  if (why) *why = "no tensor-core partition fits shared memory";
+  return false;
+}
+
+static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  TcPlan pl;
+  std::string why;
+  if (!plan_tc(c.layout, c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
+    return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit B=%d K=%d N=%d: %s", v.id, c.B,
+                c.K, c.N, why.c_str());
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  TcMaps maps;
+  memset(&maps, 0, sizeof maps);
+  const int hmax = pl.p.hmax;
+  for (int lo = 0; lo < 2; ++lo) {
+    const uint32_t hgt = static_cast<uint32_t>(std::max(1, hmax - lo));
+    if (c.layout == LAYOUT_IL) {
+      const uint64_t dims[3] = {static_cast<uint64_t>(c.K), 2, static_cast<uint64_t>(c.N)};
+      const uint64_t strides[2] = {static_cast<uint64_t>(c.K) * 2,
+                                   static_cast<uint64_t>(c.K) * 4};
+      const uint32_t box[3] = {TC_TILE_K, 1, hgt};
+      if ((rc = tensor_map(c.w0, 3, dims, strides, box, true, &maps.wg[lo]))) return rc;
+    } else {
+      if ((rc = tensor_map_2d(c.w0, c.K, c.N, static_cast<uint64_t>(c.K) * 2, TC_TILE_K, hgt,
+                              &maps.wg[lo], true)))
+        return rc;
+      if (c.nmat == 2 &&
+          (rc = tensor_map_2d(c.w1, c.K, c.N, static_cast<uint64_t>(c.K) * 2, TC_TILE_K, hgt,
+                              &maps.wu[lo], true)))
+        return rc;
+    }
+  }
+  if ((rc = tensor_map_2d(c.x, c.K, c.B, static_cast<uint64_t>(c.K) * 2, TC_TILE_K, pl.p.bn,
+                          &maps.x, true)))
+    return rc;
+  TcParams p = pl.p;
+  p.out = static_cast<uint16_t *>(c.out);
+  p.gamma = static_cast<const uint16_t *>(c.gamma);
+  p.err = ds->err;
+  p.eps = c.eps;
+  void *args[] = {&maps, &p};
+  cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TC_THREADS), pl.smem, s,
+                                pdl_enabled(), args);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "tensor-core kernel launch");
+  }
+  if (stages_used) *stages_used = p.stages;
+  return DFK_OK;
+}
+
+static int launch_variant(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
+  return v.family == DFK_FAMILY_TENSOR_CORE ? launch_tc(c, v, s, stages_used)
+                                            : launch_cc(c, v, s, stages_used);
+}
+
 // ---------------------------------------------------------------- scheduler
 
 struct TuneKey {
@@ -437,36 +603,59 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->measured_us = us;
 }
 
-// Candidates worth timing for (op, B): every j-per-thread choice at its
-// largest useful token tile; every k split for the plain GEMV.
-static std::vector<const VDef *> candidates(int op, int B) {
-  std::vector<const VDef *> c;
+// Candidates worth timing for (op, B): every CUDA-core j-per-thread / k-split
+// / tiles-per-stage choice at its largest useful token tile, plus the
+// tensor-core variants from B = 8 up (below that, fp32 FMA on CUDA cores
+// keeps up with HBM and the contraction is too thin for the MMA).
+static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
+  std::vector<const VDef *> out;
   for (const VDef &d : variants()) {
     if (d.cls != op_class(op)) continue;
+    if (d.family == DFK_FAMILY_TENSOR_CORE) {
+      if (B >= 8 && c.layout != LAYOUT_COL) out.push_back(&d);
+      continue;
+    }
     if (d.bt != bt_for(B, d.jpt)) continue;
-    c.push_back(&d);
+    out.push_back(&d);
   }
-  return c;
+  return out;
 }
 
-// Heuristic default (no timing): 4 rows per thread up to B = 4, then 2;
-// for the GEMV the largest k split whose CTA fits.  If that family does not
-// fit (shared memory), the feasible variant with the fewest passes wins.
+static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
+  if (d.family == DFK_FAMILY_TENSOR_CORE) {
+    TcPlan pl;
+    return plan_tc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+  }
+  CcPlan pl;
+  return plan_cc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+}
+
+// Heuristic default (no timing): the tensor-core family from B = 8 up (one
+// k-tile per stage for gate/up, four for the GEMV); below that CUDA cores
+// with 4 rows per thread (2 rows from B = 5), two k-tiles per stage, and for
+// the GEMV the largest k split whose CTA fits.  If nothing of that shape
+// fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
+  if (B >= 8 && c.layout != LAYOUT_COL) {
+    const int want_nt = op_class(op) == CLS_GEMV ? 4 : 1;
+    for (const VDef &d : variants())
+      if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == want_nt &&
+          feasible(d, c, ds))
+        return &d;
+  }
   const int jpt = B <= 4 ? 4 : 2;
   const VDef *best = nullptr;
   for (const VDef &d : variants()) {
-    if (d.cls != op_class(op) || d.jpt != jpt || d.bt != bt_for(B, jpt)) continue;
-    CcPlan pl;
-    if (!plan_cc(c.layout, c.nmat, c.norm, d, B, c.K, c.N, ds, &pl, nullptr)) continue;
+    if (d.cls != op_class(op) || d.family != DFK_FAMILY_CUDA_CORE) continue;
+    if (d.jpt != jpt || d.bt != bt_for(B, jpt) || d.nt != 2) continue;
+    if (!feasible(d, c, ds)) continue;
     if (!best || d.ksplit > best->ksplit) best = &d;
   }
   if (best) return best;
   int best_pass = 1 << 30;
   for (const VDef &d : variants()) {
-    if (d.cls != op_class(op)) continue;
-    CcPlan pl;
-    if (!plan_cc(c.layout, c.nmat, c.norm, d, B, c.K, c.N, ds, &pl, nullptr)) continue;
+    if (d.cls != op_class(op) || d.family != DFK_FAMILY_CUDA_CORE) continue;
+    if (!feasible(d, c, ds)) continue;
     const int passes = ceil_div(B, d.bt);
     if (passes < best_pass || (passes == best_pass && d.ksplit > best->ksplit)) {
       best = &d;
@@ -509,7 +698,7 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
   float best_t = 1e30f;
   for (const VDef *d : cands) {
     int st = 0;
-    if (launch_cc(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible variants
+    if (launch_variant(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible ones
     // Each repetition: flush L2, then a burst of back-to-back launches (the
     // way a decode loop issues them, neighbours overlapping through
     // programmatic dependent launch); the sample is the burst's mean.
@@ -519,7 +708,7 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
     for (int r = 0; r < reps && ok; ++r) {
       if (flush) cudaMemsetAsync(flush, r & 0xff, flush_bytes, s);
       cudaEventRecord(e0, s);
-      for (int b = 0; b < burst && ok; ++b) ok = launch_cc(c, *d, s, nullptr) == DFK_OK;
+      for (int b = 0; b < burst && ok; ++b) ok = launch_variant(c, *d, s, nullptr) == DFK_OK;
       cudaEventRecord(e1, s);
       if (cudaEventSynchronize(e1) != cudaSuccess) ok = false;
       float ms = 0.f;
@@ -577,7 +766,7 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
   float us = -1.f;
   int stages = 0;
   if (tune) {
-    const VDef *t = time_candidates(op, c, candidates(op, c.B), s, *ds, &us, &stages);
+    const VDef *t = time_candidates(op, c, candidates(op, c.B, c), s, *ds, &us, &stages);
     if (t) win = t;
     else us = -1.f;
   }
@@ -660,7 +849,7 @@ static int gate_up_impl(int op, const void *x, const void *gamma, float eps, con
   CcCall c{to_engine_layout(layout), 2, norm, x, gamma, eps, wg, wu, h, B, D, F};
   const VDef *v = nullptr;
   if ((rc = resolve(op, variant, c, s, &v))) return rc;
-  return launch_cc(c, *v, s, nullptr);
+  return launch_variant(c, *v, s, nullptr);
 }
 
 static int gemv_impl(int op, const void *x, const void *w, void *out, int B, int K, int N,
@@ -670,7 +859,7 @@ static int gemv_impl(int op, const void *x, const void *w, void *out, int B, int
   CcCall c{LAYOUT_ROW, 1, false, x, nullptr, 0.f, w, nullptr, out, B, K, N};
   const VDef *v = nullptr;
   if ((rc = resolve(op, variant, c, s, &v))) return rc;
-  return launch_cc(c, *v, s, nullptr);
+  return launch_variant(c, *v, s, nullptr);
 }
 
 }  // namespace dfk
@@ -778,7 +967,7 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
                     L == DFK_W_GU_INTERLEAVED ? nullptr : pw1, po, B, d_model, d_ff};
     float us = -1.f;
     int stages = 0;
-    const VDef *win = time_candidates(op, c, candidates(op, B), s, *ds, &us, &stages);
+    const VDef *win = time_candidates(op, c, candidates(op, B, c), s, *ds, &us, &stages);
     if (!win) {
       win = heuristic(op, B, c, *ds);
       us = -1.f;

@@ -1,0 +1,330 @@
+// tc_engine.cuh -- tensor-core (tcgen05 / TMEM) weight-streaming kernel for
+// the decode MLP at larger decode batches (8 <= B <= 64), where fp32 FMA on
+// CUDA cores can no longer keep up with HBM.
+//
+// Same operation as the CUDA-core engine ("Deep Kernel Fusion for
+// Transformer Decoding", episode description: gate projection, up
+// projection, SiLU and elementwise multiply in one decode kernel; the down
+// projection is the NMAT = 1 instance), formulated for the MMA with the
+// weight rows on M and the tokens on N:
+//     D_gate[j][n] = sum_k Wg[j][k] * X[n][k],  D_up likewise,
+// accumulated in fp32 in TMEM, then h[n][j] = SiLU(D_gate) * D_up.
+//
+// Work split: one CTA per SM owns a contiguous range of r ~ F / #SMs output
+// rows over the whole reduction (no split-K, no scratch memory); the range
+// is cut into MT sub-tiles of at most 128 rows, each one M = 128 MMA tile.
+// Rows of a sub-tile beyond its height come from neighbouring shared memory
+// and produce ignored accumulator rows (the MMA reads 128 rows; only the
+// loaded ones are stored).
+//
+// RMSNorm prologue (NORM): r_b = 1/sqrt(mean_k x[b][k]^2 + eps) is a
+// per-token scalar, so it factors out of the dot product:
+//     a[b][j] = r_b * sum_k (x[b][k] * gamma[k]) * Wg[j][k].
+// Four warps turn each streamed x tile into x*gamma, split exactly into two
+// bf16 halves (hi = bf16(x*gamma), lo = bf16(x*gamma - hi); the product of
+// two bf16 values has at most 16 significant bits, so hi + lo is exact),
+// accumulate sum_k x^2 on the way, and scale by r_b in the epilogue.
+//
+// Warp roles (192 threads): warp 0 issues TMA copies into an S-stage ring;
+// warp 1 owns TMEM and issues the MMAs (one thread) with tcgen05.commit
+// releasing ring stages; warps 2-5 run the x*gamma transform (NORM) and the
+// epilogue (tcgen05.ld -> SiLU * up -> one bf16 store per output).
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tc_ptx.cuh"
+
+namespace dfk {
+
+constexpr int TC_THREADS = 192;
+constexpr int TC_TILE_K = 64;       // reduction elements per k-tile (one 128-byte swizzle row)
+constexpr int TC_ATOM = 1024;       // bytes of an 8-row swizzle atom
+
+struct TcParams {
+  uint16_t *out;          // [B][N] bf16
+  const uint16_t *gamma;  // [K] bf16 (NORM)
+  unsigned *err;          // device error word
+  int B, K, N;
+  float eps;
+  int nsteps;             // ring steps = ceil(K / (64 * nt))
+  int nt;                 // k-tiles per ring stage
+  int rbase, rextra;      // rows per CTA: rbase, +1 for the first rextra CTAs
+  int hmax;               // height of the taller sub-tile box (map 0); map 1 is hmax - 1
+  int rc;                 // rows reserved per A tile in shared memory (multiple of 8)
+  int bn;                 // tokens on N: 16, 32 or 64
+  int stages, stage_bytes;
+  int a_bytes;            // A-tile bytes of one stage
+  int tmem_cols;
+  int g_off, bar_off;     // shared-memory offsets from the 1024-byte aligned base
+};
+
+// wg/wu: [0] box height hmax, [1] box height hmax - 1; x: activations box {64, bn}.
+// Interleaved weights use wg for both matrices (3-D map {k, gate|up, row}).
+struct TcMaps {
+  CUtensorMap wg[2];
+  CUtensorMap wu[2];
+  CUtensorMap x;
+};
+
+template <int NMAT, bool NORM, bool IL, int MT>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_gemv_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  static_assert(NMAT == 1 || NMAT == 2, "NMAT");
+  static_assert(!IL || NMAT == 2, "interleaved layout holds both matrices");
+  static_assert(!NORM || NMAT == 2, "the RMSNorm prologue belongs to the gate/up kernel");
+  static_assert(MT == 1 || MT == 2, "MT");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base (the host reserves the slack)
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = p.stages, NT = p.nt, BN = p.bn;
+
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+  uint64_t *empty = full + S;
+  uint64_t *xready = empty + S;
+  uint64_t *accfull = xready + S;
+  volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
+  int *s_issued = reinterpret_cast<int *>(accfull + 1) + 1;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accfull + 1) + 2;
+  float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(accfull + 1) + 16);
+  uint16_t *gs = reinterpret_cast<uint16_t *>(smem + p.g_off);
+
+  // ---- this CTA's rows [j0, j0 + r), cut into MT sub-tiles
+  const int cta = blockIdx.x;
+  const int j0 = cta * p.rbase + min(cta, p.rextra);
+  const int r = p.rbase + (cta < p.rextra ? 1 : 0);
+  int h[MT], rs[MT];
+  h[0] = (r + MT - 1) / MT;
+  rs[0] = 0;
+  if constexpr (MT == 2) {
+    h[1] = r - h[0];
+    rs[1] = h[0];
+  }
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&xready[s], 128);
+    }
+    mbar_init(accfull, 1);
+    *s_abort = 0;
+    *s_issued = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ================= TMA producer (one lane)
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_normal();
+      const uint32_t tx = static_cast<uint32_t>(NT) * (NMAT * r + BN) * 128u;
+      const int S0 = min(S, p.nsteps);
+      int issued = 0;
+      for (int i = 0; i < p.nsteps; ++i) {
+        const int st = i % S;
+        if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
+        uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[st], tx);
+        for (int kt = 0; kt < NT; ++kt) {
+          const int k0 = (i * NT + kt) * TC_TILE_K;
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            const int mi = (h[t] == p.hmax) ? 0 : 1;
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+              uint8_t *dst = sb + ((kt * MT + t) * NMAT + m) * p.rc * 128;
+              if (IL)
+                tma_load_3d(dst, &maps.wg[mi], &full[st], k0, m, j0 + rs[t], pol_w);
+              else
+                tma_load_2d(dst, m == 0 ? &maps.wg[mi] : &maps.wu[mi], &full[st], k0,
+                            j0 + rs[t], pol_w);
+            }
+          }
+          // activations: only after the previous kernel's results are visible
+          if (i >= S0)
+            tma_load_2d(sb + p.a_bytes + kt * BN * 128, &maps.x, &full[st], k0, 0, pol_x);
+        }
+        if (i == S0 - 1) {
+          pdl_wait();
+          for (int ii = 0; ii < S0; ++ii)
+            for (int kt = 0; kt < NT; ++kt)
+              tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
+                              kt * BN * 128,
+                          &maps.x, &full[ii], (ii * NT + kt) * TC_TILE_K, 0, pol_x);
+        }
+        issued = i + 1;
+      }
+      *s_issued = issued;
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (one lane)
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32(128, BN);
+      for (int i = 0; i < p.nsteps; ++i) {
+        const int st = i % S;
+        if (!mbar_wait_bounded(NORM ? &xready[st] : &full[st], (i / S) & 1, s_abort, p.err))
+          break;
+        tc_fence_after();
+        const uint32_t sb = sbase + static_cast<uint32_t>(st) * p.stage_bytes;
+        for (int kt = 0; kt < NT; ++kt) {
+          const uint64_t bx = umma_desc_sw128(sb + p.a_bytes + kt * BN * 128);
+          const uint64_t bl = umma_desc_sw128(sb + p.a_bytes + (NT + kt) * BN * 128);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+#pragma unroll
+              for (int m = 0; m < NMAT; ++m) {
+                const uint64_t a =
+                    umma_desc_sw128(sb + ((kt * MT + t) * NMAT + m) * p.rc * 128) + 2 * kk;
+                const uint32_t d = tmem + static_cast<uint32_t>((t * NMAT + m) * BN);
+                const uint32_t acc = (i > 0 || kt > 0 || kk > 0) ? 1u : 0u;
+                umma_bf16(d, a, bx + 2 * kk, idesc, acc);
+                if (NORM) umma_bf16(d, a, bl + 2 * kk, idesc, 1u);
+              }
+            }
+          }
+        }
+        umma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+      }
+      umma_commit(accfull);       // every MMA issued above has completed
+    }
+  } else {
+    // ================= x*gamma transform (NORM) and epilogue: warps 2..5
+    const int et = tid - 64;
+    if (NORM) {
+      pdl_wait();
+      const int kpad = p.nsteps * NT * TC_TILE_K;
+      for (int idx = et; idx < kpad / 8; idx += 128) {
+        const int k = idx * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (k < p.K) v = ld_nc_v4(p.gamma + k);
+        *reinterpret_cast<uint4 *>(gs + k) = v;
+      }
+      named_barrier(1, 128);
+      const int tpr = 128 / BN;       // threads per token row
+      const int n = et / tpr, part = et - n * tpr;
+      const int cpt = 8 / tpr;        // 16-byte chunks per thread per k-tile
+      float ss = 0.f;
+      for (int i = 0; i < p.nsteps; ++i) {
+        const int st = i % S;
+        const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
+        if (ok) {
+          uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
+          for (int kt = 0; kt < NT; ++kt) {
+            uint8_t *xt = sb + p.a_bytes + kt * BN * 128;
+            uint8_t *lt = sb + p.a_bytes + (NT + kt) * BN * 128;
+            for (int c = 0; c < cpt; ++c) {
+              const int pc = part * cpt + c;          // physical 16-byte chunk of row n
+              const int lc = pc ^ (n & 7);            // 128-byte swizzle: logical chunk
+              const int k = (i * NT + kt) * TC_TILE_K + 8 * lc;
+              const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
+              const uint4 gv = *reinterpret_cast<const uint4 *>(gs + k);
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float x0 = bf16_lo(xw[q]), x1 = bf16_hi(xw[q]);
+                ss = fmaf(x0, x0, ss);
+                ss = fmaf(x1, x1, ss);
+                const float p0 = x0 * bf16_lo(gw[q]), p1 = x1 * bf16_hi(gw[q]);  // exact
+                const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
+                const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+                const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+                hw[q] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                lw[q] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
+                        (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
+              }
+              *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) =
+                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4 *>(lt + n * 128 + pc * 16) =
+                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(&xready[st]);
+      }
+      // sum of squares of row n: the tpr threads of a row are adjacent lanes
+      for (int m = tpr >> 1; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      if (part == 0)
+        s_rinv[n] = (n < p.B) ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 0.f;
+      named_barrier(1, 128);
+    }
+
+    // ---- epilogue: TMEM -> registers -> SiLU(gate) * up -> bf16 h
+    const bool ok = mbar_wait_bounded(accfull, 0, s_abort, p.err);
+    tc_fence_after();
+    const bool go = __all_sync(0xffffffffu, ok && !*s_abort);
+    const int q = warp & 3;               // TMEM lanes 32q .. 32q + 31 belong to this warp
+    const int row = 32 * q + lane;
+    if (go) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        for (int c = 0; c < BN; c += 16) {
+          float g[16], u[16];
+          const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+          tmem_ld_32x32b_x16(base + (t * NMAT) * BN + c, g);
+          if (NMAT == 2) tmem_ld_32x32b_x16(base + (t * NMAT + 1) * BN + c, u);
+          tmem_ld_wait();
+          if (row < h[t]) {
+            const int j = j0 + rs[t] + row;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int n = c + e;
+              if (n < p.B) {
+                float res;
+                if (NMAT == 2) {
+                  const float sc = NORM ? s_rinv[n] : 1.0f;
+                  const float a = g[e] * sc, uu = u[e] * sc;
+                  res = (a / (1.0f + expf(-a))) * uu;
+                } else {
+                  res = g[e];
+                }
+                p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
+              }
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    // every MMA has completed before TMEM is released (bounded wait)
+    if (lane == 0) mbar_wait_bounded(accfull, 0, nullptr, p.err);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+  if (tid == 0 && *s_abort) {
+    // after an aborted pipeline, wait (bounded) for copies still in flight
+    const int issued = *s_issued;
+    for (int st = 0; st < S; ++st) {
+      int last = -1;
+      for (int i = issued - 1; i >= 0 && i >= issued - S; --i)
+        if (i % S == st) { last = i; break; }
+      if (last >= 0) mbar_wait_bounded(&full[st], (last / S) & 1, nullptr, p.err);
+    }
+  }
+}
+
+}  // namespace dfk

@@ -53,12 +53,19 @@ def test_variant_table(L):
     n = dfk.dfk_variant_count()
     assert n >= 8
     ids = set()
+    families = set()
     for i in range(1, n + 1):
         v = dfk.dfk_variant_info(i)
         assert v["variant_id"] == i
-        assert v["j_per_thread"] in (2, 4)
-        assert v["token_tile"] in (1, 2, 4, 8, 16, 32, 64)
+        families.add(v["family"])
+        if v["family"] == 0:      # CUDA-core
+            assert v["j_per_thread"] in (2, 4)
+            assert v["token_tile"] in (1, 2, 4, 8)
+        else:                     # tensor core: token tile 16/32/64 chosen from B
+            assert v["family"] == 1 and v["token_tile"] == 64
+        assert v["k_tiles_per_stage"] in (1, 2, 4, 8)
         ids.add(i)
+    assert families == {0, 1}
     with pytest.raises(dfk.DfkError) as e:
         dfk.dfk_variant_info(n + 1)
     assert e.value.status == dfk.DFK_ERR_INVALID_ARG

@@ -336,3 +336,58 @@ def test_llama3_70b_full_mlp(B):
     yrows = sample_rows(8192, 128, 4)
     assert_close(y[:, yrows], oracle.down(I.to_bits(h), I.to_bits(inp.w_down), rows=yrows),
                  "70B down (isolated) B=%d" % B)
+
+
+# ------------------------------------------------------------------ tensor-core family
+
+def tc_variants(op):
+    return [i for i in range(1, dfk.dfk_variant_count() + 1)
+            if dfk.dfk_variant_info(i)["op"] == op and dfk.dfk_variant_info(i)["family"] == 1]
+
+
+TC_SHAPES = [(1, 256, 688), (3, 320, 200), (8, 512, 1496), (13, 384, 520), (16, 1024, 2056),
+             (24, 128, 344), (32, 256, 264), (40, 448, 904), (64, 512, 776)]
+
+
+@pytest.mark.parametrize("B,D,F", TC_SHAPES)
+def test_tensor_core_gate_up(B, D, F):
+    inp = I.make_inputs(B, D, F, seed=300 + B, w_std=0.05, with_down=False, device="cuda")
+    ref_norm = oracle_gate_up(inp, True)
+    ref_plain = oracle_gate_up(inp, False)
+    for vid in tc_variants(dfk.DFK_OP_GATE_UP):
+        for layout in (I.LAYOUT_ROW, I.LAYOUT_INTERLEAVED):
+            h = run_gate_up(inp, layout, True, variant=vid)
+            torch.cuda.synchronize()
+            assert_close(h, ref_norm, "tc variant %d layout %d norm" % (vid, layout))
+            h2 = run_gate_up(inp, layout, False, variant=vid)
+            torch.cuda.synchronize()
+            assert_close(h2, ref_plain, "tc variant %d layout %d plain" % (vid, layout))
+        # the column-major layout is not a tensor-core layout: rejected, not misrouted
+        with pytest.raises(dfk.DfkError) as e:
+            run_gate_up(inp, I.LAYOUT_COL, True, variant=vid)
+        assert e.value.status == dfk.DFK_ERR_NO_VARIANT
+
+
+@pytest.mark.parametrize("B,D,F", [(8, 256, 688), (16, 4096, 1024), (64, 512, 2048)])
+def test_tensor_core_down(B, D, F):
+    g = torch.Generator(device="cuda").manual_seed(B * 7 + D)
+    h = (torch.randn(B, F, generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    wd = (torch.randn(D, F, generator=g, device="cuda") * 0.03).to(torch.bfloat16)
+    ref = oracle.down(I.to_bits(h), I.to_bits(wd))
+    for vid in tc_variants(dfk.DFK_OP_DOWN):
+        y = dfk.dfk_down_proj(h, wd, variant=vid)
+        torch.cuda.synchronize()
+        assert_close(y, ref, "tc down variant %d" % vid)
+
+
+def test_tensor_core_batch_rows_independent():
+    # tensor-core results per row do not depend on the other rows' values
+    B, D, F = 32, 512, 1000
+    inp = I.make_inputs(B, D, F, seed=41, w_std=0.05, with_down=False, device="cuda")
+    vid = tc_variants(dfk.DFK_OP_GATE_UP)[0]
+    full = run_gate_up(inp, I.LAYOUT_ROW, True, variant=vid)
+    x2 = inp.x.clone()
+    x2[1:] = x2[1:].flip(0)
+    other = I.MLPInputs(x2, inp.gamma, inp.w_gate, inp.w_up, None)
+    h2 = run_gate_up(other, I.LAYOUT_ROW, True, variant=vid)
+    assert bits_equal(full[0], h2[0])
