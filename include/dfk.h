@@ -89,6 +89,7 @@ typedef struct dfk_variant {
   int token_tile;   /* tokens per pass over the weights                              */
   int k_split;      /* thread teams splitting the reduction dimension               */
   int k_tiles_per_stage; /* consecutive 64-wide reduction tiles per ring stage       */
+  int acc_banks;    /* tensor core: independent TMEM accumulators per output        */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
 } dfk_variant;

@@ -224,6 +224,7 @@ struct VDef {
   int cls;
   int family;
   int jpt, bt, ksplit, nt;
+  int nbank;  // tensor core: independent TMEM accumulator banks per output
 };
 
 static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
@@ -234,16 +235,18 @@ static const std::vector<VDef> &variants() {
     int id = 1;
     for (int nt : {1, 2, 4})
       for (auto &jb : kJB)
-        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt});
+        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt, 1});
     for (int nt : {1, 2, 4})
       for (int ks : {1, 2, 4, 8})
         for (auto &jb : kJB)
-          t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt});
+          t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt, 1});
     // tensor-core family: token tile chosen from B at launch (16 / 32 / 64)
-    for (int nt : {1, 2})
-      t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt});
-    for (int nt : {1, 2, 4, 8})
-      t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt});
+    for (int nb : {1, 2})
+      for (int nt : {1, 2})
+        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb});
+    for (int nb : {1, 2})
+      for (int nt : {1, 2, 4, 8})
+        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb});
     return t;
   }();
   return v;
@@ -474,7 +477,8 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       const int hmax = (r_hi + mt - 1) / mt;
       const int rc = round_up(hmax, 8);
       const int a_bytes = nt * mt * nmat * rc * 128;
-      const int x_bytes = nt * bn * 128 * (norm ? 2 : 1);
+      const int xt_bytes = bn * 128 * (norm ? 2 : 1);  // hi rows (+ lo rows)
+      const int x_bytes = nt * xt_bytes;
       const int stage = a_bytes + x_bytes;
       const int slack = std::max(0, 16384 - rc * 128 - x_bytes);
       const int nsteps = ceil_div(K, TC_TILE_K * nt);
@@ -483,7 +487,11 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       const int fixed = 1024 /* alignment */ + slack + g_bytes + 1024 /* barriers */;
       const int S = std::min(8, (cap - fixed) / stage);
       if (S < 2) continue;
-      const int cols = pow2_ceil(std::max(32, mt * nmat * bn));
+      // accumulator banks per output: the variant's count, as far as TMEM holds
+      const int wn = norm ? 2 * bn : bn;  // MMA N: the tokens (hi rows, then lo rows)
+      int nbank = std::max(1, v.nbank);
+      while (nbank > 1 && mt * nmat * nbank * wn > 512) nbank >>= 1;
+      const int cols = pow2_ceil(std::max(32, mt * nmat * nbank * wn));
       if (cols > 512) continue;
       const void *fn = tc_find_kernel(nmat, norm ? 1 : 0, layout == LAYOUT_IL ? 1 : 0, mt);
       if (!fn) {
@@ -508,7 +516,9 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       p.stages = S;
       p.stage_bytes = stage;
       p.a_bytes = a_bytes;
+      p.xt_bytes = xt_bytes;
       p.tmem_cols = cols;
+      p.nbank = nbank;
       p.g_off = S * stage + slack;
       p.bar_off = p.g_off + g_bytes;
       pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
@@ -599,6 +609,7 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->token_tile = d.bt;
   out->k_split = d.ksplit;
   out->k_tiles_per_stage = d.nt;
+  out->acc_banks = d.nbank;
   out->stages = stages;
   out->measured_us = us;
 }

@@ -23,7 +23,9 @@
 // Four warps turn each streamed x tile into x*gamma, split exactly into two
 // bf16 halves (hi = bf16(x*gamma), lo = bf16(x*gamma - hi); the product of
 // two bf16 values has at most 16 significant bits, so hi + lo is exact),
-// accumulate sum_k x^2 on the way, and scale by r_b in the epilogue.
+// accumulate sum_k x^2 on the way, and scale by r_b in the epilogue.  The hi
+// and lo rows sit side by side on N (one MMA of N = 2 * bn reads each weight
+// tile once); the epilogue adds the two column halves.
 //
 // Warp roles (192 threads): warp 0 issues TMA copies into an S-stage ring;
 // warp 1 owns TMEM and issues the MMAs (one thread) with tcgen05.commit
@@ -56,7 +58,9 @@ struct TcParams {
   int bn;                 // tokens on N: 16, 32 or 64
   int stages, stage_bytes;
   int a_bytes;            // A-tile bytes of one stage
+  int xt_bytes;           // bytes of one k-tile's activation rows (bn * 128, x2 with NORM)
   int tmem_cols;
+  int nbank;              // independent TMEM accumulators per output (1, 2 or 4)
   int g_off, bar_off;     // shared-memory offsets from the 1024-byte aligned base
 };
 
@@ -67,6 +71,46 @@ struct TcMaps {
   CUtensorMap wu[2];
   CUtensorMap x;
 };
+
+// Loads 16 columns of `nb` accumulator banks (bank stride `bank_cols`
+// columns) for this warp's 32 TMEM lanes and adds them in a fixed order; with
+// lo_off > 0 each bank also holds a second column block lo_off columns
+// further (the lo products), added to its first block before the banks are
+// combined: v = ((b0.hi + b0.lo) + (b1.hi + b1.lo)) + ...
+__device__ __forceinline__ void tmem_sum_banks(uint32_t taddr, int nb, int bank_cols, int lo_off,
+                                               float (&v)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = 0.f;
+  float part[4][16];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if (b < nb) {  // nb is warp-uniform: the loads stay converged
+      float hi[16];
+      tmem_ld_32x32b_x16(taddr + b * bank_cols, hi);
+      if (lo_off > 0) {
+        float lo[16];
+        tmem_ld_32x32b_x16(taddr + b * bank_cols + lo_off, lo);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) part[b][e] = hi[e] + lo[e];
+      } else {
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) part[b][e] = hi[e];
+      }
+    }
+  }
+  if (nb == 1) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = part[0][e];
+  } else if (nb == 2) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = part[0][e] + part[1][e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = (part[0][e] + part[1][e]) + (part[2][e] + part[3][e]);
+  }
+}
 
 template <int NMAT, bool NORM, bool IL, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -157,14 +201,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           // activations: only after the previous kernel's results are visible
           if (i >= S0)
-            tma_load_2d(sb + p.a_bytes + kt * BN * 128, &maps.x, &full[st], k0, 0, pol_x);
+            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &full[st], k0, 0, pol_x);
         }
         if (i == S0 - 1) {
           pdl_wait();
           for (int ii = 0; ii < S0; ++ii)
             for (int kt = 0; kt < NT; ++kt)
               tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
-                              kt * BN * 128,
+                              kt * p.xt_bytes,
                           &maps.x, &full[ii], (ii * NT + kt) * TC_TILE_K, 0, pol_x);
         }
         issued = i + 1;
@@ -173,29 +217,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else if (warp == 1) {
     // ================= MMA issuer (one lane)
+    // Each output may accumulate into NB independent TMEM banks (k-slice kk
+    // of a tile goes to bank kk % NB); the epilogue adds the banks in a fixed
+    // order.  One MMA covers N = bn tokens, or with the prologue N = 2 bn
+    // (the hi rows, then the lo rows).
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(128, BN);
+      const int WN = NORM ? 2 * BN : BN;
+      const uint32_t idesc = umma_idesc_bf16_f32(128, WN);
+      const int NB = p.nbank;
+      // descriptors are built once; the address field (bits 0-13, 16-byte
+      // units) is then advanced by plain addition (shared memory < 256 KB)
+      const uint64_t desc0 = umma_desc_sw128(sbase);
+      const uint32_t tile_enc = static_cast<uint32_t>(p.rc * 128) >> 4;
+      const uint32_t x_enc = static_cast<uint32_t>(p.a_bytes) >> 4;
+      const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < p.nsteps; ++i) {
         const int st = i % S;
         if (!mbar_wait_bounded(NORM ? &xready[st] : &full[st], (i / S) & 1, s_abort, p.err))
           break;
         tc_fence_after();
-        const uint32_t sb = sbase + static_cast<uint32_t>(st) * p.stage_bytes;
+        const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
         for (int kt = 0; kt < NT; ++kt) {
-          const uint64_t bx = umma_desc_sw128(sb + p.a_bytes + kt * BN * 128);
-          const uint64_t bl = umma_desc_sw128(sb + p.a_bytes + (NT + kt) * BN * 128);
+          const uint64_t bx = ds + x_enc + kt * xt_enc;
+          const uint64_t at = ds + static_cast<uint64_t>(kt * MT * NMAT) * tile_enc;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            const int b = kk % NB;
+            const uint32_t acc = (i > 0 || kt > 0 || kk >= NB) ? 1u : 0u;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
 #pragma unroll
               for (int m = 0; m < NMAT; ++m) {
-                const uint64_t a =
-                    umma_desc_sw128(sb + ((kt * MT + t) * NMAT + m) * p.rc * 128) + 2 * kk;
-                const uint32_t d = tmem + static_cast<uint32_t>((t * NMAT + m) * BN);
-                const uint32_t acc = (i > 0 || kt > 0 || kk > 0) ? 1u : 0u;
+                const uint64_t a = at + static_cast<uint64_t>(t * NMAT + m) * tile_enc + 2 * kk;
+                const uint32_t d = tmem + static_cast<uint32_t>(((t * NMAT + m) * NB + b) * WN);
                 umma_bf16(d, a, bx + 2 * kk, idesc, acc);
-                if (NORM) umma_bf16(d, a, bl + 2 * kk, idesc, 1u);
               }
             }
           }
@@ -227,8 +282,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (ok) {
           uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
           for (int kt = 0; kt < NT; ++kt) {
-            uint8_t *xt = sb + p.a_bytes + kt * BN * 128;
-            uint8_t *lt = sb + p.a_bytes + (NT + kt) * BN * 128;
+            uint8_t *xt = sb + p.a_bytes + kt * p.xt_bytes;
+            uint8_t *lt = xt + BN * 128;
             for (int c = 0; c < cpt; ++c) {
               const int pc = part * cpt + c;          // physical 16-byte chunk of row n
               const int lc = pc ^ (n & 7);            // 128-byte swizzle: logical chunk
@@ -275,14 +330,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;               // TMEM lanes 32q .. 32q + 31 belong to this warp
     const int row = 32 * q + lane;
     if (go) {
+      const int NB = p.nbank;
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         for (int c = 0; c < BN; c += 16) {
           float g[16], u[16];
           const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-          tmem_ld_32x32b_x16(base + (t * NMAT) * BN + c, g);
-          if (NMAT == 2) tmem_ld_32x32b_x16(base + (t * NMAT + 1) * BN + c, u);
-          tmem_ld_wait();
+          // fixed order: per bank (hi + lo), then ((b0 + b1) + (b2 + b3))
+          const int WN = NORM ? 2 * BN : BN;
+          tmem_sum_banks(base + (t * NMAT) * NB * WN + c, NB, WN, NORM ? BN : 0, g);
+          if (NMAT == 2)
+            tmem_sum_banks(base + (t * NMAT + 1) * NB * WN + c, NB, WN, NORM ? BN : 0, u);
           if (row < h[t]) {
             const int j = j0 + rs[t] + row;
 #pragma unroll

@@ -52,6 +52,17 @@ def gate_up_variants(B):
     return out
 
 
+def cc_gate_up_variant(B, jpt=2, nt=1):
+    """Id of the CUDA-core gate/up variant (jpt, nt) at its token tile for batch B."""
+    bt = min(1 << max(B - 1, 0).bit_length(), 4 if jpt == 4 else 8)
+    for i in range(1, dfk.dfk_variant_count() + 1):
+        v = dfk.dfk_variant_info(i)
+        if (v["op"] == dfk.DFK_OP_GATE_UP and v["family"] == 0 and v["j_per_thread"] == jpt
+                and v["token_tile"] == bt and v["k_tiles_per_stage"] == nt):
+            return i
+    raise LookupError((B, jpt, nt))
+
+
 def gemv_variants():
     return [i for i in range(1, dfk.dfk_variant_count() + 1)
             if dfk.dfk_variant_info(i)["op"] == dfk.DFK_OP_DOWN]
@@ -116,11 +127,16 @@ def test_gate_up_small_shapes_all_layouts(B, D, F, norm):
                         device="cuda")
     ref = oracle_gate_up(inp, norm)
     outs = []
+    vid = cc_gate_up_variant(B)
     for layout in (I.LAYOUT_ROW, I.LAYOUT_COL, I.LAYOUT_INTERLEAVED):
-        h = run_gate_up(inp, layout, norm)
+        h = run_gate_up(inp, layout, norm)          # the scheduler's choice
         torch.cuda.synchronize()
         assert_close(h, ref, "B=%d D=%d F=%d layout=%d norm=%d" % (B, D, F, layout, norm))
-        outs.append(h)
+        hc = run_gate_up(inp, layout, norm, variant=vid)   # one CUDA-core variant
+        torch.cuda.synchronize()
+        assert_close(hc, ref, "CUDA-core B=%d layout=%d norm=%d" % (B, layout, norm))
+        outs.append(hc)
+    # within the CUDA-core family the layouts agree bit for bit
     assert bits_equal(outs[0], outs[1]), "row-major and column-major differ bitwise"
     assert bits_equal(outs[0], outs[2]), "row-major and interleaved differ bitwise"
 
@@ -141,16 +157,18 @@ def test_every_gate_up_variant_is_bitwise_identical(B):
 
 
 def test_batch_independence_and_row_permutation():
+    # CUDA-core family: row b of h depends only on row b of x, whatever the
+    # batch size, variant or layout
     B, D, F = 16, 512, 776
     inp = I.make_inputs(B, D, F, seed=21, w_std=0.05, with_down=False, device="cuda")
-    full = run_gate_up(inp, I.LAYOUT_ROW, True)
+    full = run_gate_up(inp, I.LAYOUT_ROW, True, variant=cc_gate_up_variant(B))
     for b in (0, 5, 15):
         one = I.MLPInputs(inp.x[b:b + 1].contiguous(), inp.gamma, inp.w_gate, inp.w_up, None)
-        hb = run_gate_up(one, I.LAYOUT_COL, True)
+        hb = run_gate_up(one, I.LAYOUT_COL, True, variant=cc_gate_up_variant(1, jpt=4, nt=2))
         assert bits_equal(hb, full[b:b + 1]), "row %d depends on the batch" % b
     perm = torch.randperm(B, generator=torch.Generator().manual_seed(3)).cuda()
     px = I.MLPInputs(inp.x[perm].contiguous(), inp.gamma, inp.w_gate, inp.w_up, None)
-    hp = run_gate_up(px, I.LAYOUT_INTERLEAVED, True)
+    hp = run_gate_up(px, I.LAYOUT_INTERLEAVED, True, variant=cc_gate_up_variant(B, jpt=4))
     assert bits_equal(hp, full[perm])
 
 
