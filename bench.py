@@ -437,11 +437,59 @@ def extra_measurements(args, inp, copies, h, y):
             t = timed_us(lambda i: dfk.dfk_rmsnorm_swiglu_gate_up(
                 xb, inp.gamma, inp.eps, ws[i % 2][0], ws[i % 2][1], name, h=hb), reps, flush)
             gbs = gate_up_bytes(B, D, F) / (t * 1e-6) / 1e9
-            row[name] = {"us": round(t, 2), "GBps": round(gbs, 1), "frac": round(gbs / peak, 4)}
+            v = dfk.dfk_cached_variant(dfk.DFK_OP_RMSNORM_GATE_UP, B, D, F, name) or {}
+            row[name] = {"us": round(t, 2), "GBps": round(gbs, 1), "frac": round(gbs / peak, 4),
+                         "variant": v.get("variant_id"),
+                         "family": {0: "cuda_core", 1: "tensor_core"}.get(v.get("family"))}
         row["scheduler_pick"] = "row" if row["row"]["us"] <= row["col"]["us"] else "col"
         sweep.append(row)
     out["batch_sweep"] = sweep
+    del x64, col, row_w, flush
+    torch.cuda.empty_cache()
+    out["decode_stack"] = decode_stack_measure(args.stack_steps)
     return out
+
+
+def decode_stack_measure(steps, layers=32, B=4):
+    """Long-generation decode: a 32-layer stack of Llama-3-8B-shaped MLPs
+    (11.3 GB of distinct weights, seed 4), B = 4, one step per CUDA-graph
+    replay, fused vs unfused kernels."""
+    import torch
+    from swiglu_mlp_dfk_b200 import inputs as I
+    from swiglu_mlp_dfk_b200.stack import DecodeStack
+
+    peak, _ = measured_peaks()
+    x0, params = I.make_stack(layers, B, D, F, seed=4, w_std=0.02, device="cuda")
+    res = {"layers": layers, "B": B, "steps": steps,
+           "weights_GB": round(sum(t.numel() * 2 for p in params for t in p) / 1e9, 2)}
+    for fused in (True, False):
+        st = DecodeStack(params, x0, fused=fused)
+        st.step_eager()                      # scheduler decisions outside capture
+        torch.cuda.synchronize()
+        st.capture()
+        for _ in range(3):
+            st.step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            st.step()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        key = "fused" if fused else "unfused"
+        res[key + "_ms_per_step"] = round(ms, 4)
+        res[key + "_kernels_per_step"] = st.kernels_per_step()
+        if fused:
+            gbs = st.bytes_per_step() / (ms * 1e-3) / 1e9
+            res["fused_GBps"] = round(gbs, 1)
+            res["fused_frac_of_peak"] = round(gbs / peak, 4)
+            res["roofline_ms_per_step"] = round(st.bytes_per_step() / (peak * 1e9) * 1e3, 4)
+        st.release()
+        del st
+    res["fused_speedup"] = round(res["unfused_ms_per_step"] / res["fused_ms_per_step"], 3)
+    del params, x0
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -550,7 +598,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["dfk", "reference"], default="dfk")
     ap.add_argument("--quick", action="store_true",
-                    help="skip the sweep / unfused / interleaved measurements")
+                    help="skip the sweep / unfused / interleaved / decode-stack measurements")
+    ap.add_argument("--stack-steps", type=int, default=512,
+                    help="decode steps of the 32-layer stack measurement")
     ap.add_argument("--profile", choices=["gate_up", "down"], default=None,
                     help="run only this kernel (inside an NVTX range) for ncu")
     ap.add_argument("--batch", type=int, default=1, help="batch for --profile")

@@ -150,10 +150,20 @@ DFK_API int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int
  * Returns DFK_ERR_INVALID_ARG if the stream is being captured.
  * Environment: DFK_TUNE=0 disables timing (heuristic choice),
  * DFK_TUNE_REPS (default 7) sets the timed repetitions, DFK_LOG=1 logs
- * decisions to stderr.
+ * decisions to stderr, DFK_TUNE_CACHE=<file> persists timed decisions (a
+ * text file keyed by device name, SM count and driver version; loaded on
+ * first use, appended to after each new decision; lines that do not parse
+ * are skipped with a warning on stderr), DFK_FAULT=tune makes timing fail
+ * (the heuristic is used: a host-side fault injection for tests).
  */
 DFK_API int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
                        const void *const *sample_ptrs, void *stream, dfk_variant *out);
+
+/* The scheduler's cached choice for (op, B, d_model, d_ff, layout) on the
+ * current device: DFK_OK with *out filled, or DFK_ERR_NO_VARIANT when no
+ * decision is cached yet (no call of that shape has been made). */
+DFK_API int dfk_cached_variant(int op, int B, int d_model, int d_ff, int layout,
+                               dfk_variant *out);
 
 /* Number of variant ids (valid ids are 1..count) and their description. */
 DFK_API int dfk_variant_count(void);

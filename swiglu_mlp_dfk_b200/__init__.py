@@ -49,7 +49,7 @@ _LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W
 # Every symbol the header declares (the CPU test checks the library exports them all).
 EXPORTED = (
     "dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj", "dfk_select_variant",
-    "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
+    "dfk_cached_variant", "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
     "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
 )
@@ -96,6 +96,7 @@ def lib():
                 "dfk_down_proj": [vp, vp, vp, i, i, i, i, vp],
                 "dfk_select_variant": [i, i, i, i, i, ctypes.POINTER(vp), vp,
                                        ctypes.POINTER(dfk_variant)],
+                "dfk_cached_variant": [i, i, i, i, i, ctypes.POINTER(dfk_variant)],
                 "dfk_variant_count": [],
                 "dfk_variant_info": [i, ctypes.POINTER(dfk_variant)],
                 "dfk_rmsnorm": [vp, vp, f, vp, i, i, vp],
@@ -285,6 +286,17 @@ def dfk_select_variant(op, B, d_model, d_ff, layout=DFK_W_ROW_MAJOR, sample=None
                                                 for t in sample])
     _check(lib().dfk_select_variant(int(op), int(B), int(d_model), int(d_ff), layout, arr,
                                     _stream(stream), ctypes.byref(out)))
+    return out.as_dict()
+
+
+def dfk_cached_variant(op, B, d_model, d_ff, layout=DFK_W_ROW_MAJOR):
+    """The scheduler's cached decision for the shape (dict), or None if none yet."""
+    out = dfk_variant()
+    st = lib().dfk_cached_variant(int(op), int(B), int(d_model), int(d_ff), _layout(layout),
+                                  ctypes.byref(out))
+    if st == DFK_ERR_NO_VARIANT:
+        return None
+    _check(st)
     return out.as_dict()
 
 

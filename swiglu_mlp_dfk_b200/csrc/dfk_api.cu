@@ -614,6 +614,79 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->measured_us = us;
 }
 
+// ---- persistent decisions: $DFK_TUNE_CACHE, one text line per decision
+//   dfk-tune 1 <device name> <SMs> <driver> <op> <B> <d_model> <d_ff> <layout> <variant> <us>
+// (spaces in the device name replaced by '_').  Lines for another device or
+// driver, malformed lines and unknown variant ids are skipped with a warning.
+
+static std::map<int, bool> g_cache_loaded;  // per device
+
+static std::string device_tag(int dev, int sms) {
+  cudaDeviceProp prop;
+  std::string name = "unknown";
+  if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess) name = prop.name;
+  else cudaGetLastError();
+  for (char &ch : name)
+    if (ch == ' ') ch = '_';
+  int drv = 0;
+  cudaDriverGetVersion(&drv);
+  return name + " " + std::to_string(sms) + " " + std::to_string(drv);
+}
+
+static void tune_cache_load(int dev, int sms) {  // caller holds g_tune_mu
+  if (g_cache_loaded[dev]) return;
+  g_cache_loaded[dev] = true;
+  const char *path = getenv("DFK_TUNE_CACHE");
+  if (!path || !*path) return;
+  FILE *f = fopen(path, "r");
+  if (!f) return;
+  const std::string tag = device_tag(dev, sms);
+  char line[512];
+  int lineno = 0, bad = 0, used = 0;
+  while (fgets(line, sizeof line, f)) {
+    ++lineno;
+    char magic[16], name[256];
+    int ver, n_sms, drv, op, B, D, F, layout, vid;
+    float us;
+    if (sscanf(line, "%15s %d %255s %d %d %d %d %d %d %d %d %f", magic, &ver, name, &n_sms, &drv,
+               &op, &B, &D, &F, &layout, &vid, &us) != 12 ||
+        strcmp(magic, "dfk-tune") != 0 || ver != 1) {
+      ++bad;
+      continue;
+    }
+    if (std::string(name) + " " + std::to_string(n_sms) + " " + std::to_string(drv) != tag)
+      continue;
+    const VDef *d = find_variant(vid);
+    if (!d || d->cls != op_class(op) || B < 1 || B > 64) {
+      ++bad;
+      continue;
+    }
+    dfk_variant rec;
+    fill_variant(*d, op, layout, 0, us, &rec);
+    g_tuned[TuneKey{dev, op, B, D, F, layout}] = rec;
+    ++used;
+  }
+  fclose(f);
+  if (bad)
+    fprintf(stderr, "[dfk] warning: %s: skipped %d malformed line(s) of %d\n", path, bad,
+            lineno);
+  log_msg("tune cache %s: %d decision(s) loaded", path, used);
+}
+
+static void tune_cache_append(int dev, int sms, const TuneKey &k, const dfk_variant &v) {
+  const char *path = getenv("DFK_TUNE_CACHE");
+  if (!path || !*path) return;
+  FILE *f = fopen(path, "a");
+  if (!f) {
+    log_msg("cannot append to tune cache %s", path);
+    return;
+  }
+  fprintf(f, "dfk-tune 1 %s %d %d %d %d %d %d %.3f\n", device_tag(dev, sms).c_str(), k.op, k.B,
+          k.D, k.F, k.layout, v.variant_id, v.measured_us);
+  fclose(f);
+}
+
+
 // Candidates worth timing for (op, B): every CUDA-core j-per-thread / k-split
 // / tiles-per-stage choice at its largest useful token tile, plus the
 // tensor-core variants from B = 8 up (below that, fp32 FMA on CUDA cores
@@ -764,6 +837,7 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
               c.layout};
   {
     std::lock_guard<std::mutex> lk(g_tune_mu);
+    tune_cache_load(dev, ds->sms);
     auto it = g_tuned.find(key);
     if (it != g_tuned.end()) {
       *out = find_variant(it->second.variant_id);
@@ -786,6 +860,7 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
     fill_variant(*win, op, c.layout, stages, us, &rec);
     std::lock_guard<std::mutex> lk(g_tune_mu);
     g_tuned[key] = rec;
+    if (us >= 0) tune_cache_append(dev, ds->sms, key, rec);
   }
   log_msg("op %d B=%d D=%d F=%d layout %d -> variant %d (%s)", op, c.B, key.D, key.F, c.layout,
           win->id, us >= 0 ? "timed" : "heuristic");
@@ -996,7 +1071,9 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
     {
       TuneKey key{dev, op, B, d_model, d_ff, L};
       std::lock_guard<std::mutex> lk(g_tune_mu);
+      tune_cache_load(dev, ds->sms);
       g_tuned[key] = rec;
+      if (us >= 0) tune_cache_append(dev, ds->sms, key, rec);
     }
     if (!best_set || (us >= 0 && (best.measured_us < 0 || us < best.measured_us))) {
       best = rec;
@@ -1005,6 +1082,21 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
   }
   if (!best_set) return fail(DFK_ERR_NO_VARIANT, "no variant fits this shape");
   *out = best;
+  return DFK_OK;
+}
+
+int dfk_cached_variant(int op, int B, int d_model, int d_ff, int layout, dfk_variant *out) {
+  if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  TuneKey key{dev, op, B, d_model, d_ff, layout};
+  std::lock_guard<std::mutex> lk(g_tune_mu);
+  tune_cache_load(dev, ds->sms);
+  auto it = g_tuned.find(key);
+  if (it == g_tuned.end()) return fail(DFK_ERR_NO_VARIANT, "no cached decision for this shape");
+  *out = it->second;
   return DFK_OK;
 }
 

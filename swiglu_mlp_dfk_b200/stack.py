@@ -1,0 +1,98 @@
+"""Multi-layer decode loop over the library's kernels, captured in a CUDA graph.
+
+Each decode step runs, for every layer l, the fused RMSNorm + gate/up +
+SiLU * up kernel and then the separate down projection, feeding layer l's
+output y to layer l + 1 (no residual: each layer's RMSNorm prologue keeps the
+activations in range); after the last layer the step's output is rescaled
+per row, x_{t+1} = y_t / sqrt(mean(y_t^2) + eps), and fed back.  This is the
+long-generation setting of "Deep Kernel Fusion for Transformers" (abstract:
+consistent speed-ups over generation lengths), as a stack of SwiGLU MLP
+layers only.
+
+The unfused variant runs the same step with separate kernels (RMSNorm, two
+GEMVs, SiLU, multiply, down projection) and bf16 intermediates in HBM.
+
+Everything launched here is a libdfk kernel; torch provides the buffers, the
+stream and the CUDA graph.
+"""
+import torch
+
+import swiglu_mlp_dfk_b200 as dfk
+
+
+class DecodeStack:
+    """A stack of SwiGLU MLP layers driven one decode step at a time.
+
+    layers: list of (gamma [D], W_gate [F, D], W_up [F, D], W_down [D, F]) bf16
+    x0:     [B, D] bf16 first-step input
+    """
+
+    def __init__(self, layers, x0, eps=1e-5, fused=True):
+        self.layers = layers
+        self.eps = float(eps)
+        self.fused = fused
+        self.B, self.D = x0.shape
+        self.F = layers[0][1].shape[0]
+        dev = x0.device
+        self.x = x0.clone()                       # step input (graph-static buffer)
+        self.acts = [torch.empty(self.B, self.D, dtype=torch.bfloat16, device=dev)
+                     for _ in range(2)]          # ping-pong layer outputs
+        self.h = torch.empty(self.B, self.F, dtype=torch.bfloat16, device=dev)
+        if not fused:
+            self.xn = torch.empty(self.B, self.D, dtype=torch.bfloat16, device=dev)
+            self.a = torch.empty_like(self.h)
+            self.u = torch.empty_like(self.h)
+            self.s = torch.empty_like(self.h)
+        self.graph = None
+        self.trace = None                        # optional: {(step, layer): tensor}
+
+    def layer_input(self, l):
+        return self.x if l == 0 else self.acts[(l - 1) % 2]
+
+    def _layer(self, l):
+        gamma, wg, wu, wd = self.layers[l]
+        xin = self.layer_input(l)
+        y = self.acts[l % 2]
+        if self.fused:
+            dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, "row", h=self.h)
+        else:
+            dfk.dfk_rmsnorm(xin, gamma, self.eps, out=self.xn)
+            dfk.dfk_gemv(self.xn, wg, out=self.a)
+            dfk.dfk_gemv(self.xn, wu, out=self.u)
+            dfk.dfk_silu(self.a, out=self.s)
+            dfk.dfk_mul(self.s, self.u, out=self.h)
+        dfk.dfk_down_proj(self.h, wd, y=y)
+
+    def step_eager(self):
+        """One decode step, launched kernel by kernel on the current stream."""
+        for l in range(len(self.layers)):
+            self._layer(l)
+        dfk.dfk_rms_rescale(self.acts[(len(self.layers) - 1) % 2], self.eps, out=self.x)
+
+    def capture(self):
+        """Capture one step in a CUDA graph (call after a warm-up step, so the
+        scheduler's decisions are cached and nothing is timed during capture)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step_eager()
+        self.graph = g
+        return g
+
+    def step(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.step_eager()
+
+    def release(self):
+        self.graph = None
+
+    def kernels_per_step(self):
+        return len(self.layers) * (2 if self.fused else 6) + 1
+
+    def bytes_per_step(self):
+        """Algorithmic bytes of one step: every weight once, activations in/out."""
+        B, D, F = self.B, self.D, self.F
+        per_layer = (2 * F * D * 2 + B * D * 2 + D * 2 + B * F * 2      # fused gate/up
+                     + D * F * 2 + B * F * 2 + B * D * 2)               # down projection
+        return len(self.layers) * per_layer + 2 * B * D * 2             # + rescale
