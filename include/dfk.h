@@ -90,6 +90,7 @@ typedef struct dfk_variant {
   int k_split;      /* thread teams splitting the reduction dimension               */
   int k_tiles_per_stage; /* consecutive 64-wide reduction tiles per ring stage       */
   int acc_banks;    /* tensor core: independent TMEM accumulators per output        */
+  int paired_fma;   /* CUDA core: 1 = FMAs issued two at a time (fma.rn.f32x2)      */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
 } dfk_variant;

@@ -78,11 +78,16 @@ struct CcAcc {
   float v[NMAT][JPT][BT];
 };
 
-template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NORM>
+// PAIR: issue the FMAs two at a time with fma.rn.f32x2 -- the gate and up
+// accumulators of one row (NMAT = 2) or two adjacent rows (NMAT = 1) share a
+// packed register, the activation is broadcast into both lanes.  Each lane
+// performs the same fma sequence as the scalar path: results are identical.
+template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NORM, bool PAIR>
 __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     cc_gemv_kernel(const __grid_constant__ CcMaps maps, const CcParams p) {
   static_assert(LAYOUT != LAYOUT_IL || NMAT == 2, "interleaved layout holds both matrices");
   static_assert(XF32 || !NORM, "normalised activations are kept in fp32");
+  constexpr int NPAIR = PAIR ? (NMAT == 2 ? JPT : JPT / 2) : 1;
   static_assert(JPT == 2 || JPT == 4, "JPT");
   extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -280,6 +285,11 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
         for (int jj = 0; jj < JPT; ++jj)
 #pragma unroll
           for (int bb = 0; bb < BT; ++bb) acc.v[m][jj][bb] = 0.f;
+      uint64_t acc2[NPAIR][BT];  // PAIR only: packed accumulators, +0 in both lanes
+#pragma unroll
+      for (int pr = 0; pr < NPAIR; ++pr)
+#pragma unroll
+        for (int bb = 0; bb < BT; ++bb) acc2[pr][bb] = 0ull;
 
       for (int step = 0; step < p.nsteps; ++step) {
         const int i = pass * p.nsteps + step;
@@ -322,6 +332,26 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
                     *reinterpret_cast<const uint4 *>(bse + row * rowb + tt * (TILE_K * 2) + s * 16);
                 wv[m][jj][0] = v.x; wv[m][jj][1] = v.y; wv[m][jj][2] = v.z; wv[m][jj][3] = v.w;
               }
+            if constexpr (PAIR) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                uint64_t xd[BT];
+#pragma unroll
+                for (int bb = 0; bb < BT; ++bb) xd[bb] = pack_f32x2(xv[bb][e], xv[bb][e]);
+#pragma unroll
+                for (int pr = 0; pr < NPAIR; ++pr) {
+                  // NMAT = 2: (gate, up) of row pr; NMAT = 1: rows (2 pr, 2 pr + 1)
+                  const int m1 = NMAT - 1, j0r = (NMAT == 2) ? pr : 2 * pr;
+                  const int j1r = (NMAT == 2) ? pr : 2 * pr + 1;
+                  const uint32_t w0 = wv[0][j0r][e >> 1], w1 = wv[m1][j1r][e >> 1];
+                  const uint64_t wp = (e & 1) ? pack_f32x2(bf16_hi(w0), bf16_hi(w1))
+                                              : pack_f32x2(bf16_lo(w0), bf16_lo(w1));
+#pragma unroll
+                  for (int bb = 0; bb < BT; ++bb)
+                    acc2[pr][bb] = fma_f32x2(xd[bb], wp, acc2[pr][bb]);
+                }
+              }
+            } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
 #pragma unroll
@@ -334,36 +364,69 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
                   for (int bb = 0; bb < BT; ++bb)
                     acc.v[m][jj][bb] = fmaf(xv[bb][e], wf, acc.v[m][jj][bb]);
                 }
+            }
           } else {
             // column-major tile [64 k][r j]: thread reads JPT consecutive j per k row
             const int pitch = r * 2;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int krow = tt * TILE_K + 8 * s + e;
+              uint32_t w[NMAT][JPT / 2];
 #pragma unroll
               for (int m = 0; m < NMAT; ++m) {
                 const uint8_t *src = tb + m * slot_bytes + krow * pitch + jl0 * 2;
-                uint32_t w[JPT / 2];
                 if constexpr (JPT == 4) {
                   const uint2 v = *reinterpret_cast<const uint2 *>(src);
-                  w[0] = v.x;
-                  w[1] = v.y;
+                  w[m][0] = v.x;
+                  w[m][1] = v.y;
                 } else {
-                  w[0] = *reinterpret_cast<const uint32_t *>(src);
+                  w[m][0] = *reinterpret_cast<const uint32_t *>(src);
                 }
+              }
+              if constexpr (PAIR) {
+                uint64_t xd[BT];
 #pragma unroll
-                for (int jj = 0; jj < JPT; ++jj) {
-                  const float wf = (jj & 1) ? bf16_hi(w[jj >> 1]) : bf16_lo(w[jj >> 1]);
+                for (int bb = 0; bb < BT; ++bb) xd[bb] = pack_f32x2(xv[bb][e], xv[bb][e]);
+#pragma unroll
+                for (int pr = 0; pr < NPAIR; ++pr) {
+                  const int m1 = NMAT - 1, j0r = (NMAT == 2) ? pr : 2 * pr;
+                  const int j1r = (NMAT == 2) ? pr : 2 * pr + 1;
+                  const float f0 = (j0r & 1) ? bf16_hi(w[0][j0r >> 1]) : bf16_lo(w[0][j0r >> 1]);
+                  const float f1 = (j1r & 1) ? bf16_hi(w[m1][j1r >> 1]) : bf16_lo(w[m1][j1r >> 1]);
+                  const uint64_t wp = pack_f32x2(f0, f1);
 #pragma unroll
                   for (int bb = 0; bb < BT; ++bb)
-                    acc.v[m][jj][bb] = fmaf(xv[bb][e], wf, acc.v[m][jj][bb]);
+                    acc2[pr][bb] = fma_f32x2(xd[bb], wp, acc2[pr][bb]);
                 }
+              } else {
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                  for (int jj = 0; jj < JPT; ++jj) {
+                    const float wf =
+                        (jj & 1) ? bf16_hi(w[m][jj >> 1]) : bf16_lo(w[m][jj >> 1]);
+#pragma unroll
+                    for (int bb = 0; bb < BT; ++bb)
+                      acc.v[m][jj][bb] = fmaf(xv[bb][e], wf, acc.v[m][jj][bb]);
+                  }
               }
             }
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
+      }
+
+      if constexpr (PAIR) {
+#pragma unroll
+        for (int pr = 0; pr < NPAIR; ++pr)
+#pragma unroll
+          for (int bb = 0; bb < BT; ++bb) {
+            if constexpr (NMAT == 2)
+              unpack_f32x2(acc2[pr][bb], acc.v[0][pr][bb], acc.v[NMAT - 1][pr][bb]);
+            else
+              unpack_f32x2(acc2[pr][bb], acc.v[0][2 * pr][bb], acc.v[0][2 * pr + 1][bb]);
+          }
       }
 
       // ---- reduce over the 8 slots, fold the K teams, SwiGLU epilogue

@@ -5,10 +5,13 @@
 #include "cc_engine.cuh"
 #include "cc_key.h"
 
-#define DFK_CC_CASE(L, NM, J, BT, KS, XF, NO)                    \
-  case DFK_CC_KEY(L, NM, J, BT, KS, XF, NO):                     \
-    return reinterpret_cast<const void *>(                       \
-        &dfk::cc_gemv_kernel<L, NM, J, BT, KS, (XF) != 0, (NO) != 0>);
+#define DFK_CC_CASE(L, NM, J, BT, KS, XF, NO)                                   \
+  case DFK_CC_KEY(L, NM, J, BT, KS, XF, NO, 0):                                 \
+    return reinterpret_cast<const void *>(                                      \
+        &dfk::cc_gemv_kernel<L, NM, J, BT, KS, (XF) != 0, (NO) != 0, false>);    \
+  case DFK_CC_KEY(L, NM, J, BT, KS, XF, NO, 1):                                 \
+    return reinterpret_cast<const void *>(                                      \
+        &dfk::cc_gemv_kernel<L, NM, J, BT, KS, (XF) != 0, (NO) != 0, true>);
 
 // every (j_per_thread, token_tile) pair compiled
 #define DFK_CC_JB(L, NM, KS, XF, NO)                                                 \

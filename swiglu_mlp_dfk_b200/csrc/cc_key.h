@@ -2,10 +2,10 @@
 #pragma once
 
 // layout (2 bits) | matrices (2) | j per thread (4) | token tile (4) |
-// k split (4) | fp32 activations (1) | RMSNorm prologue (1)
-#define DFK_CC_KEY(L, NM, J, BT, KS, XF, NO)                                     \
+// k split (4) | fp32 activations (1) | RMSNorm prologue (1) | paired FMA (1)
+#define DFK_CC_KEY(L, NM, J, BT, KS, XF, NO, PR)                                 \
   ((L) | ((NM) << 2) | ((J) << 4) | ((BT) << 8) | ((KS) << 12) | ((XF) << 16) | \
-   ((NO) << 17))
+   ((NO) << 17) | ((PR) << 18))
 
 namespace dfk {
 // Pointer to the __global__ function for a key, or nullptr if not compiled.

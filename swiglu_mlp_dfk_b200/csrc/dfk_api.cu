@@ -225,6 +225,7 @@ struct VDef {
   int family;
   int jpt, bt, ksplit, nt;
   int nbank;  // tensor core: independent TMEM accumulator banks per output
+  int pair;   // CUDA core: FMAs issued in pairs (fma.rn.f32x2)
 };
 
 static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
@@ -233,20 +234,22 @@ static const std::vector<VDef> &variants() {
   static std::vector<VDef> v = [] {
     std::vector<VDef> t;
     int id = 1;
-    for (int nt : {1, 2, 4})
-      for (auto &jb : kJB)
-        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt, 1});
-    for (int nt : {1, 2, 4})
-      for (int ks : {1, 2, 4, 8})
+    for (int pr : {0, 1})
+      for (int nt : {1, 2, 4})
         for (auto &jb : kJB)
-          t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt, 1});
+          t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt, 1, pr});
+    for (int pr : {0, 1})
+      for (int nt : {1, 2, 4})
+        for (int ks : {1, 2, 4, 8})
+          for (auto &jb : kJB)
+            t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt, 1, pr});
     // tensor-core family: token tile chosen from B at launch (16 / 32 / 64)
     for (int nb : {1, 2})
       for (int nt : {1, 2})
-        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb});
+        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb, 0});
     for (int nb : {1, 2})
       for (int nt : {1, 2, 4, 8})
-        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb});
+        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb, 0});
     return t;
   }();
   return v;
@@ -321,7 +324,7 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       continue;
     }
     const int key = DFK_CC_KEY(layout, nmat, v.jpt, v.bt, v.ksplit, best_xf32 ? 1 : 0,
-                               norm ? 1 : 0);
+                               norm ? 1 : 0, v.pair ? 1 : 0);
     const void *fn = cc_find_kernel(key);
     if (!fn) {
       if (why) *why = "variant not compiled for this layout";
@@ -610,6 +613,7 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->k_split = d.ksplit;
   out->k_tiles_per_stage = d.nt;
   out->acc_banks = d.nbank;
+  out->paired_fma = d.pair;
   out->stages = stages;
   out->measured_us = us;
 }
