@@ -247,9 +247,10 @@ static const std::vector<VDef> &variants() {
     for (int nb : {1, 2})
       for (int nt : {1, 2})
         t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb, 0});
-    for (int nb : {1, 2})
+    // GEMV: k-split = reduction slices across CTAs (split-K with a workspace)
+    for (int ks : {1, 2, 4})
       for (int nt : {1, 2, 4, 8})
-        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb, 0});
+        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, nt, 1, 0});
     return t;
   }();
   return v;
@@ -470,11 +471,20 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
   const int bn = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
   const int cap = std::min(ds.smem_optin, 232448);
   const int nt = v.nt;
+  const int kslices = (nmat == 1) ? std::max(1, v.ksplit) : 1;
+  const int ntiles = ceil_div(K, TC_TILE_K);
+  if (kslices > 1 && (nmat != 1 || ntiles < kslices)) {
+    if (why) *why = "split-K needs a single matrix and at least one k-tile per slice";
+    return false;
+  }
   for (int mult = 1; mult <= 8; mult *= 2) {
-    const int P = std::min(N, ds.sms * mult);
-    const int rbase = N / P, rextra = N % P;
+    // row blocks: one per CTA, or (split-K) one per kslices CTAs
+    const int nblocks = kslices > 1 ? std::min(N, ds.sms / kslices) : std::min(N, ds.sms * mult);
+    if (nblocks < 1) break;
+    const int P = nblocks * kslices;
+    const int rbase = N / nblocks, rextra = N % nblocks;
     const int r_hi = rbase + (rextra ? 1 : 0);
-    for (int mt = 1; mt <= 2; ++mt) {
+    for (int mt = 1; mt <= (kslices > 1 ? 1 : 2); ++mt) {
       if (r_hi > 128 * mt) continue;
       if (mt == 2 && rbase < 2) continue;
       const int hmax = (r_hi + mt - 1) / mt;
@@ -484,8 +494,8 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       const int x_bytes = nt * xt_bytes;
       const int stage = a_bytes + x_bytes;
       const int slack = std::max(0, 16384 - rc * 128 - x_bytes);
-      const int nsteps = ceil_div(K, TC_TILE_K * nt);
-      const int kpad = nsteps * nt * TC_TILE_K;
+      const int nsteps = ceil_div(ceil_div(ntiles, kslices), nt);
+      const int kpad = ceil_div(ntiles, nt) * nt * TC_TILE_K;
       const int g_bytes = norm ? round_up(kpad * 2, 1024) : 0;
       const int fixed = 1024 /* alignment */ + slack + g_bytes + 1024 /* barriers */;
       const int S = std::min(8, (cap - fixed) / stage);
@@ -524,12 +534,63 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       p.nbank = nbank;
       p.g_off = S * stage + slack;
       p.bar_off = p.g_off + g_bytes;
+      p.ntiles = ntiles;
+      p.kslices = kslices;
+      p.nblocks = nblocks;
       pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
       return true;
     }
+    if (kslices > 1) break;  // the split partition does not depend on `mult`
   }
   if (why) *why = "no tensor-core partition fits shared memory";
   return false;
+}
+
+// ---- split-K workspace: one per (device, stream), grown on demand outside
+// stream capture; the counter region is zeroed when allocated and every
+// kernel leaves its counters at 0.
+struct Workspace {
+  void *base = nullptr;
+  size_t bytes = 0;
+};
+static std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+static bool stream_capturing(cudaStream_t s);
+
+static int get_workspace(int dev, cudaStream_t s, size_t part_bytes, size_t counter_bytes,
+                         float **part, unsigned **counters) {
+  const size_t part_round = (part_bytes + 255) & ~static_cast<size_t>(255);
+  const size_t need = part_round + counter_bytes;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace &w = g_ws[std::make_pair(dev, s)];
+  if (w.bytes < need) {
+    if (stream_capturing(s))
+      return fail(DFK_ERR_NO_VARIANT, "split-K workspace must be allocated before capture "
+                  "(make one call of this shape on the stream first)");
+    if (w.base) {
+      cudaStreamSynchronize(s);
+      cudaFree(w.base);
+      w.base = nullptr;
+      w.bytes = 0;
+    }
+    const size_t grow = std::max(need, static_cast<size_t>(8) << 20);
+    cudaError_t e = cudaMalloc(&w.base, grow);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "cudaMalloc (split-K workspace)");
+    }
+    e = cudaMemsetAsync(w.base, 0, grow, s);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "zeroing the split-K workspace");
+    }
+    w.bytes = grow;
+  }
+  // counters at the end of the buffer: stable across shapes
+  *part = static_cast<float *>(w.base);
+  *counters = reinterpret_cast<unsigned *>(static_cast<char *>(w.base) + w.bytes - counter_bytes);
+  if (part_round > w.bytes - counter_bytes) return fail(DFK_ERR_CUDA, "workspace layout");
+  return DFK_OK;
 }
 
 static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
@@ -572,6 +633,13 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   p.gamma = static_cast<const uint16_t *>(c.gamma);
   p.err = ds->err;
   p.eps = c.eps;
+  if (p.kslices > 1) {
+    const size_t part_bytes =
+        static_cast<size_t>(p.kslices) * p.nblocks * p.bn * 128 * sizeof(float);
+    // counters: a fixed region sized for the largest partition (one per SM)
+    const size_t counter_bytes = static_cast<size_t>(ds->sms) * 8 * sizeof(unsigned);
+    if ((rc = get_workspace(dev, s, part_bytes, counter_bytes, &p.part, &p.counters))) return rc;
+  }
   void *args[] = {&maps, &p};
   cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TC_THREADS), pl.smem, s,
                                 pdl_enabled(), args);
@@ -692,15 +760,17 @@ static void tune_cache_append(int dev, int sms, const TuneKey &k, const dfk_vari
 
 
 // Candidates worth timing for (op, B): every CUDA-core j-per-thread / k-split
-// / tiles-per-stage choice at its largest useful token tile, plus the
-// tensor-core variants from B = 8 up (below that, fp32 FMA on CUDA cores
-// keeps up with HBM and the contraction is too thin for the MMA).
+// / tiles-per-stage / pairing choice at its largest useful token tile, plus the
+// tensor-core variants from B = 4 (gate/up) or B = 2 (GEMV); at B = 1 fp32
+// FMA on CUDA cores keeps up with HBM.
 static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
   std::vector<const VDef *> out;
   for (const VDef &d : variants()) {
     if (d.cls != op_class(op)) continue;
     if (d.family == DFK_FAMILY_TENSOR_CORE) {
-      if (B >= 8 && c.layout != LAYOUT_COL) out.push_back(&d);
+      // gate/up from B = 4 (where CUDA cores fall below HBM speed), the GEMV
+      // (split-K) from B = 2
+      if (B >= (d.cls == CLS_GEMV ? 2 : 4) && c.layout != LAYOUT_COL) out.push_back(&d);
       continue;
     }
     if (d.bt != bt_for(B, d.jpt)) continue;
@@ -725,10 +795,11 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
   if (B >= 8 && c.layout != LAYOUT_COL) {
-    const int want_nt = op_class(op) == CLS_GEMV ? 4 : 1;
+    const bool gemv = op_class(op) == CLS_GEMV;
+    const int want_nt = gemv ? 2 : 1, want_ks = gemv ? 4 : 1;
     for (const VDef &d : variants())
       if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == want_nt &&
-          feasible(d, c, ds))
+          d.ksplit == want_ks && d.nbank == 1 && feasible(d, c, ds))
         return &d;
   }
   const int jpt = B <= 4 ? 4 : 2;

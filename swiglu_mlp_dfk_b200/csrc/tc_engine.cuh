@@ -62,6 +62,15 @@ struct TcParams {
   int tmem_cols;
   int nbank;              // independent TMEM accumulators per output (1, 2 or 4)
   int g_off, bar_off;     // shared-memory offsets from the 1024-byte aligned base
+  // split-K (single-matrix GEMV only): CTA c handles row block c / kslices and
+  // reduction slice c % kslices; partial sums go to `part`, the last CTA to
+  // arrive on a row block (counter) adds the slices in order 0, 1, ... and
+  // stores the output, then resets the counter to 0.
+  int ntiles;             // 64-wide k-tiles covering K
+  int kslices;            // 1 = no split
+  float *part;            // [kslices][row blocks][bn][128] fp32
+  unsigned *counters;     // [row blocks], 0 between calls
+  int nblocks;            // row blocks (split-K)
 };
 
 // wg/wu: [0] box height hmax, [1] box height hmax - 1; x: activations box {64, bn}.
@@ -135,13 +144,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
   int *s_issued = reinterpret_cast<int *>(accfull + 1) + 1;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accfull + 1) + 2;
+  volatile int *s_last = reinterpret_cast<volatile int *>(accfull + 1) + 3;
   float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(accfull + 1) + 16);
   uint16_t *gs = reinterpret_cast<uint16_t *>(smem + p.g_off);
 
-  // ---- this CTA's rows [j0, j0 + r), cut into MT sub-tiles
+  // ---- this CTA's rows [j0, j0 + r), cut into MT sub-tiles, and its
+  // reduction range: k-tiles [tile0, tile1)
   const int cta = blockIdx.x;
-  const int j0 = cta * p.rbase + min(cta, p.rextra);
-  const int r = p.rbase + (cta < p.rextra ? 1 : 0);
+  const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
+  const int j0 = blk * p.rbase + min(blk, p.rextra);
+  const int r = p.rbase + (blk < p.rextra ? 1 : 0);
+  const int tile0 = (slc * p.ntiles) / p.kslices;
+  const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
+  const int nsteps = (tile1 - tile0 + NT - 1) / NT;
   int h[MT], rs[MT];
   h[0] = (r + MT - 1) / MT;
   rs[0] = 0;
@@ -176,16 +191,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_normal();
-      const uint32_t tx = static_cast<uint32_t>(NT) * (NMAT * r + BN) * 128u;
-      const int S0 = min(S, p.nsteps);
+      const int S0 = min(S, nsteps);
       int issued = 0;
-      for (int i = 0; i < p.nsteps; ++i) {
+      for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
         if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
-        mbar_arrive_expect_tx(&full[st], tx);
-        for (int kt = 0; kt < NT; ++kt) {
-          const int k0 = (i * NT + kt) * TC_TILE_K;
+        const int nv = min(NT, tile1 - (tile0 + i * NT));  // k-tiles of this step in range
+        mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nv) * (NMAT * r + BN) * 128u);
+        for (int kt = 0; kt < nv; ++kt) {
+          const int k0 = (tile0 + i * NT + kt) * TC_TILE_K;
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
             const int mi = (h[t] == p.hmax) ? 0 : 1;
@@ -205,11 +220,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (i == S0 - 1) {
           pdl_wait();
-          for (int ii = 0; ii < S0; ++ii)
-            for (int kt = 0; kt < NT; ++kt)
+          for (int ii = 0; ii < S0; ++ii) {
+            const int nvi = min(NT, tile1 - (tile0 + ii * NT));
+            for (int kt = 0; kt < nvi; ++kt)
               tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
                               kt * p.xt_bytes,
-                          &maps.x, &full[ii], (ii * NT + kt) * TC_TILE_K, 0, pol_x);
+                          &maps.x, &full[ii], (tile0 + ii * NT + kt) * TC_TILE_K, 0, pol_x);
+          }
         }
         issued = i + 1;
       }
@@ -231,13 +248,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t tile_enc = static_cast<uint32_t>(p.rc * 128) >> 4;
       const uint32_t x_enc = static_cast<uint32_t>(p.a_bytes) >> 4;
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
-      for (int i = 0; i < p.nsteps; ++i) {
+      for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
         if (!mbar_wait_bounded(NORM ? &xready[st] : &full[st], (i / S) & 1, s_abort, p.err))
           break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
-        for (int kt = 0; kt < NT; ++kt) {
+        const int nv = min(NT, tile1 - (tile0 + i * NT));
+        for (int kt = 0; kt < nv; ++kt) {
           const uint64_t bx = ds + x_enc + kt * xt_enc;
           const uint64_t at = ds + static_cast<uint64_t>(kt * MT * NMAT) * tile_enc;
 #pragma unroll
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int et = tid - 64;
     if (NORM) {
       pdl_wait();
-      const int kpad = p.nsteps * NT * TC_TILE_K;
+      const int kpad = ((p.ntiles + NT - 1) / NT) * NT * TC_TILE_K;
       for (int idx = et; idx < kpad / 8; idx += 128) {
         const int k = idx * 8;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -276,18 +294,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int n = et / tpr, part = et - n * tpr;
       const int cpt = 8 / tpr;        // 16-byte chunks per thread per k-tile
       float ss = 0.f;
-      for (int i = 0; i < p.nsteps; ++i) {
+      for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
         const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
         if (ok) {
           uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
-          for (int kt = 0; kt < NT; ++kt) {
+          const int nv = min(NT, tile1 - (tile0 + i * NT));
+          for (int kt = 0; kt < nv; ++kt) {
             uint8_t *xt = sb + p.a_bytes + kt * p.xt_bytes;
             uint8_t *lt = xt + BN * 128;
             for (int c = 0; c < cpt; ++c) {
               const int pc = part * cpt + c;          // physical 16-byte chunk of row n
               const int lc = pc ^ (n & 7);            // 128-byte swizzle: logical chunk
-              const int k = (i * NT + kt) * TC_TILE_K + 8 * lc;
+              const int k = (tile0 + i * NT + kt) * TC_TILE_K + 8 * lc;
               const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
               const uint4 gv = *reinterpret_cast<const uint4 *>(gs + k);
               const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -341,7 +360,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tmem_sum_banks(base + (t * NMAT) * NB * WN + c, NB, WN, NORM ? BN : 0, g);
           if (NMAT == 2)
             tmem_sum_banks(base + (t * NMAT + 1) * NB * WN + c, NB, WN, NORM ? BN : 0, u);
-          if (row < h[t]) {
+          if (p.kslices > 1) {
+            // split-K: this slice's partial sums, [n][row] so a warp's stores coalesce
+            float *mine = p.part + (static_cast<size_t>(slc) * p.nblocks + blk) * BN * 128;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) mine[(c + e) * 128 + row] = g[e];
+          } else if (row < h[t]) {
             const int j = j0 + rs[t] + row;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -360,6 +384,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         }
+      }
+    }
+    if (p.kslices > 1) {
+      // every CTA of the row block takes part in the count (also after an
+      // abort, so the counter stays consistent); the last one reduces
+      __threadfence();
+      named_barrier(2, 128);
+      if (et == 0) {
+        const unsigned old = atomicAdd(&p.counters[blk], 1u);
+        *s_last = (old == static_cast<unsigned>(p.kslices - 1)) ? 1 : 0;
+      }
+      named_barrier(2, 128);
+      if (*s_last) {
+        __threadfence();
+        if (row < r && !*s_abort) {
+          for (int n = 0; n < p.B; ++n) {
+            float acc = 0.f;
+            for (int sl = 0; sl < p.kslices; ++sl) {
+              const float v = __ldcg(p.part + ((static_cast<size_t>(sl) * p.nblocks + blk) * BN +
+                                               n) * 128 + row);
+              acc = (sl == 0) ? v : acc + v;
+            }
+            p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(acc);
+          }
+        }
+        named_barrier(2, 128);
+        if (et == 0) p.counters[blk] = 0u;
       }
     }
     tc_fence_before();

@@ -392,10 +392,17 @@ def test_tensor_core_down(B, D, F):
     h = (torch.randn(B, F, generator=g, device="cuda") * 0.5).to(torch.bfloat16)
     wd = (torch.randn(D, F, generator=g, device="cuda") * 0.03).to(torch.bfloat16)
     ref = oracle.down(I.to_bits(h), I.to_bits(wd))
+    ran = 0
     for vid in tc_variants(dfk.DFK_OP_DOWN):
-        y = dfk.dfk_down_proj(h, wd, variant=vid)
+        try:
+            y = dfk.dfk_down_proj(h, wd, variant=vid)
+        except dfk.DfkError as e:       # a variant that does not fit this shape
+            assert e.status == dfk.DFK_ERR_NO_VARIANT
+            continue
         torch.cuda.synchronize()
         assert_close(y, ref, "tc down variant %d" % vid)
+        ran += 1
+    assert ran >= 4
 
 
 def test_tensor_core_batch_rows_independent():
@@ -409,3 +416,34 @@ def test_tensor_core_batch_rows_independent():
     other = I.MLPInputs(x2, inp.gamma, inp.w_gate, inp.w_up, None)
     h2 = run_gate_up(other, I.LAYOUT_ROW, True, variant=vid)
     assert bits_equal(full[0], h2[0])
+
+
+def test_split_k_down_is_deterministic_and_resets():
+    # split-K tensor-core GEMV: two calls in a row give identical bits (the
+    # arrival counters are back at 0 after each call), also with a different
+    # shape in between using the same workspace
+    split = [i for i in tc_variants(dfk.DFK_OP_DOWN) if dfk.dfk_variant_info(i)["k_split"] > 1]
+    assert split
+    g = torch.Generator(device="cuda").manual_seed(77)
+    h = (torch.randn(12, 14336, generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    wd = (torch.randn(4096, 14336, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    h2 = (torch.randn(40, 2048, generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    wd2 = (torch.randn(1000, 2048, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    rows = sample_rows(4096, 256, 5)
+    ref = oracle.down(I.to_bits(h), I.to_bits(wd), rows=rows)
+    ref2 = oracle.down(I.to_bits(h2), I.to_bits(wd2))
+    ran = 0
+    for vid in split:
+        try:
+            y1 = dfk.dfk_down_proj(h, wd, variant=vid)
+            y_other = dfk.dfk_down_proj(h2, wd2, variant=vid)
+        except dfk.DfkError as e:
+            assert e.status == dfk.DFK_ERR_NO_VARIANT
+            continue
+        ran += 1
+        y2 = dfk.dfk_down_proj(h, wd, variant=vid)
+        torch.cuda.synchronize()
+        assert bits_equal(y1, y2), "variant %d not reproducible" % vid
+        assert_close(y1[:, rows], ref, "split-K variant %d" % vid)
+        assert_close(y_other, ref2, "split-K variant %d (second shape)" % vid)
+    assert ran >= 2
