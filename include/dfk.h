@@ -134,6 +134,25 @@ DFK_API int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int
                   int d_ff, int variant, void *stream);
 
 /*
+ * y = h . W_down^T without allocating device memory.  (No counterpart in the
+ * paper: this serves callers that cannot allocate while they run the MLP --
+ * a runtime that has reserved all device memory for its own pool, code that
+ * runs inside CUDA stream capture, where allocation calls are not allowed, or
+ * a host that lends the library a device it does not own.)
+ * Same arguments and result contract as dfk_down_proj; always the split-K
+ * tensor-core kernel in a fixed configuration (no scheduler timing).  Its
+ * partial sums live in a 6 MiB + 4 KiB array that is part of the library
+ * image: every device that loads the library holds it until the process
+ * exits.  The first call on a device looks up the array's device address
+ * (make that call before any stream capture).  All calls share the array:
+ * calls whose executions overlap on the GPU (different streams, or graphs
+ * replayed concurrently) race and give wrong results.  A shape whose
+ * partial sums exceed the array returns DFK_ERR_UNSUPPORTED_SHAPE.
+ */
+DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void *y, int B,
+                                         int d_model, int d_ff, void *stream);
+
+/*
  * Profiler-driven variant choice ("Deep Kernel Fusion for Transformer
  * Decoding", episode description: runtime scheduling across row-major and
  * column-major kernel variants; "Deep Kernel Fusion for Transformers",

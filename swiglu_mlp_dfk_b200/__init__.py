@@ -49,7 +49,7 @@ _LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W
 # Every symbol the header declares (the CPU test checks the library exports them all).
 EXPORTED = (
     "dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj", "dfk_select_variant",
-    "dfk_cached_variant", "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
+    "dfk_down_proj_static_scratch", "dfk_cached_variant", "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
     "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
 )
@@ -95,6 +95,7 @@ def lib():
                 "dfk_swiglu_gate_up": [vp, vp, vp, i, vp, i, i, i, i, vp],
                 "dfk_rmsnorm_swiglu_gate_up": [vp, vp, f, vp, vp, i, vp, i, i, i, i, vp],
                 "dfk_down_proj": [vp, vp, vp, i, i, i, i, vp],
+                "dfk_down_proj_static_scratch": [vp, vp, vp, i, i, i, vp],
                 "dfk_select_variant": [i, i, i, i, i, ctypes.POINTER(vp), vp,
                                        ctypes.POINTER(dfk_variant)],
                 "dfk_cached_variant": [i, i, i, i, i, ctypes.POINTER(dfk_variant)],
@@ -203,6 +204,22 @@ def dfk_down_proj(h, w_down, y=None, variant=0, stream=None):
         y = torch.empty((B, D), dtype=torch.bfloat16, device=h.device)
     _check(lib().dfk_down_proj(_ptr(h), _ptr(w_down), _ptr(y), B, D, F, int(variant),
                                _stream(stream)))
+    return y
+
+
+def dfk_down_proj_static_scratch(h, w_down, y=None, stream=None):
+    """y = h W_down^T without device allocation (library-resident scratch array).
+
+    For callers that cannot allocate while running the MLP (a pre-reserved
+    memory pool, stream capture); calls that overlap on the GPU race."""
+    for n, t in (("h", h), ("w_down", w_down), ("y", y)):
+        _dev_bf16(n, t)
+    B, F = h.shape
+    D = w_down.shape[0]
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=h.device)
+    _check(lib().dfk_down_proj_static_scratch(_ptr(h), _ptr(w_down), _ptr(y), B, D, F,
+                                              _stream(stream)))
     return y
 
 

@@ -651,6 +651,77 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   return DFK_OK;
 }
 
+static int check_gemv(const void *x, const void *w, const void *out, int B, int K, int N,
+                      int variant);
+
+// The split-K tensor-core down projection on caller-provided scratch: a
+// fixed configuration (no timing), no workspace of its own.  Used by the
+// entry point for callers that cannot allocate (noalloc.cu).
+int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, int d_model,
+                           int d_ff, float *part, size_t part_capacity, unsigned *counters,
+                           size_t counter_capacity, cudaStream_t s) {
+  int rc = check_gemv(h, w_down, y, B, d_ff, d_model, 0);
+  if (rc || B == 0) return rc;
+  DeviceState *ds;
+  int dev;
+  if ((rc = current_device(&ds, &dev))) return rc;
+  const CcCall c{LAYOUT_ROW, 1, false, h, nullptr, 0.f, w_down, nullptr, y, B, d_ff, d_model};
+  // preferred split configurations, most parallel first
+  static const int kPrefs[][2] = {{4, 2}, {4, 1}, {2, 2}, {2, 1}};
+  TcPlan pl;
+  bool found = false;
+  for (const auto &pref : kPrefs) {
+    for (const VDef &d : variants()) {
+      if (d.cls != CLS_GEMV || d.family != DFK_FAMILY_TENSOR_CORE || d.ksplit != pref[0] ||
+          d.nt != pref[1])
+        continue;
+      if (plan_tc(c.layout, 1, false, d, B, c.K, c.N, *ds, &pl, nullptr) && pl.p.kslices > 1) {
+        found = true;
+        break;
+      }
+    }
+    if (found) break;
+  }
+  if (!found)
+    return fail(DFK_ERR_NO_VARIANT, "no split-K configuration fits B=%d d_model=%d d_ff=%d", B,
+                d_model, d_ff);
+  const size_t part_bytes =
+      static_cast<size_t>(pl.p.kslices) * pl.p.nblocks * pl.p.bn * 128 * sizeof(float);
+  const size_t counter_bytes = static_cast<size_t>(pl.p.nblocks) * sizeof(unsigned);
+  if (part_bytes > part_capacity || counter_bytes > counter_capacity)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE,
+                "B=%d d_model=%d needs %zu bytes of partial sums and %zu of counters; the "
+                "static scratch holds %zu and %zu",
+                B, d_model, part_bytes, counter_bytes, part_capacity, counter_capacity);
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  TcMaps maps;
+  memset(&maps, 0, sizeof maps);
+  for (int lo = 0; lo < 2; ++lo) {
+    const uint32_t hgt = static_cast<uint32_t>(std::max(1, pl.p.hmax - lo));
+    if ((rc = tensor_map_2d(w_down, c.K, c.N, static_cast<uint64_t>(c.K) * 2, TC_TILE_K, hgt,
+                            &maps.wg[lo], true)))
+      return rc;
+  }
+  if ((rc = tensor_map_2d(h, c.K, c.B, static_cast<uint64_t>(c.K) * 2, TC_TILE_K, pl.p.bn,
+                          &maps.x, true)))
+    return rc;
+  TcParams p = pl.p;
+  p.out = static_cast<uint16_t *>(y);
+  p.gamma = nullptr;
+  p.err = ds->err;
+  p.eps = 0.f;
+  p.part = part;
+  p.counters = counters;
+  void *args[] = {&maps, &p};
+  cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TC_THREADS), pl.smem, s,
+                                pdl_enabled(), args);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "tensor-core kernel launch");
+  }
+  return DFK_OK;
+}
+
 static int launch_variant(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
   return v.family == DFK_FAMILY_TENSOR_CORE ? launch_tc(c, v, s, stages_used)
                                             : launch_cc(c, v, s, stages_used);
