@@ -638,7 +638,15 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
         static_cast<size_t>(p.kslices) * p.nblocks * p.bn * 128 * sizeof(float);
     // counters: a fixed region sized for the largest partition (one per SM)
     const size_t counter_bytes = static_cast<size_t>(ds->sms) * 8 * sizeof(unsigned);
-    if ((rc = get_workspace(dev, s, part_bytes, counter_bytes, &p.part, &p.counters))) return rc;
+    if ((rc = get_workspace(dev, s, part_bytes, counter_bytes, &p.part, &p.counters))) {
+      if (rc != DFK_ERR_NO_VARIANT || !stream_capturing(s)) return rc;
+      // being captured on a stream without a workspace (none may be allocated
+      // now): the same variant without the split
+      VDef whole = v;
+      whole.ksplit = 1;
+      log_msg("split-K workspace missing during capture: launching without the split");
+      return launch_tc(c, whole, s, stages_used);
+    }
   }
   void *args[] = {&maps, &p};
   cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TC_THREADS), pl.smem, s,

@@ -44,7 +44,10 @@ class DecodeStack:
             self.u = torch.empty_like(self.h)
             self.s = torch.empty_like(self.h)
         self.graph = None
-        self.trace = None                        # optional: {(step, layer): tensor}
+        # every launch of the stack (eager warm-up, capture, replay) goes to
+        # one stream, so the capture finds the scheduler's decisions and the
+        # split-K workspace that the warm-up made on that stream
+        self.stream = torch.cuda.Stream(device=dev)
 
     def layer_input(self, l):
         return self.x if l == 0 else self.acts[(l - 1) % 2]
@@ -63,24 +66,38 @@ class DecodeStack:
             dfk.dfk_mul(self.s, self.u, out=self.h)
         dfk.dfk_down_proj(self.h, wd, y=y)
 
-    def step_eager(self):
-        """One decode step, launched kernel by kernel on the current stream."""
+    def _launch_step(self):
         for l in range(len(self.layers)):
             self._layer(l)
         dfk.dfk_rms_rescale(self.acts[(len(self.layers) - 1) % 2], self.eps, out=self.x)
 
+    def step_eager(self):
+        """One decode step, launched kernel by kernel on the stack's stream
+        (ordered after the caller's current stream and back)."""
+        cur = torch.cuda.current_stream(self.stream.device)
+        self.stream.wait_stream(cur)
+        with torch.cuda.stream(self.stream):
+            self._launch_step()
+        cur.wait_stream(self.stream)
+
     def capture(self):
-        """Capture one step in a CUDA graph (call after a warm-up step, so the
-        scheduler's decisions are cached and nothing is timed during capture)."""
+        """Capture one step in a CUDA graph on the stack's stream (call after a
+        warm-up step, so the scheduler's decisions are cached and nothing is
+        timed during capture)."""
+        torch.cuda.synchronize(self.stream.device)
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            self.step_eager()
+        with torch.cuda.graph(g, stream=self.stream):
+            self._launch_step()
         self.graph = g
         return g
 
     def step(self):
         if self.graph is not None:
-            self.graph.replay()
+            cur = torch.cuda.current_stream(self.stream.device)
+            self.stream.wait_stream(cur)
+            with torch.cuda.stream(self.stream):
+                self.graph.replay()
+            cur.wait_stream(self.stream)
         else:
             self.step_eager()
 

@@ -85,3 +85,24 @@ def test_unfused_layer_matches_oracle():
     # the unfused chain rounds xn, a, u, SiLU(a), h to bf16 (see the unfused bound)
     ok, err = close(st.acts[0], y_ref, rtol=2.5e-2)
     assert ok, err
+
+
+def test_capture_on_fresh_stream_without_workspace():
+    # the scheduler picked a split-K variant eagerly on the default stream; a
+    # capture on a stream that never ran it cannot allocate a workspace, so
+    # the library launches the same variant without the split
+    g = torch.Generator(device="cuda").manual_seed(11)
+    h = (torch.randn(8, 14336, generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    wd = (torch.randn(4096, 14336, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    eager = dfk.dfk_down_proj(h, wd)
+    torch.cuda.synchronize()
+    y = torch.empty_like(eager)
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dfk.dfk_down_proj(h, wd, y=y)
+    graph.replay()
+    torch.cuda.synchronize()
+    ok, err = close(y, I.bf16_values(eager))
+    assert ok, err
+    del graph
