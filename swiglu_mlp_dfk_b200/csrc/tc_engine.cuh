@@ -290,10 +290,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         *reinterpret_cast<uint4 *>(gs + k) = v;
       }
       named_barrier(1, 128);
-      const int tpr = 128 / BN;       // threads per token row
-      const int n = et / tpr, part = et - n * tpr;
-      const int cpt = 8 / tpr;        // 16-byte chunks per thread per k-tile
-      float ss = 0.f;
+      // task t = et + 128 c (c < BN / 16) is 16-byte chunk (t & 7) of token row
+      // t >> 3: the 8 lanes of a shared-memory phase cover the 8 chunks of one
+      // row (conflict-free), and the 8 lanes of a row reduce its sum of squares
+      const int cpt = BN / 16;        // rows (chunks) per thread per k-tile: 1, 2 or 4
+      const int pc = et & 7;          // physical 16-byte chunk
+      float ss[4] = {0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
         const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
@@ -303,8 +305,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int kt = 0; kt < nv; ++kt) {
             uint8_t *xt = sb + p.a_bytes + kt * p.xt_bytes;
             uint8_t *lt = xt + BN * 128;
-            for (int c = 0; c < cpt; ++c) {
-              const int pc = part * cpt + c;          // physical 16-byte chunk of row n
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if (c >= cpt) break;
+              const int n = (et >> 3) + 16 * c;       // token row
               const int lc = pc ^ (n & 7);            // 128-byte swizzle: logical chunk
               const int k = (tile0 + i * NT + kt) * TC_TILE_K + 8 * lc;
               const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
@@ -315,8 +319,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float x0 = bf16_lo(xw[q]), x1 = bf16_hi(xw[q]);
-                ss = fmaf(x0, x0, ss);
-                ss = fmaf(x1, x1, ss);
+                ss[c] = fmaf(x0, x0, ss[c]);
+                ss[c] = fmaf(x1, x1, ss[c]);
                 const float p0 = x0 * bf16_lo(gw[q]), p1 = x1 * bf16_hi(gw[q]);  // exact
                 const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
                 const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
@@ -335,10 +339,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         mbar_arrive(&xready[st]);
       }
-      // sum of squares of row n: the tpr threads of a row are adjacent lanes
-      for (int m = tpr >> 1; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      if (part == 0)
-        s_rinv[n] = (n < p.B) ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 0.f;
+      // sum of squares of each row: its 8 chunks sit in 8 adjacent lanes
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v = ss[c];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        const int n = (et >> 3) + 16 * c;
+        if (c < cpt && pc == 0)
+          s_rinv[n] = (n < p.B) ? 1.0f / sqrtf(v / static_cast<float>(p.K) + p.eps) : 0.f;
+      }
       named_barrier(1, 128);
     }
 
