@@ -179,6 +179,25 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sel), "note": note}
 
 
+# ---------------------------------------------------------------- replicas
+
+def max_over_ranks(value, dist=None, device=None):
+    """Largest `value` over all ranks of the default process group (a
+    device-side time: the job ends when the slowest replica ends)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(bytes_per_step, steps, world, t_max_ms):
+    """Whole-job GB/s of `world` independent replicas that each ran `steps`
+    steps of `bytes_per_step` algorithmic bytes, the slowest taking t_max_ms."""
+    return bytes_per_step * steps * world / (t_max_ms / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def gpu_arm(args):
@@ -247,12 +266,8 @@ def gpu_arm(args):
     if world > 1:
         dist.barrier()
     total_ms = ev0.elapsed_time(ev1)
-    t_max = total_ms
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    value = step_bytes(B1, D, F) * K * world / (t_max / 1e3) / 1e9
+    t_max = max_over_ranks(total_ms, dist, "cuda")
+    value = replica_throughput(step_bytes(B1, D, F), K, world, t_max)
 
     # ---- the dominant kernel alone: K back-to-back fused gate/up launches
     # (average launch duration = elapsed / K), and the down projection alone
@@ -310,12 +325,8 @@ def gpu_arm(args):
     e1.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
-    e2e_ms = max(e0.elapsed_time(e1), wall * 1e3)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = step_bytes(B1, D, F) * Ke * world / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(max(e0.elapsed_time(e1), wall * 1e3), dist, "cuda")
+    e2e_value = replica_throughput(step_bytes(B1, D, F), Ke, world, e2e_ms)
 
     extra = {}
     if rank == 0 and not args.quick:

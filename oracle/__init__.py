@@ -30,11 +30,9 @@ LAYOUT_INTERLEAVED = 2
 _lib = None
 
 
-def _load():
-    global _lib
-    if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library; returns it."""
+    if True:
         u16p = ctypes.POINTER(ctypes.c_uint16)
         dp = ctypes.POINTER(ctypes.c_double)
         ip = ctypes.POINTER(ctypes.c_int)
@@ -61,8 +59,32 @@ def _load():
         lib.dfk_oracle_rms_rescale.restype = ctypes.c_int
         lib.dfk_oracle_rms_rescale.argtypes = [dp, ctypes.c_double, ctypes.c_int,
                                                ctypes.c_int, dp]
-        _lib = lib
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(_build.build()))
     return _lib
+
+
+class _swapped:
+    """Context manager: run the oracle functions on another build of the C
+    source (used by the mutation test, which plants mistakes in a copy)."""
+
+    def __init__(self, path):
+        self.lib = _bind(ctypes.CDLL(path))
+
+    def __enter__(self):
+        global _lib
+        self.prev, _lib = _load(), self.lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.prev
+        return False
 
 
 def _u16(a):
