@@ -460,8 +460,9 @@ static int pow2_ceil(int v) {
 // tile, so the space behind the last A tile of the ring is kept readable.
 static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
                     const DeviceState &ds, TcPlan *pl, std::string *why) {
-  if (layout == LAYOUT_COL) {
-    if (why) *why = "the tensor-core family reads K-major (row-major / interleaved) weights";
+  const bool colm = layout == LAYOUT_COL;
+  if (colm && nmat != 2) {
+    if (why) *why = "column-major tensor-core kernel is the fused gate/up only";
     return false;
   }
   if (B < 1 || B > 64) {
@@ -478,17 +479,20 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     return false;
   }
   for (int mult = 1; mult <= 8; mult *= 2) {
-    // row blocks: one per CTA, or (split-K) one per kslices CTAs
-    const int nblocks = kslices > 1 ? std::min(N, ds.sms / kslices) : std::min(N, ds.sms * mult);
+    // row blocks: one per CTA, or (split-K) one per kslices CTAs; column-major:
+    // 128 columns per CTA (two full 64-column boxes)
+    const int nblocks = colm ? ceil_div(N, 128)
+                             : (kslices > 1 ? std::min(N, ds.sms / kslices)
+                                            : std::min(N, ds.sms * mult));
     if (nblocks < 1) break;
     const int P = nblocks * kslices;
-    const int rbase = N / nblocks, rextra = N % nblocks;
+    const int rbase = colm ? 128 : N / nblocks, rextra = colm ? 0 : N % nblocks;
     const int r_hi = rbase + (rextra ? 1 : 0);
-    for (int mt = 1; mt <= (kslices > 1 ? 1 : 2); ++mt) {
+    for (int mt = 1; mt <= (kslices > 1 || colm ? 1 : 2); ++mt) {
       if (r_hi > 128 * mt) continue;
       if (mt == 2 && rbase < 2) continue;
       const int hmax = (r_hi + mt - 1) / mt;
-      const int rc = round_up(hmax, 8);
+      const int rc = colm ? 128 : round_up(hmax, 8);
       const int a_bytes = nt * mt * nmat * rc * 128;
       const int xt_bytes = bn * 128 * (norm ? 2 : 1);  // hi rows (+ lo rows)
       const int x_bytes = nt * xt_bytes;
@@ -506,7 +510,8 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       while (nbank > 1 && mt * nmat * nbank * wn > 512) nbank >>= 1;
       const int cols = pow2_ceil(std::max(32, mt * nmat * nbank * wn));
       if (cols > 512) continue;
-      const void *fn = tc_find_kernel(nmat, norm ? 1 : 0, layout == LAYOUT_IL ? 1 : 0, mt);
+      const void *fn = tc_find_kernel(nmat, norm ? 1 : 0,
+                                      layout == LAYOUT_IL ? 2 : (colm ? 1 : 0), mt);
       if (!fn) {
         if (why) *why = "tensor-core kernel not compiled for this case";
         return false;
@@ -540,7 +545,7 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
       return true;
     }
-    if (kslices > 1) break;  // the split partition does not depend on `mult`
+    if (kslices > 1 || colm) break;  // these partitions do not depend on `mult`
   }
   if (why) *why = "no tensor-core partition fits shared memory";
   return false;
@@ -609,7 +614,14 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   const int hmax = pl.p.hmax;
   for (int lo = 0; lo < 2; ++lo) {
     const uint32_t hgt = static_cast<uint32_t>(std::max(1, hmax - lo));
-    if (c.layout == LAYOUT_IL) {
+    if (c.layout == LAYOUT_COL) {
+      // [K][N] weights: boxes of 64 columns x 64 k rows
+      if ((rc = tensor_map_2d(c.w0, c.N, c.K, static_cast<uint64_t>(c.N) * 2, 64, TC_TILE_K,
+                              &maps.wg[lo], true)) ||
+          (rc = tensor_map_2d(c.w1, c.N, c.K, static_cast<uint64_t>(c.N) * 2, 64, TC_TILE_K,
+                              &maps.wu[lo], true)))
+        return rc;
+    } else if (c.layout == LAYOUT_IL) {
       const uint64_t dims[3] = {static_cast<uint64_t>(c.K), 2, static_cast<uint64_t>(c.N)};
       const uint64_t strides[2] = {static_cast<uint64_t>(c.K) * 2,
                                    static_cast<uint64_t>(c.K) * 4};
@@ -849,7 +861,7 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
     if (d.family == DFK_FAMILY_TENSOR_CORE) {
       // gate/up from B = 4 (where CUDA cores fall below HBM speed), the GEMV
       // (split-K) from B = 2
-      if (B >= (d.cls == CLS_GEMV ? 2 : 4) && c.layout != LAYOUT_COL) out.push_back(&d);
+      if (B >= (d.cls == CLS_GEMV ? 2 : 4)) out.push_back(&d);
       continue;
     }
     if (d.bt != bt_for(B, d.jpt)) continue;
@@ -873,7 +885,7 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // the GEMV the largest k split whose CTA fits.  If nothing of that shape
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
-  if (B >= 8 && c.layout != LAYOUT_COL) {
+  if (B >= 8) {
     const bool gemv = op_class(op) == CLS_GEMV;
     const int want_nt = gemv ? 2 : 1, want_ks = gemv ? 4 : 1;
     for (const VDef &d : variants())

@@ -121,11 +121,16 @@ __device__ __forceinline__ void tmem_sum_banks(uint32_t taddr, int nb, int bank_
   }
 }
 
-template <int NMAT, bool NORM, bool IL, int MT>
+// WL (weight layout): 0 row-major [N][K] (K-major A), 1 column-major [K][N]
+// (MN-major A; each CTA owns 128 columns, loaded as two 64-column boxes),
+// 2 interleaved [N][2][K].
+template <int NMAT, bool NORM, int WL, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemv_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  constexpr bool IL = WL == 2, COLM = WL == 1;
   static_assert(NMAT == 1 || NMAT == 2, "NMAT");
   static_assert(!IL || NMAT == 2, "interleaved layout holds both matrices");
+  static_assert(!COLM || MT == 1, "column-major: one 128-column tile per CTA");
   static_assert(!NORM || NMAT == 2, "the RMSNorm prologue belongs to the gate/up kernel");
   static_assert(MT == 1 || MT == 2, "MT");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int cta = blockIdx.x;
   const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
   const int j0 = blk * p.rbase + min(blk, p.rextra);
-  const int r = p.rbase + (blk < p.rextra ? 1 : 0);
+  const int r = COLM ? min(p.rbase, p.N - j0) : p.rbase + (blk < p.rextra ? 1 : 0);
   const int tile0 = (slc * p.ntiles) / p.kslices;
   const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
   const int nsteps = (tile1 - tile0 + NT - 1) / NT;
@@ -198,7 +203,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
         const int nv = min(NT, tile1 - (tile0 + i * NT));  // k-tiles of this step in range
-        mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nv) * (NMAT * r + BN) * 128u);
+        // (column-major boxes are always 64 x 64, zero-filled past the last column)
+        mbar_arrive_expect_tx(&full[st],
+                              static_cast<uint32_t>(nv) * (NMAT * (COLM ? 128 : r) + BN) * 128u);
         for (int kt = 0; kt < nv; ++kt) {
           const int k0 = (tile0 + i * NT + kt) * TC_TILE_K;
 #pragma unroll
@@ -207,11 +214,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
               uint8_t *dst = sb + ((kt * MT + t) * NMAT + m) * p.rc * 128;
-              if (IL)
+              const CUtensorMap *wm = m == 0 ? &maps.wg[mi] : &maps.wu[mi];
+              if (IL) {
                 tma_load_3d(dst, &maps.wg[mi], &full[st], k0, m, j0 + rs[t], pol_w);
-              else
-                tma_load_2d(dst, m == 0 ? &maps.wg[mi] : &maps.wu[mi], &full[st], k0,
-                            j0 + rs[t], pol_w);
+              } else if (COLM) {
+                // columns j0 .. j0 + 63 and j0 + 64 .. j0 + 127, 64 k rows each
+                tma_load_2d(dst, wm, &full[st], j0, k0, pol_w);
+                tma_load_2d(dst + 8192, wm, &full[st], j0 + 64, k0, pol_w);
+              } else {
+                tma_load_2d(dst, wm, &full[st], k0, j0 + rs[t], pol_w);
+              }
             }
           }
           // activations: only after the previous kernel's results are visible
@@ -240,7 +252,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // (the hi rows, then the lo rows).
     if (lane == 0) {
       const int WN = NORM ? 2 * BN : BN;
-      const uint32_t idesc = umma_idesc_bf16_f32(128, WN);
+      const uint32_t idesc = umma_idesc_bf16_f32(128, WN, COLM);
       const int NB = p.nbank;
       // descriptors are built once; the address field (bits 0-13, 16-byte
       // units) is then advanced by plain addition (shared memory < 256 KB)
@@ -266,7 +278,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int t = 0; t < MT; ++t) {
 #pragma unroll
               for (int m = 0; m < NMAT; ++m) {
-                const uint64_t a = at + static_cast<uint64_t>(t * NMAT + m) * tile_enc + 2 * kk;
+                // K-major: the 16-element k-slice kk starts 32 bytes into each
+                // swizzled row; MN-major: it is the atom pair 2 kk, 2 kk + 1
+                // (2048 bytes per slice), with atoms 8192 bytes apart along M
+                const uint64_t a =
+                    COLM ? umma_desc_sw128_mn(0u, 8192u, 1024u) +
+                               (((at + static_cast<uint64_t>(t * NMAT + m) * tile_enc) &
+                                 0x3FFFull) +
+                                (2048u >> 4) * kk)
+                         : at + static_cast<uint64_t>(t * NMAT + m) * tile_enc + 2 * kk;
                 const uint32_t d = tmem + static_cast<uint32_t>(((t * NMAT + m) * NB + b) * WN);
                 umma_bf16(d, a, bx + 2 * kk, idesc, acc);
               }

@@ -2,6 +2,7 @@
 #pragma once
 
 namespace dfk {
-// __global__ function for (matrices, RMSNorm prologue, interleaved, sub-tiles), or nullptr.
-const void *tc_find_kernel(int nmat, int norm, int il, int mt);
+// __global__ function for (matrices, RMSNorm prologue, weight layout 0 row /
+// 1 column / 2 interleaved, sub-tiles), or nullptr.
+const void *tc_find_kernel(int nmat, int norm, int wl, int mt);
 }  // namespace dfk

@@ -28,13 +28,31 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D,
-// shape M x N (M = 64 or 128; N a multiple of 16 up to 256 for M = 128).
+// Shared-memory descriptor for an MN-major operand in the 128-byte-swizzled
+// layout: atoms of 64 M-elements (128 bytes) x 8 K-rows (1024 bytes); `lbo`
+// bytes between atoms along M, `sbo` bytes between atoms along K.  (A TMA box
+// of 64 M-elements x 64 K-rows with 128-byte swizzle writes 8 such atoms
+// 1024 bytes apart along K.)
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo,
+                                                       uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, B K-major, A
+// K-major or MN-major, shape M x N (M = 64 or 128; N a multiple of 16 up to
+// 256 for M = 128).
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
-//   (1 = bf16), 15/16 A/B major (0 = K-major), 17-22 N >> 3, 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
+//   (1 = bf16), 15/16 A/B major (0 = K-major, 1 = MN-major), 17-22 N >> 3,
+//   24-28 M >> 4.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N, bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major ? (1u << 15) : 0u) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *slot_smem, uint32_t ncols) {
