@@ -91,6 +91,7 @@ typedef struct dfk_variant {
   int k_tiles_per_stage; /* consecutive 64-wide reduction tiles per ring stage       */
   int acc_banks;    /* tensor core: independent TMEM accumulators per output        */
   int paired_fma;   /* CUDA core: 1 = FMAs issued two at a time (fma.rn.f32x2)      */
+  int full_m_tiles; /* tensor core: 1 = each CTA owns 128 output rows (full MMA M) */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
 } dfk_variant;

@@ -68,7 +68,7 @@ class dfk_variant(ctypes.Structure):
                 ("family", ctypes.c_int), ("j_per_thread", ctypes.c_int),
                 ("token_tile", ctypes.c_int), ("k_split", ctypes.c_int),
                 ("k_tiles_per_stage", ctypes.c_int), ("acc_banks", ctypes.c_int),
-                ("paired_fma", ctypes.c_int),
+                ("paired_fma", ctypes.c_int), ("full_m_tiles", ctypes.c_int),
                 ("stages", ctypes.c_int), ("measured_us", ctypes.c_float)]
 
     def as_dict(self):

@@ -226,6 +226,7 @@ struct VDef {
   int jpt, bt, ksplit, nt;
   int nbank;  // tensor core: independent TMEM accumulator banks per output
   int pair;   // CUDA core: FMAs issued in pairs (fma.rn.f32x2)
+  int full;   // tensor core: CTAs own full 128-row M tiles (fewer CTAs than SMs)
 };
 
 static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
@@ -237,20 +238,21 @@ static const std::vector<VDef> &variants() {
     for (int pr : {0, 1})
       for (int nt : {1, 2, 4})
         for (auto &jb : kJB)
-          t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt, 1, pr});
+          t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], 1, nt, 1, pr, 0});
     for (int pr : {0, 1})
       for (int nt : {1, 2, 4})
         for (int ks : {1, 2, 4, 8})
           for (auto &jb : kJB)
-            t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt, 1, pr});
+            t.push_back({id++, CLS_GEMV, DFK_FAMILY_CUDA_CORE, jb[0], jb[1], ks, nt, 1, pr, 0});
     // tensor-core family: token tile chosen from B at launch (16 / 32 / 64)
-    for (int nb : {1, 2})
+    // gate/up: rows spread over every SM, or full 128-row tiles
+    for (int fu : {0, 1})
       for (int nt : {1, 2})
-        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, nb, 0});
+        t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, 1, 0, fu});
     // GEMV: k-split = reduction slices across CTAs (split-K with a workspace)
     for (int ks : {1, 2, 4})
       for (int nt : {1, 2, 4, 8})
-        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, nt, 1, 0});
+        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, nt, 1, 0, 0});
     return t;
   }();
   return v;
@@ -461,6 +463,7 @@ static int pow2_ceil(int v) {
 static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
                     const DeviceState &ds, TcPlan *pl, std::string *why) {
   const bool colm = layout == LAYOUT_COL;
+  const bool full = colm || (v.full != 0 && nmat == 2);  // 128 rows per CTA
   if (colm && nmat != 2) {
     if (why) *why = "column-major tensor-core kernel is the fused gate/up only";
     return false;
@@ -481,18 +484,18 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
   for (int mult = 1; mult <= 8; mult *= 2) {
     // row blocks: one per CTA, or (split-K) one per kslices CTAs; column-major:
     // 128 columns per CTA (two full 64-column boxes)
-    const int nblocks = colm ? ceil_div(N, 128)
+    const int nblocks = full ? ceil_div(N, 128)
                              : (kslices > 1 ? std::min(N, ds.sms / kslices)
                                             : std::min(N, ds.sms * mult));
     if (nblocks < 1) break;
     const int P = nblocks * kslices;
-    const int rbase = colm ? 128 : N / nblocks, rextra = colm ? 0 : N % nblocks;
+    const int rbase = full ? 128 : N / nblocks, rextra = full ? 0 : N % nblocks;
     const int r_hi = rbase + (rextra ? 1 : 0);
-    for (int mt = 1; mt <= (kslices > 1 || colm ? 1 : 2); ++mt) {
+    for (int mt = 1; mt <= (kslices > 1 || full ? 1 : 2); ++mt) {
       if (r_hi > 128 * mt) continue;
       if (mt == 2 && rbase < 2) continue;
       const int hmax = (r_hi + mt - 1) / mt;
-      const int rc = colm ? 128 : round_up(hmax, 8);
+      const int rc = full ? 128 : round_up(hmax, 8);
       const int a_bytes = nt * mt * nmat * rc * 128;
       const int xt_bytes = bn * 128 * (norm ? 2 : 1);  // hi rows (+ lo rows)
       const int x_bytes = nt * xt_bytes;
@@ -542,10 +545,11 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       p.ntiles = ntiles;
       p.kslices = kslices;
       p.nblocks = nblocks;
+      p.full = full ? 1 : 0;
       pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
       return true;
     }
-    if (kslices > 1 || colm) break;  // these partitions do not depend on `mult`
+    if (kslices > 1 || full) break;  // these partitions do not depend on `mult`
   }
   if (why) *why = "no tensor-core partition fits shared memory";
   return false;
@@ -773,6 +777,7 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->k_tiles_per_stage = d.nt;
   out->acc_banks = d.nbank;
   out->paired_fma = d.pair;
+  out->full_m_tiles = d.full;
   out->stages = stages;
   out->measured_us = us;
 }

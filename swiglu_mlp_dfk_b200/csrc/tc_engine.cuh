@@ -71,6 +71,7 @@ struct TcParams {
   float *part;            // [kslices][row blocks][bn][128] fp32
   unsigned *counters;     // [row blocks], 0 between calls
   int nblocks;            // row blocks (split-K)
+  int full;               // 1: every CTA owns 128 rows (the last one fewer); boxes of 128 rows
 };
 
 // wg/wu: [0] box height hmax, [1] box height hmax - 1; x: activations box {64, bn}.
@@ -142,8 +143,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = p.stages, NT = p.nt, BN = p.bn;
 
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-  uint64_t *empty = full + S;
+  uint64_t *fullb = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+  uint64_t *empty = fullb + S;
   uint64_t *xready = empty + S;
   uint64_t *accfull = xready + S;
   volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int cta = blockIdx.x;
   const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
   const int j0 = blk * p.rbase + min(blk, p.rextra);
-  const int r = COLM ? min(p.rbase, p.N - j0) : p.rbase + (blk < p.rextra ? 1 : 0);
+  const bool full = COLM || p.full;  // 128-row boxes, zero-filled past the last row
+  const int r = full ? min(p.rbase, p.N - j0) : p.rbase + (blk < p.rextra ? 1 : 0);
   const int tile0 = (slc * p.ntiles) / p.kslices;
   const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
   const int nsteps = (tile1 - tile0 + NT - 1) / NT;
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&fullb[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&xready[s], 128);
     }
@@ -204,31 +206,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
         const int nv = min(NT, tile1 - (tile0 + i * NT));  // k-tiles of this step in range
         // (column-major boxes are always 64 x 64, zero-filled past the last column)
-        mbar_arrive_expect_tx(&full[st],
-                              static_cast<uint32_t>(nv) * (NMAT * (COLM ? 128 : r) + BN) * 128u);
+        mbar_arrive_expect_tx(&fullb[st],
+                              static_cast<uint32_t>(nv) * (NMAT * (full ? 128 : r) + BN) * 128u);
         for (int kt = 0; kt < nv; ++kt) {
           const int k0 = (tile0 + i * NT + kt) * TC_TILE_K;
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
-            const int mi = (h[t] == p.hmax) ? 0 : 1;
+            const int mi = (full || h[t] == p.hmax) ? 0 : 1;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
               uint8_t *dst = sb + ((kt * MT + t) * NMAT + m) * p.rc * 128;
               const CUtensorMap *wm = m == 0 ? &maps.wg[mi] : &maps.wu[mi];
               if (IL) {
-                tma_load_3d(dst, &maps.wg[mi], &full[st], k0, m, j0 + rs[t], pol_w);
+                tma_load_3d(dst, &maps.wg[mi], &fullb[st], k0, m, j0 + rs[t], pol_w);
               } else if (COLM) {
                 // columns j0 .. j0 + 63 and j0 + 64 .. j0 + 127, 64 k rows each
-                tma_load_2d(dst, wm, &full[st], j0, k0, pol_w);
-                tma_load_2d(dst + 8192, wm, &full[st], j0 + 64, k0, pol_w);
+                tma_load_2d(dst, wm, &fullb[st], j0, k0, pol_w);
+                tma_load_2d(dst + 8192, wm, &fullb[st], j0 + 64, k0, pol_w);
               } else {
-                tma_load_2d(dst, wm, &full[st], k0, j0 + rs[t], pol_w);
+                tma_load_2d(dst, wm, &fullb[st], k0, j0 + rs[t], pol_w);
               }
             }
           }
           // activations: only after the previous kernel's results are visible
           if (i >= S0)
-            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &full[st], k0, 0, pol_x);
+            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &fullb[st], k0, 0, pol_x);
         }
         if (i == S0 - 1) {
           pdl_wait();
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int kt = 0; kt < nvi; ++kt)
               tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
                               kt * p.xt_bytes,
-                          &maps.x, &full[ii], (tile0 + ii * NT + kt) * TC_TILE_K, 0, pol_x);
+                          &maps.x, &fullb[ii], (tile0 + ii * NT + kt) * TC_TILE_K, 0, pol_x);
           }
         }
         issued = i + 1;
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        if (!mbar_wait_bounded(NORM ? &xready[st] : &full[st], (i / S) & 1, s_abort, p.err))
+        if (!mbar_wait_bounded(NORM ? &xready[st] : &fullb[st], (i / S) & 1, s_abort, p.err))
           break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       float ss[4] = {0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        const bool ok = mbar_wait_bounded(&full[st], (i / S) & 1, s_abort, p.err);
+        const bool ok = mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err);
         if (ok) {
           uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
           const int nv = min(NT, tile1 - (tile0 + i * NT));
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int last = -1;
       for (int i = issued - 1; i >= 0 && i >= issued - S; --i)
         if (i % S == st) { last = i; break; }
-      if (last >= 0) mbar_wait_bounded(&full[st], (last / S) & 1, nullptr, p.err);
+      if (last >= 0) mbar_wait_bounded(&fullb[st], (last / S) & 1, nullptr, p.err);
     }
   }
 }
