@@ -584,9 +584,11 @@ def profile_arm(args):
                         with_down=args.profile == "down", device="cuda")
     h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
     y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+    lay = {"row": I.LAYOUT_ROW, "col": I.LAYOUT_COL, "interleaved": I.LAYOUT_INTERLEAVED}
+    wg, wu = I.to_layout(inp.w_gate, inp.w_up, lay[args.layout])
     if args.profile == "gate_up":
-        fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate,
-                                                    inp.w_up, args.layout, h=h)
+        fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu,
+                                                    args.layout, h=h)
     else:
         fn = lambda: dfk.dfk_down_proj(h, inp.w_down, y=y)
     for _ in range(args.warmup):
