@@ -329,7 +329,9 @@ def gpu_arm(args):
     e2e_value = replica_throughput(step_bytes(B1, D, F), Ke, world, e2e_ms)
 
     extra = {}
-    if rank == 0 and not args.quick:
+    if world == 1 and not args.quick:
+        # single-GPU characterisation (sweeps, 70B layer, decode stack); with
+        # several replicas only the headline line is printed
         extra = extra_measurements(args, inp, copies, h, y)
     clocks.stop()
     err = dfk.dfk_device_error()
@@ -457,8 +459,47 @@ def extra_measurements(args, inp, copies, h, y):
     out["batch_sweep"] = sweep
     del x64, col, row_w, flush
     torch.cuda.empty_cache()
+    out["llama3_70b"] = llama70b_measure()
+    torch.cuda.empty_cache()
     out["decode_stack"] = decode_stack_measure(args.stack_steps)
     return out
+
+
+def llama70b_measure(reps=30):
+    """Llama-3-70B-shaped layer (d_model 8192, d_ff 28672, W ~ N(0, 0.015),
+    no RMSNorm, seed 3): gate/up and down at B = 1 and 8, back-to-back calls
+    over two rotated weight copies (1.9 GB each, far beyond L2)."""
+    import torch
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    peak, _ = measured_peaks()
+    D7, F7 = 8192, 28672
+    res = []
+    base = I.make_inputs(8, D7, F7, seed=3, w_std=0.015, norm=False, with_down=True,
+                         device="cuda")
+    cps = [(base.w_gate, base.w_up, base.w_down),
+           (base.w_gate.clone(), base.w_up.clone(), base.w_down.clone())]
+    for B in (1, 8):
+        x = base.x[:B].contiguous()
+        h = torch.empty(B, F7, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(B, D7, dtype=torch.bfloat16, device="cuda")
+        dfk.dfk_swiglu_gate_up(x, cps[0][0], cps[0][1], "row", h=h)   # scheduler decides
+        dfk.dfk_down_proj(h, cps[0][2], y=y)
+        tg = timed_us(lambda i: dfk.dfk_swiglu_gate_up(x, cps[i % 2][0], cps[i % 2][1], "row",
+                                                        h=h), reps)
+        td = timed_us(lambda i: dfk.dfk_down_proj(h, cps[i % 2][2], y=y), reps)
+        gg = gate_up_bytes(B, D7, F7) / (tg * 1e-6) / 1e9
+        gd = down_bytes(B, D7, F7) / (td * 1e-6) / 1e9
+        vg = dfk.dfk_cached_variant(dfk.DFK_OP_GATE_UP, B, D7, F7, "row") or {}
+        vd = dfk.dfk_cached_variant(dfk.DFK_OP_DOWN, B, D7, F7, "row") or {}
+        res.append({"B": B, "gate_up_us": round(tg, 2), "gate_up_frac": round(gg / peak, 4),
+                    "gate_up_family": {0: "cuda_core", 1: "tensor_core"}.get(vg.get("family")),
+                    "down_us": round(td, 2), "down_frac": round(gd / peak, 4),
+                    "down_family": {0: "cuda_core", 1: "tensor_core"}.get(vd.get("family")),
+                    "mlp_us": round(tg + td, 2)})
+    del base, cps
+    return res
 
 
 def decode_stack_measure(steps, layers=32, B=4):

@@ -1347,6 +1347,135 @@ int dfk_mul(const void *a, const void *b, void *out, long long n, void *stream) 
   return DFK_OK;
 }
 
+}  // extern "C"
+
+namespace dfk {
+
+// ---- dfk_mlp_forward_host: one layer from host memory.  With pinned host
+// buffers the whole step (copy in, fused gate/up, down projection, copy out)
+// is replayed as one CUDA graph per distinct argument set; the graph is
+// captured on an internal stream after one eager run there (which settles
+// the scheduler's decisions and the split-K workspace of that stream).
+
+struct HostCall {
+  const void *x_host, *gamma;
+  float eps;
+  const void *w_gate, *w_up;
+  int layout;
+  const void *w_down;
+  void *y_host, *x_dev, *h_dev, *y_dev;
+  int B, d_model, d_ff;
+};
+
+using HostKey = std::tuple<int, uintptr_t, uintptr_t, uintptr_t, uintptr_t, uintptr_t,
+                           uintptr_t, uintptr_t, uintptr_t, uintptr_t, uintptr_t, int, int,
+                           int, int, uint32_t>;
+static std::mutex g_host_mu;
+static std::map<HostKey, cudaGraphExec_t> g_host_graphs;  // nullptr: capture failed, run eager
+static std::map<int, cudaStream_t> g_capture_streams;
+
+static int forward_host_enqueue(const HostCall &a, cudaStream_t s) {
+  const size_t xb = static_cast<size_t>(a.B) * a.d_model * 2;
+  cudaError_t e = cudaMemcpyAsync(a.x_dev, a.x_host, xb, cudaMemcpyHostToDevice, s);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "copy x to device");
+  }
+  int rc = a.gamma ? dfk_rmsnorm_swiglu_gate_up(a.x_dev, a.gamma, a.eps, a.w_gate, a.w_up,
+                                                a.layout, a.h_dev, a.B, a.d_model, a.d_ff, 0, s)
+                   : dfk_swiglu_gate_up(a.x_dev, a.w_gate, a.w_up, a.layout, a.h_dev, a.B,
+                                        a.d_model, a.d_ff, 0, s);
+  if (rc) return rc;
+  if ((rc = dfk_down_proj(a.h_dev, a.w_down, a.y_dev, a.B, a.d_model, a.d_ff, 0, s))) return rc;
+  e = cudaMemcpyAsync(a.y_host, a.y_dev, xb, cudaMemcpyDeviceToHost, s);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "copy y to host");
+  }
+  return DFK_OK;
+}
+
+static bool pinned_host(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost;
+}
+
+static int forward_host_graph(const HostCall &a, int dev, cudaStream_t s, bool *done) {
+  *done = false;
+  uint32_t eps_bits;
+  memcpy(&eps_bits, &a.eps, sizeof eps_bits);
+  const HostKey key{dev, reinterpret_cast<uintptr_t>(s), reinterpret_cast<uintptr_t>(a.x_host),
+                    reinterpret_cast<uintptr_t>(a.gamma), reinterpret_cast<uintptr_t>(a.w_gate),
+                    reinterpret_cast<uintptr_t>(a.w_up), reinterpret_cast<uintptr_t>(a.w_down),
+                    reinterpret_cast<uintptr_t>(a.y_host), reinterpret_cast<uintptr_t>(a.x_dev),
+                    reinterpret_cast<uintptr_t>(a.h_dev), reinterpret_cast<uintptr_t>(a.y_dev),
+                    a.layout, a.B, a.d_model, a.d_ff, eps_bits};
+  std::lock_guard<std::mutex> lk(g_host_mu);
+  auto it = g_host_graphs.find(key);
+  if (it != g_host_graphs.end()) {
+    if (!it->second) return DFK_OK;  // known not capturable: caller runs eagerly
+    cudaError_t e = cudaGraphLaunch(it->second, s);
+    if (!e) e = cudaStreamSynchronize(s);
+    if (e) {
+      cudaGetLastError();
+      return cuda_fail(e, "forward graph replay");
+    }
+    *done = true;
+    return DFK_OK;
+  }
+  cudaStream_t &cs = g_capture_streams[dev];
+  cudaError_t e = cudaSuccess;
+  if (!cs) e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+  cudaEvent_t ready = nullptr;
+  if (!e) e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
+  if (!e) e = cudaEventRecord(ready, s);  // after the caller's earlier work on s
+  if (!e) e = cudaStreamWaitEvent(cs, ready, 0);
+  if (ready) cudaEventDestroy(ready);
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "forward graph set-up");
+  }
+  // eager run on the capture stream: this call's result
+  int rc = forward_host_enqueue(a, cs);
+  if (!rc && (e = cudaStreamSynchronize(cs))) {
+    cudaGetLastError();
+    rc = cuda_fail(e, "forward on the capture stream");
+  }
+  if (rc) return rc;
+  *done = true;
+  // capture the same step for the next calls
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (!e) {
+    rc = forward_host_enqueue(a, cs);
+    cudaError_t e2 = cudaStreamEndCapture(cs, &graph);
+    if (!rc && !e2 && graph) e = cudaGraphInstantiate(&exec, graph, 0);
+    else e = e2 ? e2 : cudaErrorUnknown;
+  }
+  if (graph) cudaGraphDestroy(graph);
+  if (e || rc) {
+    cudaGetLastError();
+    exec = nullptr;
+    log_msg("forward graph capture failed; this argument set runs eagerly");
+  }
+  if (g_host_graphs.size() >= 64) {  // bounded cache
+    for (auto &kv : g_host_graphs)
+      if (kv.second) cudaGraphExecDestroy(kv.second);
+    g_host_graphs.clear();
+  }
+  g_host_graphs[key] = exec;
+  return DFK_OK;
+}
+
+}  // namespace dfk
+
+extern "C" {
+
 int dfk_mlp_forward_host(const void *x_host, const void *gamma, float eps, const void *w_gate,
                          const void *w_up, int layout, const void *w_down, void *y_host,
                          void *x_dev, void *h_dev, void *y_dev, int B, int d_model, int d_ff,
@@ -1356,23 +1485,23 @@ int dfk_mlp_forward_host(const void *x_host, const void *gamma, float eps, const
   if (!x_host || !y_host || !x_dev || !h_dev || !y_dev || !w_down)
     return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(B) * d_model * 2;
-  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
-  if (e) {
-    cudaGetLastError();
-    return cuda_fail(e, "copy x to device");
-  }
-  int rc = gamma ? dfk_rmsnorm_swiglu_gate_up(x_dev, gamma, eps, w_gate, w_up, layout, h_dev, B,
-                                              d_model, d_ff, 0, stream)
-                 : dfk_swiglu_gate_up(x_dev, w_gate, w_up, layout, h_dev, B, d_model, d_ff, 0,
-                                      stream);
+  const HostCall a{x_host, gamma, eps, w_gate, w_up, layout, w_down, y_host, x_dev, h_dev,
+                   y_dev, B, d_model, d_ff};
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
   if (rc) return rc;
-  if ((rc = dfk_down_proj(h_dev, w_down, y_dev, B, d_model, d_ff, 0, stream))) return rc;
-  e = cudaMemcpyAsync(y_host, y_dev, xb, cudaMemcpyDeviceToHost, s);
-  if (!e) e = cudaStreamSynchronize(s);
+  if (env_flag("DFK_HOST_GRAPH", true) && !stream_capturing(s) && pinned_host(x_host) &&
+      pinned_host(y_host)) {
+    bool done = false;
+    if ((rc = forward_host_graph(a, dev, s, &done))) return rc;
+    if (done) return DFK_OK;
+  }
+  if ((rc = forward_host_enqueue(a, s))) return rc;
+  cudaError_t e = cudaStreamSynchronize(s);
   if (e) {
     cudaGetLastError();
-    return cuda_fail(e, "copy y to host");
+    return cuda_fail(e, "forward synchronise");
   }
   return DFK_OK;
 }

@@ -285,12 +285,30 @@ def test_host_entry_point_matches_device_path():
     x_dev = torch.empty_like(inp.x)
     h_dev = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
     y_dev = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
-    dfk.dfk_mlp_forward_host(x_host, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row",
-                             inp.w_down, y_host, x_dev, h_dev, y_dev)
     h = run_gate_up(inp, I.LAYOUT_ROW, True)
     y = dfk.dfk_down_proj(h, inp.w_down)
     torch.cuda.synchronize()
-    assert bits_equal(y_host, y.cpu())
+    y_ref = y.cpu()
+    # first call: eager on the library's capture stream, then captured; later
+    # calls replay the graph (pinned buffers); new x content must be picked up
+    for rep in range(3):
+        y_host.zero_()
+        dfk.dfk_mlp_forward_host(x_host, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row",
+                                 inp.w_down, y_host, x_dev, h_dev, y_dev)
+        assert bits_equal(y_host, y_ref), "call %d" % rep
+    x2 = I.make_inputs(B, D, F, seed=7, device="cuda").x
+    x_host.copy_(x2.cpu())
+    dfk.dfk_mlp_forward_host(x_host, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row",
+                             inp.w_down, y_host, x_dev, h_dev, y_dev)
+    h2 = dfk.dfk_rmsnorm_swiglu_gate_up(x2, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row")
+    y2 = dfk.dfk_down_proj(h2, inp.w_down)
+    torch.cuda.synchronize()
+    assert bits_equal(y_host, y2.cpu())
+    # pageable host buffers: eager path
+    xp, yp = x2.cpu(), torch.empty(B, D, dtype=torch.bfloat16)
+    dfk.dfk_mlp_forward_host(xp, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row", inp.w_down,
+                             yp, x_dev, h_dev, y_dev)
+    assert bits_equal(yp, y2.cpu())
 
 
 # ------------------------------------------------------------------ full-size workloads
