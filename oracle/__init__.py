@@ -56,6 +56,17 @@ def _bind(lib):
         lib.dfk_oracle_down.restype = ctypes.c_int
         lib.dfk_oracle_down.argtypes = [dp, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ip, ctypes.c_int, ctypes.c_int, dp]
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        fp = ctypes.POINTER(ctypes.c_float)
+        lib.dfk_oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.dfk_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.dfk_oracle_gate_up_fp8.restype = ctypes.c_int
+        lib.dfk_oracle_gate_up_fp8.argtypes = [u16p, u16p, ctypes.c_double, u8p, fp, u8p, fp,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ip,
+                                               ctypes.c_int, dp, dp, dp]
+        lib.dfk_oracle_down_fp8.restype = ctypes.c_int
+        lib.dfk_oracle_down_fp8.argtypes = [dp, u8p, fp, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ip, ctypes.c_int, dp]
         lib.dfk_oracle_rms_rescale.restype = ctypes.c_int
         lib.dfk_oracle_rms_rescale.argtypes = [dp, ctypes.c_double, ctypes.c_int,
                                                ctypes.c_int, dp]
@@ -241,3 +252,83 @@ def rms_rescale(y, eps=1e-5) -> np.ndarray:
     if rc != 0:
         raise ValueError("dfk_oracle_rms_rescale rejected its arguments")
     return out
+
+
+# ---------------------------------------------------------------- FP8 weights
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Exact value of FP8 E4M3 codes (numpy uint8)."""
+    lib = _load()
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    fo, fi = out.reshape(-1), c.reshape(-1)
+    for i in range(fi.size):
+        fo[i] = lib.dfk_oracle_e4m3_to_double(int(fi[i]))
+    return out
+
+
+def _u8(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint8:
+        raise TypeError("FP8 codes must be numpy uint8, got %s" % a.dtype)
+    return a
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def gate_up_fp8(x, qg, sg, qu, su, gamma=None, eps=1e-5, rows=None, return_au=False):
+    """h = SiLU(xn Wg^T) * (xn Wu^T) with Wg = diag(sg) qg, Wu = diag(su) qu.
+
+    x [B, D] bf16 bits; qg, qu [F, D] E4M3 codes (uint8); sg, su [F] float32.
+    """
+    lib = _load()
+    x, qg, qu = _u16(x), _u8(qg), _u8(qu)
+    sg, su = _f32(sg), _f32(su)
+    B, D = x.shape
+    F = qg.shape[0]
+    if qg.shape != (F, D) or qu.shape != (F, D) or sg.size != F or su.size != F:
+        raise ValueError("FP8 weights must be [F, D] with [F] scales")
+    g = None if gamma is None else _u16(gamma)
+    if rows is None:
+        r, n = None, F
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int32)
+        n = r.size
+    h = np.empty((B, n), dtype=np.float64)
+    a = np.empty((B, n), dtype=np.float64) if return_au else None
+    u = np.empty((B, n), dtype=np.float64) if return_au else None
+    rc = lib.dfk_oracle_gate_up_fp8(_p(x, ctypes.c_uint16), _p(g, ctypes.c_uint16), float(eps),
+                                    _p(qg, ctypes.c_uint8), _p(sg, ctypes.c_float),
+                                    _p(qu, ctypes.c_uint8), _p(su, ctypes.c_float), B, D, F,
+                                    _p(r, ctypes.c_int), n, _p(h, ctypes.c_double),
+                                    _p(a, ctypes.c_double), _p(u, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("dfk_oracle_gate_up_fp8 rejected its arguments")
+    return (h, a, u) if return_au else h
+
+
+def down_fp8(h, qd, sd, rows=None) -> np.ndarray:
+    """y = h Wd^T with Wd = diag(sd) qd; qd [D, F] E4M3 codes, sd [D] float32."""
+    lib = _load()
+    if np.asarray(h).dtype == np.uint16:
+        h = bf16_to_f64(h)
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    qd, sd = _u8(qd), _f32(sd)
+    B, F = h.shape
+    D = qd.shape[0]
+    if qd.shape != (D, F) or sd.size != D:
+        raise ValueError("FP8 W_down must be [D, F] with [D] scales")
+    if rows is None:
+        r, n = None, D
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int32)
+        n = r.size
+    y = np.empty((B, n), dtype=np.float64)
+    rc = lib.dfk_oracle_down_fp8(_p(h, ctypes.c_double), _p(qd, ctypes.c_uint8),
+                                 _p(sd, ctypes.c_float), B, D, F, _p(r, ctypes.c_int), n,
+                                 _p(y, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("dfk_oracle_down_fp8 rejected its arguments")
+    return y

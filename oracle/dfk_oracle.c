@@ -35,6 +35,13 @@
  *       interleaved  Wg[j,k] = W_mem[(2j)*D + k],
  *                    Wu[j,k] = W_mem[(2j+1)*D + k]      ([F][2][D])
  *
+ * Low-precision weights (the "fusing dequantize with compute" idea of
+ * GPULlama3.java PR #78, applied to the same MLP): W[j][k] = s[j] * Q[j][k]
+ * with Q an FP8 E4M3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent 0 is subnormal, S.1111.111 is NaN, no infinities) and s one
+ * fp32 scale per output row.  The dequantised weight is formed exactly in
+ * double and used in the same sums as above.
+ *
  * "Mirror" mode rounds xn, h and y to bf16 (round to nearest, ties to even)
  * at the points where the GPU kernels store bf16; it is a diagnostic only.
  * The contract check uses the pure mode (mirror = 0).
@@ -241,6 +248,79 @@ int dfk_oracle_rms_rescale(const double *y, double eps, int B, int D, double *ou
     for (int k = 0; k < D; ++k) ss += y[(size_t)b * D + k] * y[(size_t)b * D + k];
     double r = 1.0 / sqrt(ss / (double)D + eps);
     for (int k = 0; k < D; ++k) out[(size_t)b * D + k] = y[(size_t)b * D + k] * r;
+  }
+  return 0;
+}
+
+/* FP8 E4M3 code -> double (exact). */
+double dfk_oracle_e4m3_to_double(uint8_t code) {
+  const int sign = (code >> 7) & 1;
+  const int e = (code >> 3) & 15;
+  const int m = code & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);               /* m/8 * 2^(1-7) */
+  else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+static double w_fp8(const uint8_t *q, const float *sc, int j, int k, int D) {
+  return (double)sc[j] * dfk_oracle_e4m3_to_double(q[(size_t)j * D + k]);
+}
+
+/* Gate/up + SwiGLU with FP8 weights: Wg[j][k] = sg[j] * qg[j][k] (row-major
+ * [F][D] codes), likewise Wu; x, gamma as in dfk_oracle_gate_up. */
+int dfk_oracle_gate_up_fp8(const uint16_t *x, const uint16_t *gamma, double eps,
+                           const uint8_t *qg, const float *sg, const uint8_t *qu,
+                           const float *su, int B, int D, int F, const int *rows, int nrows,
+                           double *h, double *a_out, double *u_out) {
+  if (!x || !qg || !sg || !qu || !su || !h || B < 0 || D <= 0 || F <= 0) return -1;
+  if (!rows && nrows != F) return -1;
+  if (rows)
+    for (int i = 0; i < nrows; ++i)
+      if (rows[i] < 0 || rows[i] >= F) return -1;
+  double *xn = (double *)malloc(((size_t)B * D + 1) * sizeof(double));
+  if (!xn) return -1;
+  if (gamma) {
+    dfk_oracle_rmsnorm(x, gamma, eps, B, D, 0, xn);
+  } else {
+    for (size_t i = 0; i < (size_t)B * D; ++i) xn[i] = dfk_oracle_bf16_to_double(x[i]);
+  }
+#pragma omp parallel for schedule(static)
+  for (int i = 0; i < nrows; ++i) {
+    int j = rows ? rows[i] : i;
+    for (int b = 0; b < B; ++b) {
+      const double *xr = xn + (size_t)b * D;
+      double a = 0.0, u = 0.0;
+      for (int k = 0; k < D; ++k) {
+        a += xr[k] * w_fp8(qg, sg, j, k, D);
+        u += xr[k] * w_fp8(qu, su, j, k, D);
+      }
+      h[(size_t)b * nrows + i] = dfk_oracle_silu(a) * u;
+      if (a_out) a_out[(size_t)b * nrows + i] = a;
+      if (u_out) u_out[(size_t)b * nrows + i] = u;
+    }
+  }
+  free(xn);
+  return 0;
+}
+
+/* Down projection with FP8 weights: y[b][i] = sum_j h[b][j] * sd[i] * qd[i][j]. */
+int dfk_oracle_down_fp8(const double *h, const uint8_t *qd, const float *sd, int B, int D,
+                        int F, const int *rows, int nrows, double *y) {
+  if (!h || !qd || !sd || !y || B < 0 || D <= 0 || F <= 0) return -1;
+  if (!rows && nrows != D) return -1;
+  if (rows)
+    for (int i = 0; i < nrows; ++i)
+      if (rows[i] < 0 || rows[i] >= D) return -1;
+#pragma omp parallel for schedule(static)
+  for (int i = 0; i < nrows; ++i) {
+    int r = rows ? rows[i] : i;
+    for (int b = 0; b < B; ++b) {
+      double acc = 0.0;
+      for (int j = 0; j < F; ++j) acc += h[(size_t)b * F + j] * w_fp8(qd, sd, r, j, F);
+      y[(size_t)b * nrows + i] = acc;
+    }
   }
   return 0;
 }

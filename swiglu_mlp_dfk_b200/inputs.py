@@ -158,3 +158,20 @@ def bf16_values(t: torch.Tensor) -> np.ndarray:
     """Exact float64 values of a bf16 tensor (bit-level conversion, no arithmetic)."""
     bits = to_bits(t)
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def to_fp8_rows(w: torch.Tensor):
+    """FP8 E4M3 weights with one fp32 scale per row, from bf16 weights [N, K]:
+    s = max|w| / 448 per row (1 for an all-zero row), Q = E4M3(w / s) by torch's
+    round-to-nearest cast.  Returns (Q as uint8 [N, K], s float32 [N])."""
+    wf = w.float()
+    amax = wf.abs().amax(dim=1)
+    s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (wf / s[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    return q, s.contiguous()
+
+
+def fp8_values(q: torch.Tensor) -> np.ndarray:
+    """Exact float64 values of E4M3 codes (bit-level conversion through torch)."""
+    return q.detach().contiguous().view(torch.float8_e4m3fn).float().cpu().numpy().astype(
+        np.float64)

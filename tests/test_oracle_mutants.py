@@ -34,8 +34,15 @@ MUTANTS = [
      "dfk_oracle_bf16_to_double(wd[(size_t)r * F + j])",
      "dfk_oracle_bf16_to_double(wd[(size_t)j * D + r])"),
     ("first reduction term dropped",
-     "for (int k = 0; k < D; ++k) {\n        a += xr[k]",
-     "for (int k = 1; k < D; ++k) {\n        a += xr[k]"),
+     "for (int k = 0; k < D; ++k) {\n        a += xr[k] * w_gate(",
+     "for (int k = 1; k < D; ++k) {\n        a += xr[k] * w_gate("),
+    ("E4M3 exponent bias 8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("E4M3 subnormal scale", "if (e == 0) v = ldexp((double)m, -9);",
+     "if (e == 0) v = ldexp((double)m, -10);"),
+    ("FP8 row scale ignored",
+     "return (double)sc[j] * dfk_oracle_e4m3_to_double(q[(size_t)j * D + k]);",
+     "return dfk_oracle_e4m3_to_double(q[(size_t)j * D + k]);"),
     ("ties rounded away from zero",
      "(rem == 0.5 && fmod(fl, 2.0) != 0.0)", "(rem == 0.5)"),
 ]

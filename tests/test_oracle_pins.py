@@ -322,3 +322,86 @@ def test_bad_arguments_rejected(oracle_mod):
         oracle.gate_up(bits([[1.0, 2.0]]), bits([[1.0, 2.0, 3.0]]), bits([[1.0, 2.0, 3.0]]))
     with pytest.raises(ValueError):
         oracle.gate_up(bits([[1.0]]), bits([[1.0]]), bits([[1.0]]), rows=[1])
+
+
+# ---------------------------------------------------------------- FP8 weights
+
+def fp8(vals):
+    """E4M3 codes of values that E4M3 represents exactly (torch cast)."""
+    import torch
+    t = torch.tensor(vals, dtype=torch.float32).to(torch.float8_e4m3fn)
+    assert torch.equal(t.float(), torch.tensor(vals, dtype=torch.float32))
+    return t.view(torch.uint8).numpy()
+
+
+def test_e4m3_decoder_all_codes_match_torch(oracle_mod):
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2    # S.1111.111 only
+    assert np.array_equal(ours[~nan], ref[~nan].astype(np.float64))
+    signs = np.signbit(ours[~nan]) == np.signbit(ref[~nan])
+    assert signs.all()
+
+
+def test_e4m3_known_values(oracle_mod):
+    v = lambda c: oracle.e4m3_to_f64(np.array([c], np.uint8))[0]
+    assert v(0x38) == 1.0 and v(0x40) == 2.0 and v(0xB8) == -1.0
+    assert v(0x7E) == 448.0                 # largest finite
+    assert v(0x08) == 2.0 ** -6             # smallest normal
+    assert v(0x01) == 2.0 ** -9             # smallest subnormal
+    assert v(0x07) == 7 * 2.0 ** -9
+    assert v(0x80) == 0.0 and math.copysign(1.0, v(0x80)) == -1.0
+    assert math.isnan(v(0x7F)) and math.isnan(v(0xFF))
+
+
+def test_fp8_gate_up_hand_example(oracle_mod):
+    # x = [1, 2]; Wg = 0.5 * [1, 2] -> a = 0.5 * (1 + 4) = 2.5
+    #            Wu = 2 * [-1, 1]   -> u = 2 * (-1 + 2) = 2;  h = SiLU(2.5) * 2
+    h, a, u = oracle.gate_up_fp8(bits([[1.0, 2.0]]), fp8([[1.0, 2.0]]), [0.5],
+                                 fp8([[-1.0, 1.0]]), [2.0], return_au=True)
+    assert a[0, 0] == 2.5 and u[0, 0] == 2.0
+    assert h[0, 0] == pytest.approx(2.5 / (1 + math.exp(-2.5)) * 2.0, rel=1e-15)
+
+
+def test_fp8_unit_scale_reduces_to_bf16_path(oracle_mod):
+    # with s = 1 the dequantised weights are the E4M3 values, which bf16 holds
+    # exactly: the FP8 oracle must equal the bf16 oracle on those weights
+    rng = np.random.default_rng(21)
+    B, D, F = 3, 40, 24
+    x = oracle.f64_to_bf16(rng.standard_normal((B, D)))
+    g = oracle.f64_to_bf16(1.0 + 0.1 * rng.standard_normal(D))
+    qg = rng.integers(0, 256, (F, D)).astype(np.uint8)
+    qu = rng.integers(0, 256, (F, D)).astype(np.uint8)
+    qg[(qg & 0x7F) == 0x7F] = 0x38           # no NaN codes
+    qu[(qu & 0x7F) == 0x7F] = 0xB8
+    ones = np.ones(F, np.float32)
+    h8 = oracle.gate_up_fp8(x, qg, ones, qu, ones, gamma=g)
+    wg = oracle.f64_to_bf16(oracle.e4m3_to_f64(qg))
+    wu = oracle.f64_to_bf16(oracle.e4m3_to_f64(qu))
+    assert np.array_equal(oracle.bf16_to_f64(wg), oracle.e4m3_to_f64(qg))   # exact in bf16
+    assert np.array_equal(h8, oracle.gate_up(x, wg, wu, gamma=g))
+
+
+def test_fp8_scales_are_per_row_and_linear(oracle_mod):
+    rng = np.random.default_rng(22)
+    B, D, F = 2, 32, 16
+    x = oracle.f64_to_bf16(rng.standard_normal((B, D)))
+    qg = fp8(np.round(rng.standard_normal((F, D)) * 4) / 4)
+    qu = fp8(np.round(rng.standard_normal((F, D)) * 4) / 4)
+    sg = (0.01 * (1 + np.arange(F))).astype(np.float32)
+    su = np.full(F, 0.02, np.float32)
+    _, a1, u1 = oracle.gate_up_fp8(x, qg, sg, qu, su, return_au=True)
+    _, a2, u2 = oracle.gate_up_fp8(x, qg, 4 * sg, qu, su, return_au=True)
+    assert np.array_equal(4 * a1, a2) and np.array_equal(u1, u2)   # gate scale only
+    ref = oracle.bf16_to_f64(x) @ (oracle.e4m3_to_f64(qg) * sg.astype(np.float64)[:, None]).T
+    assert np.allclose(a1, ref, rtol=1e-13, atol=1e-14)
+    h = rng.standard_normal((B, F))
+    qd = fp8(np.round(rng.standard_normal((D, F)) * 2) / 2)
+    sd = (0.5 + np.arange(D)).astype(np.float32)
+    y1 = oracle.down_fp8(h, qd, sd)
+    assert np.array_equal(2 * y1, oracle.down_fp8(h, qd, 2 * sd))
+    assert np.allclose(y1, h @ (oracle.e4m3_to_f64(qd) * sd.astype(np.float64)[:, None]).T,
+                       rtol=1e-13, atol=1e-13)
