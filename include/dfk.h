@@ -72,7 +72,10 @@ typedef enum dfk_wlayout {
 typedef enum dfk_op {
   DFK_OP_GATE_UP = 0,         /* dfk_swiglu_gate_up          */
   DFK_OP_RMSNORM_GATE_UP = 1, /* dfk_rmsnorm_swiglu_gate_up  */
-  DFK_OP_DOWN = 2             /* dfk_down_proj               */
+  DFK_OP_DOWN = 2,            /* dfk_down_proj               */
+  DFK_OP_GATE_UP_FP8 = 3,     /* dfk_swiglu_gate_up_fp8      */
+  DFK_OP_RMSNORM_GATE_UP_FP8 = 4, /* dfk_rmsnorm_swiglu_gate_up_fp8 */
+  DFK_OP_DOWN_FP8 = 5         /* dfk_down_proj_fp8           */
 } dfk_op;
 
 typedef enum dfk_family {
@@ -154,6 +157,39 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
                                          int d_model, int d_ff, void *stream);
 
 /*
+ * FP8 weight streaming: the same three operations with weights stored as
+ * FP8 E4M3 codes and one fp32 scale per output row, dequantised inside the
+ * matrix-vector product (GPULlama3.java PR #78, "fusing dequantize with
+ * compute": no separate dequantise pass, no dequantised copy in memory).
+ * The weights are half the bytes of bf16, and the decode path is bound by
+ * reading them.
+ *   W[j][k] = s[j] * E4M3(q[j][k])
+ *   E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is
+ *   subnormal (m * 2^-9); S.1111.111 is NaN; no infinities; max 448.
+ *   q_gate, q_up  [d_ff][d_model] uint8 codes, row-major, device, 16-byte aligned
+ *   s_gate, s_up  [d_ff] fp32, device, 4-byte aligned
+ *   q_down        [d_model][d_ff] uint8 codes, row-major; s_down [d_model] fp32
+ *   x, gamma, h, y, eps: as for the bf16 entry points.
+ * Each code is widened to its exact fp32 value in registers; products and
+ * sums are fp32 in a fixed order; the row's sum is multiplied by s[j] once
+ * before SiLU and the bf16 rounding.  Constraints: row-major only; the
+ * reduction length (d_model for gate/up, d_ff for the down projection) a
+ * multiple of 16; CUDA-core variants only (a tensor-core id is rejected
+ * with DFK_ERR_INVALID_ARG); otherwise as for the bf16 entry points.
+ */
+DFK_API int dfk_swiglu_gate_up_fp8(const void *x, const void *q_gate, const float *s_gate,
+                                   const void *q_up, const float *s_up, void *h, int B,
+                                   int d_model, int d_ff, int variant, void *stream);
+
+DFK_API int dfk_rmsnorm_swiglu_gate_up_fp8(const void *x, const void *gamma, float eps,
+                                           const void *q_gate, const float *s_gate,
+                                           const void *q_up, const float *s_up, void *h, int B,
+                                           int d_model, int d_ff, int variant, void *stream);
+
+DFK_API int dfk_down_proj_fp8(const void *h, const void *q_down, const float *s_down, void *y,
+                              int B, int d_model, int d_ff, int variant, void *stream);
+
+/*
  * Profiler-driven variant choice ("Deep Kernel Fusion for Transformer
  * Decoding", episode description: runtime scheduling across row-major and
  * column-major kernel variants; "Deep Kernel Fusion for Transformers",
@@ -165,7 +201,10 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
  * the fastest layout in out->layout (gate/up ops only).
  *   sample_ptrs  NULL, or the caller's buffers in argument order of the op:
  *                gate_up: {x, w_gate, w_up, h}; rmsnorm_gate_up: {x, gamma,
- *                w_gate, w_up, h}; down: {h, w_down, y}.  With NULL (or with
+ *                w_gate, w_up, h}; down: {h, w_down, y}; the FP8 ops put
+ *                each scale right after its codes: {x, q_gate, s_gate, q_up,
+ *                s_up, h}, {x, gamma, q_gate, s_gate, q_up, s_up, h},
+ *                {h, q_down, s_down, y}.  With NULL (or with
  *                DFK_W_ANY) the function allocates throwaway buffers on
  *                `stream` and frees them before returning.
  * Returns DFK_ERR_INVALID_ARG if the stream is being captured.

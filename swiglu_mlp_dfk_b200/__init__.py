@@ -32,6 +32,9 @@ DFK_W_ANY = -1
 DFK_OP_GATE_UP = 0
 DFK_OP_RMSNORM_GATE_UP = 1
 DFK_OP_DOWN = 2
+DFK_OP_GATE_UP_FP8 = 3
+DFK_OP_RMSNORM_GATE_UP_FP8 = 4
+DFK_OP_DOWN_FP8 = 5
 # dfk_status
 DFK_OK = 0
 DFK_ERR_INVALID_ARG = 1
@@ -49,7 +52,9 @@ _LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W
 # Every symbol the header declares (the CPU test checks the library exports them all).
 EXPORTED = (
     "dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj", "dfk_select_variant",
-    "dfk_down_proj_static_scratch", "dfk_cached_variant", "dfk_variant_count", "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
+    "dfk_swiglu_gate_up_fp8", "dfk_rmsnorm_swiglu_gate_up_fp8", "dfk_down_proj_fp8",
+    "dfk_down_proj_static_scratch", "dfk_cached_variant", "dfk_variant_count",
+    "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
     "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
 )
@@ -96,6 +101,10 @@ def lib():
                 "dfk_rmsnorm_swiglu_gate_up": [vp, vp, f, vp, vp, i, vp, i, i, i, i, vp],
                 "dfk_down_proj": [vp, vp, vp, i, i, i, i, vp],
                 "dfk_down_proj_static_scratch": [vp, vp, vp, i, i, i, vp],
+                "dfk_swiglu_gate_up_fp8": [vp, vp, vp, vp, vp, vp, i, i, i, i, vp],
+                "dfk_rmsnorm_swiglu_gate_up_fp8": [vp, vp, f, vp, vp, vp, vp, vp, i, i, i, i,
+                                                   vp],
+                "dfk_down_proj_fp8": [vp, vp, vp, vp, i, i, i, i, vp],
                 "dfk_select_variant": [i, i, i, i, i, ctypes.POINTER(vp), vp,
                                        ctypes.POINTER(dfk_variant)],
                 "dfk_cached_variant": [i, i, i, i, i, ctypes.POINTER(dfk_variant)],
@@ -220,6 +229,68 @@ def dfk_down_proj_static_scratch(h, w_down, y=None, stream=None):
         y = torch.empty((B, D), dtype=torch.bfloat16, device=h.device)
     _check(lib().dfk_down_proj_static_scratch(_ptr(h), _ptr(w_down), _ptr(y), B, D, F,
                                               _stream(stream)))
+    return y
+
+
+def _dev_fp8(q, s, rows):
+    """FP8 weights: uint8 (or torch.float8_e4m3fn) codes [rows, K] and fp32 scales [rows]."""
+    if not isinstance(q, torch.Tensor) or not q.is_cuda or q.dim() != 2 or \
+            q.dtype not in (torch.uint8, torch.float8_e4m3fn) or not q.is_contiguous():
+        raise DfkError(DFK_ERR_INVALID_ARG, "FP8 weights must be contiguous 2-D uint8 or "
+                       "float8_e4m3fn CUDA tensors")
+    if not isinstance(s, torch.Tensor) or not s.is_cuda or s.dtype != torch.float32 or \
+            not s.is_contiguous() or s.numel() != rows:
+        raise DfkError(DFK_ERR_INVALID_ARG, "scales must be contiguous fp32 CUDA tensors of %d "
+                       "elements" % rows)
+
+
+def dfk_swiglu_gate_up_fp8(x, q_gate, s_gate, q_up, s_up, h=None, variant=0, stream=None):
+    """h = SiLU(x (s_g Q_g)^T) * (x (s_u Q_u)^T) with FP8 E4M3 codes Q [d_ff, d_model] and
+    fp32 row scales s [d_ff]; returns h [B, d_ff] bf16."""
+    _dev_bf16("x", x)
+    _dev_bf16("h", h)
+    B, D = x.shape
+    F = q_gate.shape[0]
+    _dev_fp8(q_gate, s_gate, F)
+    _dev_fp8(q_up, s_up, F)
+    if h is None:
+        h = torch.empty((B, F), dtype=torch.bfloat16, device=x.device)
+    _check(lib().dfk_swiglu_gate_up_fp8(_ptr(x), _ptr(q_gate), _ptr(s_gate), _ptr(q_up),
+                                        _ptr(s_up), _ptr(h), B, D, F, int(variant),
+                                        _stream(stream)))
+    return h
+
+
+def dfk_rmsnorm_swiglu_gate_up_fp8(x, gamma, eps, q_gate, s_gate, q_up, s_up, h=None, variant=0,
+                                   stream=None):
+    """RMSNorm(x; gamma, eps) fused in front of the FP8 gate/up kernel; returns h."""
+    _dev_bf16("x", x)
+    _dev_bf16("gamma", gamma)
+    _dev_bf16("h", h)
+    B, D = x.shape
+    F = q_gate.shape[0]
+    _dev_fp8(q_gate, s_gate, F)
+    _dev_fp8(q_up, s_up, F)
+    if h is None:
+        h = torch.empty((B, F), dtype=torch.bfloat16, device=x.device)
+    _check(lib().dfk_rmsnorm_swiglu_gate_up_fp8(_ptr(x), _ptr(gamma), float(eps), _ptr(q_gate),
+                                                _ptr(s_gate), _ptr(q_up), _ptr(s_up), _ptr(h),
+                                                B, D, F, int(variant), _stream(stream)))
+    return h
+
+
+def dfk_down_proj_fp8(h, q_down, s_down, y=None, variant=0, stream=None):
+    """y = h (s_d Q_d)^T with FP8 E4M3 codes Q_d [d_model, d_ff] and fp32 row scales s_d
+    [d_model]; returns y [B, d_model] bf16."""
+    _dev_bf16("h", h)
+    _dev_bf16("y", y)
+    B, F = h.shape
+    D = q_down.shape[0]
+    _dev_fp8(q_down, s_down, D)
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=h.device)
+    _check(lib().dfk_down_proj_fp8(_ptr(h), _ptr(q_down), _ptr(s_down), _ptr(y), B, D, F,
+                                   int(variant), _stream(stream)))
     return y
 
 

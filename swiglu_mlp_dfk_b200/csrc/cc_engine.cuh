@@ -30,7 +30,15 @@
 // With the RMSNorm prologue, xn = (x * r) * gamma stays in fp32 (it is not
 // rounded to bf16), so the products are fused multiply-adds of an fp32 and a
 // bf16 value; without it, x is bf16 and every product is exact in fp32.
-// Either way the result is fixed by the order above.  Tokens never interact, so row b of the
+// Either way the result is fixed by the order above.
+//
+// FP8 weights (W8, row-major only): W[j][k] = s[j] * Q[j][k] with Q in FP8
+// E4M3 and one fp32 scale per output row (GPULlama3.java PR #78: dequantize
+// inside the matrix-vector product instead of a separate pass).  A 128-byte
+// tile row then holds 128 codes, so the order becomes k = 128 t + 16 s + e
+// (e in [0, 16)); each code is converted to its exact fp32 value in
+// registers, the chains are the same fp32 fmas, and the row scale multiplies
+// the reduced sum once in the epilogue: out = s[j] * sum_k xn[k] Q[j][k].  Tokens never interact, so row b of the
 // output is independent of the batch size.
 #pragma once
 #include <cuda.h>
@@ -50,12 +58,14 @@ struct CcParams {
   const uint16_t *x;      // [B][K] bf16 activations
   const uint16_t *gamma;  // [K] bf16 RMSNorm weight (NORM only)
   uint16_t *out;          // [B][N] bf16
+  const float *scale[2];  // W8: per-output-row scales of each matrix [N] fp32
   unsigned *err;          // device error word
   int B, K, N;
   float eps;
   int nt;           // consecutive 64-wide tiles per team per ring stage (1, 2 or 4)
-  int nsteps;       // ring steps per pass = ceil(ceil(K/64) / (KSPLIT * nt))
-  int kpad;         // nsteps * KSPLIT * nt * 64: activation row pitch in shared memory
+  int nsteps;       // ring steps per pass = ceil(ceil(K/TK) / (KSPLIT * nt)), TK = 64
+                    // reduction elements per tile (128 with FP8 weights)
+  int kpad;         // nsteps * KSPLIT * nt * TK: activation row pitch in shared memory
   int granule;      // output rows per partition unit
   int ubase, uextra;// units per CTA: ubase, +1 for the first uextra CTAs
   int r_hi;         // largest row count of any CTA (shared-memory slot size)
@@ -82,10 +92,13 @@ struct CcAcc {
 // accumulators of one row (NMAT = 2) or two adjacent rows (NMAT = 1) share a
 // packed register, the activation is broadcast into both lanes.  Each lane
 // performs the same fma sequence as the scalar path: results are identical.
-template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NORM, bool PAIR>
+template <int LAYOUT, int NMAT, int JPT, int BT, int KSPLIT, bool XF32, bool NORM, bool PAIR,
+          bool W8 = false>
 __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     cc_gemv_kernel(const __grid_constant__ CcMaps maps, const CcParams p) {
   static_assert(LAYOUT != LAYOUT_IL || NMAT == 2, "interleaved layout holds both matrices");
+  static_assert(!W8 || LAYOUT == LAYOUT_ROW, "FP8 weights are row-major");
+  constexpr int TK = W8 ? 2 * TILE_K : TILE_K;  // reduction elements per 128-byte tile row
   static_assert(XF32 || !NORM, "normalised activations are kept in fp32");
   constexpr int NPAIR = PAIR ? (NMAT == 2 ? JPT : JPT / 2) : 1;
   static_assert(JPT == 2 || JPT == 4, "JPT");
@@ -143,7 +156,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
         mbar_arrive_expect_tx(&full[st], tx);
 #pragma unroll
         for (int kt = 0; kt < KSPLIT; ++kt) {
-          const int k0 = (step * KSPLIT + kt) * nt * TILE_K;
+          const int k0 = (step * KSPLIT + kt) * nt * TK;
           uint8_t *tb = base + static_cast<size_t>(kt) * NMAT * slot_bytes;
           if (LAYOUT == LAYOUT_ROW) {
 #pragma unroll
@@ -299,6 +312,80 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
           const int t = (step * KSPLIT + team) * nt + tt;
           const uint8_t *tb = smem + static_cast<size_t>(st) * p.stage_bytes +
                               static_cast<size_t>(team) * NMAT * slot_bytes;
+          if constexpr (W8) {
+            // slot s of 128-wide tile t: k = 128 t + 16 s + e, taken as two halves
+            // of 8 (e ascending); 16 codes per row per thread
+            uint32_t wq[NMAT][JPT][4];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+              for (int jj = 0; jj < JPT; ++jj) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(
+                    tb + m * slot_bytes + (jl0 + jj) * rowb + tt * (TILE_K * 2) + s * 16);
+                wq[m][jj][0] = v.x; wq[m][jj][1] = v.y; wq[m][jj][2] = v.z; wq[m][jj][3] = v.w;
+              }
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              float xv[BT][8];
+#pragma unroll
+              for (int bb = 0; bb < BT; ++bb) {
+                if (XF32) {
+                  // 64-wide tile 2 t + s / 4, 8-element chunk (2 s + hf) mod 8
+                  const int c = (2 * s + hf) & 7;
+                  const float *row =
+                      xs_f + static_cast<size_t>(bb) * p.kpad + (2 * t + (s >> 2)) * TILE_K;
+                  const float4 lo = *reinterpret_cast<const float4 *>(row + 4 * c);
+                  const float4 hi = *reinterpret_cast<const float4 *>(row + 32 + 4 * c);
+                  xv[bb][0] = lo.x; xv[bb][1] = lo.y; xv[bb][2] = lo.z; xv[bb][3] = lo.w;
+                  xv[bb][4] = hi.x; xv[bb][5] = hi.y; xv[bb][6] = hi.z; xv[bb][7] = hi.w;
+                } else {
+                  const uint4 v = *reinterpret_cast<const uint4 *>(
+                      xs_h + static_cast<size_t>(bb) * p.kpad + t * TK + 16 * s + 8 * hf);
+                  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                  for (int ii = 0; ii < 4; ++ii) {
+                    xv[bb][2 * ii] = bf16_lo(w[ii]);
+                    xv[bb][2 * ii + 1] = bf16_hi(w[ii]);
+                  }
+                }
+              }
+#pragma unroll
+              for (int wi = 0; wi < 2; ++wi) {  // code word 2 hf + wi: elements 4 wi .. 4 wi + 3
+                float wf[NMAT][JPT][4];
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                  for (int jj = 0; jj < JPT; ++jj) e4m3x4_to_f32(wq[m][jj][2 * hf + wi], wf[m][jj]);
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                  const int e = 4 * wi + e4;
+                  if constexpr (PAIR) {
+                    uint64_t xd[BT];
+#pragma unroll
+                    for (int bb = 0; bb < BT; ++bb) xd[bb] = pack_f32x2(xv[bb][e], xv[bb][e]);
+#pragma unroll
+                    for (int pr = 0; pr < NPAIR; ++pr) {
+                      const int m1 = NMAT - 1, j0r = (NMAT == 2) ? pr : 2 * pr;
+                      const int j1r = (NMAT == 2) ? pr : 2 * pr + 1;
+                      const uint64_t wp = pack_f32x2(wf[0][j0r][e4], wf[m1][j1r][e4]);
+#pragma unroll
+                      for (int bb = 0; bb < BT; ++bb)
+                        acc2[pr][bb] = fma_f32x2(xd[bb], wp, acc2[pr][bb]);
+                    }
+                  } else {
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                      for (int jj = 0; jj < JPT; ++jj)
+#pragma unroll
+                        for (int bb = 0; bb < BT; ++bb)
+                          acc.v[m][jj][bb] = fmaf(xv[bb][e], wf[m][jj][e4], acc.v[m][jj][bb]);
+                  }
+                }
+              }
+            }
+            continue;
+          }
           float xv[BT][8];
 #pragma unroll
           for (int bb = 0; bb < BT; ++bb) {
@@ -494,6 +581,10 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
           v[m] = tot;
         }
         if (!aborted && b < p.B && j < p.N) {
+          if constexpr (W8) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) v[m] *= __ldg(p.scale[m] + j);
+          }
           float res;
           if (NMAT == 2) {
             const float a = v[0];

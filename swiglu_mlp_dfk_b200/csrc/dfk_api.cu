@@ -88,6 +88,9 @@ const void *cc_find_kernel(int key) {
   if ((f = cc_lookup_il(key))) return f;
   if ((f = cc_lookup_gemv_a(key))) return f;
   if ((f = cc_lookup_gemv_b(key))) return f;
+  if ((f = cc_lookup_fp8_gate_up(key))) return f;
+  if ((f = cc_lookup_fp8_gemv_a(key))) return f;
+  if ((f = cc_lookup_fp8_gemv_b(key))) return f;
   return nullptr;
 }
 
@@ -161,21 +164,22 @@ static int get_encoder() {
   return DFK_OK;
 }
 
-// key: pointer, rank, dims[3], strides[2], box[3], swizzle
+// key: pointer, rank, dims[3], strides[2], box[3], swizzle, element type
 using MapKey = std::tuple<uintptr_t, int, uint64_t, uint64_t, uint64_t, uint64_t, uint64_t,
-                          uint32_t, uint32_t, uint32_t, int>;
+                          uint32_t, uint32_t, uint32_t, int, int>;
 static std::map<MapKey, CUtensorMap> g_maps;
 
-// bf16 tensor map of rank 2 or 3: dims[0] contiguous elements, strides in
-// bytes for dims 1.., box extents, 128-byte swizzle or none, zero fill
-// outside the tensor.
+// Tensor map of rank 2 or 3 (bf16 elements, or bytes for FP8 weights):
+// dims[0] contiguous elements, strides in bytes for dims 1.., box extents,
+// 128-byte swizzle or none, zero fill outside the tensor.
 static int tensor_map(const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
-                      const uint32_t *box, bool sw128, CUtensorMap *out) {
+                      const uint32_t *box, bool sw128, CUtensorMap *out,
+                      CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   int rc = get_encoder();
   if (rc) return rc;
   MapKey key{reinterpret_cast<uintptr_t>(ptr), rank, dims[0], dims[1], rank > 2 ? dims[2] : 0,
              strides[0], rank > 2 ? strides[1] : 0, box[0], box[1], rank > 2 ? box[2] : 0,
-             sw128 ? 1 : 0};
+             sw128 ? 1 : 0, static_cast<int>(dt)};
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_maps.find(key);
@@ -189,7 +193,7 @@ static int tensor_map(const void *ptr, int rank, const uint64_t *dims, const uin
   cuuint64_t st[2] = {strides[0], rank > 2 ? strides[1] : 0};
   cuuint32_t bx[3] = {box[0], box[1], rank > 2 ? box[2] : 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+  CUresult r = g_encode(&m, dt, static_cast<cuuint32_t>(rank),
                         const_cast<void *>(ptr), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -204,15 +208,16 @@ static int tensor_map(const void *ptr, int rank, const uint64_t *dims, const uin
   return DFK_OK;
 }
 
-// 2-D bf16 tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
+// 2-D tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
 // between rows, box of box_inner x box_outer.
 static int tensor_map_2d(const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
                          uint32_t box_inner, uint32_t box_outer, CUtensorMap *out,
-                         bool sw128 = false) {
+                         bool sw128 = false,
+                         CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   const uint64_t dims[2] = {inner, outer};
   const uint64_t strides[1] = {pitch};
   const uint32_t box[2] = {box_inner, box_outer};
-  return tensor_map(ptr, 2, dims, strides, box, sw128, out);
+  return tensor_map(ptr, 2, dims, strides, box, sw128, out, dt);
 }
 
 // ---------------------------------------------------------------- variants
@@ -289,8 +294,15 @@ static int ceil_div(int a, int b) { return (a + b - 1) / b; }
 static int round_up(int a, int b) { return ceil_div(a, b) * b; }
 
 // Partition N output rows over the SMs and size the shared-memory ring.
-static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
-                    const DeviceState &ds, CcPlan *pl, std::string *why) {
+static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int B, int K,
+                    int N, const DeviceState &ds, CcPlan *pl, std::string *why) {
+  // FP8 weights: 128 codes per 128-byte tile row; the TMA box is at most 256
+  // elements wide, so at most two tiles per stage
+  const int tk = w8 ? 2 * TILE_K : TILE_K;
+  if (w8 && (layout != LAYOUT_ROW || v.nt > 2)) {
+    if (why) *why = "FP8 weights: row-major, at most two tiles per stage";
+    return false;
+  }
   const int g = (layout == LAYOUT_COL) ? 8 : 4;
   const int U = ceil_div(N, g);
   const int smem_cap = std::min(ds.smem_optin, 232448);
@@ -304,9 +316,9 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     const int tpt = (layout == LAYOUT_COL) ? 256 * ceil_div(nq, 32) : round_up(8 * nq, 32);
     const int ncons = v.ksplit * tpt;
     if (ncons + 32 > CC_MAX_THREADS) continue;
-    const int nT = ceil_div(K, TILE_K);
+    const int nT = ceil_div(K, tk);
     const int nsteps = ceil_div(nT, v.ksplit * v.nt);
-    const int kpad = nsteps * v.ksplit * v.nt * TILE_K;
+    const int kpad = nsteps * v.ksplit * v.nt * tk;
     const int stage_bytes = v.ksplit * nmat * r_hi * TILE_K * 2 * v.nt;
     const int red_bytes = v.ksplit * (layout == LAYOUT_COL ? NSLOT : 1) * nmat * v.bt * r_hi * 4;
     const int bar_bytes = 256;
@@ -327,7 +339,7 @@ static bool plan_cc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       continue;
     }
     const int key = DFK_CC_KEY(layout, nmat, v.jpt, v.bt, v.ksplit, best_xf32 ? 1 : 0,
-                               norm ? 1 : 0, v.pair ? 1 : 0);
+                               norm ? 1 : 0, v.pair ? 1 : 0) | (w8 ? DFK_CC_KEY_W8 : 0);
     const void *fn = cc_find_kernel(key);
     if (!fn) {
       if (why) *why = "variant not compiled for this layout";
@@ -389,6 +401,8 @@ struct CcCall {
   const void *w0, *w1;
   void *out;
   int B, K, N;
+  bool w8 = false;               // FP8 E4M3 weights (row-major), per-row scales below
+  const float *s0 = nullptr, *s1 = nullptr;
 };
 
 static bool pdl_enabled() { return env_flag("DFK_PDL", true); }
@@ -400,7 +414,7 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   if (rc) return rc;
   CcPlan pl;
   std::string why;
-  if (!plan_cc(c.layout, c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
+  if (!plan_cc(c.layout, c.nmat, c.norm, c.w8, v, c.B, c.K, c.N, *ds, &pl, &why))
     return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit B=%d K=%d N=%d: %s", v.id, c.B,
                 c.K, c.N, why.c_str());
   if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
@@ -408,11 +422,14 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   memset(&maps, 0, sizeof maps);
   const int r_hi = pl.p.r_hi, r_lo = pl.r_lo > 0 ? pl.r_lo : pl.p.r_hi;
   const void *w[2] = {c.w0, c.w1};
-  const uint32_t kbox = TILE_K * v.nt;
+  const uint32_t kbox = (c.w8 ? 2 * TILE_K : TILE_K) * v.nt;
   for (int m = 0; m < (c.layout == LAYOUT_IL ? 1 : c.nmat); ++m) {
     for (int lo = 0; lo < 2; ++lo) {
       const uint32_t r = lo ? r_lo : r_hi;
-      if (c.layout == LAYOUT_ROW)
+      if (c.w8)
+        rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K), kbox, r,
+                           &maps.m[m * 2 + lo], false, CU_TENSOR_MAP_DATA_TYPE_UINT8);
+      else if (c.layout == LAYOUT_ROW)
         rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K) * 2, kbox, r,
                            &maps.m[m * 2 + lo]);
       else if (c.layout == LAYOUT_COL)
@@ -428,6 +445,8 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   p.x = static_cast<const uint16_t *>(c.x);
   p.gamma = static_cast<const uint16_t *>(c.gamma);
   p.out = static_cast<uint16_t *>(c.out);
+  p.scale[0] = c.s0;
+  p.scale[1] = c.s1;
   p.err = ds->err;
   p.eps = c.eps;
   void *args[] = {&maps, &p};
@@ -607,6 +626,8 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   int dev;
   int rc = current_device(&ds, &dev);
   if (rc) return rc;
+  if (c.w8)
+    return fail(DFK_ERR_NO_VARIANT, "variant %d: FP8 weights run on the CUDA-core family", v.id);
   TcPlan pl;
   std::string why;
   if (!plan_tc(c.layout, c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
@@ -763,7 +784,14 @@ struct TuneKey {
 static std::mutex g_tune_mu;
 static std::map<TuneKey, dfk_variant> g_tuned;
 
-static int op_class(int op) { return op == DFK_OP_DOWN ? CLS_GEMV : CLS_GATE_UP; }
+static bool op_is_down(int op) { return op == DFK_OP_DOWN || op == DFK_OP_DOWN_FP8; }
+static bool op_is_fp8(int op) {
+  return op == DFK_OP_GATE_UP_FP8 || op == DFK_OP_RMSNORM_GATE_UP_FP8 || op == DFK_OP_DOWN_FP8;
+}
+static bool op_is_norm(int op) {
+  return op == DFK_OP_RMSNORM_GATE_UP || op == DFK_OP_RMSNORM_GATE_UP_FP8;
+}
+static int op_class(int op) { return op_is_down(op) ? CLS_GEMV : CLS_GATE_UP; }
 
 static void fill_variant(const VDef &d, int op, int layout, int stages, float us,
                          dfk_variant *out) {
@@ -825,7 +853,8 @@ static void tune_cache_load(int dev, int sms) {  // caller holds g_tune_mu
     if (std::string(name) + " " + std::to_string(n_sms) + " " + std::to_string(drv) != tag)
       continue;
     const VDef *d = find_variant(vid);
-    if (!d || d->cls != op_class(op) || B < 1 || B > 64) {
+    if (!d || d->cls != op_class(op) || B < 1 || B > 64 ||
+        (op_is_fp8(op) && d->family != DFK_FAMILY_CUDA_CORE)) {
       ++bad;
       continue;
     }
@@ -858,11 +887,13 @@ static void tune_cache_append(int dev, int sms, const TuneKey &k, const dfk_vari
 // Candidates worth timing for (op, B): every CUDA-core j-per-thread / k-split
 // / tiles-per-stage / pairing choice at its largest useful token tile, plus the
 // tensor-core variants from B = 4 (gate/up) or B = 2 (GEMV); at B = 1 fp32
-// FMA on CUDA cores keeps up with HBM.
+// FMA on CUDA cores keeps up with HBM.  FP8 weights: CUDA-core variants with
+// one or two tiles per stage only.
 static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
   std::vector<const VDef *> out;
   for (const VDef &d : variants()) {
     if (d.cls != op_class(op)) continue;
+    if (c.w8 && (d.family == DFK_FAMILY_TENSOR_CORE || d.nt > 2)) continue;
     if (d.family == DFK_FAMILY_TENSOR_CORE) {
       // gate/up from B = 4 (where CUDA cores fall below HBM speed), the GEMV
       // (split-K) from B = 2
@@ -877,11 +908,12 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
 
 static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
   if (d.family == DFK_FAMILY_TENSOR_CORE) {
+    if (c.w8) return false;
     TcPlan pl;
     return plan_tc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
   }
   CcPlan pl;
-  return plan_cc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+  return plan_cc(c.layout, c.nmat, c.norm, c.w8, d, c.B, c.K, c.N, ds, &pl, nullptr);
 }
 
 // Heuristic default (no timing): the tensor-core family from B = 8 up (one
@@ -890,7 +922,7 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // the GEMV the largest k split whose CTA fits.  If nothing of that shape
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
-  if (B >= 8) {
+  if (B >= 8 && !c.w8) {
     const bool gemv = op_class(op) == CLS_GEMV;
     const int want_nt = gemv ? 2 : 1, want_ks = gemv ? 4 : 1;
     for (const VDef &d : variants())
@@ -1001,11 +1033,13 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
     const VDef *d = find_variant(variant);
     if (!d || d->cls != op_class(op))
       return fail(DFK_ERR_INVALID_ARG, "variant %d is not a variant of op %d", variant, op);
+    if (c.w8 && d->family == DFK_FAMILY_TENSOR_CORE)
+      return fail(DFK_ERR_INVALID_ARG, "variant %d: FP8 weights run on CUDA-core variants",
+                  variant);
     *out = d;
     return DFK_OK;
   }
-  TuneKey key{dev, op, c.B, op == DFK_OP_DOWN ? c.N : c.K, op == DFK_OP_DOWN ? c.K : c.N,
-              c.layout};
+  TuneKey key{dev, op, c.B, op_is_down(op) ? c.N : c.K, op_is_down(op) ? c.K : c.N, c.layout};
   {
     std::lock_guard<std::mutex> lk(g_tune_mu);
     tune_cache_load(dev, ds->sms);
@@ -1119,6 +1153,51 @@ static int gemv_impl(int op, const void *x, const void *w, void *out, int B, int
   return launch_variant(c, *v, s, nullptr);
 }
 
+// FP8 weights: row-major E4M3 codes (1 byte each) and fp32 row scales.
+static int check_fp8(const void *x, const void *gamma, bool norm, float eps, const void *q0,
+                     const float *s0, const void *q1, const float *s1, const void *out, int B,
+                     int K, int N, int variant, int cls) {
+  if (B < 0 || K <= 0 || N <= 0) return fail(DFK_ERR_INVALID_ARG, "negative or zero size");
+  if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
+  if (variant > 0) {
+    const VDef *d = find_variant(variant);
+    if (!d || d->cls != cls || d->family != DFK_FAMILY_CUDA_CORE)
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a CUDA-core variant of this op",
+                  variant);
+  }
+  if (norm && !(eps >= 0.f && std::isfinite(eps)))
+    return fail(DFK_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (B > 64) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "B=%d > 64 (decode batches only)", B);
+  if (K % 16)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "FP8 weights: reduction length %% 16 != 0 (%d)", K);
+  if (B == 0) return DFK_OK;
+  const bool two = cls == CLS_GATE_UP;
+  if (!x || !q0 || !s0 || !out || (norm && !gamma) || (two && (!q1 || !s1)))
+    return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if (misaligned(x) || misaligned(q0) || misaligned(out) || (two && misaligned(q1)) ||
+      (norm && misaligned(gamma)))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(s0) | reinterpret_cast<uintptr_t>(s1)) & 3u)
+    return fail(DFK_ERR_MISALIGNED, "scale pointers must be 4-byte aligned");
+  return DFK_OK;
+}
+
+static int fp8_impl(int op, const void *x, const void *gamma, float eps, const void *q0,
+                    const float *s0, const void *q1, const float *s1, void *out, int B, int K,
+                    int N, int variant, cudaStream_t s) {
+  const bool down = op_is_down(op), norm = op_is_norm(op);
+  int rc = check_fp8(x, gamma, norm, eps, q0, s0, q1, s1, out, B, K, N, variant,
+                     down ? CLS_GEMV : CLS_GATE_UP);
+  if (rc || B == 0) return rc;
+  CcCall c{LAYOUT_ROW, down ? 1 : 2, norm, x, gamma, eps, q0, down ? nullptr : q1, out, B, K, N};
+  c.w8 = true;
+  c.s0 = s0;
+  c.s1 = down ? nullptr : s1;
+  const VDef *v = nullptr;
+  if ((rc = resolve(op, variant, c, s, &v))) return rc;
+  return launch_variant(c, *v, s, nullptr);
+}
+
 }  // namespace dfk
 
 using namespace dfk;
@@ -1146,6 +1225,27 @@ int dfk_down_proj(const void *h, const void *w_down, void *y, int B, int d_model
                    static_cast<cudaStream_t>(stream));
 }
 
+int dfk_swiglu_gate_up_fp8(const void *x, const void *q_gate, const float *s_gate,
+                           const void *q_up, const float *s_up, void *h, int B, int d_model,
+                           int d_ff, int variant, void *stream) {
+  return fp8_impl(DFK_OP_GATE_UP_FP8, x, nullptr, 0.f, q_gate, s_gate, q_up, s_up, h, B,
+                  d_model, d_ff, variant, static_cast<cudaStream_t>(stream));
+}
+
+int dfk_rmsnorm_swiglu_gate_up_fp8(const void *x, const void *gamma, float eps,
+                                   const void *q_gate, const float *s_gate, const void *q_up,
+                                   const float *s_up, void *h, int B, int d_model, int d_ff,
+                                   int variant, void *stream) {
+  return fp8_impl(DFK_OP_RMSNORM_GATE_UP_FP8, x, gamma, eps, q_gate, s_gate, q_up, s_up, h, B,
+                  d_model, d_ff, variant, static_cast<cudaStream_t>(stream));
+}
+
+int dfk_down_proj_fp8(const void *h, const void *q_down, const float *s_down, void *y, int B,
+                      int d_model, int d_ff, int variant, void *stream) {
+  return fp8_impl(DFK_OP_DOWN_FP8, h, nullptr, 0.f, q_down, s_down, nullptr, nullptr, y, B,
+                  d_ff, d_model, variant, static_cast<cudaStream_t>(stream));
+}
+
 int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int variant,
              void *stream) {
   return gemv_impl(DFK_OP_DOWN, x, w, out, B, K, N, variant, static_cast<cudaStream_t>(stream));
@@ -1154,17 +1254,20 @@ int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int v
 int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
                        const void *const *sample_ptrs, void *stream, dfk_variant *out) {
   if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
-  if (op != DFK_OP_GATE_UP && op != DFK_OP_RMSNORM_GATE_UP && op != DFK_OP_DOWN)
+  if (op < DFK_OP_GATE_UP || op > DFK_OP_DOWN_FP8)
     return fail(DFK_ERR_INVALID_ARG, "unknown op %d", op);
+  const bool down = op_is_down(op), w8 = op_is_fp8(op), norm = op_is_norm(op);
   if (B <= 0 || B > 64 || d_model <= 0 || d_ff <= 0)
     return fail(DFK_ERR_UNSUPPORTED_SHAPE, "bad shape B=%d d_model=%d d_ff=%d", B, d_model, d_ff);
-  if (op == DFK_OP_DOWN && layout != DFK_W_ROW_MAJOR && layout != DFK_W_ANY)
-    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "the down projection reads row-major W_down");
+  if ((down || w8) && layout != DFK_W_ROW_MAJOR && layout != DFK_W_ANY)
+    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "op %d reads row-major weights only", op);
   if (layout != DFK_W_ANY && layout != DFK_W_ROW_MAJOR && layout != DFK_W_COL_MAJOR &&
       layout != DFK_W_GU_INTERLEAVED)
     return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "layout %d", layout);
-  if (d_model % 8 || (op == DFK_OP_DOWN && d_ff % 8))
+  if (d_model % 8 || (down && d_ff % 8))
     return fail(DFK_ERR_UNSUPPORTED_SHAPE, "sizes must be multiples of 8");
+  if (w8 && (down ? d_ff : d_model) % 16)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "FP8 weights: reduction length %% 16 != 0");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   DeviceState *ds;
   int dev;
@@ -1174,54 +1277,64 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
     return fail(DFK_ERR_INVALID_ARG, "dfk_select_variant cannot time inside stream capture");
 
   std::vector<int> layouts;
-  if (op == DFK_OP_DOWN) layouts = {DFK_W_ROW_MAJOR};
+  if (down || w8) layouts = {DFK_W_ROW_MAJOR};
   else if (layout == DFK_W_ANY) layouts = {DFK_W_ROW_MAJOR, DFK_W_COL_MAJOR, DFK_W_GU_INTERLEAVED};
   else layouts = {layout};
 
-  const size_t xb = static_cast<size_t>(B) * (op == DFK_OP_DOWN ? d_ff : d_model) * 2;
-  const size_t wb = static_cast<size_t>(d_model) * d_ff * 2;
-  const size_t ob = static_cast<size_t>(B) * (op == DFK_OP_DOWN ? d_model : d_ff) * 2;
+  const int K = down ? d_ff : d_model, N = down ? d_model : d_ff, nmat = down ? 1 : 2;
+  const size_t xb = static_cast<size_t>(B) * K * 2;
+  const size_t wb = static_cast<size_t>(d_model) * d_ff * (w8 ? 1 : 2);
+  const size_t ob = static_cast<size_t>(B) * N * 2;
+  const size_t sb = w8 ? static_cast<size_t>(N) * sizeof(float) : 0;
   bool best_set = false;
   dfk_variant best{};
   for (int L : layouts) {
     if (L == DFK_W_COL_MAJOR && d_ff % 8) continue;
     const bool own = !sample_ptrs || layout == DFK_W_ANY;
-    void *bx = nullptr, *bg = nullptr, *bw0 = nullptr, *bw1 = nullptr, *bo = nullptr;
-    const void *px, *pg = nullptr, *pw0, *pw1 = nullptr;
-    void *po;
+    void *bx = nullptr, *bg = nullptr, *bw = nullptr, *bo = nullptr, *bs = nullptr;
+    const void *px = nullptr, *pg = nullptr, *pw0 = nullptr, *pw1 = nullptr;
+    const float *ps0 = nullptr, *ps1 = nullptr;
+    void *po = nullptr;
     if (own) {
       cudaError_t e = cudaMallocAsync(&bx, xb, s);
       if (!e) e = cudaMallocAsync(&bo, ob, s);
-      if (!e && op == DFK_OP_RMSNORM_GATE_UP) e = cudaMallocAsync(&bg, d_model * 2, s);
-      if (!e) e = cudaMallocAsync(&bw0, op == DFK_OP_DOWN ? wb : 2 * wb, s);
+      if (!e && norm) e = cudaMallocAsync(&bg, d_model * 2, s);
+      if (!e) e = cudaMallocAsync(&bw, nmat * wb, s);
+      if (!e && w8) e = cudaMallocAsync(&bs, nmat * sb, s);
       if (e) {
         cudaGetLastError();
-        if (bx) cudaFreeAsync(bx, s);
-        if (bo) cudaFreeAsync(bo, s);
-        if (bg) cudaFreeAsync(bg, s);
-        if (bw0) cudaFreeAsync(bw0, s);
+        for (void *q : {bx, bo, bg, bw, bs})
+          if (q) cudaFreeAsync(q, s);
         return cuda_fail(e, "cudaMallocAsync (tuning buffers)");
       }
       cudaMemsetAsync(bx, 0, xb, s);
       if (bg) cudaMemsetAsync(bg, 0, d_model * 2, s);
-      cudaMemsetAsync(bw0, 0, op == DFK_OP_DOWN ? wb : 2 * wb, s);
-      bw1 = (op == DFK_OP_DOWN || L == DFK_W_GU_INTERLEAVED) ? nullptr
-                                                              : static_cast<char *>(bw0) + wb;
-      px = bx; pg = bg; pw0 = bw0; pw1 = bw1; po = bo;
-    } else if (op == DFK_OP_DOWN) {
-      px = sample_ptrs[0]; pw0 = sample_ptrs[1]; po = const_cast<void *>(sample_ptrs[2]);
-    } else if (op == DFK_OP_GATE_UP) {
-      px = sample_ptrs[0]; pw0 = sample_ptrs[1]; pw1 = sample_ptrs[2];
-      po = const_cast<void *>(sample_ptrs[3]);
+      cudaMemsetAsync(bw, 0, nmat * wb, s);
+      if (bs) cudaMemsetAsync(bs, 0, nmat * sb, s);
+      px = bx; pg = bg; po = bo; pw0 = bw;
+      pw1 = (down || L == DFK_W_GU_INTERLEAVED) ? nullptr : static_cast<char *>(bw) + wb;
+      ps0 = static_cast<const float *>(bs);
+      ps1 = (bs && !down) ? static_cast<const float *>(bs) + N : nullptr;
     } else {
-      px = sample_ptrs[0]; pg = sample_ptrs[1]; pw0 = sample_ptrs[2]; pw1 = sample_ptrs[3];
-      po = const_cast<void *>(sample_ptrs[4]);
+      // argument order of the op's entry point
+      int i = 0;
+      px = sample_ptrs[i++];
+      if (norm) pg = sample_ptrs[i++];
+      pw0 = sample_ptrs[i++];
+      if (w8) ps0 = static_cast<const float *>(sample_ptrs[i++]);
+      if (!down) {
+        pw1 = sample_ptrs[i++];
+        if (w8) ps1 = static_cast<const float *>(sample_ptrs[i++]);
+      }
+      po = const_cast<void *>(sample_ptrs[i++]);
     }
     CcCall c;
-    if (op == DFK_OP_DOWN) c = CcCall{LAYOUT_ROW, 1, false, px, nullptr, 0.f, pw0, nullptr, po,
-                                      B, d_ff, d_model};
-    else c = CcCall{to_engine_layout(L), 2, op == DFK_OP_RMSNORM_GATE_UP, px, pg, 1e-5f, pw0,
-                    L == DFK_W_GU_INTERLEAVED ? nullptr : pw1, po, B, d_model, d_ff};
+    if (down) c = CcCall{LAYOUT_ROW, 1, false, px, nullptr, 0.f, pw0, nullptr, po, B, K, N};
+    else c = CcCall{to_engine_layout(L), 2, norm, px, pg, 1e-5f, pw0,
+                    L == DFK_W_GU_INTERLEAVED ? nullptr : pw1, po, B, K, N};
+    c.w8 = w8;
+    c.s0 = ps0;
+    c.s1 = ps1;
     float us = -1.f;
     int stages = 0;
     const VDef *win = time_candidates(op, c, candidates(op, B, c), s, *ds, &us, &stages);
@@ -1230,10 +1343,8 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
       us = -1.f;
     }
     if (own) {
-      cudaFreeAsync(bx, s);
-      cudaFreeAsync(bo, s);
-      if (bg) cudaFreeAsync(bg, s);
-      cudaFreeAsync(bw0, s);
+      for (void *q : {bx, bo, bg, bw, bs})
+        if (q) cudaFreeAsync(q, s);
       cudaStreamSynchronize(s);
     }
     if (!win) continue;

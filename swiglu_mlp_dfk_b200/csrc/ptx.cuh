@@ -127,6 +127,29 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Four FP8 E4M3 codes (byte i of w = element i) -> their fp32 values.  Each
+// pair goes through the hardware E4M3x2 -> f16x2 conversion and then f16 ->
+// f32; both steps are exact (every E4M3 value, subnormals included, is an
+// f16 value), so f[i] is the code's value with no rounding.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
+  uint32_t h01, h23;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(h01), "=r"(h23)
+      : "r"(w));
+  asm("{\n\t.reg .b16 a, b, c, d;\n\t"
+      "mov.b32 {a, b}, %4;\n\t"
+      "mov.b32 {c, d}, %5;\n\t"
+      "cvt.f32.f16 %0, a;\n\t"
+      "cvt.f32.f16 %1, b;\n\t"
+      "cvt.f32.f16 %2, c;\n\t"
+      "cvt.f32.f16 %3, d;\n\t}"
+      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
+      : "r"(h01), "r"(h23));
+}
+
 // Two fp32 values in one 64-bit register (lo = first element).
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   uint64_t r;

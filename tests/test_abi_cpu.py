@@ -110,6 +110,28 @@ MIS = ctypes.c_void_p(0x10008)
     (lambda L: L.dfk_down_proj(P, P2, P3, 1, 64, 64, 1, None),   # id 1 is a gate/up variant
      dfk.DFK_ERR_INVALID_ARG),
     (lambda L: L.dfk_silu(P, P2, -5, None), dfk.DFK_ERR_INVALID_ARG),
+    # FP8 weights: reduction length % 16, null scales, misaligned scales, tensor-core ids
+    (lambda L: L.dfk_swiglu_gate_up_fp8(P, P2, P3, P2, P3, P, 1, 72, 64, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_swiglu_gate_up_fp8(P, P2, None, P2, P3, P, 1, 64, 64, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_swiglu_gate_up_fp8(P, P2, P3, P2, ctypes.c_void_p(0x30002), P, 1, 64, 64,
+                                        0, None), dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_swiglu_gate_up_fp8(P, P2, P3, P2, P3, P, 65, 64, 64, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_rmsnorm_swiglu_gate_up_fp8(P, None, 1e-5, P2, P3, P2, P3, P, 1, 64, 64, 0,
+                                                None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_swiglu_gate_up_fp8(P, P, 1e-5, P2, P3, P2, P3, P, 1, 64, 64,
+                                                dfk.dfk_variant_count(), None),
+     dfk.DFK_ERR_INVALID_ARG),                              # last id: a tensor-core GEMV
+    (lambda L: L.dfk_down_proj_fp8(P, P2, P3, P, 1, 64, 72, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_down_proj_fp8(P, MIS, P3, P, 1, 64, 64, 0, None), dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_down_proj_fp8(P, P2, P3, P, 1, 64, 64, 1, None),   # gate/up id
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_select_variant(dfk.DFK_OP_DOWN_FP8, 1, 64, 64, 1, None, None,
+                                    ctypes.byref(dfk.dfk_variant())),
+     dfk.DFK_ERR_UNSUPPORTED_LAYOUT),
     (lambda L: L.dfk_select_variant(9, 1, 64, 64, 0, None, None, None), dfk.DFK_ERR_INVALID_ARG),
 ])
 def test_validation_rejects_without_launch(L, call, status):
@@ -121,6 +143,8 @@ def test_empty_batch_is_a_no_op(L):
     assert L.dfk_swiglu_gate_up(None, P2, P3, 0, None, 0, 64, 64, 0, None) == dfk.DFK_OK
     assert L.dfk_down_proj(None, P2, None, 0, 64, 64, 0, None) == dfk.DFK_OK
     assert L.dfk_silu(None, None, 0, None) == dfk.DFK_OK
+    assert L.dfk_swiglu_gate_up_fp8(None, P2, P3, P2, P3, None, 0, 64, 64, 0, None) == dfk.DFK_OK
+    assert L.dfk_down_proj_fp8(None, P2, P3, None, 0, 64, 64, 0, None) == dfk.DFK_OK
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device behaviour")
