@@ -461,6 +461,9 @@ def extra_measurements(args, inp, copies, h, y):
     torch.cuda.empty_cache()
     out["llama3_70b"] = llama70b_measure()
     torch.cuda.empty_cache()
+    out["fp8_weights"] = fp8_measure()
+    out["fp8_weights"]["bf16_b1_fused_us"] = round(t_fus, 2)
+    torch.cuda.empty_cache()
     out["decode_stack"] = decode_stack_measure(args.stack_steps)
     return out
 
@@ -500,6 +503,56 @@ def llama70b_measure(reps=30):
                     "mlp_us": round(tg + td, 2)})
     del base, cps
     return res
+
+
+def fp8_gate_up_bytes(B, D, F):
+    """FP8 E4M3 codes of both matrices, their fp32 row scales, x, gamma, h."""
+    return 2 * F * D + 2 * F * 4 + B * D * 2 + D * 2 + B * F * 2
+
+
+def fp8_down_bytes(B, D, F):
+    return D * F + D * 4 + B * F * 2 + B * D * 2
+
+
+def fp8_measure(reps=100, ncopies=4):
+    """FP8 E4M3 weight streaming (row scales, fused dequantisation) on the
+    Llama-3-8B-shaped layer: the bench's seeded bf16 weights encoded per row,
+    fused RMSNorm + gate/up and the down projection at B = 1..16, back-to-back
+    calls over `ncopies` weight copies (176 MB each; together beyond L2)."""
+    import torch
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    peak, _ = measured_peaks()
+    base = I.make_inputs(16, D, F, seed=2, norm=True, with_down=True, device="cuda")
+    qg, sg = I.to_fp8_rows(base.w_gate)
+    qu, su = I.to_fp8_rows(base.w_up)
+    qd, sd = I.to_fp8_rows(base.w_down)
+    del base.w_gate, base.w_up, base.w_down
+    cps = [(qg, qu, qd)] + [(qg.clone(), qu.clone(), qd.clone()) for _ in range(ncopies - 1)]
+    res = []
+    for B in (1, 2, 4, 8, 16):
+        x = base.x[:B].contiguous()
+        h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+        dfk.dfk_rmsnorm_swiglu_gate_up_fp8(x, base.gamma, base.eps, qg, sg, qu, su, h=h)
+        dfk.dfk_down_proj_fp8(h, qd, sd, y=y)        # first calls: the scheduler decides
+        tg = timed_us(lambda i: dfk.dfk_rmsnorm_swiglu_gate_up_fp8(
+            x, base.gamma, base.eps, cps[i % ncopies][0], sg, cps[i % ncopies][1], su, h=h), reps)
+        td = timed_us(lambda i: dfk.dfk_down_proj_fp8(h, cps[i % ncopies][2], sd, y=y), reps)
+        gg = fp8_gate_up_bytes(B, D, F) / (tg * 1e-6) / 1e9
+        gd = fp8_down_bytes(B, D, F) / (td * 1e-6) / 1e9
+        vg = dfk.dfk_cached_variant(dfk.DFK_OP_RMSNORM_GATE_UP_FP8, B, D, F, "row") or {}
+        vd = dfk.dfk_cached_variant(dfk.DFK_OP_DOWN_FP8, B, D, F, "row") or {}
+        res.append({"B": B, "gate_up_us": round(tg, 2), "gate_up_GBps": round(gg, 1),
+                    "gate_up_frac": round(gg / peak, 4), "gate_up_variant": vg.get("variant_id"),
+                    "down_us": round(td, 2), "down_GBps": round(gd, 1),
+                    "down_frac": round(gd / peak, 4), "down_variant": vd.get("variant_id"),
+                    "mlp_us": round(tg + td, 2)})
+    del cps, qg, qu, qd, base
+    torch.cuda.empty_cache()
+    return {"workload": "llama3_8b_fp8_e4m3_row_scales", "weights": "E4M3 codes + fp32 row "
+            "scales from the seeded bf16 weights (absmax / 448 per row)", "sweep": res}
 
 
 def decode_stack_measure(steps, layers=32, B=4):
@@ -622,16 +675,24 @@ def profile_arm(args):
     torch.cuda.set_device(0)
     B = args.batch
     inp = I.make_inputs(B, D, F, seed=SEED, w_std=0.02, norm=True,
-                        with_down=args.profile == "down", device="cuda")
+                        with_down=args.profile.startswith("down"), device="cuda")
     h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
     y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
     lay = {"row": I.LAYOUT_ROW, "col": I.LAYOUT_COL, "interleaved": I.LAYOUT_INTERLEAVED}
     wg, wu = I.to_layout(inp.w_gate, inp.w_up, lay[args.layout])
     if args.profile == "gate_up":
         fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu,
-                                                    args.layout, h=h)
+                                                    args.layout, h=h, variant=args.variant)
+    elif args.profile == "gate_up_fp8":
+        qg, sg = I.to_fp8_rows(inp.w_gate)
+        qu, su = I.to_fp8_rows(inp.w_up)
+        fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up_fp8(inp.x, inp.gamma, inp.eps, qg, sg, qu,
+                                                        su, h=h, variant=args.variant)
+    elif args.profile == "down_fp8":
+        qd, sd = I.to_fp8_rows(inp.w_down)
+        fn = lambda: dfk.dfk_down_proj_fp8(h, qd, sd, y=y, variant=args.variant)
     else:
-        fn = lambda: dfk.dfk_down_proj(h, inp.w_down, y=y)
+        fn = lambda: dfk.dfk_down_proj(h, inp.w_down, y=y, variant=args.variant)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -655,10 +716,13 @@ def main():
                     help="skip the sweep / unfused / interleaved / decode-stack measurements")
     ap.add_argument("--stack-steps", type=int, default=512,
                     help="decode steps of the 32-layer stack measurement")
-    ap.add_argument("--profile", choices=["gate_up", "down"], default=None,
+    ap.add_argument("--profile", choices=["gate_up", "down", "gate_up_fp8", "down_fp8"],
+                    default=None,
                     help="run only this kernel (inside an NVTX range) for ncu")
     ap.add_argument("--batch", type=int, default=1, help="batch for --profile")
     ap.add_argument("--layout", default="row", help="weight layout for --profile")
+    ap.add_argument("--variant", type=int, default=0,
+                    help="variant id for --profile (0 = the scheduler's choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -172,10 +172,15 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
  *   x, gamma, h, y, eps: as for the bf16 entry points.
  * Each code is widened to its exact fp32 value in registers; products and
  * sums are fp32 in a fixed order; the row's sum is multiplied by s[j] once
- * before SiLU and the bf16 rounding.  Constraints: row-major only; the
- * reduction length (d_model for gate/up, d_ff for the down projection) a
- * multiple of 16; CUDA-core variants only (a tensor-core id is rejected
- * with DFK_ERR_INVALID_ARG); otherwise as for the bf16 entry points.
+ * before SiLU and the bf16 rounding.  Two variant families: CUDA-core
+ * variants (fp32 FMA on the widened codes; at most two k tiles per stage) and
+ * a tensor-core kernel (the tensor-core ids with one k tile per stage and
+ * rows spread over the SMs: codes widened to bf16 into TMEM, bf16 MMA with
+ * fp32 accumulation; at most 128 output rows per SM, or per SM / k_split for
+ * the down projection); other ids are rejected with DFK_ERR_INVALID_ARG.
+ * Constraints: row-major only; the reduction length (d_model for gate/up,
+ * d_ff for the down projection) a multiple of 16; otherwise as for the bf16
+ * entry points.
  */
 DFK_API int dfk_swiglu_gate_up_fp8(const void *x, const void *q_gate, const float *s_gate,
                                    const void *q_up, const float *s_up, void *h, int B,

@@ -33,6 +33,8 @@
 #include "launch_util.h"
 #include "tc_engine.cuh"
 #include "tc_key.h"
+#include "tf8_engine.cuh"
+#include "tf8_key.h"
 
 // Device error word: bit 0 = a pipeline wait in some kernel gave up.
 __device__ unsigned g_dfk_err;
@@ -261,6 +263,12 @@ static const std::vector<VDef> &variants() {
     return t;
   }();
   return v;
+}
+
+// Variants that can run FP8 weights: CUDA-core ones, and tensor-core ones with
+// one k tile per stage whose rows are spread over the SMs.
+static bool fp8_capable(const VDef &d) {
+  return d.family == DFK_FAMILY_CUDA_CORE || (d.nt == 1 && d.full == 0);
 }
 
 static const VDef *find_variant(int id) {
@@ -626,8 +634,6 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   int dev;
   int rc = current_device(&ds, &dev);
   if (rc) return rc;
-  if (c.w8)
-    return fail(DFK_ERR_NO_VARIANT, "variant %d: FP8 weights run on the CUDA-core family", v.id);
   TcPlan pl;
   std::string why;
   if (!plan_tc(c.layout, c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
@@ -767,9 +773,153 @@ int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, in
   return DFK_OK;
 }
 
+// ---------------------------------------------------------------- FP8 tensor-core plan
+
+struct Tf8Plan {
+  const void *fn = nullptr;
+  int grid = 0;
+  size_t smem = 0;
+  Tf8Params p{};
+};
+
+// Row blocks of at most 128 rows (one per SM, or per SM / kslices for the
+// split-K GEMV), one 128-wide k tile per ring stage.  FP8 weights use the
+// tensor-core variants with one k tile per stage that own no full M tiles.
+static bool plan_tf8(int nmat, bool norm, const VDef &v, int B, int K, int N,
+                     const DeviceState &ds, Tf8Plan *pl, std::string *why) {
+  if (v.nt != 1 || v.full != 0) {
+    if (why) *why = "FP8 tensor-core kernel: one k tile per stage, rows spread over the SMs";
+    return false;
+  }
+  if (B < 1 || B > 64) {
+    if (why) *why = "batch outside 1..64";
+    return false;
+  }
+  const int bn = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
+  const int ks = nmat == 1 ? v.ksplit : 1;
+  const int ntiles = ceil_div(K, TF8_TILE_K);
+  if (ks > ntiles) {
+    if (why) *why = "more k slices than k tiles";
+    return false;
+  }
+  const int nblocks = std::max(1, std::min(N, ds.sms / ks));
+  const int rbase = N / nblocks, rextra = N % nblocks;
+  const int hmax = rbase + (rextra ? 1 : 0);
+  if (hmax > 128) {
+    if (why) *why = "more than 128 output rows per CTA";
+    return false;
+  }
+  const int r8 = round_up(hmax, 8);
+  const int a8 = nmat * r8 * 128;
+  const int xt = bn * 128 * (norm ? 2 : 1);
+  const int stage = a8 + 2 * xt;  // both multiples of 1024
+  const int g_bytes = norm ? round_up(ntiles * TF8_TILE_K * 2, 1024) : 0;
+  const int bar_bytes = 512;      // 2 S + 5 barriers, flags, r_b of 64 tokens
+  const int smem_cap = std::min(ds.smem_optin, 232448);
+  const int avail = smem_cap - 1024 - g_bytes - bar_bytes;
+  const int S = std::min(8, avail / stage);
+  if (S < 2) {
+    if (why) *why = "shared memory too small for two ring stages";
+    return false;
+  }
+  const int wn = norm ? 2 * bn : bn;
+  const int acol = round_up(nmat * wn, 64);
+  const int cols = acol + 2 * nmat * 64;
+  const int tmem_cols = std::max(32, pow2_ceil(cols));
+  if (tmem_cols > 512) {
+    if (why) *why = "accumulators and A buffers exceed TMEM";
+    return false;
+  }
+  const void *fn = tf8_find_kernel(nmat, norm);
+  if (!fn) {
+    if (why) *why = "FP8 tensor-core kernel not compiled for this op";
+    return false;
+  }
+  Tf8Params &p = pl->p;
+  p = Tf8Params{};
+  p.B = B;
+  p.K = K;
+  p.N = N;
+  p.rbase = rbase;
+  p.rextra = rextra;
+  p.hmax = hmax;
+  p.r8 = r8;
+  p.bn = bn;
+  p.stages = S;
+  p.stage_bytes = stage;
+  p.a8_bytes = a8;
+  p.xt_bytes = xt;
+  p.tmem_cols = tmem_cols;
+  p.acol = acol;
+  p.g_off = S * stage;
+  p.bar_off = p.g_off + g_bytes;
+  p.ntiles = ntiles;
+  p.kslices = ks;
+  p.nblocks = nblocks;
+  pl->fn = fn;
+  pl->grid = nblocks * ks;
+  pl->smem = 1024 + static_cast<size_t>(p.bar_off) + bar_bytes;
+  return true;
+}
+
+static int launch_tf8(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  Tf8Plan pl;
+  std::string why;
+  if (!plan_tf8(c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
+    return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit FP8 B=%d K=%d N=%d: %s", v.id, c.B,
+                c.K, c.N, why.c_str());
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  Tf8Maps maps;
+  memset(&maps, 0, sizeof maps);
+  const void *w[2] = {c.w0, c.w1};
+  for (int m = 0; m < c.nmat; ++m)
+    for (int lo = 0; lo < 2; ++lo) {
+      const uint32_t hgt = static_cast<uint32_t>(std::max(1, pl.p.hmax - lo));
+      if ((rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K), TF8_TILE_K, hgt,
+                              &maps.w[m][lo], true, CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+        return rc;
+    }
+  if ((rc = tensor_map_2d(c.x, c.K, c.B, static_cast<uint64_t>(c.K) * 2, 64, pl.p.bn, &maps.x,
+                          true)))
+    return rc;
+  Tf8Params p = pl.p;
+  p.out = static_cast<uint16_t *>(c.out);
+  p.gamma = static_cast<const uint16_t *>(c.gamma);
+  p.scale[0] = c.s0;
+  p.scale[1] = c.s1;
+  p.err = ds->err;
+  p.eps = c.eps;
+  if (p.kslices > 1) {
+    const size_t part_bytes =
+        static_cast<size_t>(p.kslices) * p.nblocks * p.bn * 128 * sizeof(float);
+    const size_t counter_bytes = static_cast<size_t>(ds->sms) * 8 * sizeof(unsigned);
+    if ((rc = get_workspace(dev, s, part_bytes, counter_bytes, &p.part, &p.counters))) {
+      if (rc != DFK_ERR_NO_VARIANT || !stream_capturing(s)) return rc;
+      VDef whole = v;
+      whole.ksplit = 1;
+      log_msg("split-K workspace missing during capture: launching without the split");
+      return launch_tf8(c, whole, s, stages_used);
+    }
+  }
+  void *args[] = {&maps, &p};
+  cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TF8_THREADS), pl.smem, s,
+                                pdl_enabled(), args);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "FP8 tensor-core kernel launch");
+  }
+  if (stages_used) *stages_used = p.stages;
+  return DFK_OK;
+}
+
 static int launch_variant(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
-  return v.family == DFK_FAMILY_TENSOR_CORE ? launch_tc(c, v, s, stages_used)
-                                            : launch_cc(c, v, s, stages_used);
+  if (v.family == DFK_FAMILY_TENSOR_CORE)
+    return c.w8 ? launch_tf8(c, v, s, stages_used) : launch_tc(c, v, s, stages_used);
+  return launch_cc(c, v, s, stages_used);
 }
 
 // ---------------------------------------------------------------- scheduler
@@ -854,7 +1004,7 @@ static void tune_cache_load(int dev, int sms) {  // caller holds g_tune_mu
       continue;
     const VDef *d = find_variant(vid);
     if (!d || d->cls != op_class(op) || B < 1 || B > 64 ||
-        (op_is_fp8(op) && d->family != DFK_FAMILY_CUDA_CORE)) {
+        (op_is_fp8(op) && !fp8_capable(*d))) {
       ++bad;
       continue;
     }
@@ -893,7 +1043,12 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
   std::vector<const VDef *> out;
   for (const VDef &d : variants()) {
     if (d.cls != op_class(op)) continue;
-    if (c.w8 && (d.family == DFK_FAMILY_TENSOR_CORE || d.nt > 2)) continue;
+    if (c.w8 && d.family == DFK_FAMILY_TENSOR_CORE) {
+      // FP8: the tensor-core kernel from B = 2 (one k tile per stage)
+      if (d.nt == 1 && d.full == 0 && B >= 2) out.push_back(&d);
+      continue;
+    }
+    if (c.w8 && d.nt > 2) continue;
     if (d.family == DFK_FAMILY_TENSOR_CORE) {
       // gate/up from B = 4 (where CUDA cores fall below HBM speed), the GEMV
       // (split-K) from B = 2
@@ -908,7 +1063,10 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
 
 static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
   if (d.family == DFK_FAMILY_TENSOR_CORE) {
-    if (c.w8) return false;
+    if (c.w8) {
+      Tf8Plan pl;
+      return plan_tf8(c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+    }
     TcPlan pl;
     return plan_tc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
   }
@@ -922,6 +1080,14 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // the GEMV the largest k split whose CTA fits.  If nothing of that shape
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
+  if (c.w8 && B >= 2) {
+    // FP8 weights: the tensor-core kernel (split-K 4 for the GEMV)
+    const int want_ks = op_class(op) == CLS_GEMV ? 4 : 1;
+    for (const VDef &d : variants())
+      if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == 1 &&
+          d.full == 0 && d.ksplit == want_ks && feasible(d, c, ds))
+        return &d;
+  }
   if (B >= 8 && !c.w8) {
     const bool gemv = op_class(op) == CLS_GEMV;
     const int want_nt = gemv ? 2 : 1, want_ks = gemv ? 4 : 1;
@@ -1033,9 +1199,8 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
     const VDef *d = find_variant(variant);
     if (!d || d->cls != op_class(op))
       return fail(DFK_ERR_INVALID_ARG, "variant %d is not a variant of op %d", variant, op);
-    if (c.w8 && d->family == DFK_FAMILY_TENSOR_CORE)
-      return fail(DFK_ERR_INVALID_ARG, "variant %d: FP8 weights run on CUDA-core variants",
-                  variant);
+    if (c.w8 && !fp8_capable(*d))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d cannot run FP8 weights", variant);
     *out = d;
     return DFK_OK;
   }
@@ -1161,9 +1326,8 @@ static int check_fp8(const void *x, const void *gamma, bool norm, float eps, con
   if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
   if (variant > 0) {
     const VDef *d = find_variant(variant);
-    if (!d || d->cls != cls || d->family != DFK_FAMILY_CUDA_CORE)
-      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a CUDA-core variant of this op",
-                  variant);
+    if (!d || d->cls != cls || !fp8_capable(*d))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d cannot run this FP8 op", variant);
   }
   if (norm && !(eps >= 0.f && std::isfinite(eps)))
     return fail(DFK_ERR_INVALID_ARG, "eps must be finite and >= 0");

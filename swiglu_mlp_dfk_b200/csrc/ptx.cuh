@@ -150,6 +150,49 @@ __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
       : "r"(h01), "r"(h23));
 }
 
+// Four FP8 E4M3 codes (byte i of w = element i) -> two bf16x2 words (lo holds
+// elements 0, 1; hi holds 2, 3; lower element in the low half).  E4M3 -> f16
+// is exact (hardware pair conversion), and so is f16 -> bf16 for these values
+// (at most 4 significant bits, exponents -9 .. 8).
+__device__ __forceinline__ void e4m3x4_to_bf16x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 c01, c23, a, b, c, d;\n\t"
+      ".reg .b32 h01, h23;\n\t"
+      "mov.b32 {c01, c23}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h01, c01;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h23, c23;\n\t"
+      "mov.b32 {a, b}, h01;\n\t"
+      "mov.b32 {c, d}, h23;\n\t"
+      "cvt.rn.bf16.f16 a, a;\n\t"
+      "cvt.rn.bf16.f16 b, b;\n\t"
+      "cvt.rn.bf16.f16 c, c;\n\t"
+      "cvt.rn.bf16.f16 d, d;\n\t"
+      "mov.b32 %0, {a, b};\n\t"
+      "mov.b32 %1, {c, d};\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// The same conversion without the conversion unit (whose throughput is a
+// quarter of the ALU's): for a code c = s.eeee.mmm, the 16 bits
+// (c & 0x7F) << 4 read as bf16 have exponent field e and mantissa mmm0000,
+// i.e. the value |E4M3(c)| * 2^-120 exactly (e = 0 gives the bf16 subnormal
+// m * 2^-129); one bf16x2 multiply by 2^120 (exact) restores the scale and
+// the sign bit is or-ed in.  Per pair of codes: a byte permute, a shift, a
+// mask, a multiply and an or.  The NaN code S.1111.111 is not special:
+// it comes out as +-480.
+__device__ __forceinline__ uint32_t e4m3x2_bits_to_bf16x2(uint32_t b) {
+  // b holds code 0 in bits 15..8 and code 1 in bits 31..24 (other bits 0)
+  const uint32_t mag = (b >> 4) & 0x07F007F0u;
+  uint32_t v;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(v) : "r"(mag), "r"(0x7B807B80u));  // x 2^120
+  return v | (b & 0x80008000u);
+}
+
+__device__ __forceinline__ void e4m3x4_to_bf16x2_alu(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  lo = e4m3x2_bits_to_bf16x2(__byte_perm(w, 0u, 0x1404));  // [c1, 0, c0, 0]
+  hi = e4m3x2_bits_to_bf16x2(__byte_perm(w, 0u, 0x3424));  // [c3, 0, c2, 0]
+}
+
 // Two fp32 values in one 64-bit register (lo = first element).
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   uint64_t r;

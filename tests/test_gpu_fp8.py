@@ -136,12 +136,16 @@ def test_fp8_down_small_shapes(B, D, F):
 
 @pytest.mark.parametrize("B", [1, 3, 8])
 def test_every_fp8_gate_up_variant_is_bitwise_identical(B):
+    # the CUDA-core family is bitwise invariant; the tensor-core kernel (which
+    # the scheduler may pick) is held to the tolerance only
     L = Fp8Layer(B, 384, 1000, seed=300 + B, norm=True, with_down=False)
-    ref = L.gate_up(True)
+    ids = [v for v in cc_ids(dfk.DFK_OP_GATE_UP_FP8)
+           if v["token_tile"] == bt_for(B, v["j_per_thread"])]
+    ref = L.gate_up(True, variant=ids[0]["variant_id"])
     torch.cuda.synchronize()
     assert_close(ref, L.oracle_gate_up(True), "fp8 gate/up reference run")
     ran = 0
-    for v in cc_ids(dfk.DFK_OP_GATE_UP_FP8):
+    for v in ids:
         if v["token_tile"] != bt_for(B, v["j_per_thread"]):
             continue
         h = try_variant(lambda vid: L.gate_up(True, variant=vid), v["variant_id"])
@@ -157,28 +161,36 @@ def test_every_fp8_down_variant_is_bitwise_identical():
     B, D, F = 2, 512, 2064
     L = Fp8Layer(B, D, F, seed=310, norm=False)
     h = (torch.randn(B, F, device="cuda")).to(torch.bfloat16)
-    ref = dfk.dfk_down_proj_fp8(h, L.qd, L.sd)
-    torch.cuda.synchronize()
-    assert_close(ref, L.oracle_down(h), "fp8 down reference run")
+    # the k split and (when it is above 1) the tiles per stage fix which tiles
+    # each team sums, so bits agree within one such pair; across pairs the
+    # results are held to the tolerance
+    ids = [v for v in cc_ids(dfk.DFK_OP_DOWN_FP8)
+           if v["token_tile"] == bt_for(B, v["j_per_thread"])]
+    want = L.oracle_down(h)
+    refs = {}
     ran = 0
-    for v in cc_ids(dfk.DFK_OP_DOWN_FP8):
-        if v["token_tile"] != bt_for(B, v["j_per_thread"]):
-            continue
+    for v in ids:
         y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid),
                         v["variant_id"])
         if y is None:
             continue
         torch.cuda.synchronize()
+        assert_close(y, want, "fp8 down variant %d" % v["variant_id"])
+        key = (v["k_split"], v["k_tiles_per_stage"] if v["k_split"] > 1 else 0)
+        ref = refs.setdefault(key, y)
         assert bits_equal(y, ref), "variant %d differs" % v["variant_id"]
         ran += 1
-    assert ran >= 8
+    assert ran >= 8 and len(refs) >= 2
 
 
 def test_fp8_rows_do_not_depend_on_batch():
+    # CUDA-core family: row b is independent of B for any tile (one variant forced)
     L = Fp8Layer(8, 512, 688, seed=320, norm=True, with_down=False)
-    full = L.gate_up(True)
+    vid = next(v["variant_id"] for v in cc_ids(dfk.DFK_OP_GATE_UP_FP8)
+               if v["j_per_thread"] == 2 and v["token_tile"] == 8)
+    full = L.gate_up(True, variant=vid)
     for b in (1, 2, 5):
-        part = L.gate_up(True, x=L.inp.x[:b].contiguous())
+        part = L.gate_up(True, variant=vid, x=L.inp.x[:b].contiguous())
         torch.cuda.synchronize()
         assert bits_equal(part, full[:b].contiguous()), b
 
@@ -247,3 +259,107 @@ def test_fp8_scheduler_select_variant():
     h2 = L.gate_up(True)
     torch.cuda.synchronize()
     assert_close(h2, L.oracle_gate_up(True), "fp8 gate/up after tuning")
+
+
+# ------------------------------------------------------------------ tensor-core FP8 kernel
+
+def tc_fp8_ids(down):
+    """Tensor-core variant ids that run FP8 weights (one k tile per stage, rows spread)."""
+    want = dfk.DFK_OP_DOWN if down else dfk.DFK_OP_GATE_UP
+    return [v for v in (dfk.dfk_variant_info(i) for i in range(1, dfk.dfk_variant_count() + 1))
+            if v["op"] == want and v["family"] == 1 and v["k_tiles_per_stage"] == 1
+            and v["full_m_tiles"] == 0]
+
+
+TC_SHAPES = [(1, 256, 688), (2, 144, 200), (5, 400, 1000), (16, 1024, 1496), (17, 272, 96),
+             (33, 512, 520), (64, 256, 264)]
+
+
+@pytest.mark.parametrize("B,D,F", TC_SHAPES)
+@pytest.mark.parametrize("norm", [False, True])
+def test_fp8_tensor_core_gate_up(B, D, F, norm):
+    (v,) = tc_fp8_ids(False)
+    L = Fp8Layer(B, D, F, seed=400 + B, norm=norm, with_down=False)
+    h = L.gate_up(norm, variant=v["variant_id"])
+    torch.cuda.synchronize()
+    assert_close(h, L.oracle_gate_up(norm), "fp8 tc gate/up B=%d D=%d F=%d" % (B, D, F))
+
+
+@pytest.mark.parametrize("B,D,F", [(1, 256, 688), (3, 520, 400), (16, 1024, 2048),
+                                   (40, 272, 1024), (64, 384, 2064)])
+def test_fp8_tensor_core_down_every_split(B, D, F):
+    L = Fp8Layer(B, D, F, seed=410 + B, norm=False)
+    h = (torch.randn(B, F, device="cuda") * 0.5).to(torch.bfloat16)
+    want = L.oracle_down(h)
+    ran = 0
+    for v in tc_fp8_ids(True):
+        y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid),
+                        v["variant_id"])
+        if y is None:
+            continue
+        y2 = dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=v["variant_id"])  # counters reset
+        torch.cuda.synchronize()
+        assert_close(y, want, "fp8 tc down ks=%d B=%d" % (v["k_split"], B))
+        assert bits_equal(y, y2), "split-K result not repeatable"
+        ran += 1
+    assert ran >= 2
+
+
+def test_fp8_tensor_core_rows_do_not_depend_on_batch_within_a_tile():
+    # tokens are columns of one MMA: row b of h does not change with B while
+    # the token tile (16) stays the same
+    (v,) = tc_fp8_ids(False)
+    L = Fp8Layer(16, 512, 688, seed=420, norm=True, with_down=False)
+    full = L.gate_up(True, variant=v["variant_id"])
+    part = L.gate_up(True, variant=v["variant_id"], x=L.inp.x[:5].contiguous())
+    torch.cuda.synchronize()
+    assert bits_equal(part, full[:5].contiguous())
+
+
+@pytest.mark.parametrize("B", [2, 16, 64])
+def test_fp8_tensor_core_llama3_8b_sampled_rows(B):
+    w = I.WORKLOADS["llama3_8b"]
+    L = Fp8Layer(B, w.d_model, w.d_ff, seed=w.seed, norm=True)
+    (vg,) = tc_fp8_ids(False)
+    h = L.gate_up(True, variant=vg["variant_id"])
+    ys = []
+    for v in tc_fp8_ids(True):
+        y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid),
+                        v["variant_id"])
+        if y is not None:
+            ys.append(y)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.d_ff, 160, 11)
+    idx = torch.from_numpy(rows).long().cuda()
+    assert_close(h[:, idx].contiguous(), L.oracle_gate_up(True, rows=rows),
+                 "fp8 tc 8B gate/up rows B=%d" % B)
+    drows = sample_rows(w.d_model, 96, 12)
+    didx = torch.from_numpy(drows).long().cuda()
+    want = L.oracle_down(h, rows=drows)
+    assert ys
+    for y in ys:
+        assert_close(y[:, didx].contiguous(), want, "fp8 tc 8B down rows B=%d" % B)
+
+
+def test_fp8_tensor_core_is_exact_dequantisation():
+    # unit scales, weights covering every finite E4M3 code: the FP8 tensor-core
+    # kernel must give the bits of the bf16 tensor-core kernel on the decoded
+    # weights (same MMA k-slice sequence into one accumulator, same epilogue),
+    # so a lost subnormal or a wrong exponent shows up bitwise
+    (v,) = tc_fp8_ids(False)
+    B, D, F = 4, 512, 688
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    rng = np.random.default_rng(430)
+    qg = torch.from_numpy(codes[rng.integers(0, codes.size, (F, D))]).cuda()
+    qu = torch.from_numpy(codes[rng.integers(0, codes.size, (F, D))]).cuda()
+    ones = torch.ones(F, dtype=torch.float32, device="cuda")
+    inp = I.make_inputs(B, D, F, seed=431, norm=True, with_down=False, device="cuda")
+    x = (inp.x.float() * 0.05).to(torch.bfloat16)       # keeps |a| moderate
+    h8 = dfk.dfk_rmsnorm_swiglu_gate_up_fp8(x, inp.gamma, 1e-5, qg, ones, qu, ones,
+                                            variant=v["variant_id"])
+    wg = qg.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    wu = qu.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    h16 = dfk.dfk_rmsnorm_swiglu_gate_up(x, inp.gamma, 1e-5, wg, wu, "row",
+                                         variant=v["variant_id"])
+    torch.cuda.synchronize()
+    assert bits_equal(h8, h16)
