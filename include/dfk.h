@@ -97,6 +97,9 @@ typedef struct dfk_variant {
   int full_m_tiles; /* tensor core: 1 = each CTA owns 128 output rows (full MMA M) */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
+  int e4m3_mma;     /* tensor core, FP8 weights only: 1 = E4M3 MMA on the codes
+                       (kind::f8f6f4, activations as E4M3 terms); dfk_variant_info
+                       reports these under the FP8 ops                           */
 } dfk_variant;
 
 /*
@@ -172,12 +175,18 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
  *   x, gamma, h, y, eps: as for the bf16 entry points.
  * Each code is widened to its exact fp32 value in registers; products and
  * sums are fp32 in a fixed order; the row's sum is multiplied by s[j] once
- * before SiLU and the bf16 rounding.  Two variant families: CUDA-core
- * variants (fp32 FMA on the widened codes; at most two k tiles per stage) and
- * a tensor-core kernel (the tensor-core ids with one k tile per stage and
- * rows spread over the SMs: codes widened to bf16 into TMEM, bf16 MMA with
- * fp32 accumulation; at most 128 output rows per SM, or per SM / k_split for
- * the down projection); other ids are rejected with DFK_ERR_INVALID_ARG.
+ * before SiLU and the bf16 rounding.  Variant families: CUDA-core variants
+ * (fp32 FMA on the widened codes; at most two k tiles per stage); a
+ * widening tensor-core kernel (the tensor-core ids with one k tile per stage
+ * and rows spread over the SMs: codes widened to bf16 into TMEM, bf16 MMA
+ * with fp32 accumulation); and the E4M3-MMA kernel (ids with e4m3_mma = 1:
+ * the codes feed the E4M3 tensor-core MMA directly, each token's activations
+ * are first written as E4M3 terms -- two for bf16 x, four for x * gamma,
+ * after a power-of-two scale -- by a small kernel launched before it, into a
+ * library-owned buffer per (device, stream) allocated at first use outside
+ * stream capture).  Tensor-core kernels take at most 128 output rows per SM
+ * (per SM / k_split for the down projection).  Other ids are rejected with
+ * DFK_ERR_INVALID_ARG; E4M3-MMA ids are rejected by the bf16 entry points.
  * Constraints: row-major only; the reduction length (d_model for gate/up,
  * d_ff for the down projection) a multiple of 16; otherwise as for the bf16
  * entry points.

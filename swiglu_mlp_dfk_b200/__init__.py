@@ -74,7 +74,8 @@ class dfk_variant(ctypes.Structure):
                 ("token_tile", ctypes.c_int), ("k_split", ctypes.c_int),
                 ("k_tiles_per_stage", ctypes.c_int), ("acc_banks", ctypes.c_int),
                 ("paired_fma", ctypes.c_int), ("full_m_tiles", ctypes.c_int),
-                ("stages", ctypes.c_int), ("measured_us", ctypes.c_float)]
+                ("stages", ctypes.c_int), ("measured_us", ctypes.c_float),
+                ("e4m3_mma", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -35,6 +35,7 @@
 #include "tc_key.h"
 #include "tf8_engine.cuh"
 #include "tf8_key.h"
+#include "tf8mma_engine.cuh"
 
 // Device error word: bit 0 = a pipeline wait in some kernel gave up.
 __device__ unsigned g_dfk_err;
@@ -234,6 +235,7 @@ struct VDef {
   int nbank;  // tensor core: independent TMEM accumulator banks per output
   int pair;   // CUDA core: FMAs issued in pairs (fma.rn.f32x2)
   int full;   // tensor core: CTAs own full 128-row M tiles (fewer CTAs than SMs)
+  int e4m3mma;  // tensor core, FP8 weights only: E4M3 MMA on the codes (kind::f8f6f4)
 };
 
 static const int kJB[][2] = {{4, 1}, {4, 2}, {4, 4}, {2, 1}, {2, 2}, {2, 4}, {2, 8}};
@@ -260,6 +262,10 @@ static const std::vector<VDef> &variants() {
     for (int ks : {1, 2, 4})
       for (int nt : {1, 2, 4, 8})
         t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, nt, 1, 0, 0});
+    // FP8 weights only: the E4M3 MMA on the codes (activations as E4M3 terms)
+    t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, 1, 1, 0, 0, 1});
+    for (int ks : {1, 2, 4})
+      t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, 1, 1, 0, 0, 1});
     return t;
   }();
   return v;
@@ -270,6 +276,9 @@ static const std::vector<VDef> &variants() {
 static bool fp8_capable(const VDef &d) {
   return d.family == DFK_FAMILY_CUDA_CORE || (d.nt == 1 && d.full == 0);
 }
+
+// Variants that can run bf16 weights: all but the E4M3-MMA ones.
+static bool bf16_capable(const VDef &d) { return d.e4m3mma == 0; }
 
 static const VDef *find_variant(int id) {
   for (const VDef &d : variants())
@@ -489,6 +498,10 @@ static int pow2_ceil(int v) {
 // tile, so the space behind the last A tile of the ring is kept readable.
 static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K, int N,
                     const DeviceState &ds, TcPlan *pl, std::string *why) {
+  if (v.e4m3mma) {
+    if (why) *why = "E4M3-MMA variants run FP8 weights only";
+    return false;
+  }
   const bool colm = layout == LAYOUT_COL;
   const bool full = colm || (v.full != 0 && nmat == 2);  // 128 rows per CTA
   if (colm && nmat != 2) {
@@ -787,7 +800,7 @@ struct Tf8Plan {
 // tensor-core variants with one k tile per stage that own no full M tiles.
 static bool plan_tf8(int nmat, bool norm, const VDef &v, int B, int K, int N,
                      const DeviceState &ds, Tf8Plan *pl, std::string *why) {
-  if (v.nt != 1 || v.full != 0) {
+  if (v.nt != 1 || v.full != 0 || v.e4m3mma) {
     if (why) *why = "FP8 tensor-core kernel: one k tile per stage, rows spread over the SMs";
     return false;
   }
@@ -916,9 +929,213 @@ static int launch_tf8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
   return DFK_OK;
 }
 
+// ---------------------------------------------------------------- FP8 E4M3-MMA plan
+
+struct Tm8Plan {
+  const void *fn = nullptr;
+  int grid = 0;
+  size_t smem = 0;
+  Tm8Params p{};
+  size_t term_bytes = 0;  // activation-term buffer: codes + per-token factors
+};
+
+// Terms per token: 2 carry a bf16 activation exactly, 4 the 16-bit x * gamma
+// products of the RMSNorm path.  Rows of <= 128 per CTA as for the other
+// tensor-core kernels; one 128-wide k tile per stage.
+static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
+                     const DeviceState &ds, Tm8Plan *pl, std::string *why) {
+  if (!v.e4m3mma) {
+    if (why) *why = "not an E4M3-MMA variant";
+    return false;
+  }
+  if (B < 1 || B > 64) {
+    if (why) *why = "batch outside 1..64";
+    return false;
+  }
+  const int T = norm ? 4 : 2;
+  const int bnp = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
+  const int np = T * bnp;
+  if (np > 256 || nmat * np > 512) {
+    if (why) *why = "activation terms exceed N = 256";
+    return false;
+  }
+  const int ks = nmat == 1 ? v.ksplit : 1;
+  const int ntiles = ceil_div(K, TM8_TILE_K);
+  if (ks > ntiles) {
+    if (why) *why = "more k slices than k tiles";
+    return false;
+  }
+  const int nblocks = std::max(1, std::min(N, ds.sms / ks));
+  const int rbase = N / nblocks, rextra = N % nblocks;
+  const int hmax = rbase + (rextra ? 1 : 0);
+  if (hmax > 128) {
+    if (why) *why = "more than 128 output rows per CTA";
+    return false;
+  }
+  const int r8 = round_up(hmax, 8);
+  const int a8 = nmat * r8 * 128;
+  const int stage = a8 + np * 128;  // both multiples of 1024
+  // the last code tile's 128-row MMA read may run past the last stage
+  const int over = (nmat - 1) * r8 * 128 + 128 * 128;
+  const int slack = std::max(0, over - stage);
+  const int bar_bytes = 256;        // 2 S + 1 barriers and flags
+  const int smem_cap = std::min(ds.smem_optin, 232448);
+  const int S = std::min(8, (smem_cap - 1024 - bar_bytes - slack) / stage);
+  if (S < 2) {
+    if (why) *why = "shared memory too small for two ring stages";
+    return false;
+  }
+  const void *fn = tf8mma_find_kernel(nmat);
+  if (!fn) {
+    if (why) *why = "E4M3-MMA kernel not compiled for this op";
+    return false;
+  }
+  Tm8Params &p = pl->p;
+  p = Tm8Params{};
+  p.B = B;
+  p.K = K;
+  p.N = N;
+  p.rbase = rbase;
+  p.rextra = rextra;
+  p.hmax = hmax;
+  p.r8 = r8;
+  p.bnp = bnp;
+  p.T = T;
+  p.np = np;
+  p.stages = S;
+  p.stage_bytes = stage;
+  p.a8_bytes = a8;
+  p.tmem_cols = std::max(32, pow2_ceil(nmat * np));
+  p.bar_off = S * stage + slack;
+  p.ntiles = ntiles;
+  p.kslices = ks;
+  p.nblocks = nblocks;
+  pl->fn = fn;
+  pl->grid = nblocks * ks;
+  pl->smem = 1024 + static_cast<size_t>(p.bar_off) + bar_bytes;
+  pl->term_bytes = static_cast<size_t>(ntiles) * np * 128 + 64 * sizeof(float);
+  return true;
+}
+
+// Activation-term buffer: one per (device, stream), grown on demand outside
+// stream capture.
+static std::map<std::pair<int, cudaStream_t>, Workspace> g_terms;
+
+static int get_term_buffer(int dev, cudaStream_t s, size_t bytes, void **out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace &w = g_terms[std::make_pair(dev, s)];
+  if (w.bytes < bytes) {
+    if (stream_capturing(s))
+      return fail(DFK_ERR_NO_VARIANT, "FP8 activation-term buffer must be allocated before "
+                  "capture (make one call of this shape on the stream first)");
+    if (w.base) {
+      cudaStreamSynchronize(s);
+      cudaFree(w.base);
+      w.base = nullptr;
+      w.bytes = 0;
+    }
+    const size_t grow = std::max(bytes, static_cast<size_t>(4) << 20);
+    cudaError_t e = cudaMalloc(&w.base, grow);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "cudaMalloc (FP8 activation-term buffer)");
+    }
+    w.bytes = grow;
+  }
+  *out = w.base;
+  return DFK_OK;
+}
+
+static int launch_tf8(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used);
+
+static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  Tm8Plan pl;
+  std::string why;
+  if (!plan_tm8(c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
+    return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit FP8 B=%d K=%d N=%d: %s", v.id, c.B,
+                c.K, c.N, why.c_str());
+  void *terms = nullptr;
+  if ((rc = get_term_buffer(dev, s, pl.term_bytes, &terms))) {
+    if (rc != DFK_ERR_NO_VARIANT || !stream_capturing(s)) return rc;
+    // captured on a stream without the buffer: the widening tensor-core kernel
+    VDef alt = v;
+    alt.e4m3mma = 0;
+    log_msg("FP8 term buffer missing during capture: launching the widening kernel");
+    return launch_tf8(c, alt, s, stages_used);
+  }
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  Tm8Params p = pl.p;
+  const size_t code_bytes = static_cast<size_t>(p.ntiles) * p.np * 128;
+  float *fac = reinterpret_cast<float *>(static_cast<char *>(terms) + code_bytes);
+  Tm8Maps maps;
+  memset(&maps, 0, sizeof maps);
+  const void *w[2] = {c.w0, c.w1};
+  for (int m = 0; m < c.nmat; ++m)
+    for (int lo = 0; lo < 2; ++lo) {
+      const uint32_t hgt = static_cast<uint32_t>(std::max(1, p.hmax - lo));
+      if ((rc = tensor_map_2d(w[m], c.K, c.N, static_cast<uint64_t>(c.K), TM8_TILE_K, hgt,
+                              &maps.w[m][lo], true, CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+        return rc;
+    }
+  if ((rc = tensor_map_2d(terms, TM8_TILE_K, static_cast<uint64_t>(p.ntiles) * p.np, TM8_TILE_K,
+                          TM8_TILE_K, static_cast<uint32_t>(p.np), &maps.x, true,
+                          CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+    return rc;
+  p.out = static_cast<uint16_t *>(c.out);
+  p.scale[0] = c.s0;
+  p.scale[1] = c.s1;
+  p.fac = fac;
+  p.err = ds->err;
+  if (p.kslices > 1) {
+    const size_t part_bytes =
+        static_cast<size_t>(p.kslices) * p.nblocks * p.bnp * 128 * sizeof(float);
+    const size_t counter_bytes = static_cast<size_t>(ds->sms) * 8 * sizeof(unsigned);
+    if ((rc = get_workspace(dev, s, part_bytes, counter_bytes, &p.part, &p.counters))) {
+      if (rc != DFK_ERR_NO_VARIANT || !stream_capturing(s)) return rc;
+      VDef whole = v;
+      whole.ksplit = 1;
+      log_msg("split-K workspace missing during capture: launching without the split");
+      return launch_tm8(c, whole, s, stages_used);
+    }
+  }
+  // prep: scales, r_b and the E4M3 terms of the activations
+  Tm8PrepParams pp{};
+  pp.x = static_cast<const uint16_t *>(c.x);
+  pp.gamma = c.norm ? static_cast<const uint16_t *>(c.gamma) : nullptr;
+  pp.terms = static_cast<uint8_t *>(terms);
+  pp.fac = fac;
+  pp.B = c.B;
+  pp.K = c.K;
+  pp.bnp = p.bnp;
+  pp.T = p.T;
+  pp.ntiles = p.ntiles;
+  pp.eps = c.eps;
+  void *pargs[] = {&pp};
+  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
+                                pdl_enabled(), pargs);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "FP8 activation-term kernel launch");
+  }
+  void *args[] = {&maps, &p};
+  e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TM8_THREADS), pl.smem, s, pdl_enabled(), args);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "FP8 E4M3-MMA kernel launch");
+  }
+  if (stages_used) *stages_used = p.stages;
+  return DFK_OK;
+}
+
 static int launch_variant(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
-  if (v.family == DFK_FAMILY_TENSOR_CORE)
-    return c.w8 ? launch_tf8(c, v, s, stages_used) : launch_tc(c, v, s, stages_used);
+  if (v.family == DFK_FAMILY_TENSOR_CORE) {
+    if (!c.w8) return launch_tc(c, v, s, stages_used);
+    return v.e4m3mma ? launch_tm8(c, v, s, stages_used) : launch_tf8(c, v, s, stages_used);
+  }
   return launch_cc(c, v, s, stages_used);
 }
 
@@ -956,6 +1173,7 @@ static void fill_variant(const VDef &d, int op, int layout, int stages, float us
   out->acc_banks = d.nbank;
   out->paired_fma = d.pair;
   out->full_m_tiles = d.full;
+  out->e4m3_mma = d.e4m3mma;
   out->stages = stages;
   out->measured_us = us;
 }
@@ -1004,7 +1222,7 @@ static void tune_cache_load(int dev, int sms) {  // caller holds g_tune_mu
       continue;
     const VDef *d = find_variant(vid);
     if (!d || d->cls != op_class(op) || B < 1 || B > 64 ||
-        (op_is_fp8(op) && !fp8_capable(*d))) {
+        (op_is_fp8(op) && !fp8_capable(*d)) || (!op_is_fp8(op) && !bf16_capable(*d))) {
       ++bad;
       continue;
     }
@@ -1044,10 +1262,11 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
   for (const VDef &d : variants()) {
     if (d.cls != op_class(op)) continue;
     if (c.w8 && d.family == DFK_FAMILY_TENSOR_CORE) {
-      // FP8: the tensor-core kernel from B = 2 (one k tile per stage)
-      if (d.nt == 1 && d.full == 0 && B >= 2) out.push_back(&d);
+      // FP8: the tensor-core kernels (widening, E4M3 MMA) at every batch
+      if (d.nt == 1 && d.full == 0) out.push_back(&d);
       continue;
     }
+    if (!c.w8 && !bf16_capable(d)) continue;
     if (c.w8 && d.nt > 2) continue;
     if (d.family == DFK_FAMILY_TENSOR_CORE) {
       // gate/up from B = 4 (where CUDA cores fall below HBM speed), the GEMV
@@ -1063,6 +1282,10 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
 
 static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
   if (d.family == DFK_FAMILY_TENSOR_CORE) {
+    if (c.w8 && d.e4m3mma) {
+      Tm8Plan pl;
+      return plan_tm8(c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+    }
     if (c.w8) {
       Tf8Plan pl;
       return plan_tf8(c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
@@ -1081,18 +1304,21 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
   if (c.w8 && B >= 2) {
-    // FP8 weights: the tensor-core kernel (split-K 4 for the GEMV)
+    // FP8 weights: the E4M3-MMA kernel, else the widening one (split-K 4 for
+    // the GEMV)
     const int want_ks = op_class(op) == CLS_GEMV ? 4 : 1;
-    for (const VDef &d : variants())
-      if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == 1 &&
-          d.full == 0 && d.ksplit == want_ks && feasible(d, c, ds))
-        return &d;
+    for (int mma : {1, 0})
+      for (const VDef &d : variants())
+        if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == 1 &&
+            d.full == 0 && d.e4m3mma == mma && d.ksplit == want_ks && feasible(d, c, ds))
+          return &d;
   }
   if (B >= 8 && !c.w8) {
     const bool gemv = op_class(op) == CLS_GEMV;
     const int want_nt = gemv ? 2 : 1, want_ks = gemv ? 4 : 1;
     for (const VDef &d : variants())
-      if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == want_nt &&
+      if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && bf16_capable(d) &&
+          d.nt == want_nt &&
           d.ksplit == want_ks && d.nbank == 1 && feasible(d, c, ds))
         return &d;
   }
@@ -1201,6 +1427,8 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
       return fail(DFK_ERR_INVALID_ARG, "variant %d is not a variant of op %d", variant, op);
     if (c.w8 && !fp8_capable(*d))
       return fail(DFK_ERR_INVALID_ARG, "variant %d cannot run FP8 weights", variant);
+    if (!c.w8 && !bf16_capable(*d))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d runs FP8 weights only", variant);
     *out = d;
     return DFK_OK;
   }
@@ -1251,8 +1479,8 @@ static int check_gate_up(const void *x, const void *gamma, bool norm, float eps,
   if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
   if (variant > 0) {
     const VDef *d = find_variant(variant);
-    if (!d || d->cls != CLS_GATE_UP)
-      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a gate/up variant", variant);
+    if (!d || d->cls != CLS_GATE_UP || !bf16_capable(*d))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a bf16 gate/up variant", variant);
   }
   if (norm && !(eps >= 0.f && std::isfinite(eps)))
     return fail(DFK_ERR_INVALID_ARG, "eps must be finite and >= 0");
@@ -1279,8 +1507,8 @@ static int check_gemv(const void *x, const void *w, const void *out, int B, int 
   if (variant < 0) return fail(DFK_ERR_INVALID_ARG, "variant id %d < 0", variant);
   if (variant > 0) {
     const VDef *d = find_variant(variant);
-    if (!d || d->cls != CLS_GEMV)
-      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a GEMV variant", variant);
+    if (!d || d->cls != CLS_GEMV || !bf16_capable(*d))
+      return fail(DFK_ERR_INVALID_ARG, "variant %d is not a bf16 GEMV variant", variant);
   }
   if (B > 64) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "B=%d > 64 (decode batches only)", B);
   if (K % 8) return fail(DFK_ERR_UNSUPPORTED_SHAPE, "reduction length %% 8 != 0 (K=%d)", K);
@@ -1552,7 +1780,9 @@ int dfk_variant_info(int variant_id, dfk_variant *out) {
   if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
   const VDef *d = find_variant(variant_id);
   if (!d) return fail(DFK_ERR_INVALID_ARG, "no variant %d", variant_id);
-  fill_variant(*d, d->cls == CLS_GEMV ? DFK_OP_DOWN : DFK_OP_GATE_UP, -1, 0, -1.f, out);
+  const int op = d->e4m3mma ? (d->cls == CLS_GEMV ? DFK_OP_DOWN_FP8 : DFK_OP_GATE_UP_FP8)
+                            : (d->cls == CLS_GEMV ? DFK_OP_DOWN : DFK_OP_GATE_UP);
+  fill_variant(*d, op, -1, 0, -1.f, out);
   return DFK_OK;
 }
 

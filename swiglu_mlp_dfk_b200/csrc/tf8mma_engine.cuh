@@ -1,0 +1,428 @@
+// tf8mma_engine.cuh -- FP8 weights on the E4M3 tensor-core MMA
+// (tcgen05.mma kind::f8f6f4): the weight codes are the MMA's A operand as
+// they arrive from HBM, with no per-weight work on the CUDA cores.
+//
+// Same operation as the other FP8 kernels (W[j][k] = s[j] * E4M3(q[j][k]);
+// "Deep Kernel Fusion for Transformer Decoding", episode description, with
+// the dequantisation inside the product as GPULlama3.java PR #78 does).  The
+// MMA multiplies E4M3 by E4M3, so the activations are written as a short sum
+// of E4M3 terms per token b (a prep kernel does this once per call):
+//   v[k] = x[b][k] * gamma[k]  (RMSNorm; exact in fp32)  or  x[b][k],
+//   u[k] = v[k] * 2^e_b         (e_b puts max_k |u| in [128, 256)),
+//   c_0 = E4M3(u), c_t = E4M3((u - sum_{i<t} c_i 16^-i) 16^t)  (t < T),
+// so u = sum_t c_t 16^-t up to the last residual.  Two terms carry a bf16
+// value exactly (8 significant bits, 4 per E4M3 term) and four terms the
+// 16-bit x * gamma products, for every element within 2^17 of the token's
+// largest (smaller ones are carried to about 2^-21 of it).  Term t of token
+// b is row t * bnp + b of the MMA's B operand, so one MMA of N = T * bnp
+// reads each weight tile once for all terms and tokens, and
+//   sum_k W[j][k] v[k] = s[j] * 2^-e_b * sum_t 16^-t D[j][t * bnp + b],
+// the terms combined smallest first (Horner in 1/16, exact scalings).
+// The prep kernel also computes r_b = 1 / sqrt(mean x^2 + eps) for the
+// RMSNorm and stores f_b = r_b * 2^-e_b (1 * 2^-e_b without it).
+//
+// Main kernel: one CTA per SM owns r <= 128 weight rows (the MMA's M) over its
+// reduction range (split-K slices for the down projection); a TMA ring
+// carries 128-wide k tiles of codes (128-byte swizzle) and of the activation
+// terms; one thread issues 4 MMAs (K = 32) per matrix per tile; warps 2-5
+// read the accumulators, combine the terms, apply f_b, s[j], SiLU(gate) * up
+// and store bf16.  Rows of the 128-row MMA beyond r read neighbouring shared
+// memory and give ignored accumulator rows.
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tc_ptx.cuh"
+
+namespace dfk {
+
+constexpr int TM8_THREADS = 192;
+constexpr int TM8_TILE_K = 128;
+constexpr int TM8_PREP_THREADS = 256;
+
+// kind::f8f6f4 instruction descriptor: E4M3 A and B (format 0), fp32 D,
+// both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], one CTA, kind::f8f6f4 (K = 32).
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Two fp32 values -> two E4M3 codes (round to nearest even, saturating to
+// +-448), lo in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Exact value of the E4M3 code in byte 0 / byte 1 of a 16-bit pair.
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float &lo, float &hi) {
+  asm("{\n\t.reg .b16 c, a, b;\n\t.reg .b32 h;\n\t"
+      "cvt.u16.u32 c, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h, c;\n\t"
+      "mov.b32 {a, b}, h;\n\t"
+      "cvt.f32.f16 %0, a;\n\t"
+      "cvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(pair));
+}
+
+struct Tm8PrepParams {
+  const uint16_t *x;      // [B][K] bf16
+  const uint16_t *gamma;  // [K] bf16 or nullptr (no RMSNorm)
+  uint8_t *terms;         // [ntiles][T * bnp][128] E4M3 codes
+  float *fac;             // [bnp]: f_b (0 for padding tokens)
+  int B, K, bnp, T, ntiles;
+  float eps;
+};
+
+// One CTA per token slot b < bnp: pass 1 finds max |v| (and sum x^2 in a
+// fixed order), pass 2 writes the T term codes of every k (zeros past K and
+// for b >= B).  Defined in the one file that instantiates the kernels.
+#ifdef DFK_TF8MMA_KERNELS
+__global__ void __launch_bounds__(TM8_PREP_THREADS)
+    tf8mma_prep_kernel(const Tm8PrepParams p) {
+  __shared__ float s_max[TM8_PREP_THREADS / 32], s_ss[TM8_PREP_THREADS / 32];
+  __shared__ float s_scale, s_fac;
+  pdl_launch_dependents();
+  pdl_wait();  // x comes from the previous kernel
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool real = b < p.B;
+  const int nchunk = (p.ntiles * TM8_TILE_K) / 8;  // 8-element chunks incl. padding
+  const int kchunks = p.K / 8;
+  float mx = 0.f, ss = 0.f;
+  if (real) {
+    for (int c = tid; c < kchunks; c += TM8_PREP_THREADS) {
+      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
+      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
+      if (p.gamma) gv = ld_nc_v4(p.gamma + 8 * c);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
+        ss = fmaf(x0, x0, ss);
+        ss = fmaf(x1, x1, ss);
+        const float v0 = p.gamma ? x0 * bf16_lo(gw[u]) : x0;
+        const float v1 = p.gamma ? x1 * bf16_hi(gw[u]) : x1;
+        mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  }
+  if (lane == 0) {
+    s_max[warp] = mx;
+    s_ss[warp] = ss;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float m = 0.f, t = 0.f;
+    for (int w = 0; w < TM8_PREP_THREADS / 32; ++w) {
+      m = fmaxf(m, s_max[w]);
+      t += s_ss[w];
+    }
+    int e = 0;
+    if (m > 0.f) {
+      int E;
+      frexpf(m, &E);            // m = f * 2^E, f in [0.5, 1)
+      e = min(max(8 - E, -126), 126);  // m * 2^e in [128, 256)
+    }
+    s_scale = ldexpf(1.0f, e);
+    const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
+    s_fac = real ? r * ldexpf(1.0f, -e) : 0.f;
+  }
+  __syncthreads();
+  const float sc = s_scale;
+  if (tid == 0) p.fac[b] = s_fac;
+  const int rows = p.T * p.bnp;
+  for (int c = tid; c < nchunk; c += TM8_PREP_THREADS) {
+    const int k = 8 * c, tile = k / TM8_TILE_K, kk = k % TM8_TILE_K;
+    float u[8];
+    if (real && c < kchunks) {
+      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + k);
+      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
+      if (p.gamma) gv = ld_nc_v4(p.gamma + k);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x0 = bf16_lo(xw[i]), x1 = bf16_hi(xw[i]);
+        u[2 * i] = (p.gamma ? x0 * bf16_lo(gw[i]) : x0) * sc;
+        u[2 * i + 1] = (p.gamma ? x1 * bf16_hi(gw[i]) : x1) * sc;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[i] = 0.f;
+    }
+    for (int t = 0; t < p.T; ++t) {
+      uint32_t w[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t c01 = f32x2_to_e4m3x2(u[4 * h + 0], u[4 * h + 1]);
+        const uint32_t c23 = f32x2_to_e4m3x2(u[4 * h + 2], u[4 * h + 3]);
+        w[h] = c01 | (c23 << 16);
+        float d0, d1, d2, d3;
+        e4m3x2_to_f32(c01, d0, d1);
+        e4m3x2_to_f32(c23, d2, d3);
+        // residual, scaled for the next term (exact: |residual| <= half an
+        // E4M3 step of u, and times 16 stays below 448)
+        u[4 * h + 0] = (u[4 * h + 0] - d0) * 16.f;
+        u[4 * h + 1] = (u[4 * h + 1] - d1) * 16.f;
+        u[4 * h + 2] = (u[4 * h + 2] - d2) * 16.f;
+        u[4 * h + 3] = (u[4 * h + 3] - d3) * 16.f;
+      }
+      uint8_t *dst = p.terms + (static_cast<size_t>(tile) * rows + t * p.bnp + b) * TM8_TILE_K + kk;
+      *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+    }
+  }
+}
+#endif  // DFK_TF8MMA_KERNELS
+
+struct Tm8Params {
+  uint16_t *out;          // [B][N] bf16
+  const float *scale[2];  // per-row scales [N]
+  const float *fac;       // [bnp] per-token factor f_b (prep kernel)
+  unsigned *err;
+  int B, K, N;
+  int rbase, rextra, hmax, r8;
+  int bnp, T, np;         // tokens per term block, terms, np = T * bnp (the MMA's N)
+  int stages, stage_bytes, a8_bytes;
+  int tmem_cols;
+  int bar_off;
+  int ntiles, kslices, nblocks;
+  float *part;            // split-K partial sums [kslices][nblocks][bnp][128]
+  unsigned *counters;     // [nblocks]
+};
+
+// w[m][0]: codes of matrix m, box {128, hmax}; w[m][1]: box {128, hmax - 1};
+// x: the term codes [ntiles * np][128], box {128, np}.  128-byte swizzle.
+struct Tm8Maps {
+  CUtensorMap w[2][2];
+  CUtensorMap x;
+};
+
+template <int NMAT>
+__global__ void __launch_bounds__(TM8_THREADS, 1)
+    tf8mma_kernel(const __grid_constant__ Tm8Maps maps, const Tm8Params p) {
+  static_assert(NMAT == 1 || NMAT == 2, "NMAT");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = p.stages, NP = p.np;
+
+  uint64_t *fullb = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+  uint64_t *empty = fullb + S;
+  uint64_t *accfull = empty + S;
+  volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
+  int *s_issued = reinterpret_cast<int *>(accfull + 1) + 1;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accfull + 1) + 2;
+  volatile int *s_last = reinterpret_cast<volatile int *>(accfull + 1) + 3;
+
+  const int cta = blockIdx.x;
+  const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
+  const int j0 = blk * p.rbase + min(blk, p.rextra);
+  const int r = p.rbase + (blk < p.rextra ? 1 : 0);
+  const int mi = (r == p.hmax) ? 0 : 1;
+  const int tile0 = (slc * p.ntiles) / p.kslices;
+  const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
+  const int nsteps = tile1 - tile0;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&fullb[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    *s_abort = 0;
+    *s_issued = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ================= TMA producer (one lane): codes first; the term tiles
+    // only after the prep kernel's results are visible
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_normal();
+      const int S0 = min(S, nsteps);
+      int issued = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int st = i % S;
+        if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
+        uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
+        const int tile = tile0 + i;
+        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>((NMAT * r + NP) * 128));
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+          tma_load_2d(sb + m * p.r8 * 128, &maps.w[m][mi], &fullb[st], tile * TM8_TILE_K, j0,
+                      pol_w);
+        if (i >= S0) tma_load_2d(sb + p.a8_bytes, &maps.x, &fullb[st], 0, tile * NP, pol_x);
+        if (i == S0 - 1) {
+          pdl_wait();
+          for (int ii = 0; ii < S0; ++ii)
+            tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a8_bytes, &maps.x,
+                        &fullb[ii], 0, (tile0 + ii) * NP, pol_x);
+        }
+        issued = i + 1;
+      }
+      *s_issued = issued;
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (one lane): per tile and matrix, 4 MMAs of
+    // K = 32 (32 bytes further into each swizzled 128-byte row)
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_e4m3_f32(128, NP);
+      const uint64_t desc0 = umma_desc_sw128(sbase);
+      const uint32_t tile_enc = static_cast<uint32_t>(p.r8 * 128) >> 4;
+      const uint32_t x_enc = static_cast<uint32_t>(p.a8_bytes) >> 4;
+      for (int i = 0; i < nsteps; ++i) {
+        const int st = i % S;
+        if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
+        tc_fence_after();
+        const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+            umma_e4m3(tmem + static_cast<uint32_t>(m * NP), ds + m * tile_enc + 2 * kk,
+                      ds + x_enc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[st]);
+      }
+      umma_commit(accfull);
+    }
+  } else {
+    // ================= epilogue (warps 2..5, one per TMEM lane quarter)
+    const int et = tid - 64;
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const bool okw = mbar_wait_bounded(accfull, 0, s_abort, p.err);
+    tc_fence_after();
+    const bool go = __all_sync(0xffffffffu, okw && !*s_abort);
+    if (go) {
+      const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      const int j = j0 + row;
+      float sg = 0.f, su = 0.f;
+      if (p.kslices == 1 && row < r) {
+        sg = __ldg(p.scale[0] + j);
+        if (NMAT == 2) su = __ldg(p.scale[1] + j);
+      }
+      for (int c = 0; c < p.bnp; c += 16) {
+        // terms combined smallest first: S = D_0 + (D_1 + (...) / 16) / 16
+        float g[16], u[16];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+          float acc[16];
+          for (int t = p.T - 1; t >= 0; --t) {
+            float d[16];
+            tmem_ld_32x32b_x16(base + m * NP + t * p.bnp + c, d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = (t == p.T - 1) ? d[e] : d[e] + acc[e] * 0.0625f;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            if (m == 0) g[e] = acc[e];
+            else u[e] = acc[e];
+          }
+        }
+        if (p.kslices > 1) {
+          float *mine = p.part + (static_cast<size_t>(slc) * p.nblocks + blk) * p.bnp * 128;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mine[(c + e) * 128 + row] = g[e];
+        } else if (row < r) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int n = c + e;
+            if (n < p.B) {
+              const float f = __ldg(p.fac + n);
+              float res;
+              if (NMAT == 2) {
+                const float a = (g[e] * f) * sg, uu = (u[e] * f) * su;
+                res = (a / (1.0f + expf(-a))) * uu;
+              } else {
+                res = (g[e] * f) * sg;
+              }
+              p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
+            }
+          }
+        }
+      }
+    }
+    if (p.kslices > 1) {
+      // every CTA of the row block takes part in the count (also after an
+      // abort); the last one adds the slices in order, scales and stores
+      __threadfence();
+      named_barrier(2, 128);
+      if (et == 0) {
+        const unsigned old = atomicAdd(&p.counters[blk], 1u);
+        *s_last = (old == static_cast<unsigned>(p.kslices - 1)) ? 1 : 0;
+      }
+      named_barrier(2, 128);
+      if (*s_last) {
+        __threadfence();
+        if (row < r && !*s_abort) {
+          const float sd = __ldg(p.scale[0] + j0 + row);
+          for (int n = 0; n < p.B; ++n) {
+            float acc = 0.f;
+            for (int sl = 0; sl < p.kslices; ++sl) {
+              const float v = __ldcg(p.part + ((static_cast<size_t>(sl) * p.nblocks + blk) * p.bnp +
+                                               n) * 128 + row);
+              acc = (sl == 0) ? v : acc + v;
+            }
+            p.out[static_cast<size_t>(n) * p.N + j0 + row] =
+                f32_to_bf16_bits((acc * __ldg(p.fac + n)) * sd);
+          }
+        }
+        named_barrier(2, 128);
+        if (et == 0) p.counters[blk] = 0u;
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) mbar_wait_bounded(accfull, 0, nullptr, p.err);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+  if (tid == 0 && *s_abort) {
+    const int issued = *s_issued;
+    for (int st = 0; st < S; ++st) {
+      int last = -1;
+      for (int i = issued - 1; i >= 0 && i >= issued - S; --i)
+        if (i % S == st) { last = i; break; }
+      if (last >= 0) mbar_wait_bounded(&fullb[st], (last / S) & 1, nullptr, p.err);
+    }
+  }
+}
+
+}  // namespace dfk

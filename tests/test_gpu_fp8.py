@@ -264,11 +264,11 @@ def test_fp8_scheduler_select_variant():
 # ------------------------------------------------------------------ tensor-core FP8 kernel
 
 def tc_fp8_ids(down):
-    """Tensor-core variant ids that run FP8 weights (one k tile per stage, rows spread)."""
+    """Ids of the widening FP8 tensor-core kernel (one k tile per stage, rows spread)."""
     want = dfk.DFK_OP_DOWN if down else dfk.DFK_OP_GATE_UP
     return [v for v in (dfk.dfk_variant_info(i) for i in range(1, dfk.dfk_variant_count() + 1))
             if v["op"] == want and v["family"] == 1 and v["k_tiles_per_stage"] == 1
-            and v["full_m_tiles"] == 0]
+            and v["full_m_tiles"] == 0 and v["e4m3_mma"] == 0]
 
 
 TC_SHAPES = [(1, 256, 688), (2, 144, 200), (5, 400, 1000), (16, 1024, 1496), (17, 272, 96),
@@ -363,3 +363,92 @@ def test_fp8_tensor_core_is_exact_dequantisation():
                                          variant=v["variant_id"])
     torch.cuda.synchronize()
     assert bits_equal(h8, h16)
+
+
+# ------------------------------------------------------------------ E4M3-MMA kernel
+
+def e4m3_mma_ids(down):
+    want = dfk.DFK_OP_DOWN_FP8 if down else dfk.DFK_OP_GATE_UP_FP8
+    return [v for v in (dfk.dfk_variant_info(i) for i in range(1, dfk.dfk_variant_count() + 1))
+            if v["op"] == want and v["e4m3_mma"] == 1]
+
+
+def test_e4m3_mma_ids_are_fp8_only():
+    gu, dn = e4m3_mma_ids(False), e4m3_mma_ids(True)
+    assert len(gu) == 1 and len(dn) == 3
+    x = torch.zeros(2, 256, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(264, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dfk.DfkError) as e:
+        dfk.dfk_swiglu_gate_up(x, w, w, "row", variant=gu[0]["variant_id"])
+    assert e.value.status == dfk.DFK_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,D,F", TC_SHAPES)
+@pytest.mark.parametrize("norm", [False, True])
+def test_fp8_e4m3_mma_gate_up(B, D, F, norm):
+    (v,) = e4m3_mma_ids(False)
+    L = Fp8Layer(B, D, F, seed=500 + B, norm=norm, with_down=False)
+    h = L.gate_up(norm, variant=v["variant_id"])
+    torch.cuda.synchronize()
+    assert_close(h, L.oracle_gate_up(norm), "fp8 e4m3-mma gate/up B=%d D=%d F=%d" % (B, D, F))
+
+
+@pytest.mark.parametrize("B,D,F", [(1, 256, 688), (3, 520, 400), (16, 1024, 2048),
+                                   (40, 272, 1024), (64, 384, 2064)])
+def test_fp8_e4m3_mma_down_every_split(B, D, F):
+    L = Fp8Layer(B, D, F, seed=510 + B, norm=False)
+    h = (torch.randn(B, F, device="cuda") * 0.5).to(torch.bfloat16)
+    want = L.oracle_down(h)
+    ran = 0
+    for v in e4m3_mma_ids(True):
+        y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid),
+                        v["variant_id"])
+        if y is None:
+            continue
+        y2 = dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=v["variant_id"])
+        torch.cuda.synchronize()
+        assert_close(y, want, "fp8 e4m3-mma down ks=%d B=%d" % (v["k_split"], B))
+        assert bits_equal(y, y2), "split-K result not repeatable"
+        ran += 1
+    assert ran >= 2
+
+
+@pytest.mark.parametrize("norm", [False, True])
+def test_fp8_e4m3_mma_encodes_activations_closely(norm):
+    # the CUDA-core FP8 kernel multiplies by the exact activations; the E4M3
+    # terms (2 for bf16 x, 4 for x * gamma) must leave only accumulation-order
+    # and output-rounding differences: within two bf16 steps of each other
+    (v,) = e4m3_mma_ids(False)
+    B, D, F = 8, 1024, 1496
+    L = Fp8Layer(B, D, F, seed=520 + norm, norm=norm, with_down=False)
+    cc = next(w["variant_id"] for w in cc_ids(dfk.DFK_OP_GATE_UP_FP8)
+              if w["j_per_thread"] == 2 and w["token_tile"] == 8)
+    a = I.bf16_values(L.gate_up(norm, variant=v["variant_id"]))
+    b = I.bf16_values(L.gate_up(norm, variant=cc))
+    torch.cuda.synchronize()
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.abs(b) + 1e-4)
+
+
+@pytest.mark.parametrize("B", [1, 16, 64])
+def test_fp8_e4m3_mma_llama3_8b_sampled_rows(B):
+    w = I.WORKLOADS["llama3_8b"]
+    L = Fp8Layer(B, w.d_model, w.d_ff, seed=w.seed, norm=True)
+    (vg,) = e4m3_mma_ids(False)
+    h = L.gate_up(True, variant=vg["variant_id"])
+    ys = []
+    for v in e4m3_mma_ids(True):
+        y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid),
+                        v["variant_id"])
+        if y is not None:
+            ys.append(y)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.d_ff, 160, 13)
+    idx = torch.from_numpy(rows).long().cuda()
+    assert_close(h[:, idx].contiguous(), L.oracle_gate_up(True, rows=rows),
+                 "fp8 e4m3-mma 8B gate/up rows B=%d" % B)
+    drows = sample_rows(w.d_model, 96, 14)
+    didx = torch.from_numpy(drows).long().cuda()
+    want = L.oracle_down(h, rows=drows)
+    assert ys
+    for y in ys:
+        assert_close(y[:, didx].contiguous(), want, "fp8 e4m3-mma 8B down rows B=%d" % B)
