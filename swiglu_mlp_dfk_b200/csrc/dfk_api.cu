@@ -266,6 +266,10 @@ static const std::vector<VDef> &variants() {
     t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, 1, 1, 0, 0, 1});
     for (int ks : {1, 2, 4})
       t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, 1, 1, 0, 0, 1});
+    // ... with two 128-wide k tiles per ring stage
+    t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, 2, 1, 0, 0, 1});
+    for (int ks : {1, 2, 4})
+      t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, 2, 1, 0, 0, 1});
     return t;
   }();
   return v;
@@ -274,7 +278,7 @@ static const std::vector<VDef> &variants() {
 // Variants that can run FP8 weights: CUDA-core ones, and tensor-core ones with
 // one k tile per stage whose rows are spread over the SMs.
 static bool fp8_capable(const VDef &d) {
-  return d.family == DFK_FAMILY_CUDA_CORE || (d.nt == 1 && d.full == 0);
+  return d.family == DFK_FAMILY_CUDA_CORE || (d.nt == 1 && d.full == 0) || d.e4m3mma;
 }
 
 // Variants that can run bf16 weights: all but the E4M3-MMA ones.
@@ -972,11 +976,15 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
     if (why) *why = "more than 128 output rows per CTA";
     return false;
   }
+  if (v.nt < 1 || v.nt > 2) {
+    if (why) *why = "one or two k tiles per stage";
+    return false;
+  }
   const int r8 = round_up(hmax, 8);
   const int a8 = nmat * r8 * 128;
-  const int stage = a8 + np * 128;  // both multiples of 1024
+  const int stage = v.nt * (a8 + np * 128);  // multiples of 1024
   // the last code tile's 128-row MMA read may run past the last stage
-  const int over = (nmat - 1) * r8 * 128 + 128 * 128;
+  const int over = (v.nt * nmat - 1) * r8 * 128 + 128 * 128;
   const int slack = std::max(0, over - stage);
   const int bar_bytes = 256;        // 2 S + 1 barriers and flags
   const int smem_cap = std::min(ds.smem_optin, 232448);
@@ -1002,6 +1010,7 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   p.bnp = bnp;
   p.T = T;
   p.np = np;
+  p.nt = v.nt;
   p.stages = S;
   p.stage_bytes = stage;
   p.a8_bytes = a8;
@@ -1115,8 +1124,11 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
   pp.ntiles = p.ntiles;
   pp.eps = c.eps;
   void *pargs[] = {&pp};
-  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
-                                pdl_enabled(), pargs);
+  // P CTAs per token (a cluster), one 256-thread pass over ~K / P elements each
+  const unsigned P = static_cast<unsigned>(
+      std::min(8, std::max(1, ceil_div(p.ntiles * TM8_TILE_K / 8, TM8_PREP_THREADS))));
+  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(P, p.bnp), dim3(TM8_PREP_THREADS), 0, s,
+                                pdl_enabled(), pargs, P);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_fail(e, "FP8 activation-term kernel launch");
@@ -1263,7 +1275,7 @@ static std::vector<const VDef *> candidates(int op, int B, const CcCall &c) {
     if (d.cls != op_class(op)) continue;
     if (c.w8 && d.family == DFK_FAMILY_TENSOR_CORE) {
       // FP8: the tensor-core kernels (widening, E4M3 MMA) at every batch
-      if (d.nt == 1 && d.full == 0) out.push_back(&d);
+      if (fp8_capable(d)) out.push_back(&d);
       continue;
     }
     if (!c.w8 && !bf16_capable(d)) continue;

@@ -8,18 +8,32 @@ namespace dfk {
 // the launch may begin while the previous kernel in the stream finishes;
 // kernels here call griddepcontrol.wait before touching data that the
 // previous kernel writes, so this only overlaps their prologues.
+// `cluster_x` > 1 groups that many consecutive blocks along x into a
+// thread-block cluster (portable sizes: at most 8).
 inline cudaError_t launch_kernel(const void *fn, dim3 grid, dim3 block, size_t smem,
-                                 cudaStream_t stream, bool pdl, void **args) {
+                                 cudaStream_t stream, bool pdl, void **args,
+                                 unsigned cluster_x = 1) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 

@@ -18,8 +18,9 @@
 // reads each weight tile once for all terms and tokens, and
 //   sum_k W[j][k] v[k] = s[j] * 2^-e_b * sum_t 16^-t D[j][t * bnp + b],
 // the terms combined smallest first (Horner in 1/16, exact scalings).
-// The prep kernel also computes r_b = 1 / sqrt(mean x^2 + eps) for the
-// RMSNorm and stores f_b = r_b * 2^-e_b (1 * 2^-e_b without it).
+// The prep kernel (a cluster of up to 8 CTAs per token, partials combined
+// through distributed shared memory) also computes r_b = 1 / sqrt(mean x^2 +
+// eps) for the RMSNorm and stores f_b = r_b * 2^-e_b (1 * 2^-e_b without it).
 //
 // Main kernel: one CTA per SM owns r <= 128 weight rows (the MMA's M) over its
 // reduction range (split-K slices for the down projection); a TMA ring
@@ -31,6 +32,8 @@
 #pragma once
 #include <cuda.h>
 #include <cstdint>
+
+#include <cooperative_groups.h>
 
 #include "ptx.cuh"
 #include "tc_ptx.cuh"
@@ -88,23 +91,31 @@ struct Tm8PrepParams {
   float eps;
 };
 
-// One CTA per token slot b < bnp: pass 1 finds max |v| (and sum x^2 in a
-// fixed order), pass 2 writes the T term codes of every k (zeros past K and
-// for b >= B).  Defined in the one file that instantiates the kernels.
+// One cluster of P CTAs (blockIdx.x = rank) per token slot b = blockIdx.y;
+// each CTA takes a contiguous range of 8-element chunks.  Pass 1: max |v| and
+// sum x^2 of the range (fixed order: thread chains, warp butterfly, warps in
+// order); the ranks' partials are combined in rank order through distributed
+// shared memory; pass 2 writes the T term codes of the range (zeros past K
+// and for b >= B).  Defined in the one file that instantiates the kernels.
 #ifdef DFK_TF8MMA_KERNELS
 __global__ void __launch_bounds__(TM8_PREP_THREADS)
     tf8mma_prep_kernel(const Tm8PrepParams p) {
-  __shared__ float s_max[TM8_PREP_THREADS / 32], s_ss[TM8_PREP_THREADS / 32];
-  __shared__ float s_scale, s_fac;
+  __shared__ float s_part[2];  // this CTA's max |v| and sum x^2
+  __shared__ float s_wmax[TM8_PREP_THREADS / 32], s_wss[TM8_PREP_THREADS / 32];
+  __shared__ float s_scale;
+  cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
   pdl_launch_dependents();
   pdl_wait();  // x comes from the previous kernel
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rank = blockIdx.x, P = gridDim.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool real = b < p.B;
   const int nchunk = (p.ntiles * TM8_TILE_K) / 8;  // 8-element chunks incl. padding
   const int kchunks = p.K / 8;
+  const int per = (nchunk + P - 1) / P;
+  const int c0 = rank * per, c1 = min(nchunk, c0 + per);
   float mx = 0.f, ss = 0.f;
   if (real) {
-    for (int c = tid; c < kchunks; c += TM8_PREP_THREADS) {
+    for (int c = c0 + tid; c < min(c1, kchunks); c += TM8_PREP_THREADS) {
       const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
       uint4 gv = make_uint4(0u, 0u, 0u, 0u);
       if (p.gamma) gv = ld_nc_v4(p.gamma + 8 * c);
@@ -126,31 +137,43 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS)
     ss += __shfl_xor_sync(0xffffffffu, ss, m);
   }
   if (lane == 0) {
-    s_max[warp] = mx;
-    s_ss[warp] = ss;
+    s_wmax[warp] = mx;
+    s_wss[warp] = ss;
   }
   __syncthreads();
   if (tid == 0) {
     float m = 0.f, t = 0.f;
     for (int w = 0; w < TM8_PREP_THREADS / 32; ++w) {
-      m = fmaxf(m, s_max[w]);
-      t += s_ss[w];
+      m = fmaxf(m, s_wmax[w]);
+      t += s_wss[w];
+    }
+    s_part[0] = m;
+    s_part[1] = t;
+  }
+  cl.sync();  // every rank's partials are in its shared memory
+  if (tid == 0) {
+    float m = 0.f, t = 0.f;
+    for (int q = 0; q < P; ++q) {
+      const float *rp = cl.map_shared_rank(s_part, q);
+      m = fmaxf(m, rp[0]);
+      t += rp[1];
     }
     int e = 0;
     if (m > 0.f) {
       int E;
-      frexpf(m, &E);            // m = f * 2^E, f in [0.5, 1)
+      frexpf(m, &E);                   // m = f * 2^E, f in [0.5, 1)
       e = min(max(8 - E, -126), 126);  // m * 2^e in [128, 256)
     }
     s_scale = ldexpf(1.0f, e);
-    const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
-    s_fac = real ? r * ldexpf(1.0f, -e) : 0.f;
+    if (rank == 0) {
+      const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
+      p.fac[b] = real ? r * ldexpf(1.0f, -e) : 0.f;
+    }
   }
-  __syncthreads();
+  cl.sync();  // remote reads done (no CTA leaves early); s_scale visible
   const float sc = s_scale;
-  if (tid == 0) p.fac[b] = s_fac;
   const int rows = p.T * p.bnp;
-  for (int c = tid; c < nchunk; c += TM8_PREP_THREADS) {
+  for (int c = c0 + tid; c < c1; c += TM8_PREP_THREADS) {
     const int k = 8 * c, tile = k / TM8_TILE_K, kk = k % TM8_TILE_K;
     float u[8];
     if (real && c < kchunks) {
@@ -200,7 +223,8 @@ struct Tm8Params {
   int B, K, N;
   int rbase, rextra, hmax, r8;
   int bnp, T, np;         // tokens per term block, terms, np = T * bnp (the MMA's N)
-  int stages, stage_bytes, a8_bytes;
+  int nt;                 // 128-wide k tiles per ring stage (1 or 2)
+  int stages, stage_bytes, a8_bytes;  // a8_bytes: code bytes of one tile (NMAT * r8 * 128)
   int tmem_cols;
   int bar_off;
   int ntiles, kslices, nblocks;
@@ -242,7 +266,10 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
   const int mi = (r == p.hmax) ? 0 : 1;
   const int tile0 = (slc * p.ntiles) / p.kslices;
   const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
-  const int nsteps = tile1 - tile0;
+  const int NT = p.nt;
+  const int nsteps = (tile1 - tile0 + NT - 1) / NT;
+  // stage layout: code tiles [tt][m] (r8 rows each), then term tiles [tt] (np rows)
+  const int codes_bytes = NT * p.a8_bytes;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -276,18 +303,27 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
         const int st = i % S;
         if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
-        const int tile = tile0 + i;
-        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>((NMAT * r + NP) * 128));
+        const int nv = min(NT, tile1 - (tile0 + i * NT));  // k tiles of this stage
+        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>(nv * (NMAT * r + NP) * 128));
+        for (int tt = 0; tt < nv; ++tt) {
+          const int tile = tile0 + i * NT + tt;
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-          tma_load_2d(sb + m * p.r8 * 128, &maps.w[m][mi], &fullb[st], tile * TM8_TILE_K, j0,
-                      pol_w);
-        if (i >= S0) tma_load_2d(sb + p.a8_bytes, &maps.x, &fullb[st], 0, tile * NP, pol_x);
+          for (int m = 0; m < NMAT; ++m)
+            tma_load_2d(sb + tt * p.a8_bytes + m * p.r8 * 128, &maps.w[m][mi], &fullb[st],
+                        tile * TM8_TILE_K, j0, pol_w);
+          if (i >= S0)
+            tma_load_2d(sb + codes_bytes + tt * NP * 128, &maps.x, &fullb[st], 0, tile * NP,
+                        pol_x);
+        }
         if (i == S0 - 1) {
           pdl_wait();
-          for (int ii = 0; ii < S0; ++ii)
-            tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a8_bytes, &maps.x,
-                        &fullb[ii], 0, (tile0 + ii) * NP, pol_x);
+          for (int ii = 0; ii < S0; ++ii) {
+            const int nvi = min(NT, tile1 - (tile0 + ii * NT));
+            for (int tt = 0; tt < nvi; ++tt)
+              tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + codes_bytes +
+                              tt * NP * 128,
+                          &maps.x, &fullb[ii], 0, (tile0 + ii * NT + tt) * NP, pol_x);
+          }
         }
         issued = i + 1;
       }
@@ -300,18 +336,24 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
       const uint32_t idesc = umma_idesc_e4m3_f32(128, NP);
       const uint64_t desc0 = umma_desc_sw128(sbase);
       const uint32_t tile_enc = static_cast<uint32_t>(p.r8 * 128) >> 4;
-      const uint32_t x_enc = static_cast<uint32_t>(p.a8_bytes) >> 4;
+      const uint32_t a_enc = static_cast<uint32_t>(p.a8_bytes) >> 4;
+      const uint32_t x_enc = static_cast<uint32_t>(codes_bytes) >> 4;
+      const uint32_t xt_enc = static_cast<uint32_t>(NP * 128) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
         if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
+        const int nv = min(NT, tile1 - (tile0 + i * NT));
+        for (int tt = 0; tt < nv; ++tt) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-          for (int m = 0; m < NMAT; ++m)
-            umma_e4m3(tmem + static_cast<uint32_t>(m * NP), ds + m * tile_enc + 2 * kk,
-                      ds + x_enc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            for (int m = 0; m < NMAT; ++m)
+              umma_e4m3(tmem + static_cast<uint32_t>(m * NP),
+                        ds + tt * a_enc + m * tile_enc + 2 * kk, ds + x_enc + tt * xt_enc + 2 * kk,
+                        idesc, (i > 0 || tt > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty[st]);
       }
