@@ -25,13 +25,19 @@
 // two bf16 values has at most 16 significant bits, so hi + lo is exact),
 // accumulate sum_k x^2 on the way, and scale by r_b in the epilogue.  The hi
 // and lo rows sit side by side on N (one MMA of N = 2 * bn reads each weight
-// tile once); the epilogue adds the two column halves.
+// tile once); the epilogue adds the two column halves.  NORM = 1 does this
+// transform inside the kernel; NORM = 2 reads tiles that a prep kernel (a
+// thread-block cluster per token, launched just before) wrote in the same
+// layout, with r_b, so the kernel streams them like plain activations (the
+// in-kernel transform serialises with the MMAs and costs a third of the time
+// at 64 tokens; the host uses NORM = 2 above 32 tokens).
 //
 // Warp roles (192 threads): warp 0 issues TMA copies into an S-stage ring;
 // warp 1 owns TMEM and issues the MMAs (one thread) with tcgen05.commit
 // releasing ring stages; warps 2-5 run the x*gamma transform (NORM) and the
 // epilogue (tcgen05.ld -> SiLU * up -> one bf16 store per output).
 #pragma once
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cstdint>
 
@@ -46,7 +52,8 @@ constexpr int TC_ATOM = 1024;       // bytes of an 8-row swizzle atom
 
 struct TcParams {
   uint16_t *out;          // [B][N] bf16
-  const uint16_t *gamma;  // [K] bf16 (NORM)
+  const uint16_t *gamma;  // [K] bf16 (NORM = 1)
+  const float *rinv;      // [bn] r_b from the prep kernel (NORM = 2)
   unsigned *err;          // device error word
   int B, K, N;
   float eps;
@@ -125,7 +132,8 @@ __device__ __forceinline__ void tmem_sum_banks(uint32_t taddr, int nb, int bank_
 // WL (weight layout): 0 row-major [N][K] (K-major A), 1 column-major [K][N]
 // (MN-major A; each CTA owns 128 columns, loaded as two 64-column boxes),
 // 2 interleaved [N][2][K].
-template <int NMAT, bool NORM, int WL, int MT>
+// NORM: 0 none, 1 x * gamma transform in the kernel, 2 prepared tiles.
+template <int NMAT, int NORM, int WL, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemv_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
   constexpr bool IL = WL == 2, COLM = WL == 1;
@@ -133,6 +141,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   static_assert(!IL || NMAT == 2, "interleaved layout holds both matrices");
   static_assert(!COLM || MT == 1, "column-major: one 128-column tile per CTA");
   static_assert(!NORM || NMAT == 2, "the RMSNorm prologue belongs to the gate/up kernel");
+  static_assert(NORM >= 0 && NORM <= 2, "NORM");
+  constexpr int XROWS = NORM == 2 ? 2 : 1;  // activation rows per token loaded by TMA
   static_assert(MT == 1 || MT == 2, "MT");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base (the host reserves the slack)
@@ -206,8 +216,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
         const int nv = min(NT, tile1 - (tile0 + i * NT));  // k-tiles of this step in range
         // (column-major boxes are always 64 x 64, zero-filled past the last column)
-        mbar_arrive_expect_tx(&fullb[st],
-                              static_cast<uint32_t>(nv) * (NMAT * (full ? 128 : r) + BN) * 128u);
+        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>(nv) *
+                                              (NMAT * (full ? 128 : r) + XROWS * BN) * 128u);
         for (int kt = 0; kt < nv; ++kt) {
           const int k0 = (tile0 + i * NT + kt) * TC_TILE_K;
 #pragma unroll
@@ -229,17 +239,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           // activations: only after the previous kernel's results are visible
-          if (i >= S0)
-            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &fullb[st], k0, 0, pol_x);
+          // (prepared tiles: rows tile * 2 bn .. of the prep kernel's buffer)
+          if (i >= S0) {
+            const int tl = tile0 + i * NT + kt;
+            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &fullb[st],
+                        NORM == 2 ? 0 : k0, NORM == 2 ? tl * 2 * BN : 0, pol_x);
+          }
         }
         if (i == S0 - 1) {
           pdl_wait();
           for (int ii = 0; ii < S0; ++ii) {
             const int nvi = min(NT, tile1 - (tile0 + ii * NT));
-            for (int kt = 0; kt < nvi; ++kt)
+            for (int kt = 0; kt < nvi; ++kt) {
+              const int tl = tile0 + ii * NT + kt;
               tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
                               kt * p.xt_bytes,
-                          &maps.x, &fullb[ii], (tile0 + ii * NT + kt) * TC_TILE_K, 0, pol_x);
+                          &maps.x, &fullb[ii], NORM == 2 ? 0 : tl * TC_TILE_K,
+                          NORM == 2 ? tl * 2 * BN : 0, pol_x);
+            }
           }
         }
         issued = i + 1;
@@ -264,7 +281,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        if (!mbar_wait_bounded(NORM ? &xready[st] : &fullb[st], (i / S) & 1, s_abort, p.err))
+        if (!mbar_wait_bounded(NORM == 1 ? &xready[st] : &fullb[st], (i / S) & 1, s_abort, p.err))
           break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
@@ -300,9 +317,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       umma_commit(accfull);       // every MMA issued above has completed
     }
   } else {
-    // ================= x*gamma transform (NORM) and epilogue: warps 2..5
+    // ================= x*gamma transform (NORM = 1) and epilogue: warps 2..5
     const int et = tid - 64;
-    if (NORM) {
+    if (NORM == 2) pdl_wait();  // r_b comes from the prep kernel
+    if (NORM == 1) {
       pdl_wait();
       const int kpad = ((p.ntiles + NT - 1) / NT) * NT * TC_TILE_K;
       for (int idx = et; idx < kpad / 8; idx += 128) {
@@ -406,7 +424,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (n < p.B) {
                 float res;
                 if (NMAT == 2) {
-                  const float sc = NORM ? s_rinv[n] : 1.0f;
+                  const float sc = NORM == 1 ? s_rinv[n] : (NORM == 2 ? p.rinv[n] : 1.0f);
                   const float a = g[e] * sc, uu = u[e] * sc;
                   res = (a / (1.0f + expf(-a))) * uu;
                 } else {
@@ -468,5 +486,94 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   }
 }
+
+// ---- prep for NORM = 2: one cluster of P CTAs (blockIdx.x = rank) per
+// token slot b = blockIdx.y, each over a contiguous range of 8-element
+// chunks.  sum x^2 in a fixed order (thread chains, warp butterfly, warps in
+// order, ranks in order through distributed shared memory) gives r_b; x *
+// gamma (exact in fp32) is split into bf16 hi + lo and written as rows
+// tile * 2 bn + b (hi) and tile * 2 bn + bn + b (lo) of 64 bf16 per k tile;
+// zeros past K and for b >= B.  Defined in the one file that instantiates
+// the kernels.
+struct TcPrepParams {
+  const uint16_t *x;      // [B][K] bf16
+  const uint16_t *gamma;  // [K] bf16
+  uint16_t *xg;           // [ntiles][2 bn][64] bf16
+  float *rinv;            // [bn]
+  int B, K, bn, ntiles;
+  float eps;
+};
+
+constexpr int TC_PREP_THREADS = 256;
+
+#ifdef DFK_TC_KERNELS
+__global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcPrepParams p) {
+  __shared__ float s_part, s_wss[TC_PREP_THREADS / 32];
+  cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+  pdl_launch_dependents();
+  pdl_wait();  // x comes from the previous kernel
+  const int rank = blockIdx.x, P = gridDim.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool real = b < p.B;
+  const int nchunk = p.ntiles * TC_TILE_K / 8, kchunks = p.K / 8;
+  const int per = (nchunk + P - 1) / P;
+  const int c0 = rank * per, c1 = min(nchunk, c0 + per);
+  float ss = 0.f;
+  if (real) {
+    for (int c = c0 + tid; c < min(c1, kchunks); c += TC_PREP_THREADS) {
+      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
+        ss = fmaf(x0, x0, ss);
+        ss = fmaf(x1, x1, ss);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  if (lane == 0) s_wss[warp] = ss;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < TC_PREP_THREADS / 32; ++w) t += s_wss[w];
+    s_part = t;
+  }
+  cl.sync();  // every rank's partial sum is in its shared memory
+  if (tid == 0 && rank == 0) {
+    float t = 0.f;
+    for (int q = 0; q < P; ++q) t += *cl.map_shared_rank(&s_part, q);
+    p.rinv[b] = real ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 0.f;
+  }
+  cl.sync();  // remote reads done before any CTA of the cluster leaves
+  for (int c = c0 + tid; c < c1; c += TC_PREP_THREADS) {
+    const int k = 8 * c, tile = k / TC_TILE_K, kk = k % TC_TILE_K;
+    uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = make_uint4(0u, 0u, 0u, 0u);
+    if (real && c < kchunks) {
+      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + k);
+      const uint4 gv = ld_nc_v4(p.gamma + k);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float p0 = bf16_lo(xw[u]) * bf16_lo(gw[u]);  // exact
+        const float p1 = bf16_hi(xw[u]) * bf16_hi(gw[u]);
+        const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
+        const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+        const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+        hw[u] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+        lw[u] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
+                (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
+      }
+      hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    uint16_t *hrow = p.xg + (static_cast<size_t>(tile) * 2 * p.bn + b) * TC_TILE_K;
+    *reinterpret_cast<uint4 *>(hrow + kk) = hv;
+    *reinterpret_cast<uint4 *>(hrow + static_cast<size_t>(p.bn) * TC_TILE_K + kk) = lv;
+  }
+}
+#endif  // DFK_TC_KERNELS
 
 }  // namespace dfk

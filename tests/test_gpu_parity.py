@@ -461,3 +461,29 @@ def test_split_k_down_is_deterministic_and_resets():
         assert_close(y1[:, rows], ref, "split-K variant %d" % vid)
         assert_close(y_other, ref2, "split-K variant %d (second shape)" % vid)
     assert ran >= 2
+
+
+def test_tensor_core_rmsnorm_captured_on_a_fresh_stream():
+    # above 32 tokens the tensor-core RMSNorm path takes its activations from a
+    # prep kernel and a per-stream buffer; captured on a stream that has no
+    # buffer yet (none may be allocated during capture) it transforms in the
+    # kernel instead -- both must match the oracle
+    B, D, F = 64, 512, 776
+    inp = I.make_inputs(B, D, F, seed=777, w_std=0.05, with_down=False, device="cuda")
+    ref = oracle_gate_up(inp, True)
+    vid = tc_variants(dfk.DFK_OP_GATE_UP)[0]
+    h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row",
+                                       h=h, variant=vid)
+    g.replay()
+    torch.cuda.synchronize()
+    assert_close(h, ref, "captured in-kernel RMSNorm transform")
+    h2 = dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row",
+                                        variant=vid)
+    torch.cuda.synchronize()
+    assert_close(h2, ref, "prepared RMSNorm activations")
+    del g
