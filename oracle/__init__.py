@@ -14,6 +14,13 @@ PR #78 (description of the ``rms_ffn_gate_up`` task):
     h  = SiLU(xn @ Wg^T) * (xn @ Wu^T),  SiLU(a) = a / (1 + exp(-a))
     y  = h @ Wd^T
 
+and, for the packed QKV projection ("Optimizing QKV Projection with Operator
+Fusion", section "Implementing Fusion: Packed Projections": one wider linear
+layer replaces the three, its output split into Q, K and V; the RMSNorm in
+front as in the PR's ``fusedRmsNormQKVMatmul``):
+
+    o = xn @ Wqkv^T,  Wqkv = [Wq; Wk; Wv],  q, k, v = o[:, :nq], o[:, nq:nq+nk], o[:, nq+nk:]
+
 Inputs are bf16 bit patterns (numpy uint16); outputs are float64.
 """
 import ctypes
@@ -332,3 +339,21 @@ def down_fp8(h, qd, sd, rows=None) -> np.ndarray:
     if rc != 0:
         raise ValueError("dfk_oracle_down_fp8 rejected its arguments")
     return y
+
+
+def qkv(x, w_qkv, nq, nk, nv, gamma=None, eps=1e-5, rows=None):
+    """RMSNorm (optional) + packed QKV projection; returns (q, k, v) float64.
+
+    x [B, D] bf16 bits; w_qkv [nq + nk + nv, D] bf16 bits (rows of W_q, then
+    W_k, then W_v).  With ``rows`` (indices into the packed output), returns
+    the packed output o[:, rows] instead.  Composition of the RMSNorm and
+    matrix-product oracles: xn stays float64, the product is the same
+    definition as the down projection (sum_k xn[b][k] W[j][k])."""
+    w = np.asarray(w_qkv)
+    if w.shape[0] != nq + nk + nv:
+        raise ValueError("w_qkv must have nq + nk + nv rows")
+    xn = rmsnorm(x, gamma, eps) if gamma is not None else bf16_to_f64(np.asarray(x))
+    o = down(xn, w, rows=rows)
+    if rows is not None:
+        return o
+    return o[:, :nq], o[:, nq:nq + nk], o[:, nq + nk:]

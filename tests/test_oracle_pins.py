@@ -405,3 +405,55 @@ def test_fp8_scales_are_per_row_and_linear(oracle_mod):
     assert np.array_equal(2 * y1, oracle.down_fp8(h, qd, 2 * sd))
     assert np.allclose(y1, h @ (oracle.e4m3_to_f64(qd) * sd.astype(np.float64)[:, None]).T,
                        rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- packed QKV
+
+def test_qkv_hand_example(oracle_mod):
+    # D = 2, nq = 2, nk = 1, nv = 1; x = [3, 4] -> mean(x^2) = 12.5, r = 1/sqrt(12.5)
+    # gamma = [2, 1] -> xn = [6 r, 4 r]
+    x = bits([[3.0, 4.0]])
+    w = bits([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [1.0, -1.0]])
+    q, k, v = oracle.qkv(x, w, 2, 1, 1, gamma=bits([2.0, 1.0]), eps=0.0)
+    r = 1.0 / math.sqrt(12.5)
+    assert q[0] == pytest.approx([6 * r, 4 * r], rel=1e-15)
+    assert k[0, 0] == pytest.approx(10 * r, rel=1e-15)
+    assert v[0, 0] == pytest.approx(2 * r, rel=1e-15)
+    # without RMSNorm the product of the raw x
+    q, k, v = oracle.qkv(x, w, 2, 1, 1)
+    assert q[0].tolist() == [3.0, 4.0] and k[0, 0] == 7.0 and v[0, 0] == -1.0
+
+
+def test_qkv_packed_equals_three_projections_and_numpy(oracle_mod):
+    # the packed projection computes what three separate linear layers do
+    # (the fusion changes no math), checked against numpy's matmul as an
+    # independent routine
+    rng = np.random.default_rng(41)
+    B, D, nq, nk, nv = 3, 48, 32, 8, 8
+    x = oracle.f64_to_bf16(rng.standard_normal((B, D)))
+    g = oracle.f64_to_bf16(1.0 + 0.1 * rng.standard_normal(D))
+    wq = oracle.f64_to_bf16(0.05 * rng.standard_normal((nq, D)))
+    wk = oracle.f64_to_bf16(0.05 * rng.standard_normal((nk, D)))
+    wv = oracle.f64_to_bf16(0.05 * rng.standard_normal((nv, D)))
+    w = np.concatenate([wq, wk, wv])
+    q, k, v = oracle.qkv(x, w, nq, nk, nv, gamma=g, eps=1e-5)
+    xn = oracle.rmsnorm(x, g, eps=1e-5)
+    for got, ws in ((q, wq), (k, wk), (v, wv)):
+        assert np.array_equal(got, oracle.down(xn, ws))                  # separate layer
+        assert np.allclose(got, xn @ oracle.bf16_to_f64(ws).T, rtol=1e-13, atol=1e-14)
+    # packed rows subset
+    rows = np.array([0, nq, nq + nk, nq + nk + nv - 1], np.int32)
+    o = oracle.qkv(x, w, nq, nk, nv, gamma=g, eps=1e-5, rows=rows)
+    assert np.array_equal(o, np.concatenate([q[:, :1], k[:, :1], v[:, :1], v[:, -1:]], axis=1))
+
+
+def test_qkv_identity_weights_return_the_normalised_input(oracle_mod):
+    rng = np.random.default_rng(42)
+    D = 16
+    x = oracle.f64_to_bf16(rng.standard_normal((2, D)))
+    g = oracle.f64_to_bf16(1.0 + 0.1 * rng.standard_normal(D))
+    eye = oracle.f64_to_bf16(np.eye(D))
+    w = np.concatenate([eye, eye[:4], eye[4:8]])
+    q, k, v = oracle.qkv(x, w, D, 4, 4, gamma=g, eps=1e-5)
+    xn = oracle.rmsnorm(x, g, eps=1e-5)
+    assert np.array_equal(q, xn) and np.array_equal(k, xn[:, :4]) and np.array_equal(v, xn[:, 4:8])
