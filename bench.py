@@ -464,6 +464,7 @@ def extra_measurements(args, inp, copies, h, y):
     out["fp8_weights"] = fp8_measure()
     out["fp8_weights"]["bf16_b1_fused_us"] = round(t_fus, 2)
     torch.cuda.empty_cache()
+    out["qkv_projection"] = qkv_measure()
     out["decode_stack"] = decode_stack_measure(args.stack_steps)
     return out
 
@@ -553,6 +554,61 @@ def fp8_measure(reps=100, ncopies=4):
     torch.cuda.empty_cache()
     return {"workload": "llama3_8b_fp8_e4m3_row_scales", "weights": "E4M3 codes + fp32 row "
             "scales from the seeded bf16 weights (absmax / 448 per row)", "sweep": res}
+
+
+def qkv_bytes(B, D, N):
+    """Packed QKV projection: the weights once, x, gamma, the outputs."""
+    return N * D * 2 + B * D * 2 + D * 2 + B * N * 2
+
+
+def qkv_measure(reps=100, ncopies=4):
+    """RMSNorm + packed QKV projection on the Llama-3-8B attention input shape
+    (d_model 4096, n_q 4096, n_k = n_v = 1024; seeded weights ~ N(0, 0.02)):
+    fused (one kernel, one weight stream) against the pages' unfused form
+    (an RMSNorm kernel, then three separate projections), B = 1..64,
+    back-to-back calls over `ncopies` weight copies (50 MB each)."""
+    import torch
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    peak, _ = measured_peaks()
+    Dq, nq, nk, nv = 4096, 4096, 1024, 1024
+    N = nq + nk + nv
+    g = I.make_generator(7, "cuda")
+    x64 = torch.randn(64, Dq, generator=g, device="cuda").to(torch.bfloat16)
+    gamma = (1.0 + 0.1 * torch.randn(Dq, generator=g, device="cuda")).to(torch.bfloat16)
+    ws = [(0.02 * torch.randn(N, Dq, generator=g, device="cuda")).to(torch.bfloat16)
+          for _ in range(ncopies)]
+    res = []
+    for B in (1, 4, 16, 64):
+        x = x64[:B].contiguous()
+        q = torch.empty(B, nq, dtype=torch.bfloat16, device="cuda")
+        k = torch.empty(B, nk, dtype=torch.bfloat16, device="cuda")
+        v = torch.empty(B, nv, dtype=torch.bfloat16, device="cuda")
+        xn = torch.empty_like(x)
+        dfk.dfk_rmsnorm_qkv_proj(x, gamma, 1e-5, ws[0], nq, nk, nv, q=q, k=k, v=v)
+
+        def unfused(i):
+            w = ws[i % ncopies]
+            dfk.dfk_rmsnorm(x, gamma, 1e-5, out=xn)
+            dfk.dfk_gemv(xn, w[:nq], out=q)
+            dfk.dfk_gemv(xn, w[nq:nq + nk], out=k)
+            dfk.dfk_gemv(xn, w[nq + nk:], out=v)
+
+        unfused(0)                                    # scheduler decisions first
+        tf = timed_us(lambda i: dfk.dfk_rmsnorm_qkv_proj(x, gamma, 1e-5, ws[i % ncopies], nq, nk,
+                                                         nv, q=q, k=k, v=v), reps)
+        tu = timed_us(unfused, reps)
+        gbs = qkv_bytes(B, Dq, N) / (tf * 1e-6) / 1e9
+        vq = dfk.dfk_cached_variant(dfk.DFK_OP_RMSNORM_QKV, B, Dq, N) or {}
+        res.append({"B": B, "fused_us": round(tf, 2), "fused_GBps": round(gbs, 1),
+                    "fused_frac": round(gbs / peak, 4), "unfused_us": round(tu, 2),
+                    "speedup": round(tu / tf, 3), "variant": vq.get("variant_id"),
+                    "family": {0: "cuda_core", 1: "tensor_core"}.get(vq.get("family"))})
+    del ws, x64
+    torch.cuda.empty_cache()
+    return {"workload": "llama3_8b_qkv (d_model 4096, n_q 4096, n_k 1024, n_v 1024)",
+            "unfused": "rmsnorm + gemv(W_q) + gemv(W_k) + gemv(W_v)", "sweep": res}
 
 
 def decode_stack_measure(steps, layers=32, B=4):
@@ -688,6 +744,11 @@ def profile_arm(args):
         qu, su = I.to_fp8_rows(inp.w_up)
         fn = lambda: dfk.dfk_rmsnorm_swiglu_gate_up_fp8(inp.x, inp.gamma, inp.eps, qg, sg, qu,
                                                         su, h=h, variant=args.variant)
+    elif args.profile == "qkv":
+        nq, nk, nv = 4096, 1024, 1024
+        w_qkv = torch.cat([inp.w_gate[:nq], inp.w_up[:nk + nv]]).contiguous()  # seeded weights
+        fn = lambda: dfk.dfk_rmsnorm_qkv_proj(inp.x, inp.gamma, inp.eps, w_qkv, nq, nk, nv,
+                                              variant=args.variant)
     elif args.profile == "down_fp8":
         qd, sd = I.to_fp8_rows(inp.w_down)
         fn = lambda: dfk.dfk_down_proj_fp8(h, qd, sd, y=y, variant=args.variant)
@@ -716,7 +777,7 @@ def main():
                     help="skip the sweep / unfused / interleaved / decode-stack measurements")
     ap.add_argument("--stack-steps", type=int, default=512,
                     help="decode steps of the 32-layer stack measurement")
-    ap.add_argument("--profile", choices=["gate_up", "down", "gate_up_fp8", "down_fp8"],
+    ap.add_argument("--profile", choices=["gate_up", "down", "gate_up_fp8", "down_fp8", "qkv"],
                     default=None,
                     help="run only this kernel (inside an NVTX range) for ncu")
     ap.add_argument("--batch", type=int, default=1, help="batch for --profile")

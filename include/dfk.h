@@ -75,7 +75,9 @@ typedef enum dfk_op {
   DFK_OP_DOWN = 2,            /* dfk_down_proj               */
   DFK_OP_GATE_UP_FP8 = 3,     /* dfk_swiglu_gate_up_fp8      */
   DFK_OP_RMSNORM_GATE_UP_FP8 = 4, /* dfk_rmsnorm_swiglu_gate_up_fp8 */
-  DFK_OP_DOWN_FP8 = 5         /* dfk_down_proj_fp8           */
+  DFK_OP_DOWN_FP8 = 5,        /* dfk_down_proj_fp8           */
+  DFK_OP_QKV = 6,             /* dfk_rmsnorm_qkv_proj, gamma == NULL */
+  DFK_OP_RMSNORM_QKV = 7      /* dfk_rmsnorm_qkv_proj with RMSNorm   */
 } dfk_op;
 
 typedef enum dfk_family {
@@ -204,13 +206,40 @@ DFK_API int dfk_down_proj_fp8(const void *h, const void *q_down, const float *s_
                               int B, int d_model, int d_ff, int variant, void *stream);
 
 /*
+ * RMSNorm + packed QKV projection ("Optimizing QKV Projection with Operator
+ * Fusion", section "Implementing Fusion: Packed Projections": one wider
+ * projection replaces the separate Q, K and V ones and its output is split;
+ * the RMSNorm in front as the fusedRmsNormQKVMatmul task of GPULlama3.java
+ * PR #78):
+ *   xn = RMSNorm(x; gamma, eps) as for dfk_rmsnorm_swiglu_gate_up, or x when
+ *        gamma is NULL;
+ *   o[b][j] = sum_k xn[b][k] * w_qkv[j][k]  for j < n_q + n_k + n_v;
+ *   q[b][j] = o[b][j], k[b][j] = o[b][n_q + j], v[b][j] = o[b][n_q + n_k + j].
+ *   x      [B][d_model] bf16, device
+ *   w_qkv  [n_q + n_k + n_v][d_model] bf16 row-major (W_q rows, then W_k,
+ *          then W_v), device
+ *   q, k, v  [B][n_q], [B][n_k], [B][n_v] bf16, device, each written once;
+ *          a part of size 0 may be NULL
+ * One weight stream for all three parts and every token; the normalised
+ * activations never reach HBM.  Runs on the GEMV variants (variant 0 = the
+ * scheduler's choice, timed per shape under DFK_OP_QKV / DFK_OP_RMSNORM_QKV;
+ * for dfk_select_variant pass d_ff = n_q + n_k + n_v and a packed output).
+ * Part sizes >= 0 with a positive sum; otherwise as for dfk_down_proj.
+ */
+DFK_API int dfk_rmsnorm_qkv_proj(const void *x, const void *gamma, float eps,
+                                 const void *w_qkv, void *q, void *k, void *v, int B,
+                                 int d_model, int n_q, int n_k, int n_v, int variant,
+                                 void *stream);
+
+/*
  * Profiler-driven variant choice ("Deep Kernel Fusion for Transformer
  * Decoding", episode description: runtime scheduling across row-major and
  * column-major kernel variants; "Deep Kernel Fusion for Transformers",
  * abstract: the kernel is paired with a kernel scheduler).
  * Times every feasible variant of `op` for (B, d_model, d_ff, layout) with
  * CUDA events (each sample: L2 flushed, then a burst of 4 back-to-back
- * launches; median of DFK_TUNE_REPS samples), caches the fastest and
+ * launches -- or a single launch when one call's weights fit in L2; median
+ * of DFK_TUNE_REPS samples), caches the fastest and
  * returns it in *out.  layout == DFK_W_ANY times every layout and reports
  * the fastest layout in out->layout (gate/up ops only).
  *   sample_ptrs  NULL, or the caller's buffers in argument order of the op:

@@ -35,6 +35,8 @@ DFK_OP_DOWN = 2
 DFK_OP_GATE_UP_FP8 = 3
 DFK_OP_RMSNORM_GATE_UP_FP8 = 4
 DFK_OP_DOWN_FP8 = 5
+DFK_OP_QKV = 6
+DFK_OP_RMSNORM_QKV = 7
 # dfk_status
 DFK_OK = 0
 DFK_ERR_INVALID_ARG = 1
@@ -53,6 +55,7 @@ _LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W
 EXPORTED = (
     "dfk_swiglu_gate_up", "dfk_rmsnorm_swiglu_gate_up", "dfk_down_proj", "dfk_select_variant",
     "dfk_swiglu_gate_up_fp8", "dfk_rmsnorm_swiglu_gate_up_fp8", "dfk_down_proj_fp8",
+    "dfk_rmsnorm_qkv_proj",
     "dfk_down_proj_static_scratch", "dfk_cached_variant", "dfk_variant_count",
     "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
@@ -106,6 +109,7 @@ def lib():
                 "dfk_rmsnorm_swiglu_gate_up_fp8": [vp, vp, f, vp, vp, vp, vp, vp, i, i, i, i,
                                                    vp],
                 "dfk_down_proj_fp8": [vp, vp, vp, vp, i, i, i, i, vp],
+                "dfk_rmsnorm_qkv_proj": [vp, vp, f, vp, vp, vp, vp, i, i, i, i, i, i, vp],
                 "dfk_select_variant": [i, i, i, i, i, ctypes.POINTER(vp), vp,
                                        ctypes.POINTER(dfk_variant)],
                 "dfk_cached_variant": [i, i, i, i, i, ctypes.POINTER(dfk_variant)],
@@ -293,6 +297,26 @@ def dfk_down_proj_fp8(h, q_down, s_down, y=None, variant=0, stream=None):
     _check(lib().dfk_down_proj_fp8(_ptr(h), _ptr(q_down), _ptr(s_down), _ptr(y), B, D, F,
                                    int(variant), _stream(stream)))
     return y
+
+
+def dfk_rmsnorm_qkv_proj(x, gamma, eps, w_qkv, n_q, n_k, n_v, q=None, k=None, v=None,
+                         variant=0, stream=None):
+    """RMSNorm(x; gamma, eps) (skipped when gamma is None) + packed QKV projection with
+    w_qkv [n_q + n_k + n_v, d_model]; returns (q, k, v), [B, n_q] / [B, n_k] / [B, n_v]."""
+    for n, t in (("x", x), ("gamma", gamma), ("w_qkv", w_qkv), ("q", q), ("k", k), ("v", v)):
+        _dev_bf16(n, t)
+    B, D = x.shape
+    if w_qkv.shape != (n_q + n_k + n_v, D):
+        raise DfkError(DFK_ERR_INVALID_ARG, "w_qkv must be [n_q + n_k + n_v, d_model]")
+    outs = []
+    for t, n in ((q, n_q), (k, n_k), (v, n_v)):
+        outs.append(torch.empty((B, n), dtype=torch.bfloat16, device=x.device) if t is None else t)
+    _check(lib().dfk_rmsnorm_qkv_proj(_ptr(x), _ptr(gamma), float(eps), _ptr(w_qkv),
+                                      _ptr(outs[0]) if n_q else None,
+                                      _ptr(outs[1]) if n_k else None,
+                                      _ptr(outs[2]) if n_v else None,
+                                      B, D, n_q, n_k, n_v, int(variant), _stream(stream)))
+    return tuple(outs)
 
 
 def dfk_gemv(x, w, out=None, variant=0, stream=None):

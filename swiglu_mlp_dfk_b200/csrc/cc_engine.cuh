@@ -58,6 +58,8 @@ struct CcParams {
   const uint16_t *x;      // [B][K] bf16 activations
   const uint16_t *gamma;  // [K] bf16 RMSNorm weight (NORM only)
   uint16_t *out;          // [B][N] bf16
+  uint16_t *outs[3];      // split output (packed QKV) when outs[0] != nullptr: rows
+  int split[2];           // [0, split0) -> outs[0], [split0, split1) -> outs[1], rest -> outs[2]
   const float *scale[2];  // W8: per-output-row scales of each matrix [N] fp32
   unsigned *err;          // device error word
   int B, K, N;
@@ -592,7 +594,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
           } else {
             res = v[0];
           }
-          p.out[static_cast<size_t>(b) * p.N + j] = f32_to_bf16_bits(res);
+          store_out(p, b, j, f32_to_bf16_bits(res));
         }
       }
       named_barrier(1, ncons);  // `red` / activations are rewritten by the next pass

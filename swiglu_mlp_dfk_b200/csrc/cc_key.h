@@ -20,4 +20,6 @@ const void *cc_lookup_gemv_b(int key);
 const void *cc_lookup_fp8_gate_up(int key);
 const void *cc_lookup_fp8_gemv_a(int key);
 const void *cc_lookup_fp8_gemv_b(int key);
+const void *cc_lookup_qkv_a(int key);
+const void *cc_lookup_qkv_b(int key);
 }  // namespace dfk

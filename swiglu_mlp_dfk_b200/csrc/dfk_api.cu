@@ -94,6 +94,8 @@ const void *cc_find_kernel(int key) {
   if ((f = cc_lookup_fp8_gate_up(key))) return f;
   if ((f = cc_lookup_fp8_gemv_a(key))) return f;
   if ((f = cc_lookup_fp8_gemv_b(key))) return f;
+  if ((f = cc_lookup_qkv_a(key))) return f;
+  if ((f = cc_lookup_qkv_b(key))) return f;
   return nullptr;
 }
 
@@ -270,6 +272,10 @@ static const std::vector<VDef> &variants() {
     t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, 2, 1, 0, 0, 1});
     for (int ks : {1, 2, 4})
       t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, 2, 1, 0, 0, 1});
+    // GEMV in full 128-row tiles (every MMA row used), k split 0 = as many
+    // slices as fill the SMs: ceil(N / 128) row blocks x floor(SMs / blocks)
+    for (int nt : {1, 2, 4, 8})
+      t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 0, nt, 1, 0, 1, 0});
     return t;
   }();
   return v;
@@ -424,6 +430,8 @@ struct CcCall {
   int B, K, N;
   bool w8 = false;               // FP8 E4M3 weights (row-major), per-row scales below
   const float *s0 = nullptr, *s1 = nullptr;
+  void *outs[3] = {nullptr, nullptr, nullptr};  // packed QKV: q / k / v parts of the output
+  int split[2] = {0, 0};                         // row ranges of the parts
 };
 
 static bool pdl_enabled() { return env_flag("DFK_PDL", true); }
@@ -468,6 +476,9 @@ static int launch_cc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   p.out = static_cast<uint16_t *>(c.out);
   p.scale[0] = c.s0;
   p.scale[1] = c.s1;
+  for (int i = 0; i < 3; ++i) p.outs[i] = static_cast<uint16_t *>(c.outs[i]);
+  p.split[0] = c.split[0];
+  p.split[1] = c.split[1];
   p.err = ds->err;
   p.eps = c.eps;
   void *args[] = {&maps, &p};
@@ -508,8 +519,12 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     if (why) *why = "E4M3-MMA variants run FP8 weights only";
     return false;
   }
+  if (norm && nmat == 1 && v.ksplit != 1 && !prepped) {
+    if (why) *why = "RMSNorm with split-K needs the prepared activations (r_b over all of K)";
+    return false;
+  }
   const bool colm = layout == LAYOUT_COL;
-  const bool full = colm || (v.full != 0 && nmat == 2);  // 128 rows per CTA
+  const bool full = colm || v.full != 0;  // 128 rows per CTA
   if (colm && nmat != 2) {
     if (why) *why = "column-major tensor-core kernel is the fused gate/up only";
     return false;
@@ -521,8 +536,16 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
   const int bn = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
   const int cap = std::min(ds.smem_optin, 232448);
   const int nt = v.nt;
-  const int kslices = (nmat == 1) ? std::max(1, v.ksplit) : 1;
   const int ntiles = ceil_div(K, TC_TILE_K);
+  // GEMV in full tiles: k slices = SMs per row block (k split 0 = automatic)
+  const int kslices = nmat != 1 ? 1
+                      : (v.ksplit == 0 ? std::max(1, std::min({ntiles, SPLITK_MAX,
+                                                               ds.sms / ceil_div(N, 128)}))
+                                       : std::max(1, v.ksplit));
+  if (kslices > SPLITK_MAX) {
+    if (why) *why = "more than 8 k slices";
+    return false;
+  }
   if (kslices > 1 && (nmat != 1 || ntiles < kslices)) {
     if (why) *why = "split-K needs a single matrix and at least one k-tile per slice";
     return false;
@@ -650,21 +673,25 @@ static int get_workspace(int dev, cudaStream_t s, size_t part_bytes, size_t coun
 
 static int get_term_buffer(int dev, cudaStream_t s, size_t bytes, void **out);
 
+// Tensor-core RMSNorm from the prep kernel (mode 2): for the fused gate/up
+// above 32 tokens (measured on the 8B layer: 66 -> 54 us at 64 tokens; at 16
+// and 32 tokens the in-kernel transform is ~3 us faster, the prep latency not
+// hidden), and always for the one-matrix GEMV (packed QKV), where it also
+// allows split-K across CTAs (r_b over all of K).
+static bool tc_prepared(const CcCall &c) { return c.norm && (c.B > 32 || c.nmat == 1); }
+
 static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages_used) {
   DeviceState *ds;
   int dev;
   int rc = current_device(&ds, &dev);
   if (rc) return rc;
-  // RMSNorm above 32 tokens: activations prepared by the prep kernel into the
-  // per-stream buffer (measured on the 8B layer: 66 -> 54 us at 64 tokens;
-  // at 16 and 32 tokens the in-kernel transform is ~3 us faster because the
-  // prep kernel's latency is not hidden); the in-kernel transform also when
-  // the buffer cannot be had (stream capture before any call of this shape
-  // on the stream)
+  // RMSNorm: prepared activations (tc_prepared) in the per-stream buffer; the
+  // in-kernel transform when the buffer cannot be had (stream capture before
+  // any call of this shape on the stream)
   void *xg = nullptr;
   bool prepped = false;
   size_t xg_bytes = 0;
-  if (c.norm && c.B > 32) {
+  if (tc_prepared(c)) {
     const int bn = c.B <= 16 ? 16 : (c.B <= 32 ? 32 : 64);
     xg_bytes = static_cast<size_t>(ceil_div(c.K, TC_TILE_K)) * 2 * bn * TC_TILE_K * 2;
     rc = get_term_buffer(dev, s, xg_bytes + 64 * sizeof(float), &xg);
@@ -672,6 +699,11 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
     else if (rc == DFK_ERR_NO_VARIANT && stream_capturing(s)) log_msg("RMSNorm prep buffer "
              "missing during capture: transforming in the kernel");
     else return rc;
+    if (!prepped && c.nmat == 1 && v.ksplit != 1) {
+      VDef whole = v;  // the in-kernel transform cannot split K
+      whole.ksplit = 1;
+      return launch_tc(c, whole, s, stages_used);
+    }
   }
   TcPlan pl;
   std::string why;
@@ -721,6 +753,9 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
   p.gamma = static_cast<const uint16_t *>(c.gamma);
   p.rinv = prepped ? reinterpret_cast<const float *>(static_cast<char *>(xg) + xg_bytes)
                    : nullptr;
+  for (int i = 0; i < 3; ++i) p.outs[i] = static_cast<uint16_t *>(c.outs[i]);
+  p.split[0] = c.split[0];
+  p.split[1] = c.split[1];
   p.err = ds->err;
   p.eps = c.eps;
   if (p.kslices > 1) {
@@ -1215,13 +1250,15 @@ static std::mutex g_tune_mu;
 static std::map<TuneKey, dfk_variant> g_tuned;
 
 static bool op_is_down(int op) { return op == DFK_OP_DOWN || op == DFK_OP_DOWN_FP8; }
+static bool op_is_qkv(int op) { return op == DFK_OP_QKV || op == DFK_OP_RMSNORM_QKV; }
 static bool op_is_fp8(int op) {
   return op == DFK_OP_GATE_UP_FP8 || op == DFK_OP_RMSNORM_GATE_UP_FP8 || op == DFK_OP_DOWN_FP8;
 }
 static bool op_is_norm(int op) {
-  return op == DFK_OP_RMSNORM_GATE_UP || op == DFK_OP_RMSNORM_GATE_UP_FP8;
+  return op == DFK_OP_RMSNORM_GATE_UP || op == DFK_OP_RMSNORM_GATE_UP_FP8 ||
+         op == DFK_OP_RMSNORM_QKV;
 }
-static int op_class(int op) { return op_is_down(op) ? CLS_GEMV : CLS_GATE_UP; }
+static int op_class(int op) { return (op_is_down(op) || op_is_qkv(op)) ? CLS_GEMV : CLS_GATE_UP; }
 
 static void fill_variant(const VDef &d, int op, int layout, int stages, float us,
                          dfk_variant *out) {
@@ -1354,7 +1391,8 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
       return plan_tf8(c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
     }
     TcPlan pl;
-    return plan_tc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr);
+    return plan_tc(c.layout, c.nmat, c.norm, d, c.B, c.K, c.N, ds, &pl, nullptr,
+                   tc_prepared(c));
   }
   CcPlan pl;
   return plan_cc(c.layout, c.nmat, c.norm, c.w8, d, c.B, c.K, c.N, ds, &pl, nullptr);
@@ -1443,8 +1481,11 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
     if (launch_variant(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible ones
     // Each repetition: flush L2, then a burst of back-to-back launches (the
     // way a decode loop issues them, neighbours overlapping through
-    // programmatic dependent launch); the sample is the burst's mean.
-    const int burst = 4;
+    // programmatic dependent launch); the sample is the burst's mean.  When
+    // one call's weights fit in L2 the later launches of a burst would read
+    // them from L2, so each sample is then one launch after its own flush.
+    const size_t wbytes = static_cast<size_t>(c.K) * c.N * c.nmat * (c.w8 ? 1 : 2);
+    const int burst = (flush && wbytes < static_cast<size_t>(ds.l2_bytes)) ? 1 : 4;
     std::vector<float> ts;
     bool ok = true;
     for (int r = 0; r < reps && ok; ++r) {
@@ -1653,6 +1694,37 @@ static int fp8_impl(int op, const void *x, const void *gamma, float eps, const v
   return launch_variant(c, *v, s, nullptr);
 }
 
+// RMSNorm (optional) + packed QKV projection: one GEMV over W_qkv
+// [n_q + n_k + n_v][d_model], the output rows routed to q, k and v.
+static int qkv_impl(const void *x, const void *gamma, float eps, const void *w, void *q, void *k,
+                    void *v, int B, int D, int nq, int nk, int nv, int variant,
+                    cudaStream_t s) {
+  const bool norm = gamma != nullptr;
+  if (nq < 0 || nk < 0 || nv < 0 || static_cast<long long>(nq) + nk + nv <= 0 ||
+      static_cast<long long>(nq) + nk + nv > (1 << 30))
+    return fail(DFK_ERR_INVALID_ARG, "bad part sizes n_q=%d n_k=%d n_v=%d", nq, nk, nv);
+  if (norm && !(eps >= 0.f && std::isfinite(eps)))
+    return fail(DFK_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  const int N = nq + nk + nv;
+  int rc = check_gemv(x, w, B > 0 ? (q ? q : (k ? k : v)) : nullptr, B, D, N, variant);
+  if (rc || B == 0) return rc;
+  if ((nq && !q) || (nk && !k) || (nv && !v))
+    return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if ((q && misaligned(q)) || (k && misaligned(k)) || (v && misaligned(v)) ||
+      (norm && misaligned(gamma)))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  CcCall c{LAYOUT_ROW, 1, norm, x, gamma, eps, w, nullptr, q, B, D, N};
+  c.outs[0] = q;
+  c.outs[1] = k;
+  c.outs[2] = v;
+  c.split[0] = nq;
+  c.split[1] = nq + nk;
+  const VDef *vd = nullptr;
+  const int op = norm ? DFK_OP_RMSNORM_QKV : DFK_OP_QKV;
+  if ((rc = resolve(op, variant, c, s, &vd))) return rc;
+  return launch_variant(c, *vd, s, nullptr);
+}
+
 }  // namespace dfk
 
 using namespace dfk;
@@ -1701,6 +1773,13 @@ int dfk_down_proj_fp8(const void *h, const void *q_down, const float *s_down, vo
                   d_ff, d_model, variant, static_cast<cudaStream_t>(stream));
 }
 
+int dfk_rmsnorm_qkv_proj(const void *x, const void *gamma, float eps, const void *w_qkv,
+                         void *q, void *k, void *v, int B, int d_model, int n_q, int n_k,
+                         int n_v, int variant, void *stream) {
+  return qkv_impl(x, gamma, eps, w_qkv, q, k, v, B, d_model, n_q, n_k, n_v, variant,
+                  static_cast<cudaStream_t>(stream));
+}
+
 int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int variant,
              void *stream) {
   return gemv_impl(DFK_OP_DOWN, x, w, out, B, K, N, variant, static_cast<cudaStream_t>(stream));
@@ -1709,12 +1788,13 @@ int dfk_gemv(const void *x, const void *w, void *out, int B, int K, int N, int v
 int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
                        const void *const *sample_ptrs, void *stream, dfk_variant *out) {
   if (!out) return fail(DFK_ERR_INVALID_ARG, "out is NULL");
-  if (op < DFK_OP_GATE_UP || op > DFK_OP_DOWN_FP8)
+  if (op < DFK_OP_GATE_UP || op > DFK_OP_RMSNORM_QKV)
     return fail(DFK_ERR_INVALID_ARG, "unknown op %d", op);
   const bool down = op_is_down(op), w8 = op_is_fp8(op), norm = op_is_norm(op);
+  const bool qkv = op_is_qkv(op);  // d_ff = n_q + n_k + n_v; one packed output
   if (B <= 0 || B > 64 || d_model <= 0 || d_ff <= 0)
     return fail(DFK_ERR_UNSUPPORTED_SHAPE, "bad shape B=%d d_model=%d d_ff=%d", B, d_model, d_ff);
-  if ((down || w8) && layout != DFK_W_ROW_MAJOR && layout != DFK_W_ANY)
+  if ((down || w8 || qkv) && layout != DFK_W_ROW_MAJOR && layout != DFK_W_ANY)
     return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "op %d reads row-major weights only", op);
   if (layout != DFK_W_ANY && layout != DFK_W_ROW_MAJOR && layout != DFK_W_COL_MAJOR &&
       layout != DFK_W_GU_INTERLEAVED)
@@ -1732,11 +1812,11 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
     return fail(DFK_ERR_INVALID_ARG, "dfk_select_variant cannot time inside stream capture");
 
   std::vector<int> layouts;
-  if (down || w8) layouts = {DFK_W_ROW_MAJOR};
+  if (down || w8 || qkv) layouts = {DFK_W_ROW_MAJOR};
   else if (layout == DFK_W_ANY) layouts = {DFK_W_ROW_MAJOR, DFK_W_COL_MAJOR, DFK_W_GU_INTERLEAVED};
   else layouts = {layout};
 
-  const int K = down ? d_ff : d_model, N = down ? d_model : d_ff, nmat = down ? 1 : 2;
+  const int K = down ? d_ff : d_model, N = down ? d_model : d_ff, nmat = (down || qkv) ? 1 : 2;
   const size_t xb = static_cast<size_t>(B) * K * 2;
   const size_t wb = static_cast<size_t>(d_model) * d_ff * (w8 ? 1 : 2);
   const size_t ob = static_cast<size_t>(B) * N * 2;
@@ -1767,9 +1847,9 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
       cudaMemsetAsync(bw, 0, nmat * wb, s);
       if (bs) cudaMemsetAsync(bs, 0, nmat * sb, s);
       px = bx; pg = bg; po = bo; pw0 = bw;
-      pw1 = (down || L == DFK_W_GU_INTERLEAVED) ? nullptr : static_cast<char *>(bw) + wb;
+      pw1 = (nmat == 1 || L == DFK_W_GU_INTERLEAVED) ? nullptr : static_cast<char *>(bw) + wb;
       ps0 = static_cast<const float *>(bs);
-      ps1 = (bs && !down) ? static_cast<const float *>(bs) + N : nullptr;
+      ps1 = (bs && nmat == 2) ? static_cast<const float *>(bs) + N : nullptr;
     } else {
       // argument order of the op's entry point
       int i = 0;
@@ -1777,14 +1857,14 @@ int dfk_select_variant(int op, int B, int d_model, int d_ff, int layout,
       if (norm) pg = sample_ptrs[i++];
       pw0 = sample_ptrs[i++];
       if (w8) ps0 = static_cast<const float *>(sample_ptrs[i++]);
-      if (!down) {
+      if (!down && !qkv) {
         pw1 = sample_ptrs[i++];
         if (w8) ps1 = static_cast<const float *>(sample_ptrs[i++]);
       }
       po = const_cast<void *>(sample_ptrs[i++]);
     }
     CcCall c;
-    if (down) c = CcCall{LAYOUT_ROW, 1, false, px, nullptr, 0.f, pw0, nullptr, po, B, K, N};
+    if (down || qkv) c = CcCall{LAYOUT_ROW, 1, norm, px, pg, 1e-5f, pw0, nullptr, po, B, K, N};
     else c = CcCall{to_engine_layout(L), 2, norm, px, pg, 1e-5f, pw0,
                     L == DFK_W_GU_INTERLEAVED ? nullptr : pw1, po, B, K, N};
     c.w8 = w8;

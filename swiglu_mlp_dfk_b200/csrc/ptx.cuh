@@ -223,4 +223,52 @@ __device__ __forceinline__ float round_bf16(float f) {
   return __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(f)) << 16);
 }
 
+// Output element (b, j): row j of the one output, or of its q / k / v part.
+template <typename P>
+__device__ __forceinline__ void store_out(const P &p, int b, int j, uint16_t v) {
+  if (p.outs[0] == nullptr) {
+    p.out[static_cast<size_t>(b) * p.N + j] = v;
+  } else if (j < p.split[0]) {
+    p.outs[0][static_cast<size_t>(b) * p.split[0] + j] = v;
+  } else if (j < p.split[1]) {
+    p.outs[1][static_cast<size_t>(b) * (p.split[1] - p.split[0]) + (j - p.split[0])] = v;
+  } else {
+    p.outs[2][static_cast<size_t>(b) * (p.N - p.split[1]) + (j - p.split[1])] = v;
+  }
+}
+
+// Split-K tail for output row `row` of row block `blk`: adds the kslices
+// (<= 8) fp32 partial sums of tokens 0 .. B-1 in slice order (slice 0
+// first) and hands each total to emit(n, total).  The loads of 8 tokens x
+// all slices are issued before any add, so the tail costs a few L2 round
+// trips rather than one per token.  part: [kslices][nblocks][bnp][128].
+constexpr int SPLITK_MAX = 8;
+
+template <typename Emit>
+__device__ __forceinline__ void splitk_reduce_row(const float *part, int kslices, int nblocks,
+                                                  int blk, int bnp, int B, int row, Emit emit) {
+  constexpr int TB = 8;
+  for (int n0 = 0; n0 < B; n0 += TB) {
+    float v[TB][SPLITK_MAX];
+#pragma unroll
+    for (int i = 0; i < TB; ++i)
+#pragma unroll
+      for (int sl = 0; sl < SPLITK_MAX; ++sl)
+        v[i][sl] = (n0 + i < B && sl < kslices)
+                       ? __ldcg(part + ((static_cast<size_t>(sl) * nblocks + blk) * bnp + n0 + i) *
+                                           128 + row)
+                       : 0.f;
+#pragma unroll
+    for (int i = 0; i < TB; ++i) {
+      if (n0 + i < B) {
+        float acc = v[i][0];
+#pragma unroll
+        for (int sl = 1; sl < SPLITK_MAX; ++sl)
+          if (sl < kslices) acc = acc + v[i][sl];
+        emit(n0 + i, acc);
+      }
+    }
+  }
+}
+
 }  // namespace dfk

@@ -52,6 +52,8 @@ constexpr int TC_ATOM = 1024;       // bytes of an 8-row swizzle atom
 
 struct TcParams {
   uint16_t *out;          // [B][N] bf16
+  uint16_t *outs[3];      // split output (packed QKV) when outs[0] != nullptr
+  int split[2];           // row ranges of the q / k / v parts
   const uint16_t *gamma;  // [K] bf16 (NORM = 1)
   const float *rinv;      // [bn] r_b from the prep kernel (NORM = 2)
   unsigned *err;          // device error word
@@ -140,7 +142,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   static_assert(NMAT == 1 || NMAT == 2, "NMAT");
   static_assert(!IL || NMAT == 2, "interleaved layout holds both matrices");
   static_assert(!COLM || MT == 1, "column-major: one 128-column tile per CTA");
-  static_assert(!NORM || NMAT == 2, "the RMSNorm prologue belongs to the gate/up kernel");
   static_assert(NORM >= 0 && NORM <= 2, "NORM");
   constexpr int XROWS = NORM == 2 ? 2 : 1;  // activation rows per token loaded by TMA
   static_assert(MT == 1 || MT == 2, "MT");
@@ -423,14 +424,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const int n = c + e;
               if (n < p.B) {
                 float res;
+                const float sc = NORM == 1 ? s_rinv[n] : (NORM == 2 ? p.rinv[n] : 1.0f);
                 if (NMAT == 2) {
-                  const float sc = NORM == 1 ? s_rinv[n] : (NORM == 2 ? p.rinv[n] : 1.0f);
                   const float a = g[e] * sc, uu = u[e] * sc;
                   res = (a / (1.0f + expf(-a))) * uu;
                 } else {
-                  res = g[e];
+                  res = NORM ? g[e] * sc : g[e];
                 }
-                p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
+                store_out(p, n, j, f32_to_bf16_bits(res));
               }
             }
           }
@@ -449,17 +450,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       named_barrier(2, 128);
       if (*s_last) {
         __threadfence();
-        if (row < r && !*s_abort) {
-          for (int n = 0; n < p.B; ++n) {
-            float acc = 0.f;
-            for (int sl = 0; sl < p.kslices; ++sl) {
-              const float v = __ldcg(p.part + ((static_cast<size_t>(sl) * p.nblocks + blk) * BN +
-                                               n) * 128 + row);
-              acc = (sl == 0) ? v : acc + v;
-            }
-            p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(acc);
-          }
-        }
+        if (row < r && !*s_abort)
+          splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, BN, p.B, row,
+                            [&](int n, float acc) {
+                              // RMSNorm with split-K only in mode 2 (r_b over all of K)
+                              if (NORM == 2) acc *= p.rinv[n];
+                              store_out(p, n, j0 + row, f32_to_bf16_bits(acc));
+                            });
         named_barrier(2, 128);
         if (et == 0) p.counters[blk] = 0u;
       }

@@ -364,15 +364,11 @@ __global__ void __launch_bounds__(TF8_THREADS, 1)
           __threadfence();
           if (row < r && !*s_abort) {
             const float sd = __ldg(p.scale[0] + j0 + row);
-            for (int n = 0; n < p.B; ++n) {
-              float acc = 0.f;
-              for (int sl = 0; sl < p.kslices; ++sl) {
-                const float v = __ldcg(p.part + ((static_cast<size_t>(sl) * p.nblocks + blk) * BN +
-                                                 n) * 128 + row);
-                acc = (sl == 0) ? v : acc + v;
-              }
-              p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(acc * sd);
-            }
+            splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, BN, p.B, row,
+                              [&](int n, float acc) {
+                                p.out[static_cast<size_t>(n) * p.N + j0 + row] =
+                                    f32_to_bf16_bits(acc * sd);
+                              });
           }
           named_barrier(2, 128);
           if (et == 0) p.counters[blk] = 0u;

@@ -132,6 +132,21 @@ MIS = ctypes.c_void_p(0x10008)
     (lambda L: L.dfk_select_variant(dfk.DFK_OP_DOWN_FP8, 1, 64, 64, 1, None, None,
                                     ctypes.byref(dfk.dfk_variant())),
      dfk.DFK_ERR_UNSUPPORTED_LAYOUT),
+    # packed QKV: part sizes, null parts, misaligned parts, eps, bf16-only ids
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, P3, P3, 1, 64, -1, 8, 8, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, P3, P3, 1, 64, 0, 0, 0, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, None, P3, 1, 64, 8, 8, 8, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, MIS, P3, 1, 64, 8, 8, 8, 0, None),
+     dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, -1.0, P2, P3, P3, P3, 1, 64, 8, 8, 8, 0, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, P3, P3, 1, 60, 8, 8, 8, 0, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_rmsnorm_qkv_proj(P, P, 1e-5, P2, P3, P3, P3, 1, 64, 8, 8, 8, 1, None),
+     dfk.DFK_ERR_INVALID_ARG),                                   # id 1: a gate/up variant
     (lambda L: L.dfk_select_variant(9, 1, 64, 64, 0, None, None, None), dfk.DFK_ERR_INVALID_ARG),
 ])
 def test_validation_rejects_without_launch(L, call, status):
