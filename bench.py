@@ -373,11 +373,16 @@ def gpu_arm(args):
     return line
 
 
-def timed_us(fn, reps, flush=None):
-    """Mean duration of `reps` back-to-back calls (after an L2 flush), in us."""
+def timed_us(fn, reps, flush=None, warm=3):
+    """Mean duration of `reps` back-to-back calls, in us.  `warm` untimed calls
+    run first (after the optional L2 flush, whose dirty lines they write back),
+    so the timed calls see the steady state; every caller rotates weight copies
+    whose total exceeds L2, so no timed call finds its weights cached."""
     import torch
     if flush is not None:
         flush.add_(1)
+    for i in range(warm):
+        fn(reps + i)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for i in range(reps):
@@ -397,7 +402,7 @@ def extra_measurements(args, inp, copies, h, y):
     from swiglu_mlp_dfk_b200 import inputs as I
 
     peak, _ = measured_peaks()
-    reps = 30
+    reps = 100
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")  # 256 MB > L2
     out = {}
     # interleaved layout of the same weights (two copies, rotated)
