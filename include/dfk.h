@@ -303,7 +303,11 @@ DFK_API int dfk_rms_rescale(const void *y, float eps, void *x_next, int B, int d
  * kernel (gamma may be NULL: no RMSNorm) and the down projection, and copies
  * y back to y_host ([B][d_model] bf16).  Weights are device-resident.
  * x_dev, h_dev, y_dev are caller-owned device work buffers of the sizes of
- * x, h and y.  Synchronises `stream` before returning.
+ * x, h and y.  Synchronises `stream` before returning.  Pinned host
+ * buffers (device-addressable, 16-byte aligned): the copies are small
+ * kernels chained to the MLP kernels by programmatic dependent launch, and
+ * the whole sequence is captured once per argument set and replayed as one
+ * CUDA graph; pageable buffers use copy-engine transfers, eagerly.
  */
 DFK_API int dfk_mlp_forward_host(const void *x_host, const void *gamma, float eps,
                          const void *w_gate, const void *w_up, int layout,

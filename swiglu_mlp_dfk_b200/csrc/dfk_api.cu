@@ -2022,9 +2022,26 @@ static std::mutex g_host_mu;
 static std::map<HostKey, cudaGraphExec_t> g_host_graphs;  // nullptr: capture failed, run eager
 static std::map<int, cudaStream_t> g_capture_streams;
 
+// Device address of a pinned host buffer (unified addressing), or nullptr.
+static void *mapped_host_ptr(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 static int forward_host_enqueue(const HostCall &a, cudaStream_t s) {
   const size_t xb = static_cast<size_t>(a.B) * a.d_model * 2;
-  cudaError_t e = cudaMemcpyAsync(a.x_dev, a.x_host, xb, cudaMemcpyHostToDevice, s);
+  // pinned, device-addressable host buffers: copy kernels (which overlap the
+  // neighbouring kernels through programmatic dependent launch); otherwise
+  // copy-engine transfers
+  void *xh = mapped_host_ptr(a.x_host), *yh = mapped_host_ptr(a.y_host);
+  const bool kern = xh && yh && xb % 16 == 0 &&
+                    ((reinterpret_cast<uintptr_t>(xh) | reinterpret_cast<uintptr_t>(yh)) & 15u) == 0;
+  cudaError_t e = kern ? launch_copy16(xh, a.x_dev, xb, false, s, pdl_enabled())
+                       : cudaMemcpyAsync(a.x_dev, a.x_host, xb, cudaMemcpyHostToDevice, s);
   if (e) {
     cudaGetLastError();
     return cuda_fail(e, "copy x to device");
@@ -2035,7 +2052,8 @@ static int forward_host_enqueue(const HostCall &a, cudaStream_t s) {
                                         a.d_model, a.d_ff, 0, s);
   if (rc) return rc;
   if ((rc = dfk_down_proj(a.h_dev, a.w_down, a.y_dev, a.B, a.d_model, a.d_ff, 0, s))) return rc;
-  e = cudaMemcpyAsync(a.y_host, a.y_dev, xb, cudaMemcpyDeviceToHost, s);
+  e = kern ? launch_copy16(a.y_dev, yh, xb, true, s, pdl_enabled())
+           : cudaMemcpyAsync(a.y_host, a.y_dev, xb, cudaMemcpyDeviceToHost, s);
   if (e) {
     cudaGetLastError();
     return cuda_fail(e, "copy y to host");

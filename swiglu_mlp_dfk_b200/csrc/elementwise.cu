@@ -5,6 +5,7 @@
 // Projection with Operator Fusion", section "The Why of Operator Fusion":
 // every intermediate is written to HBM and read back by the next kernel).
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <cstdint>
 
 #include "launch_util.h"
@@ -121,6 +122,47 @@ cudaError_t launch_mul(const void *a, const void *b, void *out, long long n, cud
   void *args[] = {&ap, &bp, &op, &n};
   return launch_kernel(reinterpret_cast<const void *>(&mul_kernel), dim3(ew_blocks(n)),
                        dim3(256), 0, s, pdl, args);
+}
+
+// Device copy of `n16` 16-byte chunks, used by the host-memory entry point
+// to move x into and y out of pinned host buffers that the device addresses
+// directly (in place of copy-engine transfers, so the copies take part in
+// programmatic dependent launch).  WAIT_FIRST: the source is the previous
+// kernel's output (wait before reading); otherwise the loads are issued
+// first and only the stores wait for the previous kernel.
+template <bool WAIT_FIRST>
+__global__ void copy16_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst,
+                              size_t n16) {
+  if (WAIT_FIRST) pdl_wait();
+  pdl_launch_dependents();
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint4 v[4];
+  for (; i < n16; i += 4 * stride) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * stride < n16) v[u] = src[i + u * stride];
+    if (!WAIT_FIRST) pdl_wait();
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * stride < n16) dst[i + u * stride] = v[u];
+  }
+  if (!WAIT_FIRST) pdl_wait();  // threads without work still order after the previous kernel
+}
+
+cudaError_t launch_copy16(const void *src, void *dst, size_t bytes, bool wait_first,
+                          cudaStream_t s, bool pdl) {
+  const size_t n16 = bytes / 16;
+  if (n16 == 0) return cudaSuccess;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>(148, (n16 + threads - 1) / threads));
+  const uint4 *a = static_cast<const uint4 *>(src);
+  uint4 *b = static_cast<uint4 *>(dst);
+  size_t n = n16;
+  void *args[] = {&a, &b, &n};
+  return launch_kernel(wait_first ? reinterpret_cast<const void *>(&copy16_kernel<true>)
+                                  : reinterpret_cast<const void *>(&copy16_kernel<false>),
+                       dim3(blocks), dim3(threads), 0, s, pdl, args);
 }
 
 }  // namespace dfk

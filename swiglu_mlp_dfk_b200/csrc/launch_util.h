@@ -43,5 +43,7 @@ cudaError_t launch_rmsnorm_rows(const void *x, const void *gamma, float eps, voi
 cudaError_t launch_silu(const void *a, void *out, long long n, cudaStream_t s, bool pdl);
 cudaError_t launch_mul(const void *a, const void *b, void *out, long long n, cudaStream_t s,
                        bool pdl);
+cudaError_t launch_copy16(const void *src, void *dst, size_t bytes, bool wait_first,
+                          cudaStream_t s, bool pdl);
 
 }  // namespace dfk
