@@ -470,6 +470,7 @@ def extra_measurements(args, inp, copies, h, y):
     out["fp8_weights"]["bf16_b1_fused_us"] = round(t_fus, 2)
     torch.cuda.empty_cache()
     out["qkv_projection"] = qkv_measure()
+    out["torch_eager_mlp"] = torch_eager_measure()
     out["decode_stack"] = decode_stack_measure(args.stack_steps)
     return out
 
@@ -616,10 +617,56 @@ def qkv_measure(reps=100, ncopies=4):
             "unfused": "rmsnorm + gemv(W_q) + gemv(W_k) + gemv(W_v)", "sweep": res}
 
 
+def torch_eager_measure(reps=50):
+    """Informational: the same Llama-3-8B-shaped MLP layer in torch eager ops
+    (RMSNorm, two cuBLAS linears, SiLU, multiply, cuBLAS down projection),
+    two rotated weight copies, back-to-back calls.  Library kernels, not this
+    repository's; reported for context only."""
+    import torch
+    import torch.nn.functional as Fn
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import inputs as I
+
+    base = I.make_inputs(64, D, F, seed=2, norm=True, with_down=True, device="cuda")
+    cps = [(base.w_gate, base.w_up, base.w_down),
+           (base.w_gate.clone(), base.w_up.clone(), base.w_down.clone())]
+    res = []
+    for B in (1, 16, 64):
+        x = base.x[:B].contiguous()
+
+        def step(i):
+            wg, wu, wd = cps[i % 2]
+            xn = Fn.rms_norm(x, (D,), base.gamma, base.eps)
+            return Fn.linear(Fn.silu(Fn.linear(xn, wg)) * Fn.linear(xn, wu), wd)
+
+        t = timed_us(step, reps)
+        h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+
+        def ours(i):
+            wg, wu, wd = cps[i % 2]
+            dfk.dfk_rmsnorm_swiglu_gate_up(x, base.gamma, base.eps, wg, wu, "row", h=h)
+            dfk.dfk_down_proj(h, wd, y=y)
+
+        ours(0)
+        t2 = timed_us(ours, reps)
+        res.append({"B": B, "torch_mlp_us": round(t, 2),
+                    "torch_GBps": round(step_bytes(B, D, F) / (t * 1e-6) / 1e9, 1),
+                    "dfk_mlp_us": round(t2, 2),
+                    "dfk_GBps": round(step_bytes(B, D, F) / (t2 * 1e-6) / 1e9, 1),
+                    "dfk_speedup": round(t / t2, 3)})
+    del cps, base
+    torch.cuda.empty_cache()
+    return {"what": "torch eager: rms_norm + linear(Wg), linear(Wu) + silu * mul + linear(Wd) "
+            "(cuBLAS), against this library's fused RMSNorm+gate/up + down on the same "
+            "weights; informational", "sweep": res}
+
+
 def decode_stack_measure(steps, layers=32, B=4):
     """Long-generation decode: a 32-layer stack of Llama-3-8B-shaped MLPs
     (11.3 GB of distinct weights, seed 4), B = 4, one step per CUDA-graph
-    replay, fused vs unfused kernels."""
+    replay: fused vs unfused kernels, and the fused stack with the weights
+    encoded as FP8 E4M3 + row scales (5.6 GB per step)."""
     import torch
     from swiglu_mlp_dfk_b200 import inputs as I
     from swiglu_mlp_dfk_b200.stack import DecodeStack
@@ -628,8 +675,8 @@ def decode_stack_measure(steps, layers=32, B=4):
     x0, params = I.make_stack(layers, B, D, F, seed=4, w_std=0.02, device="cuda")
     res = {"layers": layers, "B": B, "steps": steps,
            "weights_GB": round(sum(t.numel() * 2 for p in params for t in p) / 1e9, 2)}
-    for fused in (True, False):
-        st = DecodeStack(params, x0, fused=fused)
+    for fused, fp8 in ((True, False), (False, False), (True, True)):
+        st = DecodeStack(params, x0, fused=fused, fp8=fp8)
         st.step_eager()                      # scheduler decisions outside capture
         torch.cuda.synchronize()
         st.capture()
@@ -642,10 +689,18 @@ def decode_stack_measure(steps, layers=32, B=4):
         b.record()
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / steps
-        key = "fused" if fused else "unfused"
+        key = "fp8" if fp8 else ("fused" if fused else "unfused")
         res[key + "_ms_per_step"] = round(ms, 4)
-        res[key + "_kernels_per_step"] = st.kernels_per_step()
-        if fused:
+        if fp8:  # the E4M3-MMA calls launch two kernels each (prep + main)
+            res["fp8_calls_per_step"] = st.kernels_per_step()
+        else:
+            res[key + "_kernels_per_step"] = st.kernels_per_step()
+        if fp8:
+            gbs = st.bytes_per_step() / (ms * 1e-3) / 1e9
+            res["fp8_GBps"] = round(gbs, 1)
+            res["fp8_frac_of_peak"] = round(gbs / peak, 4)
+            res["fp8_weights_GB"] = round(st.bytes_per_step() / 1e9, 2)
+        elif fused:
             gbs = st.bytes_per_step() / (ms * 1e-3) / 1e9
             res["fused_GBps"] = round(gbs, 1)
             res["fused_frac_of_peak"] = round(gbs / peak, 4)
@@ -653,6 +708,7 @@ def decode_stack_measure(steps, layers=32, B=4):
         st.release()
         del st
     res["fused_speedup"] = round(res["unfused_ms_per_step"] / res["fused_ms_per_step"], 3)
+    res["fp8_speedup_over_bf16_fused"] = round(res["fused_ms_per_step"] / res["fp8_ms_per_step"], 3)
     del params, x0
     torch.cuda.empty_cache()
     return res

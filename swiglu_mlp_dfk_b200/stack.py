@@ -10,7 +10,10 @@ consistent speed-ups over generation lengths), as a stack of SwiGLU MLP
 layers only.
 
 The unfused variant runs the same step with separate kernels (RMSNorm, two
-GEMVs, SiLU, multiply, down projection) and bf16 intermediates in HBM.
+GEMVs, SiLU, multiply, down projection) and bf16 intermediates in HBM.  The
+FP8 variant encodes every layer's weights once as E4M3 codes with one fp32
+scale per output row (the library's FP8 entry points: half the weight bytes
+per step, dequantised inside the kernels).
 
 Everything launched here is a libdfk kernel; torch provides the buffers, the
 stream and the CUDA graph.
@@ -27,12 +30,21 @@ class DecodeStack:
     x0:     [B, D] bf16 first-step input
     """
 
-    def __init__(self, layers, x0, eps=1e-5, fused=True):
-        self.layers = layers
+    def __init__(self, layers, x0, eps=1e-5, fused=True, fp8=False):
+        if fp8 and not fused:
+            raise ValueError("the FP8 stack runs the fused kernels")
         self.eps = float(eps)
         self.fused = fused
+        self.fp8 = fp8
+        if fp8:
+            from . import inputs as I
+            enc = []
+            for gamma, wg, wu, wd in layers:
+                enc.append((gamma,) + I.to_fp8_rows(wg) + I.to_fp8_rows(wu) + I.to_fp8_rows(wd))
+            layers = enc
+        self.layers = layers
         self.B, self.D = x0.shape
-        self.F = layers[0][1].shape[0]
+        self.F = layers[0][1].shape[0]     # W_gate rows (bf16 or FP8 codes)
         dev = x0.device
         self.x = x0.clone()                       # step input (graph-static buffer)
         self.acts = [torch.empty(self.B, self.D, dtype=torch.bfloat16, device=dev)
@@ -53,9 +65,14 @@ class DecodeStack:
         return self.x if l == 0 else self.acts[(l - 1) % 2]
 
     def _layer(self, l):
-        gamma, wg, wu, wd = self.layers[l]
         xin = self.layer_input(l)
         y = self.acts[l % 2]
+        if self.fp8:
+            gamma, qg, sg, qu, su, qd, sd = self.layers[l]
+            dfk.dfk_rmsnorm_swiglu_gate_up_fp8(xin, gamma, self.eps, qg, sg, qu, su, h=self.h)
+            dfk.dfk_down_proj_fp8(self.h, qd, sd, y=y)
+            return
+        gamma, wg, wu, wd = self.layers[l]
         if self.fused:
             dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, "row", h=self.h)
         else:
@@ -105,11 +122,17 @@ class DecodeStack:
         self.graph = None
 
     def kernels_per_step(self):
+        """Library calls per step (one kernel each, except the FP8 tensor-core
+        calls that launch a prep kernel first)."""
         return len(self.layers) * (2 if self.fused else 6) + 1
 
     def bytes_per_step(self):
         """Algorithmic bytes of one step: every weight once, activations in/out."""
         B, D, F = self.B, self.D, self.F
+        if self.fp8:  # codes (1 byte) + fp32 row scales
+            per_layer = (2 * F * D + 2 * F * 4 + B * D * 2 + D * 2 + B * F * 2
+                         + D * F + D * 4 + B * F * 2 + B * D * 2)
+            return len(self.layers) * per_layer + 2 * B * D * 2
         per_layer = (2 * F * D * 2 + B * D * 2 + D * 2 + B * F * 2      # fused gate/up
                      + D * F * 2 + B * F * 2 + B * D * 2)               # down projection
         return len(self.layers) * per_layer + 2 * B * D * 2             # + rescale

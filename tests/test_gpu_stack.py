@@ -106,3 +106,40 @@ def test_capture_on_fresh_stream_without_workspace():
     ok, err = close(y, I.bf16_values(eager))
     assert ok, err
     del graph
+
+
+def test_fp8_stack_graph_replay_equals_eager():
+    x0, params = I.make_stack(3, 4, 1024, 2048, seed=5, w_std=0.02, device="cuda")
+    st = DecodeStack(params, x0, fp8=True)
+    ref = DecodeStack(params, x0, fp8=True)
+    st.step_eager()
+    ref.step_eager()
+    st.capture()
+    for _ in range(4):
+        st.step()
+        ref.step_eager()
+    torch.cuda.synchronize()
+    assert torch.equal(st.x.view(torch.int16), ref.x.view(torch.int16))
+    st.release()
+
+
+def test_fp8_stack_teacher_forced_layers_match_oracle():
+    x0, params = I.make_stack(4, 4, 1024, 2048, seed=6, w_std=0.02, device="cuda")
+    st = DecodeStack(params, x0, fp8=True)
+    checked = 0
+    for step in range(2):
+        for l in range(len(params)):
+            xin = st.layer_input(l).clone()
+            st._layer(l)
+            if l in (0, 3):
+                torch.cuda.synchronize()
+                gamma, qg, sg, qu, su, qd, sd = st.layers[l]
+                host = lambda t: t.detach().cpu().numpy()
+                h_ref = oracle.gate_up_fp8(I.to_bits(xin), host(qg), host(sg), host(qu), host(su),
+                                           gamma=I.to_bits(gamma), eps=1e-5)
+                y_ref = oracle.down_fp8(h_ref, host(qd), host(sd))
+                ok, err = close(st.acts[l % 2], y_ref)
+                assert ok, "fp8 step %d layer %d: max err %g" % (step, l, err)
+                checked += 1
+        dfk.dfk_rms_rescale(st.acts[(len(params) - 1) % 2], 1e-5, out=st.x)
+    assert checked == 4
