@@ -78,6 +78,7 @@ struct CcParams {
   int xs_off;       // shared-memory offset of the activation / reduction area
   int g_off;        // shared-memory offset of gamma (bf16 bits, NORM only)
   int bar_off;      // shared-memory offset of the barrier area
+  int pf_steps;     // ring steps after the first fill whose weight boxes are prefetched into L2
 };
 
 // Tensor maps: index matrix * 2 + (CTA has the short row count ? 1 : 0).
@@ -175,6 +176,28 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
           }
         }
         issued = i + 1;
+        if (i == S - 1) {
+          // ring full: pull the next pf_steps steps' boxes into L2 while the
+          // consumers wait for the previous kernel's activations
+          const int pf_end = min(total_steps, S + p.pf_steps);
+          for (int ii = S; ii < pf_end; ++ii) {
+            const int pstep = ii % p.nsteps;
+#pragma unroll
+            for (int kt = 0; kt < KSPLIT; ++kt) {
+              const int k0 = (pstep * KSPLIT + kt) * nt * TK;
+              if (LAYOUT == LAYOUT_ROW) {
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) tma_prefetch_2d(&maps.m[m * 2 + mi], k0, j0);
+              } else if (LAYOUT == LAYOUT_COL) {
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) tma_prefetch_2d(&maps.m[m * 2 + mi], j0, k0);
+              } else {
+                tma_prefetch_2d(&maps.m[mi], k0, 2 * j0);
+                tma_prefetch_2d(&maps.m[mi], k0, 2 * j0 + r);
+              }
+            }
+          }
+        }
       }
       *s_issued = issued;
     }

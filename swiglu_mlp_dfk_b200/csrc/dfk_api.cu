@@ -320,6 +320,21 @@ struct CcPlan {
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
 static int round_up(int a, int b) { return ceil_div(a, b) * b; }
 
+// L2 bytes (over the whole grid) that a weight-streaming kernel prefetches
+// ahead of its shared-memory ring while it waits on the previous kernel; a
+// fraction of the 126 MB L2, so the boxes are still there when loaded.
+static constexpr long long kPrefetchBytes = 48LL << 20;
+
+// Where the prefetch pays (measured on the 8B shapes, back-to-back calls):
+// a bf16 single-matrix GEMV whose weights are at least twice the budget (the
+// down projection, 117 MB: 0.5-2 us saved at 1-64 tokens).  It was neutral
+// to harmful where the budget covers most of the weights (packed QKV, 50 MB;
+// FP8 down, 59 MB: up to 2 us lost) and on the fused gate/up (up to 1.5 us
+// lost: the deeper per-CTA sweep is already covered by the ring).
+static bool prefetch_pays(int nmat, bool w8, int N, int K) {
+  return nmat == 1 && !w8 && 2LL * N * K >= 2 * kPrefetchBytes;
+}
+
 // Partition N output rows over the SMs and size the shared-memory ring.
 static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int B, int K,
                     int N, const DeviceState &ds, CcPlan *pl, std::string *why) {
@@ -396,6 +411,12 @@ static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int
     p.xs_off = best_s * stage_bytes;
     p.g_off = p.xs_off + v.bt * kpad * (best_xf32 ? 4 : 2);
     p.bar_off = p.xs_off + best_region;
+    // single-matrix GEMV: L2 prefetch of the steps after the ring fill
+    p.pf_steps = !prefetch_pays(nmat, w8, N, K)
+                     ? 0
+                     : static_cast<int>(std::max(0LL, std::min<long long>(
+                                 p.npass * nsteps - best_s,
+                                 kPrefetchBytes / P / stage_bytes)));
     pl->smem = static_cast<size_t>(p.bar_off) + bar_bytes;
     return true;
   }
@@ -615,6 +636,13 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
       p.kslices = kslices;
       p.nblocks = nblocks;
       p.full = full ? 1 : 0;
+      // weight boxes prefetched into L2 ahead of the ring while the previous
+      // kernel finishes, at most kPrefetchBytes over the grid
+      const long long step_w = static_cast<long long>(nmat) * mt * nt * (full ? 128 : hmax) * 128;
+      p.pf_steps = !prefetch_pays(nmat, false, N, K)
+                       ? 0
+                       : static_cast<int>(std::max(0LL, std::min<long long>(
+                                   nsteps - S, kPrefetchBytes / P / step_w)));
       pl->smem = 1024 + static_cast<size_t>(p.bar_off) + 1024;
       return true;
     }

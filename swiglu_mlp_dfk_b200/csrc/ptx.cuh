@@ -87,6 +87,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// Bulk tensor prefetch global -> L2 of the box a tma_load_2d with the same map
+// and coordinates would copy (no shared memory, no barrier; boxes past the
+// tensor bounds are clipped by the map).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // L2 policy: weights are streamed once per call -> evict first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
@@ -150,29 +160,7 @@ __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
       : "r"(h01), "r"(h23));
 }
 
-// Four FP8 E4M3 codes (byte i of w = element i) -> two bf16x2 words (lo holds
-// elements 0, 1; hi holds 2, 3; lower element in the low half).  E4M3 -> f16
-// is exact (hardware pair conversion), and so is f16 -> bf16 for these values
-// (at most 4 significant bits, exponents -9 .. 8).
-__device__ __forceinline__ void e4m3x4_to_bf16x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
-  asm("{\n\t.reg .b16 c01, c23, a, b, c, d;\n\t"
-      ".reg .b32 h01, h23;\n\t"
-      "mov.b32 {c01, c23}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h01, c01;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h23, c23;\n\t"
-      "mov.b32 {a, b}, h01;\n\t"
-      "mov.b32 {c, d}, h23;\n\t"
-      "cvt.rn.bf16.f16 a, a;\n\t"
-      "cvt.rn.bf16.f16 b, b;\n\t"
-      "cvt.rn.bf16.f16 c, c;\n\t"
-      "cvt.rn.bf16.f16 d, d;\n\t"
-      "mov.b32 %0, {a, b};\n\t"
-      "mov.b32 %1, {c, d};\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
-// The same conversion without the conversion unit (whose throughput is a
+// FP8 E4M3 -> bf16 without the conversion unit (whose throughput is a
 // quarter of the ALU's): for a code c = s.eeee.mmm, the 16 bits
 // (c & 0x7F) << 4 read as bf16 have exponent field e and mantissa mmm0000,
 // i.e. the value |E4M3(c)| * 2^-120 exactly (e = 0 gives the bf16 subnormal

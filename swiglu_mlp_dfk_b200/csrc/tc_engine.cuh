@@ -81,6 +81,8 @@ struct TcParams {
   unsigned *counters;     // [row blocks], 0 between calls
   int nblocks;            // row blocks (split-K)
   int full;               // 1: every CTA owns 128 rows (the last one fewer); boxes of 128 rows
+  int pf_steps;           // ring steps after the first fill whose weight boxes are prefetched
+                          // into L2 before the wait on the previous kernel
 };
 
 // wg/wu: [0] box height hmax, [1] box height hmax - 1; x: activations box {64, bn}.
@@ -248,6 +250,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
         if (i == S0 - 1) {
+          // the weights never depend on the previous kernel: pull the next
+          // pf_steps steps' boxes into L2 while it finishes
+          const int pf_end = min(nsteps, S0 + p.pf_steps);
+          for (int ii = S0; ii < pf_end; ++ii) {
+            const int nvi = min(NT, tile1 - (tile0 + ii * NT));
+            for (int kt = 0; kt < nvi; ++kt) {
+              const int k0 = (tile0 + ii * NT + kt) * TC_TILE_K;
+#pragma unroll
+              for (int t = 0; t < MT; ++t) {
+                const int mi = (full || h[t] == p.hmax) ? 0 : 1;
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                  const CUtensorMap *wm = m == 0 ? &maps.wg[mi] : &maps.wu[mi];
+                  if (IL) {
+                    tma_prefetch_3d(&maps.wg[mi], k0, m, j0 + rs[t]);
+                  } else if (COLM) {
+                    tma_prefetch_2d(wm, j0, k0);
+                    tma_prefetch_2d(wm, j0 + 64, k0);
+                  } else {
+                    tma_prefetch_2d(wm, k0, j0 + rs[t]);
+                  }
+                }
+              }
+            }
+          }
           pdl_wait();
           for (int ii = 0; ii < S0; ++ii) {
             const int nvi = min(NT, tile1 - (tile0 + ii * NT));
