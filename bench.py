@@ -665,8 +665,10 @@ def torch_eager_measure(reps=50):
 def decode_stack_measure(steps, layers=32, B=4):
     """Long-generation decode: a 32-layer stack of Llama-3-8B-shaped MLPs
     (11.3 GB of distinct weights, seed 4), B = 4, one step per CUDA-graph
-    replay: fused vs unfused kernels, and the fused stack with the weights
-    encoded as FP8 E4M3 + row scales (5.6 GB per step)."""
+    replay: fused vs unfused kernels, the fused stack with W_gate / W_up in
+    the layout the scheduler picks for the shape (layout "auto"), and the
+    fused stack with the weights encoded as FP8 E4M3 + row scales (5.6 GB
+    per step)."""
     import torch
     from swiglu_mlp_dfk_b200 import inputs as I
     from swiglu_mlp_dfk_b200.stack import DecodeStack
@@ -675,8 +677,9 @@ def decode_stack_measure(steps, layers=32, B=4):
     x0, params = I.make_stack(layers, B, D, F, seed=4, w_std=0.02, device="cuda")
     res = {"layers": layers, "B": B, "steps": steps,
            "weights_GB": round(sum(t.numel() * 2 for p in params for t in p) / 1e9, 2)}
-    for fused, fp8 in ((True, False), (False, False), (True, True)):
-        st = DecodeStack(params, x0, fused=fused, fp8=fp8)
+    for fused, fp8, layout in ((True, False, "row"), (False, False, "row"),
+                               (True, False, "auto"), (True, True, "row")):
+        st = DecodeStack(params, x0, fused=fused, fp8=fp8, layout=layout)
         st.step_eager()                      # scheduler decisions outside capture
         torch.cuda.synchronize()
         st.capture()
@@ -689,8 +692,17 @@ def decode_stack_measure(steps, layers=32, B=4):
         b.record()
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / steps
-        key = "fp8" if fp8 else ("fused" if fused else "unfused")
+        key = "fp8" if fp8 else ("fused_auto" if layout == "auto" else
+                                 ("fused" if fused else "unfused"))
         res[key + "_ms_per_step"] = round(ms, 4)
+        if layout == "auto":
+            gbs = st.bytes_per_step() / (ms * 1e-3) / 1e9
+            res["fused_auto_layout"] = st.layout
+            res["fused_auto_GBps"] = round(gbs, 1)
+            res["fused_auto_frac_of_peak"] = round(gbs / peak, 4)
+            st.release()
+            del st
+            continue
         if fp8:  # the E4M3-MMA calls launch two kernels each (prep + main)
             res["fp8_calls_per_step"] = st.kernels_per_step()
         else:
@@ -708,6 +720,8 @@ def decode_stack_measure(steps, layers=32, B=4):
         st.release()
         del st
     res["fused_speedup"] = round(res["unfused_ms_per_step"] / res["fused_ms_per_step"], 3)
+    res["fused_auto_speedup_over_row"] = round(res["fused_ms_per_step"] /
+                                               res["fused_auto_ms_per_step"], 3)
     res["fp8_speedup_over_bf16_fused"] = round(res["fused_ms_per_step"] / res["fp8_ms_per_step"], 3)
     del params, x0
     torch.cuda.empty_cache()

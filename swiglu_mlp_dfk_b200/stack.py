@@ -9,6 +9,15 @@ long-generation setting of "Deep Kernel Fusion for Transformers" (abstract:
 consistent speed-ups over generation lengths), as a stack of SwiGLU MLP
 layers only.
 
+The fused bf16 stack can hold W_gate / W_up in any of the library's gate/up
+layouts: row-major [d_ff][d_model] as given, column-major [d_model][d_ff],
+or gate/up rows interleaved [d_ff][2][d_model].  With layout="auto" the
+library's scheduler times the fused RMSNorm + gate/up op for the stack's
+shape over every layout (dfk_select_variant with DFK_W_ANY) and the weights
+are stored once in the winner's layout: the profiler-driven choice between
+row- and column-major kernels of "Deep Kernel Fusion for Transformer
+Decoding" (episode description), made per model at load time.
+
 The unfused variant runs the same step with separate kernels (RMSNorm, two
 GEMVs, SiLU, multiply, down projection) and bf16 intermediates in HBM.  The
 FP8 variant encodes every layer's weights once as E4M3 codes with one fp32
@@ -28,11 +37,18 @@ class DecodeStack:
 
     layers: list of (gamma [D], W_gate [F, D], W_up [F, D], W_down [D, F]) bf16
     x0:     [B, D] bf16 first-step input
+    layout: "row", "col", "interleaved" or "auto" -- how the fused bf16
+            stack stores W_gate / W_up (converted copies; "auto" asks the
+            scheduler); the unfused and FP8 stacks are row-major only
     """
 
-    def __init__(self, layers, x0, eps=1e-5, fused=True, fp8=False):
+    def __init__(self, layers, x0, eps=1e-5, fused=True, fp8=False, layout="row"):
         if fp8 and not fused:
             raise ValueError("the FP8 stack runs the fused kernels")
+        if layout not in ("row", "col", "interleaved", "auto"):
+            raise ValueError("layout must be row, col, interleaved or auto")
+        if layout != "row" and (fp8 or not fused):
+            raise ValueError("only the fused bf16 stack takes another weight layout")
         self.eps = float(eps)
         self.fused = fused
         self.fp8 = fp8
@@ -42,10 +58,27 @@ class DecodeStack:
             for gamma, wg, wu, wd in layers:
                 enc.append((gamma,) + I.to_fp8_rows(wg) + I.to_fp8_rows(wu) + I.to_fp8_rows(wd))
             layers = enc
-        self.layers = layers
         self.B, self.D = x0.shape
         self.F = layers[0][1].shape[0]     # W_gate rows (bf16 or FP8 codes)
         dev = x0.device
+        # the stream exists before the layout choice so the scheduler's
+        # timing and every later launch share it
+        self.stream = torch.cuda.Stream(device=dev)
+        if layout == "auto":
+            with torch.cuda.stream(self.stream):
+                rec = dfk.dfk_select_variant(dfk.DFK_OP_RMSNORM_GATE_UP, self.B, self.D, self.F,
+                                             layout=dfk.DFK_W_ANY, stream=self.stream)
+            self.stream.synchronize()
+            layout = {dfk.DFK_W_ROW_MAJOR: "row", dfk.DFK_W_COL_MAJOR: "col",
+                      dfk.DFK_W_GU_INTERLEAVED: "interleaved"}[rec["layout"]]
+        self.layout = layout
+        if layout == "col":
+            layers = [(g, wg.t().contiguous(), wu.t().contiguous(), wd)
+                      for g, wg, wu, wd in layers]
+        elif layout == "interleaved":
+            layers = [(g, torch.stack([wg, wu], 1).contiguous(), None, wd)
+                      for g, wg, wu, wd in layers]
+        self.layers = layers
         self.x = x0.clone()                       # step input (graph-static buffer)
         self.acts = [torch.empty(self.B, self.D, dtype=torch.bfloat16, device=dev)
                      for _ in range(2)]          # ping-pong layer outputs
@@ -57,9 +90,8 @@ class DecodeStack:
             self.s = torch.empty_like(self.h)
         self.graph = None
         # every launch of the stack (eager warm-up, capture, replay) goes to
-        # one stream, so the capture finds the scheduler's decisions and the
+        # self.stream, so the capture finds the scheduler's decisions and the
         # split-K workspace that the warm-up made on that stream
-        self.stream = torch.cuda.Stream(device=dev)
 
     def layer_input(self, l):
         return self.x if l == 0 else self.acts[(l - 1) % 2]
@@ -74,7 +106,7 @@ class DecodeStack:
             return
         gamma, wg, wu, wd = self.layers[l]
         if self.fused:
-            dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, "row", h=self.h)
+            dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, self.layout, h=self.h)
         else:
             dfk.dfk_rmsnorm(xin, gamma, self.eps, out=self.xn)
             dfk.dfk_gemv(self.xn, wg, out=self.a)

@@ -143,3 +143,44 @@ def test_fp8_stack_teacher_forced_layers_match_oracle():
                 checked += 1
         dfk.dfk_rms_rescale(st.acts[(len(params) - 1) % 2], 1e-5, out=st.x)
     assert checked == 4
+
+
+@pytest.mark.parametrize("layout", ["col", "interleaved", "auto"])
+def test_stack_weight_layouts_match_oracle(layout):
+    # the same stack with W_gate / W_up stored column-major or interleaved
+    # (or as the scheduler picks): graph replay equals eager launches, and
+    # each layer, teacher-forced, matches the oracle on the row-major weights
+    x0, params = I.make_stack(3, 4, 1024, 2048, seed=7, w_std=0.02, device="cuda")
+    st = DecodeStack(params, x0, layout=layout)
+    ref = DecodeStack(params, x0, layout=st.layout)
+    assert st.layout in ("row", "col", "interleaved")
+    for l in range(len(params)):
+        xin = st.layer_input(l).clone()
+        st._layer(l)
+        torch.cuda.synchronize()
+        gamma, wg, wu, wd = params[l]
+        _, y_ref = oracle.mlp(I.to_bits(xin), I.to_bits(wg), I.to_bits(wu), I.to_bits(wd),
+                              gamma=I.to_bits(gamma), eps=1e-5)
+        ok, err = close(st.acts[l % 2], y_ref)
+        assert ok, "layout %s layer %d: max err %g" % (st.layout, l, err)
+    dfk.dfk_rms_rescale(st.acts[(len(params) - 1) % 2], 1e-5, out=st.x)
+    ref.step_eager()
+    torch.cuda.synchronize()
+    assert torch.equal(st.x.view(torch.int16), ref.x.view(torch.int16))
+    st.capture()
+    for _ in range(3):
+        st.step()
+        ref.step_eager()
+    torch.cuda.synchronize()
+    assert torch.equal(st.x.view(torch.int16), ref.x.view(torch.int16))
+    st.release()
+
+
+def test_stack_layout_arguments_are_checked():
+    x0, params = I.make_stack(1, 2, 256, 512, seed=8, w_std=0.02, device="cuda")
+    with pytest.raises(ValueError):
+        DecodeStack(params, x0, layout="diagonal")
+    with pytest.raises(ValueError):
+        DecodeStack(params, x0, fused=False, layout="col")
+    with pytest.raises(ValueError):
+        DecodeStack(params, x0, fp8=True, layout="col")
