@@ -813,10 +813,9 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
     pp.ntiles = p.ntiles;
     pp.eps = c.eps;
     void *pargs[] = {&pp};
-    const unsigned P = static_cast<unsigned>(
-        std::min(8, std::max(1, ceil_div(p.ntiles * TC_TILE_K / 8, TC_PREP_THREADS))));
-    cudaError_t e = launch_kernel(tc_norm_prep_fn(), dim3(P, p.bn), dim3(TC_PREP_THREADS), 0, s,
-                                  pdl_enabled(), pargs, P);
+    // one CTA per token slot
+    cudaError_t e = launch_kernel(tc_norm_prep_fn(), dim3(p.bn), dim3(TC_PREP_THREADS), 0, s,
+                                  pdl_enabled(), pargs);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return cuda_fail(e, "RMSNorm prep kernel launch");
@@ -1238,11 +1237,9 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
   pp.ntiles = p.ntiles;
   pp.eps = c.eps;
   void *pargs[] = {&pp};
-  // P CTAs per token (a cluster), one 256-thread pass over ~K / P elements each
-  const unsigned P = static_cast<unsigned>(
-      std::min(8, std::max(1, ceil_div(p.ntiles * TM8_TILE_K / 8, TM8_PREP_THREADS))));
-  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(P, p.bnp), dim3(TM8_PREP_THREADS), 0, s,
-                                pdl_enabled(), pargs, P);
+  // one CTA per token slot
+  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
+                                pdl_enabled(), pargs);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_fail(e, "FP8 activation-term kernel launch");

@@ -27,7 +27,7 @@
 // and lo rows sit side by side on N (one MMA of N = 2 * bn reads each weight
 // tile once); the epilogue adds the two column halves.  NORM = 1 does this
 // transform inside the kernel; NORM = 2 reads tiles that a prep kernel (a
-// thread-block cluster per token, launched just before) wrote in the same
+// CTA per token, launched just before) wrote in the same
 // layout, with r_b, so the kernel streams them like plain activations (the
 // in-kernel transform serialises with the MMAs and costs a third of the time
 // at 64 tokens; the host uses NORM = 2 above 32 tokens).
@@ -37,7 +37,6 @@
 // releasing ring stages; warps 2-5 run the x*gamma transform (NORM) and the
 // epilogue (tcgen05.ld -> SiLU * up -> one bf16 store per output).
 #pragma once
-#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cstdint>
 
@@ -511,14 +510,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
-// ---- prep for NORM = 2: one cluster of P CTAs (blockIdx.x = rank) per
-// token slot b = blockIdx.y, each over a contiguous range of 8-element
-// chunks.  sum x^2 in a fixed order (thread chains, warp butterfly, warps in
-// order, ranks in order through distributed shared memory) gives r_b; x *
-// gamma (exact in fp32) is split into bf16 hi + lo and written as rows
-// tile * 2 bn + b (hi) and tile * 2 bn + bn + b (lo) of 64 bf16 per k tile;
-// zeros past K and for b >= B.  Defined in the one file that instantiates
-// the kernels.
+// ---- prep for NORM = 2: one CTA per token slot b = blockIdx.x, one pass
+// over x.  x * gamma (exact in fp32) is split into bf16 hi + lo and written
+// as rows tile * 2 bn + b (hi) and tile * 2 bn + bn + b (lo) of 64 bf16 per
+// k tile -- zeros past K and for b >= B -- as each chunk of 8 elements
+// arrives (the split does not depend on r_b); sum x^2 in a fixed order (each
+// thread chains its chunks c = t + TC_PREP_THREADS * i, i then e ascending;
+// a xor butterfly per warp; the warps in order) gives r_b.  Defined in the
+// one file that instantiates the kernels.
 struct TcPrepParams {
   const uint16_t *x;      // [B][K] bf16
   const uint16_t *gamma;  // [K] bf16
@@ -528,31 +527,54 @@ struct TcPrepParams {
   float eps;
 };
 
-constexpr int TC_PREP_THREADS = 256;
+constexpr int TC_PREP_THREADS = 512;
 
 #ifdef DFK_TC_KERNELS
 __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcPrepParams p) {
-  __shared__ float s_part, s_wss[TC_PREP_THREADS / 32];
-  cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+  __shared__ float s_wss[TC_PREP_THREADS / 32];
   pdl_launch_dependents();
   pdl_wait();  // x comes from the previous kernel
-  const int rank = blockIdx.x, P = gridDim.x, b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool real = b < p.B;
   const int nchunk = p.ntiles * TC_TILE_K / 8, kchunks = p.K / 8;
-  const int per = (nchunk + P - 1) / P;
-  const int c0 = rank * per, c1 = min(nchunk, c0 + per);
   float ss = 0.f;
-  if (real) {
-    for (int c = c0 + tid; c < min(c1, kchunks); c += TC_PREP_THREADS) {
-      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  for (int c0 = tid; c0 < nchunk; c0 += 4 * TC_PREP_THREADS) {
+    uint4 xv[4], gv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // up to four chunks' loads in flight per thread
+      const int c = c0 + i * TC_PREP_THREADS;
+      xv[i] = gv[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (real && c < kchunks) {
+        xv[i] = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
+        gv[i] = ld_nc_v4(p.gamma + 8 * c);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = c0 + i * TC_PREP_THREADS;
+      if (c >= nchunk) continue;
+      const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+      const uint32_t gw[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+      uint32_t hw[4], lw[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
         ss = fmaf(x0, x0, ss);
         ss = fmaf(x1, x1, ss);
+        const float p0 = x0 * bf16_lo(gw[u]);  // exact
+        const float p1 = x1 * bf16_hi(gw[u]);
+        const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
+        const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+        const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+        hw[u] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+        lw[u] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
+                (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
       }
+      const int k = 8 * c, tile = k / TC_TILE_K, kk = k % TC_TILE_K;
+      uint16_t *hrow = p.xg + (static_cast<size_t>(tile) * 2 * p.bn + b) * TC_TILE_K;
+      *reinterpret_cast<uint4 *>(hrow + kk) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4 *>(hrow + static_cast<size_t>(p.bn) * TC_TILE_K + kk) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
 #pragma unroll
@@ -562,40 +584,7 @@ __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcP
   if (tid == 0) {
     float t = 0.f;
     for (int w = 0; w < TC_PREP_THREADS / 32; ++w) t += s_wss[w];
-    s_part = t;
-  }
-  cl.sync();  // every rank's partial sum is in its shared memory
-  if (tid == 0 && rank == 0) {
-    float t = 0.f;
-    for (int q = 0; q < P; ++q) t += *cl.map_shared_rank(&s_part, q);
     p.rinv[b] = real ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 0.f;
-  }
-  cl.sync();  // remote reads done before any CTA of the cluster leaves
-  for (int c = c0 + tid; c < c1; c += TC_PREP_THREADS) {
-    const int k = 8 * c, tile = k / TC_TILE_K, kk = k % TC_TILE_K;
-    uint4 hv = make_uint4(0u, 0u, 0u, 0u), lv = make_uint4(0u, 0u, 0u, 0u);
-    if (real && c < kchunks) {
-      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + k);
-      const uint4 gv = ld_nc_v4(p.gamma + k);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float p0 = bf16_lo(xw[u]) * bf16_lo(gw[u]);  // exact
-        const float p1 = bf16_hi(xw[u]) * bf16_hi(gw[u]);
-        const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
-        const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
-        const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
-        hw[u] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-        lw[u] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
-                (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
-      }
-      hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-    uint16_t *hrow = p.xg + (static_cast<size_t>(tile) * 2 * p.bn + b) * TC_TILE_K;
-    *reinterpret_cast<uint4 *>(hrow + kk) = hv;
-    *reinterpret_cast<uint4 *>(hrow + static_cast<size_t>(p.bn) * TC_TILE_K + kk) = lv;
   }
 }
 #endif  // DFK_TC_KERNELS

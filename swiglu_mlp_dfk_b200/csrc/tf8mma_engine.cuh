@@ -18,9 +18,11 @@
 // reads each weight tile once for all terms and tokens, and
 //   sum_k W[j][k] v[k] = s[j] * 2^-e_b * sum_t 16^-t D[j][t * bnp + b],
 // the terms combined smallest first (Horner in 1/16, exact scalings).
-// The prep kernel (a cluster of up to 8 CTAs per token, partials combined
-// through distributed shared memory) also computes r_b = 1 / sqrt(mean x^2 +
-// eps) for the RMSNorm and stores f_b = r_b * 2^-e_b (1 * 2^-e_b without it).
+// The prep kernel (one CTA per token, a single pass over x held in
+// registers: the x-dependent chain between the previous kernel and this one
+// is one L2 round trip and one block reduction) also computes r_b = 1 /
+// sqrt(mean x^2 + eps) for the RMSNorm and stores f_b = r_b * 2^-e_b
+// (1 * 2^-e_b without it).
 //
 // Main kernel: one CTA per SM owns r <= 128 weight rows (the MMA's M) over its
 // reduction range (split-K slices for the down projection); a TMA ring
@@ -33,8 +35,6 @@
 #include <cuda.h>
 #include <cstdint>
 
-#include <cooperative_groups.h>
-
 #include "ptx.cuh"
 #include "tc_ptx.cuh"
 
@@ -42,7 +42,8 @@ namespace dfk {
 
 constexpr int TM8_THREADS = 192;
 constexpr int TM8_TILE_K = 128;
-constexpr int TM8_PREP_THREADS = 256;
+constexpr int TM8_PREP_THREADS = 512;
+constexpr int TM8_PREP_CPT = 4;  // chunks per prep thread kept in registers
 
 // kind::f8f6f4 instruction descriptor: E4M3 A and B (format 0), fp32 D,
 // both K-major, shape M x N.
@@ -91,45 +92,110 @@ struct Tm8PrepParams {
   float eps;
 };
 
-// One cluster of P CTAs (blockIdx.x = rank) per token slot b = blockIdx.y;
-// each CTA takes a contiguous range of 8-element chunks.  Pass 1: max |v| and
-// sum x^2 of the range (fixed order: thread chains, warp butterfly, warps in
-// order); the ranks' partials are combined in rank order through distributed
-// shared memory; pass 2 writes the T term codes of the range (zeros past K
-// and for b >= B).  Defined in the one file that instantiates the kernels.
+// One CTA per token slot b = blockIdx.x, one pass over x: thread t holds
+// chunks c = t + TM8_PREP_THREADS * i (8 elements each) in registers for
+// i < TM8_PREP_CPT and re-reads any further ones.  max |v| and sum x^2 in a
+// fixed order (each thread chains its chunks, i then e ascending; a xor
+// butterfly per warp; the warps in order), then the T term codes of every
+// chunk (zeros past K and for b >= B).  Defined in the one file that
+// instantiates the kernels.
 #ifdef DFK_TF8MMA_KERNELS
-__global__ void __launch_bounds__(TM8_PREP_THREADS)
-    tf8mma_prep_kernel(const Tm8PrepParams p) {
-  __shared__ float s_part[2];  // this CTA's max |v| and sum x^2
+__device__ __forceinline__ void tm8_load_chunk(const Tm8PrepParams &p, int b, int c, uint4 &xv,
+                                               uint4 &gv) {
+  xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
+  gv = p.gamma ? ld_nc_v4(p.gamma + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// v = x (or x * gamma, exact in fp32) of one chunk
+__device__ __forceinline__ void tm8_chunk_values(const Tm8PrepParams &p, const uint4 &xv,
+                                                 const uint4 &gv, float (&v)[8]) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
+    v[2 * u] = p.gamma ? x0 * bf16_lo(gw[u]) : x0;
+    v[2 * u + 1] = p.gamma ? x1 * bf16_hi(gw[u]) : x1;
+  }
+}
+
+__device__ __forceinline__ void tm8_chunk_stats(const uint4 &xv, const float (&v)[8], float &mx,
+                                                float &ss) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
+    ss = fmaf(x0, x0, ss);
+    ss = fmaf(x1, x1, ss);
+    mx = fmaxf(mx, fmaxf(fabsf(v[2 * u]), fabsf(v[2 * u + 1])));
+  }
+}
+
+// The T term codes of one chunk (u = v * 2^e, already scaled) at k = 8 c.
+__device__ __forceinline__ void tm8_write_terms(const Tm8PrepParams &p, int b, int c,
+                                                float (&u)[8]) {
+  const int k = 8 * c, tile = k / TM8_TILE_K, kk = k % TM8_TILE_K;
+  const int rows = p.T * p.bnp;
+  for (int t = 0; t < p.T; ++t) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t c01 = f32x2_to_e4m3x2(u[4 * h + 0], u[4 * h + 1]);
+      const uint32_t c23 = f32x2_to_e4m3x2(u[4 * h + 2], u[4 * h + 3]);
+      w[h] = c01 | (c23 << 16);
+      float d0, d1, d2, d3;
+      e4m3x2_to_f32(c01, d0, d1);
+      e4m3x2_to_f32(c23, d2, d3);
+      // residual, scaled for the next term (exact: |residual| <= half an
+      // E4M3 step of u, and times 16 stays below 448)
+      u[4 * h + 0] = (u[4 * h + 0] - d0) * 16.f;
+      u[4 * h + 1] = (u[4 * h + 1] - d1) * 16.f;
+      u[4 * h + 2] = (u[4 * h + 2] - d2) * 16.f;
+      u[4 * h + 3] = (u[4 * h + 3] - d3) * 16.f;
+    }
+    uint8_t *dst = p.terms + (static_cast<size_t>(tile) * rows + t * p.bnp + b) * TM8_TILE_K + kk;
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+  }
+}
+
+__global__ void __launch_bounds__(TM8_PREP_THREADS) tf8mma_prep_kernel(const Tm8PrepParams p) {
   __shared__ float s_wmax[TM8_PREP_THREADS / 32], s_wss[TM8_PREP_THREADS / 32];
   __shared__ float s_scale;
-  cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
   pdl_launch_dependents();
   pdl_wait();  // x comes from the previous kernel
-  const int rank = blockIdx.x, P = gridDim.x, b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool real = b < p.B;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nchunk = (p.ntiles * TM8_TILE_K) / 8;  // 8-element chunks incl. padding
   const int kchunks = p.K / 8;
-  const int per = (nchunk + P - 1) / P;
-  const int c0 = rank * per, c1 = min(nchunk, c0 + per);
-  float mx = 0.f, ss = 0.f;
-  if (real) {
-    for (int c = c0 + tid; c < min(c1, kchunks); c += TM8_PREP_THREADS) {
-      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
-      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
-      if (p.gamma) gv = ld_nc_v4(p.gamma + 8 * c);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+  constexpr int NT = TM8_PREP_THREADS, CPT = TM8_PREP_CPT;
+  if (b >= p.B) {  // padding token slot: zero codes, zero factor
+    float z[8];
+    for (int c = tid; c < nchunk; c += NT) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float x0 = bf16_lo(xw[u]), x1 = bf16_hi(xw[u]);
-        ss = fmaf(x0, x0, ss);
-        ss = fmaf(x1, x1, ss);
-        const float v0 = p.gamma ? x0 * bf16_lo(gw[u]) : x0;
-        const float v1 = p.gamma ? x1 * bf16_hi(gw[u]) : x1;
-        mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
-      }
+      for (int i = 0; i < 8; ++i) z[i] = 0.f;
+      tm8_write_terms(p, b, c, z);
     }
+    if (tid == 0) p.fac[b] = 0.f;
+    return;
+  }
+  uint4 xr[CPT], gr[CPT];
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {  // every load issued before any use
+    const int c = tid + NT * i;
+    xr[i] = gr[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < kchunks) tm8_load_chunk(p, b, c, xr[i], gr[i]);
+  }
+  float mx = 0.f, ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    float v[8];
+    tm8_chunk_values(p, xr[i], gr[i], v);
+    tm8_chunk_stats(xr[i], v, mx, ss);
+  }
+  for (int c = tid + NT * CPT; c < kchunks; c += NT) {
+    uint4 xv, gv;
+    tm8_load_chunk(p, b, c, xv, gv);
+    float v[8];
+    tm8_chunk_values(p, xv, gv, v);
+    tm8_chunk_stats(xv, v, mx, ss);
   }
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) {
@@ -143,20 +209,9 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS)
   __syncthreads();
   if (tid == 0) {
     float m = 0.f, t = 0.f;
-    for (int w = 0; w < TM8_PREP_THREADS / 32; ++w) {
+    for (int w = 0; w < NT / 32; ++w) {
       m = fmaxf(m, s_wmax[w]);
       t += s_wss[w];
-    }
-    s_part[0] = m;
-    s_part[1] = t;
-  }
-  cl.sync();  // every rank's partials are in its shared memory
-  if (tid == 0) {
-    float m = 0.f, t = 0.f;
-    for (int q = 0; q < P; ++q) {
-      const float *rp = cl.map_shared_rank(s_part, q);
-      m = fmaxf(m, rp[0]);
-      t += rp[1];
     }
     int e = 0;
     if (m > 0.f) {
@@ -165,52 +220,30 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS)
       e = min(max(8 - E, -126), 126);  // m * 2^e in [128, 256)
     }
     s_scale = ldexpf(1.0f, e);
-    if (rank == 0) {
-      const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
-      p.fac[b] = real ? r * ldexpf(1.0f, -e) : 0.f;
+    const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
+    p.fac[b] = r * ldexpf(1.0f, -e);
+  }
+  __syncthreads();
+  const float sc = s_scale;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = tid + NT * i;
+    if (c < nchunk) {
+      float u[8];
+      tm8_chunk_values(p, xr[i], gr[i], u);  // zeros past K
+#pragma unroll
+      for (int q = 0; q < 8; ++q) u[q] *= sc;
+      tm8_write_terms(p, b, c, u);
     }
   }
-  cl.sync();  // remote reads done (no CTA leaves early); s_scale visible
-  const float sc = s_scale;
-  const int rows = p.T * p.bnp;
-  for (int c = c0 + tid; c < c1; c += TM8_PREP_THREADS) {
-    const int k = 8 * c, tile = k / TM8_TILE_K, kk = k % TM8_TILE_K;
+  for (int c = tid + NT * CPT; c < nchunk; c += NT) {
+    uint4 xv = make_uint4(0u, 0u, 0u, 0u), gv = make_uint4(0u, 0u, 0u, 0u);
+    if (c < kchunks) tm8_load_chunk(p, b, c, xv, gv);
     float u[8];
-    if (real && c < kchunks) {
-      const uint4 xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + k);
-      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
-      if (p.gamma) gv = ld_nc_v4(p.gamma + k);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    tm8_chunk_values(p, xv, gv, u);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float x0 = bf16_lo(xw[i]), x1 = bf16_hi(xw[i]);
-        u[2 * i] = (p.gamma ? x0 * bf16_lo(gw[i]) : x0) * sc;
-        u[2 * i + 1] = (p.gamma ? x1 * bf16_hi(gw[i]) : x1) * sc;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) u[i] = 0.f;
-    }
-    for (int t = 0; t < p.T; ++t) {
-      uint32_t w[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t c01 = f32x2_to_e4m3x2(u[4 * h + 0], u[4 * h + 1]);
-        const uint32_t c23 = f32x2_to_e4m3x2(u[4 * h + 2], u[4 * h + 3]);
-        w[h] = c01 | (c23 << 16);
-        float d0, d1, d2, d3;
-        e4m3x2_to_f32(c01, d0, d1);
-        e4m3x2_to_f32(c23, d2, d3);
-        // residual, scaled for the next term (exact: |residual| <= half an
-        // E4M3 step of u, and times 16 stays below 448)
-        u[4 * h + 0] = (u[4 * h + 0] - d0) * 16.f;
-        u[4 * h + 1] = (u[4 * h + 1] - d1) * 16.f;
-        u[4 * h + 2] = (u[4 * h + 2] - d2) * 16.f;
-        u[4 * h + 3] = (u[4 * h + 3] - d3) * 16.f;
-      }
-      uint8_t *dst = p.terms + (static_cast<size_t>(tile) * rows + t * p.bnp + b) * TM8_TILE_K + kk;
-      *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
-    }
+    for (int q = 0; q < 8; ++q) u[q] *= sc;
+    tm8_write_terms(p, b, c, u);
   }
 }
 #endif  // DFK_TF8MMA_KERNELS
