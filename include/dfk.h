@@ -99,9 +99,11 @@ typedef struct dfk_variant {
   int full_m_tiles; /* tensor core: 1 = each CTA owns 128 output rows (full MMA M) */
   int stages;       /* ring stages used at the queried shape (0 = not resolved)      */
   float measured_us;/* median timed duration; < 0 when chosen without timing        */
-  int e4m3_mma;     /* tensor core, FP8 weights only: 1 = E4M3 MMA on the codes
-                       (kind::f8f6f4, activations as E4M3 terms); dfk_variant_info
-                       reports these under the FP8 ops                           */
+  int e4m3_mma;     /* tensor core, FP8 weights only: E4M3 MMA on the codes
+                       (kind::f8f6f4, activations as E4M3 terms); 1 = terms
+                       written by a prep kernel, 2 = derived inside the kernel
+                       (up to 16 tokens); dfk_variant_info reports these under
+                       the FP8 ops                                               */
 } dfk_variant;
 
 /*
@@ -181,12 +183,14 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
  * (fp32 FMA on the widened codes; at most two k tiles per stage); a
  * widening tensor-core kernel (the tensor-core ids with one k tile per stage
  * and rows spread over the SMs: codes widened to bf16 into TMEM, bf16 MMA
- * with fp32 accumulation); and the E4M3-MMA kernel (ids with e4m3_mma = 1:
+ * with fp32 accumulation); and the E4M3-MMA kernel (ids with e4m3_mma >= 1:
  * the codes feed the E4M3 tensor-core MMA directly, each token's activations
- * are first written as E4M3 terms -- two for bf16 x, four for x * gamma,
- * after a power-of-two scale -- by a small kernel launched before it, into a
- * library-owned buffer per (device, stream) allocated at first use outside
- * stream capture).  Tensor-core kernels take at most 128 output rows per SM
+ * are written as E4M3 terms -- two for bf16 x, four for x * gamma, after a
+ * power-of-two scale -- either (e4m3_mma = 1) by a small kernel launched
+ * before it, into a library-owned buffer per (device, stream) allocated at
+ * first use outside stream capture, or (e4m3_mma = 2, B <= 16) inside the
+ * kernel from each ring stage's raw activations; with a k split the latter
+ * scales each slice's partial sums by the slice's own power of two).  Tensor-core kernels take at most 128 output rows per SM
  * (per SM / k_split for the down projection).  Other ids are rejected with
  * DFK_ERR_INVALID_ARG; E4M3-MMA ids are rejected by the bf16 entry points.
  * Constraints: row-major only; the reduction length (d_model for gate/up,

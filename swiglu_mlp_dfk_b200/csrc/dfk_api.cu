@@ -276,6 +276,13 @@ static const std::vector<VDef> &variants() {
     // slices as fill the SMs: ceil(N / 128) row blocks x floor(SMs / blocks)
     for (int nt : {1, 2, 4, 8})
       t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, 0, nt, 1, 0, 1, 0});
+    // FP8 weights, up to 16 tokens: the E4M3 MMA with the activation terms
+    // derived inside the kernel (no prep kernel)
+    for (int nt : {1, 2}) {
+      t.push_back({id++, CLS_GATE_UP, DFK_FAMILY_TENSOR_CORE, 0, 64, 1, nt, 1, 0, 0, 2});
+      for (int ks : {1, 2, 4})
+        t.push_back({id++, CLS_GEMV, DFK_FAMILY_TENSOR_CORE, 0, 64, ks, nt, 1, 0, 0, 2});
+    }
     return t;
   }();
   return v;
@@ -1050,7 +1057,7 @@ static int launch_tf8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
 
 struct Tm8Plan {
   const void *fn = nullptr;
-  int grid = 0;
+  int grid = 0, threads = TM8_THREADS;
   size_t smem = 0;
   Tm8Params p{};
   size_t term_bytes = 0;  // activation-term buffer: codes + per-token factors
@@ -1069,8 +1076,16 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
     if (why) *why = "batch outside 1..64";
     return false;
   }
+  const bool ink = v.e4m3mma == 2;  // activation terms derived in the kernel
   const int T = norm ? 4 : 2;
-  const int bnp = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
+  // in-kernel terms: the fewest token slots holding B with 16 or 32 MMA columns
+  const int ibp = !ink ? 0 : (T == 4 ? (B <= 4 ? 4 : (B <= 8 ? 8 : 0))
+                                     : (B <= 8 ? 8 : (B <= 16 ? 16 : 0)));
+  if (ink && !ibp) {
+    if (why) *why = "in-kernel activation terms: up to 8 tokens with RMSNorm, 16 without";
+    return false;
+  }
+  const int bnp = ink ? ibp : (B <= 16 ? 16 : (B <= 32 ? 32 : 64));
   const int np = T * bnp;
   if (np > 256 || nmat * np > 512) {
     if (why) *why = "activation terms exceed N = 256";
@@ -1095,18 +1110,21 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   }
   const int r8 = round_up(hmax, 8);
   const int a8 = nmat * r8 * 128;
-  const int stage = v.nt * (a8 + np * 128);  // multiples of 1024
+  // stage: code tiles (+ the term tiles with prep terms); in-kernel terms
+  // keep the whole k range's terms resident after the ring
+  const int stage = v.nt * (a8 + (ink ? 0 : np * 128));  // multiples of 1024
+  const int tarea = ink ? ceil_div(ntiles, ks) * np * 128 : 0;
   // the last code tile's 128-row MMA read may run past the last stage
   const int over = (v.nt * nmat - 1) * r8 * 128 + 128 * 128;
-  const int slack = std::max(0, over - stage);
-  const int bar_bytes = 256;        // 2 S + 1 barriers and flags
+  const int slack = std::max(0, over - stage - tarea);
+  const int bar_bytes = 512;  // 2 S + 2 barriers, flags, per-token factors and scales
   const int smem_cap = std::min(ds.smem_optin, 232448);
-  const int S = std::min(8, (smem_cap - 1024 - bar_bytes - slack) / stage);
+  const int S = std::min(8, (smem_cap - 1024 - bar_bytes - slack - tarea) / stage);
   if (S < 2) {
     if (why) *why = "shared memory too small for two ring stages";
     return false;
   }
-  const void *fn = tf8mma_find_kernel(nmat);
+  const void *fn = tf8mma_find_kernel(nmat, ibp, ink ? T : 0);
   if (!fn) {
     if (why) *why = "E4M3-MMA kernel not compiled for this op";
     return false;
@@ -1128,14 +1146,16 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   p.stage_bytes = stage;
   p.a8_bytes = a8;
   p.tmem_cols = std::max(32, pow2_ceil(nmat * np));
-  p.bar_off = S * stage + slack;
+  p.bar_off = S * stage + tarea + slack;
   p.ntiles = ntiles;
   p.kslices = ks;
   p.nblocks = nblocks;
+  p.term_off = ink ? S * stage : v.nt * a8;
   pl->fn = fn;
   pl->grid = nblocks * ks;
+  pl->threads = ink ? TM8_INK_THREADS : TM8_THREADS;
   pl->smem = 1024 + static_cast<size_t>(p.bar_off) + bar_bytes;
-  pl->term_bytes = static_cast<size_t>(ntiles) * np * 128 + 64 * sizeof(float);
+  pl->term_bytes = ink ? 0 : static_cast<size_t>(ntiles) * np * 128 + 64 * sizeof(float);
   return true;
 }
 
@@ -1180,8 +1200,9 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
   if (!plan_tm8(c.nmat, c.norm, v, c.B, c.K, c.N, *ds, &pl, &why))
     return fail(DFK_ERR_NO_VARIANT, "variant %d does not fit FP8 B=%d K=%d N=%d: %s", v.id, c.B,
                 c.K, c.N, why.c_str());
+  const bool ink = v.e4m3mma == 2;  // no prep kernel, no term buffer
   void *terms = nullptr;
-  if ((rc = get_term_buffer(dev, s, pl.term_bytes, &terms))) {
+  if (!ink && (rc = get_term_buffer(dev, s, pl.term_bytes, &terms))) {
     if (rc != DFK_ERR_NO_VARIANT || !stream_capturing(s)) return rc;
     // captured on a stream without the buffer: the widening tensor-core kernel
     VDef alt = v;
@@ -1192,7 +1213,7 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
   if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
   Tm8Params p = pl.p;
   const size_t code_bytes = static_cast<size_t>(p.ntiles) * p.np * 128;
-  float *fac = reinterpret_cast<float *>(static_cast<char *>(terms) + code_bytes);
+  float *fac = ink ? nullptr : reinterpret_cast<float *>(static_cast<char *>(terms) + code_bytes);
   Tm8Maps maps;
   memset(&maps, 0, sizeof maps);
   const void *w[2] = {c.w0, c.w1};
@@ -1203,10 +1224,13 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
                               &maps.w[m][lo], true, CU_TENSOR_MAP_DATA_TYPE_UINT8)))
         return rc;
     }
-  if ((rc = tensor_map_2d(terms, TM8_TILE_K, static_cast<uint64_t>(p.ntiles) * p.np, TM8_TILE_K,
-                          TM8_TILE_K, static_cast<uint32_t>(p.np), &maps.x, true,
-                          CU_TENSOR_MAP_DATA_TYPE_UINT8)))
+  if (!ink && (rc = tensor_map_2d(terms, TM8_TILE_K, static_cast<uint64_t>(p.ntiles) * p.np,
+                                  TM8_TILE_K, TM8_TILE_K, static_cast<uint32_t>(p.np), &maps.x,
+                                  true, CU_TENSOR_MAP_DATA_TYPE_UINT8)))
     return rc;
+  p.x = static_cast<const uint16_t *>(c.x);
+  p.gamma = c.norm ? static_cast<const uint16_t *>(c.gamma) : nullptr;
+  p.eps = c.eps;
   p.out = static_cast<uint16_t *>(c.out);
   p.scale[0] = c.s0;
   p.scale[1] = c.s1;
@@ -1224,28 +1248,31 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
       return launch_tm8(c, whole, s, stages_used);
     }
   }
-  // prep: scales, r_b and the E4M3 terms of the activations
-  Tm8PrepParams pp{};
-  pp.x = static_cast<const uint16_t *>(c.x);
-  pp.gamma = c.norm ? static_cast<const uint16_t *>(c.gamma) : nullptr;
-  pp.terms = static_cast<uint8_t *>(terms);
-  pp.fac = fac;
-  pp.B = c.B;
-  pp.K = c.K;
-  pp.bnp = p.bnp;
-  pp.T = p.T;
-  pp.ntiles = p.ntiles;
-  pp.eps = c.eps;
-  void *pargs[] = {&pp};
-  // one CTA per token slot
-  cudaError_t e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
-                                pdl_enabled(), pargs);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return cuda_fail(e, "FP8 activation-term kernel launch");
+  cudaError_t e = cudaSuccess;
+  if (!ink) {
+    // prep: scales, r_b and the E4M3 terms of the activations
+    Tm8PrepParams pp{};
+    pp.x = static_cast<const uint16_t *>(c.x);
+    pp.gamma = c.norm ? static_cast<const uint16_t *>(c.gamma) : nullptr;
+    pp.terms = static_cast<uint8_t *>(terms);
+    pp.fac = fac;
+    pp.B = c.B;
+    pp.K = c.K;
+    pp.bnp = p.bnp;
+    pp.T = p.T;
+    pp.ntiles = p.ntiles;
+    pp.eps = c.eps;
+    void *pargs[] = {&pp};
+    // one CTA per token slot
+    e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
+                      pdl_enabled(), pargs);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "FP8 activation-term kernel launch");
+    }
   }
   void *args[] = {&maps, &p};
-  e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TM8_THREADS), pl.smem, s, pdl_enabled(), args);
+  e = launch_kernel(pl.fn, dim3(pl.grid), dim3(pl.threads), pl.smem, s, pdl_enabled(), args);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_fail(e, "FP8 E4M3-MMA kernel launch");
@@ -1430,10 +1457,10 @@ static bool feasible(const VDef &d, const CcCall &c, const DeviceState &ds) {
 // fits, the feasible CUDA-core variant with the fewest passes wins.
 static const VDef *heuristic(int op, int B, const CcCall &c, const DeviceState &ds) {
   if (c.w8 && B >= 2) {
-    // FP8 weights: the E4M3-MMA kernel, else the widening one (split-K 4 for
-    // the GEMV)
+    // FP8 weights: the E4M3-MMA kernel (with in-kernel activation terms up
+    // to 16 tokens), else the widening one (split-K 4 for the GEMV)
     const int want_ks = op_class(op) == CLS_GEMV ? 4 : 1;
-    for (int mma : {1, 0})
+    for (int mma : {2, 1, 0})
       for (const VDef &d : variants())
         if (d.cls == op_class(op) && d.family == DFK_FAMILY_TENSOR_CORE && d.nt == 1 &&
             d.full == 0 && d.e4m3mma == mma && d.ksplit == want_ks && feasible(d, c, ds))

@@ -42,6 +42,10 @@ namespace dfk {
 
 constexpr int TM8_THREADS = 192;
 constexpr int TM8_TILE_K = 128;
+// in-kernel activation terms (no prep kernel): 8 more warps write the terms
+// of the CTA's whole k range into shared memory once
+constexpr int TM8_XF_THREADS = 256;
+constexpr int TM8_INK_THREADS = TM8_THREADS + TM8_XF_THREADS;
 constexpr int TM8_PREP_THREADS = 512;
 constexpr int TM8_PREP_CPT = 4;  // chunks per prep thread kept in registers
 
@@ -81,6 +85,28 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float &lo, float &h
       "cvt.f32.f16 %1, b;\n\t}"
       : "=f"(lo), "=f"(hi)
       : "r"(pair));
+}
+
+// One E4M3 term of 8 scaled activations u (codes packed little-endian into
+// w0, w1); u becomes the residual times 16, the next term's input (exact:
+// |residual| <= half an E4M3 step of u, and times 16 stays below 448).
+__device__ __forceinline__ void tm8_encode_term(float (&u)[8], uint32_t &w0, uint32_t &w1) {
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t c01 = f32x2_to_e4m3x2(u[4 * h + 0], u[4 * h + 1]);
+    const uint32_t c23 = f32x2_to_e4m3x2(u[4 * h + 2], u[4 * h + 3]);
+    w[h] = c01 | (c23 << 16);
+    float d0, d1, d2, d3;
+    e4m3x2_to_f32(c01, d0, d1);
+    e4m3x2_to_f32(c23, d2, d3);
+    u[4 * h + 0] = (u[4 * h + 0] - d0) * 16.f;
+    u[4 * h + 1] = (u[4 * h + 1] - d1) * 16.f;
+    u[4 * h + 2] = (u[4 * h + 2] - d2) * 16.f;
+    u[4 * h + 3] = (u[4 * h + 3] - d3) * 16.f;
+  }
+  w0 = w[0];
+  w1 = w[1];
 }
 
 struct Tm8PrepParams {
@@ -136,24 +162,15 @@ __device__ __forceinline__ void tm8_write_terms(const Tm8PrepParams &p, int b, i
   const int k = 8 * c, tile = k / TM8_TILE_K, kk = k % TM8_TILE_K;
   const int rows = p.T * p.bnp;
   for (int t = 0; t < p.T; ++t) {
-    uint32_t w[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t c01 = f32x2_to_e4m3x2(u[4 * h + 0], u[4 * h + 1]);
-      const uint32_t c23 = f32x2_to_e4m3x2(u[4 * h + 2], u[4 * h + 3]);
-      w[h] = c01 | (c23 << 16);
-      float d0, d1, d2, d3;
-      e4m3x2_to_f32(c01, d0, d1);
-      e4m3x2_to_f32(c23, d2, d3);
-      // residual, scaled for the next term (exact: |residual| <= half an
-      // E4M3 step of u, and times 16 stays below 448)
-      u[4 * h + 0] = (u[4 * h + 0] - d0) * 16.f;
-      u[4 * h + 1] = (u[4 * h + 1] - d1) * 16.f;
-      u[4 * h + 2] = (u[4 * h + 2] - d2) * 16.f;
-      u[4 * h + 3] = (u[4 * h + 3] - d3) * 16.f;
+    uint32_t w0, w1;
+    if (t + 1 < p.T) {
+      tm8_encode_term(u, w0, w1);
+    } else {  // the last term: no residual needed
+      w0 = f32x2_to_e4m3x2(u[0], u[1]) | (f32x2_to_e4m3x2(u[2], u[3]) << 16);
+      w1 = f32x2_to_e4m3x2(u[4], u[5]) | (f32x2_to_e4m3x2(u[6], u[7]) << 16);
     }
     uint8_t *dst = p.terms + (static_cast<size_t>(tile) * rows + t * p.bnp + b) * TM8_TILE_K + kk;
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
   }
 }
 
@@ -263,19 +280,38 @@ struct Tm8Params {
   int ntiles, kslices, nblocks;
   float *part;            // split-K partial sums [kslices][nblocks][bnp][128]
   unsigned *counters;     // [nblocks]
+  int term_off;           // prep terms: offset of the term tiles within a stage;
+                          // in-kernel terms: offset of the resident term area
+                          // ([tiles of this CTA][np rows][128], after the ring)
+  const uint16_t *x;      // in-kernel terms: [B][K] bf16 activations
+  const uint16_t *gamma;  // in-kernel terms: [K] bf16, or nullptr (no RMSNorm)
+  float eps;
 };
 
 // w[m][0]: codes of matrix m, box {128, hmax}; w[m][1]: box {128, hmax - 1};
-// x: the term codes [ntiles * np][128], box {128, np}.  128-byte swizzle.
+// x: the term codes [ntiles * np][128], box {128, np} (prep terms only).
+// 128-byte swizzle.
 struct Tm8Maps {
   CUtensorMap w[2][2];
   CUtensorMap x;
 };
 
-template <int NMAT>
-__global__ void __launch_bounds__(TM8_THREADS, 1)
+// IBP > 0: in-kernel terms, no prep kernel.  IBP token slots (4, 8 or 16)
+// and IT terms per token (IR = IBP * IT = 16 or 32 MMA columns).  Warps
+// 6..13 wait for the previous kernel, read this CTA's k range of x once,
+// derive each token's scale 2^e_b (and r_b) from it, and write the terms of
+// the whole range into a resident shared-memory area (128-byte swizzle, as
+// TMA would write them), then release it to the MMA thread (tready).  The
+// TMA ring carries only the weight codes, so the producer never waits for
+// the previous kernel.  With a k split each slice's partial sums are scaled
+// by the slice's own 2^-e before they are added.
+template <int NMAT, int IBP, int IT>
+__global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
     tf8mma_kernel(const __grid_constant__ Tm8Maps maps, const Tm8Params p) {
   static_assert(NMAT == 1 || NMAT == 2, "NMAT");
+  constexpr bool INK = IBP > 0;
+  constexpr int IR = IBP * IT;  // B-operand rows / TMEM columns per matrix (INK)
+  static_assert(!INK || (IR == 16 || IR == 32), "in-kernel terms: 16 or 32 MMA columns");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -287,10 +323,15 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
   uint64_t *fullb = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   uint64_t *empty = fullb + S;
   uint64_t *accfull = empty + S;
-  volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
-  int *s_issued = reinterpret_cast<int *>(accfull + 1) + 1;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accfull + 1) + 2;
-  volatile int *s_last = reinterpret_cast<volatile int *>(accfull + 1) + 3;
+  uint64_t *tready = accfull + 1;  // INK: the resident term area is written
+  uint64_t *bend = tready + 1;
+  volatile int *s_abort = reinterpret_cast<volatile int *>(bend);
+  int *s_issued = reinterpret_cast<int *>(bend) + 1;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bend) + 2;
+  volatile int *s_last = reinterpret_cast<volatile int *>(bend) + 3;
+  float *s_fac = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bend) + 16);  // [16]
+  float *s_sc = s_fac + 16;                                                             // [16]
+  float *s_rmx = s_sc + 16, *s_rss = s_rmx + 8;  // per-warp partials of the term warps
 
   const int cta = blockIdx.x;
   const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
@@ -301,8 +342,8 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
   const int tile1 = ((slc + 1) * p.ntiles) / p.kslices;
   const int NT = p.nt;
   const int nsteps = (tile1 - tile0 + NT - 1) / NT;
-  // stage layout: code tiles [tt][m] (r8 rows each), then term tiles [tt] (np rows)
-  const int codes_bytes = NT * p.a8_bytes;
+  // stage layout: code tiles [tt][m] (r8 rows each), then (prep terms) the
+  // term tiles [tt] (np rows)
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -310,6 +351,7 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(accfull, 1);
+    mbar_init(tready, TM8_XF_THREADS);
     *s_abort = 0;
     *s_issued = 0;
     fence_mbar_init();
@@ -325,8 +367,8 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
   pdl_launch_dependents();
 
   if (warp == 0) {
-    // ================= TMA producer (one lane): codes first; the term tiles
-    // only after the prep kernel's results are visible
+    // ================= TMA producer (one lane): codes; the term tiles (prep
+    // terms) only after the prep kernel's results are visible
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_normal();
@@ -337,23 +379,24 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
         if (i >= S && !mbar_wait_bounded(&empty[st], ((i / S) - 1) & 1, s_abort, p.err)) break;
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
         const int nv = min(NT, tile1 - (tile0 + i * NT));  // k tiles of this stage
-        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>(nv * (NMAT * r + NP) * 128));
+        mbar_arrive_expect_tx(&fullb[st],
+                              static_cast<uint32_t>(nv * (NMAT * r + (INK ? 0 : NP)) * 128));
         for (int tt = 0; tt < nv; ++tt) {
           const int tile = tile0 + i * NT + tt;
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
             tma_load_2d(sb + tt * p.a8_bytes + m * p.r8 * 128, &maps.w[m][mi], &fullb[st],
                         tile * TM8_TILE_K, j0, pol_w);
-          if (i >= S0)
-            tma_load_2d(sb + codes_bytes + tt * NP * 128, &maps.x, &fullb[st], 0, tile * NP,
+          if (!INK && i >= S0)
+            tma_load_2d(sb + p.term_off + tt * NP * 128, &maps.x, &fullb[st], 0, tile * NP,
                         pol_x);
         }
-        if (i == S0 - 1) {
+        if (!INK && i == S0 - 1) {
           pdl_wait();
           for (int ii = 0; ii < S0; ++ii) {
             const int nvi = min(NT, tile1 - (tile0 + ii * NT));
             for (int tt = 0; tt < nvi; ++tt)
-              tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + codes_bytes +
+              tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.term_off +
                               tt * NP * 128,
                           &maps.x, &fullb[ii], 0, (tile0 + ii * NT + tt) * NP, pol_x);
           }
@@ -366,37 +409,43 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
     // ================= MMA issuer (one lane): per tile and matrix, 4 MMAs of
     // K = 32 (32 bytes further into each swizzled 128-byte row)
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_e4m3_f32(128, NP);
+      const uint32_t idesc = umma_idesc_e4m3_f32(128, INK ? IR : NP);
       const uint64_t desc0 = umma_desc_sw128(sbase);
       const uint32_t tile_enc = static_cast<uint32_t>(p.r8 * 128) >> 4;
       const uint32_t a_enc = static_cast<uint32_t>(p.a8_bytes) >> 4;
-      const uint32_t x_enc = static_cast<uint32_t>(codes_bytes) >> 4;
-      const uint32_t xt_enc = static_cast<uint32_t>(NP * 128) >> 4;
-      for (int i = 0; i < nsteps; ++i) {
+      const uint32_t x_enc = static_cast<uint32_t>(p.term_off) >> 4;
+      const uint32_t xt_enc = static_cast<uint32_t>((INK ? IR : NP) * 128) >> 4;
+      bool ok = !INK || mbar_wait_bounded(tready, 0, s_abort, p.err);
+      if (ok) tc_fence_after();
+      for (int i = 0; ok && i < nsteps; ++i) {
         const int st = i % S;
         if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
         const int nv = min(NT, tile1 - (tile0 + i * NT));
         for (int tt = 0; tt < nv; ++tt) {
+          // B operand: this stage's term tile, or the resident one of the tile
+          const uint64_t bx = INK ? desc0 + x_enc + (i * NT + tt) * xt_enc
+                                  : ds + x_enc + tt * xt_enc;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              umma_e4m3(tmem + static_cast<uint32_t>(m * NP),
-                        ds + tt * a_enc + m * tile_enc + 2 * kk, ds + x_enc + tt * xt_enc + 2 * kk,
-                        idesc, (i > 0 || tt > 0 || kk > 0) ? 1u : 0u);
+              umma_e4m3(tmem + static_cast<uint32_t>(m * (INK ? IR : NP)),
+                        ds + tt * a_enc + m * tile_enc + 2 * kk, bx + 2 * kk, idesc,
+                        (i > 0 || tt > 0 || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(&empty[st]);
       }
       umma_commit(accfull);
     }
-  } else {
+  } else if (warp < 6) {
     // ================= epilogue (warps 2..5, one per TMEM lane quarter)
     const int et = tid - 64;
     const int q = warp & 3;
     const int row = 32 * q + lane;
+    if (INK) named_barrier(4, 128 + TM8_XF_THREADS);  // the term warps' s_fac is written
     const bool okw = mbar_wait_bounded(accfull, 0, s_abort, p.err);
     tc_fence_after();
     const bool go = __all_sync(0xffffffffu, okw && !*s_abort);
@@ -408,18 +457,43 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
         sg = __ldg(p.scale[0] + j);
         if (NMAT == 2) su = __ldg(p.scale[1] + j);
       }
-      for (int c = 0; c < p.bnp; c += 16) {
+      const int cstep = INK ? IBP : 16;  // token slots per pass
+      for (int c = 0; c < p.bnp; c += cstep) {
         // terms combined smallest first: S = D_0 + (D_1 + (...) / 16) / 16
         float g[16], u[16];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
           float acc[16];
-          for (int t = p.T - 1; t >= 0; --t) {
-            float d[16];
-            tmem_ld_32x32b_x16(base + m * NP + t * p.bnp + c, d);
+          if constexpr (INK) {
+            // columns t * IBP + b of this matrix (IR = 16 or 32; the loops
+            // unroll, so every index is a constant)
+            float d0[16], d1[16];
+            tmem_ld_32x32b_x16(base + m * IR, d0);
+            if constexpr (IR == 32) tmem_ld_32x32b_x16(base + m * IR + 16, d1);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = (t == p.T - 1) ? d[e] : d[e] + acc[e] * 0.0625f;
+            for (int e = 0; e < 16; ++e) {
+              if (e < IBP) {
+                constexpr int top = (IT - 1) * IBP;
+                float a = (top + e < 16) ? d0[(top + e) & 15] : d1[(top + e) & 15];
+#pragma unroll
+                for (int t = IT - 2; t >= 0; --t) {
+                  const int col = t * IBP + e;
+                  a = ((col < 16) ? d0[col & 15] : d1[col & 15]) + a * 0.0625f;
+                }
+                acc[e] = a;
+              } else {
+                acc[e] = 0.f;
+              }
+            }
+          } else {
+            for (int t = p.T - 1; t >= 0; --t) {
+              float d[16];
+              tmem_ld_32x32b_x16(base + m * NP + t * p.bnp + c, d);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) acc[e] = (t == p.T - 1) ? d[e] : d[e] + acc[e] * 0.0625f;
+            }
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -428,15 +502,18 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
           }
         }
         if (p.kslices > 1) {
+          // in-kernel terms: each slice's partial sums at their true scale
+          // (times the slice's 2^-e_b; exact)
           float *mine = p.part + (static_cast<size_t>(slc) * p.nblocks + blk) * p.bnp * 128;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) mine[(c + e) * 128 + row] = g[e];
+          for (int e = 0; e < 16; ++e)
+            if (e < cstep) mine[(c + e) * 128 + row] = INK ? g[e] * s_fac[c + e] : g[e];
         } else if (row < r) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int n = c + e;
-            if (n < p.B) {
-              const float f = __ldg(p.fac + n);
+            if (e < cstep && n < p.B) {
+              const float f = INK ? s_fac[n] : __ldg(p.fac + n);
               float res;
               if (NMAT == 2) {
                 const float a = (g[e] * f) * sg, uu = (u[e] * f) * su;
@@ -466,8 +543,8 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
           const float sd = __ldg(p.scale[0] + j0 + row);
           splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, p.bnp, p.B, row,
                             [&](int n, float acc) {
-                              p.out[static_cast<size_t>(n) * p.N + j0 + row] =
-                                  f32_to_bf16_bits((acc * __ldg(p.fac + n)) * sd);
+                              p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(
+                                  INK ? acc * sd : (acc * __ldg(p.fac + n)) * sd);
                             });
         }
         named_barrier(2, 128);
@@ -475,6 +552,158 @@ __global__ void __launch_bounds__(TM8_THREADS, 1)
       }
     }
     tc_fence_before();
+  } else if (INK) {
+    // ================= activation terms (warps 6..13)
+    const int xt = tid - TM8_THREADS;  // 0 .. 255
+    // the B real token slots share the 256 threads: tpt per slot (256 .. 16)
+    const int bp = p.B <= 1 ? 1 : (p.B <= 2 ? 2 : (p.B <= 4 ? 4 : (p.B <= 8 ? 8 : 16)));
+    const int tpt = TM8_XF_THREADS / bp;
+    const int tok = xt / tpt, sub = xt % tpt;
+    const int c_lo = tile0 * (TM8_TILE_K / 8);   // first 8-element chunk of this CTA's range
+    const int c_end = tile1 * (TM8_TILE_K / 8);  // past its last chunk (whole tiles)
+    const int c_k = min(c_end, p.K / 8);         // chunks inside K
+    const bool real = tok < p.B;
+    const uint16_t *xr = p.x + static_cast<size_t>(real ? tok : 0) * p.K;
+    uint8_t *tarea = smem + p.term_off;
+    // chunk c of token slot tok: values v (x, or x * gamma: exact in fp32)
+    auto load = [&](int c, uint4 &xv, uint4 &gv) {
+      xv = gv = make_uint4(0u, 0u, 0u, 0u);
+      if (real && c < c_k) {
+        xv = ld_nc_v4(xr + 8 * c);
+        if (p.gamma) gv = ld_nc_v4(p.gamma + 8 * c);
+      }
+    };
+    auto values = [&](const uint4 &xv, const uint4 &gv, float (&v)[8]) {
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float x0 = bf16_lo(xw[h]), x1 = bf16_hi(xw[h]);
+        v[2 * h] = p.gamma ? x0 * bf16_lo(gw[h]) : x0;
+        v[2 * h + 1] = p.gamma ? x1 * bf16_hi(gw[h]) : x1;
+      }
+    };
+    float mx = 0.f, ss = 0.f;
+    auto stats = [&](const uint4 &xv, const uint4 &gv) {
+      float v[8];
+      values(xv, gv, v);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float x0 = bf16_lo(xw[h]), x1 = bf16_hi(xw[h]);
+        ss = fmaf(x0, x0, ss);
+        ss = fmaf(x1, x1, ss);
+        mx = fmaxf(mx, fmaxf(fabsf(v[2 * h]), fabsf(v[2 * h + 1])));
+      }
+    };
+    // the IT term codes of chunk c into the resident area: tile (c - c_lo) / 16,
+    // rows t * IBP + tok, 16-byte granule (chunk / 2) xor (row % 8) (128-byte
+    // swizzle)
+    auto emit = [&](int c, const uint4 &xv, const uint4 &gv, float scb) {
+      float u[8];
+      values(xv, gv, u);
+#pragma unroll
+      for (int h = 0; h < 8; ++h) u[h] *= scb;
+      const int kl = 8 * (c - c_lo), jc = (kl & (TM8_TILE_K - 1)) >> 3;
+      uint8_t *tb = tarea + (kl / TM8_TILE_K) * IR * 128;
+#pragma unroll
+      for (int t = 0; t < IT; ++t) {
+        uint32_t w0, w1;
+        if (t + 1 < IT) {
+          tm8_encode_term(u, w0, w1);
+        } else {  // the last term: no residual needed
+          w0 = f32x2_to_e4m3x2(u[0], u[1]) | (f32x2_to_e4m3x2(u[2], u[3]) << 16);
+          w1 = f32x2_to_e4m3x2(u[4], u[5]) | (f32x2_to_e4m3x2(u[6], u[7]) << 16);
+        }
+        const int rw = t * IBP + tok;
+        *reinterpret_cast<uint2 *>(tb + rw * 128 + (((jc >> 1) ^ (rw & 7)) << 4) + ((jc & 1) << 3)) =
+            make_uint2(w0, w1);
+      }
+    };
+    // rows of the slots past B are zero in every tile (no conversion needed)
+    {
+      const int ntl = tile1 - tile0, zrows = IBP - p.B;
+      constexpr int ITS = IT > 0 ? IT : 1;
+      const int nz = ntl * ITS * zrows * 8;  // 16-byte stores
+      for (int z = xt; z < nz; z += TM8_XF_THREADS) {
+        const int g = z & 7, rz = (z >> 3) % zrows, rest = (z >> 3) / zrows;
+        const int t = rest % ITS, tl = rest / ITS;
+        *reinterpret_cast<uint4 *>(tarea + tl * IR * 128 + (t * IBP + p.B + rz) * 128 + 16 * g) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    pdl_wait();  // x comes from the previous kernel
+    // pass 1: max |v| and sum x^2 of slot tok over [c_lo, c_k); the thread
+    // chains its chunks c = c_lo + sub + tpt * i (i, then the 8 elements,
+    // ascending)
+    constexpr int W = 8;  // chunks per thread in flight
+    const bool one = (c_end - c_lo) <= tpt * W;  // the whole range in one window
+    uint4 xv[W], gv[W];
+    for (int c0 = c_lo + sub; real && c0 < c_end; c0 += tpt * W) {
+#pragma unroll
+      for (int u = 0; u < W; ++u) load(c0 + tpt * u, xv[u], gv[u]);
+#pragma unroll
+      for (int u = 0; u < W; ++u) stats(xv[u], gv[u]);
+    }
+    // combine the tpt threads of the slot: xor butterfly inside the warp (or
+    // half warp), then the slot's warps in order
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      if (m < tpt) {  // tpt >= 16: warp-uniform
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+        ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      }
+    }
+    if (tpt > 32) {
+      const int w = xt >> 5;
+      if (lane == 0) {
+        s_rmx[w] = mx;
+        s_rss[w] = ss;
+      }
+      named_barrier(5, TM8_XF_THREADS);
+      const int nw = tpt >> 5, w0 = tok * nw;
+      mx = s_rmx[w0];
+      ss = s_rss[w0];
+      for (int q = 1; q < nw; ++q) {
+        mx = fmaxf(mx, s_rmx[w0 + q]);
+        ss += s_rss[w0 + q];
+      }
+    }
+    if (sub == 0) {
+      int e = 0;
+      if (mx > 0.f) {
+        int E;
+        frexpf(mx, &E);                  // mx = f * 2^E, f in [0.5, 1)
+        e = min(max(8 - E, -126), 126);  // mx * 2^e in [128, 256)
+      }
+      s_sc[tok] = ldexpf(1.0f, e);
+      const float rr = p.gamma ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 1.0f;
+      s_fac[tok] = real ? rr * ldexpf(1.0f, -e) : 0.f;
+    }
+    if (xt < IBP && xt >= bp) s_fac[xt] = 0.f;  // slots no thread group covers
+    named_barrier(5, TM8_XF_THREADS);
+    const float scb = s_sc[tok];
+    // pass 2: the terms of the real slots (from the registers when the range
+    // fit in one window)
+    if (real) {
+      if (one) {
+#pragma unroll
+        for (int u = 0; u < W; ++u) {
+          const int c = c_lo + sub + tpt * u;
+          if (c < c_end) emit(c, xv[u], gv[u], scb);
+        }
+      } else {
+        for (int c0 = c_lo + sub; c0 < c_end; c0 += tpt * W) {
+#pragma unroll
+          for (int u = 0; u < W; ++u) load(c0 + tpt * u, xv[u], gv[u]);
+#pragma unroll
+          for (int u = 0; u < W; ++u)
+            if (c0 + tpt * u < c_end) emit(c0 + tpt * u, xv[u], gv[u], scb);
+        }
+      }
+    }
+    fence_proxy_async_smem();  // the MMA (async proxy) reads these shared-memory writes
+    mbar_arrive(tready);
+    named_barrier(4, 128 + TM8_XF_THREADS);  // with the epilogue warps: s_fac is written
   }
 
   __syncthreads();

@@ -366,15 +366,17 @@ def test_fp8_tensor_core_is_exact_dequantisation():
 
 # ------------------------------------------------------------------ E4M3-MMA kernel
 
-def e4m3_mma_ids(down):
+def e4m3_mma_ids(down, kinds=(1, 2)):
+    # kind 1: activation terms from the prep kernel; kind 2: derived inside
+    # the kernel (up to 16 tokens)
     want = dfk.DFK_OP_DOWN_FP8 if down else dfk.DFK_OP_GATE_UP_FP8
     return [v for v in (dfk.dfk_variant_info(i) for i in range(1, dfk.dfk_variant_count() + 1))
-            if v["op"] == want and v["e4m3_mma"] == 1]
+            if v["op"] == want and v["e4m3_mma"] in kinds]
 
 
 def test_e4m3_mma_ids_are_fp8_only():
     gu, dn = e4m3_mma_ids(False), e4m3_mma_ids(True)
-    assert len(gu) == 2 and len(dn) == 6       # one or two k tiles per stage
+    assert len(gu) == 4 and len(dn) == 12      # one or two k tiles per stage, both kinds
     x = torch.zeros(2, 256, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(264, 256, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(dfk.DfkError) as e:
@@ -421,15 +423,32 @@ def test_fp8_e4m3_mma_encodes_activations_closely(norm):
     # the CUDA-core FP8 kernel multiplies by the exact activations; the E4M3
     # terms (2 for bf16 x, 4 for x * gamma) must leave only accumulation-order
     # and output-rounding differences: within two bf16 steps of each other
-    v = e4m3_mma_ids(False)[0]
     B, D, F = 8, 1024, 1496
     L = Fp8Layer(B, D, F, seed=520 + norm, norm=norm, with_down=False)
     cc = next(w["variant_id"] for w in cc_ids(dfk.DFK_OP_GATE_UP_FP8)
               if w["j_per_thread"] == 2 and w["token_tile"] == 8)
-    a = I.bf16_values(L.gate_up(norm, variant=v["variant_id"]))
     b = I.bf16_values(L.gate_up(norm, variant=cc))
-    torch.cuda.synchronize()
-    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.abs(b) + 1e-4)
+    for kind in (1, 2):
+        v = e4m3_mma_ids(False, kinds=(kind,))[0]
+        a = I.bf16_values(L.gate_up(norm, variant=v["variant_id"]))
+        torch.cuda.synchronize()
+        assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.abs(b) + 1e-4), kind
+
+
+@pytest.mark.parametrize("B,D,F", [(1, 256, 688), (5, 1024, 1496), (16, 4096, 2048)])
+def test_fp8_in_kernel_terms_equal_prep_kernel_terms(B, D, F):
+    # without RMSNorm and without a k split both kinds scale by the same
+    # power of two (from max |x| over K) and write the same term codes: the
+    # tensor cores see identical operands, so the results agree bit for bit
+    L = Fp8Layer(B, D, F, seed=530 + B, norm=False, with_down=False)
+    for nt in (1, 2):
+        ids = [next(v["variant_id"] for v in e4m3_mma_ids(False, kinds=(k,))
+                    if v["k_tiles_per_stage"] == nt) for k in (1, 2)]
+        outs = [try_variant(lambda vid: L.gate_up(False, variant=vid), vid) for vid in ids]
+        if outs[0] is None or outs[1] is None:
+            continue
+        torch.cuda.synchronize()
+        assert bits_equal(outs[0], outs[1]), "nt=%d" % nt
 
 
 @pytest.mark.parametrize("B", [1, 16, 64])
