@@ -1526,6 +1526,35 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   cudaEventCreate(&e0);
   cudaEventCreate(&e1);
+  // When one call's weights fit in L2, a burst's later launches would read
+  // them from L2: the burst then rotates over copies of the weights that
+  // together exceed L2 (made here, freed below); without memory for them
+  // each sample is one launch after its own flush.
+  const size_t wbytes = static_cast<size_t>(c.K) * c.N * c.nmat * (c.w8 ? 1 : 2);
+  const size_t l2 = static_cast<size_t>(std::max(ds.l2_bytes, 1 << 20));
+  std::vector<CcCall> rot;
+  void *wcopies = nullptr;
+  if (flush && wbytes < l2) {
+    const int ncopy = static_cast<int>(std::min<size_t>(8, l2 / wbytes + 2));
+    const size_t b0 = c.w1 ? wbytes / c.nmat : wbytes;  // bytes at w0 (w1 holds the rest)
+    const size_t stride = (wbytes + 1023) & ~static_cast<size_t>(1023);
+    if (cudaMallocAsync(&wcopies, stride * ncopy, s) == cudaSuccess) {
+      for (int i = 0; i < ncopy; ++i) {
+        char *base = static_cast<char *>(wcopies) + stride * i;
+        CcCall ci = c;
+        cudaMemcpyAsync(base, c.w0, b0, cudaMemcpyDeviceToDevice, s);
+        ci.w0 = base;
+        if (c.w1) {
+          cudaMemcpyAsync(base + b0, c.w1, wbytes - b0, cudaMemcpyDeviceToDevice, s);
+          ci.w1 = base + b0;
+        }
+        rot.push_back(ci);
+      }
+    } else {
+      cudaGetLastError();
+      wcopies = nullptr;
+    }
+  }
   const VDef *best = nullptr;
   float best_t = 1e30f;
   for (const VDef *d : cands) {
@@ -1533,17 +1562,15 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
     if (launch_variant(c, *d, s, &st) != DFK_OK) continue;  // warm-up; skips infeasible ones
     // Each repetition: flush L2, then a burst of back-to-back launches (the
     // way a decode loop issues them, neighbours overlapping through
-    // programmatic dependent launch); the sample is the burst's mean.  When
-    // one call's weights fit in L2 the later launches of a burst would read
-    // them from L2, so each sample is then one launch after its own flush.
-    const size_t wbytes = static_cast<size_t>(c.K) * c.N * c.nmat * (c.w8 ? 1 : 2);
-    const int burst = (flush && wbytes < static_cast<size_t>(ds.l2_bytes)) ? 1 : 4;
+    // programmatic dependent launch); the sample is the burst's mean.
+    const int burst = (flush && wbytes < l2 && rot.empty()) ? 1 : 4;
     std::vector<float> ts;
     bool ok = true;
     for (int r = 0; r < reps && ok; ++r) {
       if (flush) cudaMemsetAsync(flush, r & 0xff, flush_bytes, s);
       cudaEventRecord(e0, s);
-      for (int b = 0; b < burst && ok; ++b) ok = launch_variant(c, *d, s, nullptr) == DFK_OK;
+      for (int b = 0; b < burst && ok; ++b)
+        ok = launch_variant(rot.empty() ? c : rot[b % rot.size()], *d, s, nullptr) == DFK_OK;
       cudaEventRecord(e1, s);
       if (cudaEventSynchronize(e1) != cudaSuccess) ok = false;
       float ms = 0.f;
@@ -1563,6 +1590,7 @@ static const VDef *time_candidates(int op, const CcCall &c, const std::vector<co
     }
   }
   if (flush) cudaFreeAsync(flush, s);
+  if (wcopies) cudaFreeAsync(wcopies, s);
   cudaStreamSynchronize(s);
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
