@@ -790,7 +790,9 @@ def reference_arm(args):
     value = sample_bytes * args.steps / el / 1e9
     sample = ("1/8 of the Llama-3-8B-shaped layer per step (1792 gate/up columns + 512 "
               "down rows, B=1)")
-    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0,
+    # n_gpus: the N this arm was launched with (the oracle itself runs on rank
+    # 0's host cores only)
+    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el * 1e3 / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
