@@ -477,3 +477,35 @@ def test_fp8_e4m3_mma_llama3_8b_sampled_rows(B):
     assert ys
     for y in ys:
         assert_close(y[:, didx].contiguous(), want, "fp8 e4m3-mma 8B down rows B=%d" % B)
+
+
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_fp8_in_kernel_terms_capture_on_a_fresh_stream(B):
+    # the in-kernel-term variants need no per-stream buffer: captured into a
+    # CUDA graph on a stream that never ran them, the replay gives the eager
+    # result bit for bit (gate/up with RMSNorm, then the split-K down)
+    L = Fp8Layer(B, 1024, 2048, seed=540 + B, norm=True)
+    gu = next(v["variant_id"] for v in e4m3_mma_ids(False, kinds=(2,)) if v["k_tiles_per_stage"] == 1)
+    dn = next(v["variant_id"] for v in e4m3_mma_ids(True, kinds=(2,)) if v["k_split"] == 4)
+    h_ref = L.gate_up(True, variant=gu)
+    y_ref = dfk.dfk_down_proj_fp8(h_ref, L.qd, L.sd, variant=dn)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    h = torch.empty_like(h_ref)
+    y = torch.empty_like(y_ref)
+    # the split-K workspace is per stream: one eager call on the new stream first
+    with torch.cuda.stream(s):
+        dfk.dfk_down_proj_fp8(h_ref, L.qd, L.sd, y=y, variant=dn)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dfk.dfk_rmsnorm_swiglu_gate_up_fp8(L.inp.x, L.inp.gamma, L.inp.eps, L.qg, L.sg, L.qu,
+                                           L.su, h=h, variant=gu, stream=s)
+        dfk.dfk_down_proj_fp8(h, L.qd, L.sd, y=y, variant=dn, stream=s)
+    h.zero_()
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert bits_equal(h, h_ref)
+    assert bits_equal(y, y_ref)
+    del g
