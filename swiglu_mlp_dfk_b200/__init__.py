@@ -146,19 +146,32 @@ def _check(status):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain int: the c_void_p argtypes convert it (None passes NULL)
+    return None if t is None else t.data_ptr()
+
+
+# The current stream's handle.  torch.cuda.current_stream() builds a Stream
+# object (about 3 us a call); the raw accessor under it returns the handle
+# directly and is used when this torch has it.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream(stream):
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+_BF16 = torch.bfloat16
 
 
 def _dev_bf16(name, t):
+    # on every call of the host-memory entry point: kept to a few attribute reads
     if t is None:
         return
-    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+    if not (isinstance(t, torch.Tensor) and t.dtype is _BF16 and t.is_cuda):
         raise DfkError(DFK_ERR_INVALID_ARG, "%s must be a bf16 CUDA tensor" % name)
     if not t.is_contiguous():
         raise DfkError(DFK_ERR_INVALID_ARG, "%s must be contiguous" % name)

@@ -311,6 +311,26 @@ def test_host_entry_point_matches_device_path():
     assert bits_equal(yp, y2.cpu())
 
 
+
+def test_binding_uses_the_current_torch_stream():
+    # the binding reads the current stream's handle without building a Stream
+    # object; it must name the same stream as torch.cuda.current_stream()
+    assert dfk._stream(None) == torch.cuda.current_stream().cuda_stream
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        assert dfk._stream(None) == s.cuda_stream
+        # and work launched there is ordered on that stream
+        inp = I.make_inputs(3, 256, 512, seed=8, device="cuda")
+        h = dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row")
+        done = torch.cuda.Event()
+        done.record(s)
+    done.synchronize()
+    want = run_gate_up(inp, I.LAYOUT_ROW, True)
+    torch.cuda.synchronize()
+    assert bits_equal(h, want)
+    assert dfk._stream(s) == s.cuda_stream
+
+
 # ------------------------------------------------------------------ full-size workloads
 
 def sample_rows(F, n, seed):
