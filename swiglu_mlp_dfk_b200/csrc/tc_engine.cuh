@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t *fullb = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   uint64_t *empty = fullb + S;
   uint64_t *xready = empty + S;
-  uint64_t *accfull = xready + S;
+  uint64_t *xfull = xready + S;  // NORM = 1: a stage's activation tiles have landed
+  uint64_t *accfull = xfull + S;
   volatile int *s_abort = reinterpret_cast<volatile int *>(accfull + 1);
   int *s_issued = reinterpret_cast<int *>(accfull + 1) + 1;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accfull + 1) + 2;
@@ -189,6 +190,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&fullb[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&xready[s], 128);
+      mbar_init(&xfull[s], 1);
     }
     mbar_init(accfull, 1);
     *s_abort = 0;
@@ -218,10 +220,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
         const int nv = min(NT, tile1 - (tile0 + i * NT));  // k-tiles of this step in range
         // (column-major boxes are always 64 x 64, zero-filled past the last column)
-        mbar_arrive_expect_tx(&fullb[st], static_cast<uint32_t>(nv) *
-                                              (NMAT * (full ? 128 : r) + XROWS * BN) * 128u);
+        const uint32_t wbytes = static_cast<uint32_t>(nv) * NMAT * (full ? 128 : r) * 128u;
+        const uint32_t xbytes = static_cast<uint32_t>(nv) * XROWS * BN * 128u;
+        // with the in-kernel transform the activation tiles have a barrier of
+        // their own: they come from L2 and land long before the weights, so
+        // the transform is done by the time the weights arrive
+        if (NORM == 1) {
+          mbar_arrive_expect_tx(&xfull[st], xbytes);
+          mbar_arrive_expect_tx(&fullb[st], wbytes);
+        } else {
+          mbar_arrive_expect_tx(&fullb[st], wbytes + xbytes);
+        }
+        uint64_t *xbar = NORM == 1 ? &xfull[st] : &fullb[st];
         for (int kt = 0; kt < nv; ++kt) {
           const int k0 = (tile0 + i * NT + kt) * TC_TILE_K;
+          // activations: only after the previous kernel's results are visible
+          // (prepared tiles: rows tile * 2 bn .. of the prep kernel's buffer)
+          if (i >= S0) {
+            const int tl = tile0 + i * NT + kt;
+            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, xbar,
+                        NORM == 2 ? 0 : k0, NORM == 2 ? tl * 2 * BN : 0, pol_x);
+          }
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
             const int mi = (full || h[t] == p.hmax) ? 0 : 1;
@@ -239,13 +258,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 tma_load_2d(dst, wm, &fullb[st], k0, j0 + rs[t], pol_w);
               }
             }
-          }
-          // activations: only after the previous kernel's results are visible
-          // (prepared tiles: rows tile * 2 bn .. of the prep kernel's buffer)
-          if (i >= S0) {
-            const int tl = tile0 + i * NT + kt;
-            tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, &fullb[st],
-                        NORM == 2 ? 0 : k0, NORM == 2 ? tl * 2 * BN : 0, pol_x);
           }
         }
         if (i == S0 - 1) {
@@ -281,7 +293,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const int tl = tile0 + ii * NT + kt;
               tma_load_2d(smem + static_cast<size_t>(ii) * p.stage_bytes + p.a_bytes +
                               kt * p.xt_bytes,
-                          &maps.x, &fullb[ii], NORM == 2 ? 0 : tl * TC_TILE_K,
+                          &maps.x, NORM == 1 ? &xfull[ii] : &fullb[ii],
+                          NORM == 2 ? 0 : tl * TC_TILE_K,
                           NORM == 2 ? tl * 2 * BN : 0, pol_x);
             }
           }
@@ -308,8 +321,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        if (!mbar_wait_bounded(NORM == 1 ? &xready[st] : &fullb[st], (i / S) & 1, s_abort, p.err))
-          break;
+        if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
+        if (NORM == 1 && !mbar_wait_bounded(&xready[st], (i / S) & 1, s_abort, p.err)) break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
         const int nv = min(NT, tile1 - (tile0 + i * NT));
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       float ss[4] = {0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        const bool ok = mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err);
+        const bool ok = mbar_wait_bounded(&xfull[st], (i / S) & 1, s_abort, p.err);
         if (ok) {
           uint8_t *sb = smem + static_cast<size_t>(st) * p.stage_bytes;
           const int nv = min(NT, tile1 - (tile0 + i * NT));
@@ -505,7 +518,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int last = -1;
       for (int i = issued - 1; i >= 0 && i >= issued - S; --i)
         if (i % S == st) { last = i; break; }
-      if (last >= 0) mbar_wait_bounded(&fullb[st], (last / S) & 1, nullptr, p.err);
+      if (last >= 0) {
+        mbar_wait_bounded(&fullb[st], (last / S) & 1, nullptr, p.err);
+        if (NORM == 1) mbar_wait_bounded(&xfull[st], (last / S) & 1, nullptr, p.err);
+      }
     }
   }
 }
