@@ -304,12 +304,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       *s_issued = issued;
     }
   } else if (warp == 1) {
-    // ================= MMA issuer (one lane)
+    // ================= MMA issuer
+    // The whole warp walks the ring, so every descriptor below is a
+    // warp-uniform value; one elected lane issues the MMAs and commits.
+    // (Issued from a single-lane branch each MMA cost ~50 cycles of issue,
+    // holding its ring stage for that long.)
     // Each output may accumulate into NB independent TMEM banks (k-slice kk
     // of a tile goes to bank kk % NB); the epilogue adds the banks in a fixed
     // order.  One MMA covers N = bn tokens, or with the prologue N = 2 bn
     // (the hi rows, then the lo rows).
-    if (lane == 0) {
+    __syncwarp();
+    const uint32_t leader = elect_one_sync();
+    {
       const int WN = NORM ? 2 * BN : BN;
       const uint32_t idesc = umma_idesc_bf16_f32(128, WN, COLM);
       const int NB = p.nbank;
@@ -321,8 +327,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S;
-        if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
-        if (NORM == 1 && !mbar_wait_bounded(&xready[st], (i / S) & 1, s_abort, p.err)) break;
+        bool ok = mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err);
+        if (NORM == 1 && ok) ok = mbar_wait_bounded(&xready[st], (i / S) & 1, s_abort, p.err);
+        if (!__all_sync(0xffffffffu, ok)) break;  // the warp leaves together
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
         const int nv = min(NT, tile1 - (tile0 + i * NT));
@@ -347,14 +354,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                 (2048u >> 4) * kk)
                          : at + static_cast<uint64_t>(t * NMAT + m) * tile_enc + 2 * kk;
                 const uint32_t d = tmem + static_cast<uint32_t>(((t * NMAT + m) * NB + b) * WN);
-                umma_bf16(d, a, bx + 2 * kk, idesc, acc);
+                if (leader) umma_bf16(d, a, bx + 2 * kk, idesc, acc);
               }
             }
           }
         }
-        umma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+        if (leader) umma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+        __syncwarp();
       }
-      umma_commit(accfull);       // every MMA issued above has completed
+      if (leader) umma_commit(accfull);       // every MMA issued above has completed
     }
   } else {
     // ================= x*gamma transform (NORM = 1) and epilogue: warps 2..5
