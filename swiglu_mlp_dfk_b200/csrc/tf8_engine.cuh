@@ -177,17 +177,23 @@ __global__ void __launch_bounds__(TF8_THREADS, 1)
       *s_issued = issued;
     }
   } else if (warp == 1) {
-    // ================= MMA issuer (one lane): per stage, the k-slices of
-    // 16 inside K, A from TMEM buffer (i mod NAB), B from the activation sub-tile
-    // (k-slice kk: sub-tile kk / 4, 32 bytes per slice inside its swizzled rows)
-    if (lane == 0) {
+    // ================= MMA issuer: per stage, the k-slices of 16 inside K,
+    // A from TMEM buffer (i mod NAB), B from the activation sub-tile (k-slice
+    // kk: sub-tile kk / 4, 32 bytes per slice inside its swizzled rows).  The
+    // whole warp walks the ring (warp-uniform descriptors); one elected lane
+    // issues.
+    __syncwarp();
+    const uint32_t leader = elect_one_sync();
+    {
       const uint32_t idesc = umma_idesc_bf16_f32(128, WN);
       const uint64_t desc0 = umma_desc_sw128(sbase);
       const uint32_t x_enc = static_cast<uint32_t>(p.a8_bytes) >> 4;
       const uint32_t xt_enc = static_cast<uint32_t>(p.xt_bytes) >> 4;
       for (int i = 0; i < nsteps; ++i) {
         const int st = i % S, slot = i % NAB;
-        if (!mbar_wait_bounded(&aready[slot], (i / NAB) & 1, s_abort, p.err)) break;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_bounded(&aready[slot], (i / NAB) & 1, s_abort, p.err)))
+          break;
         tc_fence_after();
         const int k0 = (tile0 + i) * TF8_TILE_K;
         const int nk = min(8, (p.K - k0) / 16);
@@ -197,14 +203,18 @@ __global__ void __launch_bounds__(TF8_THREADS, 1)
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             const uint32_t a = tmem + static_cast<uint32_t>(p.acol + (slot * NMAT + m) * 64 + 8 * kk);
-            umma_bf16_ts(tmem + static_cast<uint32_t>(m * WN), a, b, idesc,
-                         (i > 0 || kk > 0) ? 1u : 0u);
+            if (leader)
+              umma_bf16_ts(tmem + static_cast<uint32_t>(m * WN), a, b, idesc,
+                           (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&empty[st]);     // the stage's activations have been read
-        umma_commit(&aempty[slot]);  // and so has the A buffer
+        if (leader) {
+          umma_commit(&empty[st]);     // the stage's activations have been read
+          umma_commit(&aempty[slot]);  // and so has the A buffer
+        }
+        __syncwarp();
       }
-      umma_commit(accfull);          // every MMA issued above has completed
+      if (leader) umma_commit(accfull);  // every MMA issued above has completed
     }
   } else {
     // ================= dequantise / x * gamma transform: warps 2..17

@@ -406,9 +406,12 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
       *s_issued = issued;
     }
   } else if (warp == 1) {
-    // ================= MMA issuer (one lane): per tile and matrix, 4 MMAs of
-    // K = 32 (32 bytes further into each swizzled 128-byte row)
-    if (lane == 0) {
+    // ================= MMA issuer: per tile and matrix, 4 MMAs of K = 32
+    // (32 bytes further into each swizzled 128-byte row).  The whole warp
+    // walks the ring (warp-uniform descriptors); one elected lane issues.
+    __syncwarp();
+    const uint32_t leader = elect_one_sync();
+    {
       const uint32_t idesc = umma_idesc_e4m3_f32(128, INK ? IR : NP);
       const uint64_t desc0 = umma_desc_sw128(sbase);
       const uint32_t tile_enc = static_cast<uint32_t>(p.r8 * 128) >> 4;
@@ -416,10 +419,12 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
       const uint32_t x_enc = static_cast<uint32_t>(p.term_off) >> 4;
       const uint32_t xt_enc = static_cast<uint32_t>((INK ? IR : NP) * 128) >> 4;
       bool ok = !INK || mbar_wait_bounded(tready, 0, s_abort, p.err);
+      ok = __all_sync(0xffffffffu, ok);
       if (ok) tc_fence_after();
       for (int i = 0; ok && i < nsteps; ++i) {
         const int st = i % S;
-        if (!mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&fullb[st], (i / S) & 1, s_abort, p.err)))
+          break;
         tc_fence_after();
         const uint64_t ds = desc0 + (static_cast<uint32_t>(st * p.stage_bytes) >> 4);
         const int nv = min(NT, tile1 - (tile0 + i * NT));
@@ -431,14 +436,16 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
           for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
-              umma_e4m3(tmem + static_cast<uint32_t>(m * (INK ? IR : NP)),
-                        ds + tt * a_enc + m * tile_enc + 2 * kk, bx + 2 * kk, idesc,
-                        (i > 0 || tt > 0 || kk > 0) ? 1u : 0u);
+              if (leader)
+                umma_e4m3(tmem + static_cast<uint32_t>(m * (INK ? IR : NP)),
+                          ds + tt * a_enc + m * tile_enc + 2 * kk, bx + 2 * kk, idesc,
+                          (i > 0 || tt > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&empty[st]);
+        if (leader) umma_commit(&empty[st]);
+        __syncwarp();
       }
-      umma_commit(accfull);
+      if (leader) umma_commit(accfull);
     }
   } else if (warp < 6) {
     // ================= epilogue (warps 2..5, one per TMEM lane quarter)
