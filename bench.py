@@ -708,6 +708,26 @@ def decode_stack_measure(steps, layers=32, B=4):
         key = "fp8" if fp8 else ("fused_auto" if layout == "auto" else
                                  ("fused" if fused else "unfused"))
         res[key + "_ms_per_step"] = round(ms, 4)
+        if layout == "auto" or fp8:
+            # in-context tuning: the step timed with forced variants of each
+            # call, then the same timed loop again with the winners
+            st.release()
+            tuned = st.tune_variants()
+            st.step_eager()
+            torch.cuda.synchronize()
+            st.capture()
+            for _ in range(3):
+                st.step()
+            a.record()
+            for _ in range(steps):
+                st.step()
+            b.record()
+            torch.cuda.synchronize()
+            tms = a.elapsed_time(b) / steps
+            res[key + "_tuned_ms_per_step"] = round(tms, 4)
+            res[key + "_tuned_variants"] = {"gate_up": tuned["gate_up"], "down": tuned["down"]}
+            res[key + "_tuned_frac_of_peak"] = round(
+                st.bytes_per_step() / (tms * 1e-3) / 1e9 / peak, 4)
         if layout == "auto":
             gbs = st.bytes_per_step() / (ms * 1e-3) / 1e9
             res["fused_auto_layout"] = st.layout

@@ -24,6 +24,16 @@ FP8 variant encodes every layer's weights once as E4M3 codes with one fp32
 scale per output row (the library's FP8 entry points: half the weight bytes
 per step, dequantised inside the kernels).
 
+In-context tuning (``tune_variants``): the library's scheduler times each
+operation on its own, in bursts of back-to-back launches of that one
+operation.  Inside the stack every gate/up call follows a down projection and
+every down projection follows a gate/up call, and a variant that wins in a
+burst can lose there (with FP8 weights the in-kernel-term E4M3 variants win
+the bursts at B = 4 but cost ~5 us per layer in the stack).  The tuner
+times the captured step itself with each candidate variant of one
+operation while the other keeps its current choice, first for the gate/up
+call, then for the down projection, and keeps the fastest.
+
 Everything launched here is a libdfk kernel; torch provides the buffers, the
 stream and the CUDA graph.
 """
@@ -89,6 +99,9 @@ class DecodeStack:
             self.u = torch.empty_like(self.h)
             self.s = torch.empty_like(self.h)
         self.graph = None
+        # forced variants of the two per-layer calls (0 = the library's choice)
+        self.gu_variant = 0
+        self.dn_variant = 0
         # every launch of the stack (eager warm-up, capture, replay) goes to
         # self.stream, so the capture finds the scheduler's decisions and the
         # split-K workspace that the warm-up made on that stream
@@ -101,19 +114,21 @@ class DecodeStack:
         y = self.acts[l % 2]
         if self.fp8:
             gamma, qg, sg, qu, su, qd, sd = self.layers[l]
-            dfk.dfk_rmsnorm_swiglu_gate_up_fp8(xin, gamma, self.eps, qg, sg, qu, su, h=self.h)
-            dfk.dfk_down_proj_fp8(self.h, qd, sd, y=y)
+            dfk.dfk_rmsnorm_swiglu_gate_up_fp8(xin, gamma, self.eps, qg, sg, qu, su, h=self.h,
+                                               variant=self.gu_variant)
+            dfk.dfk_down_proj_fp8(self.h, qd, sd, y=y, variant=self.dn_variant)
             return
         gamma, wg, wu, wd = self.layers[l]
         if self.fused:
-            dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, self.layout, h=self.h)
+            dfk.dfk_rmsnorm_swiglu_gate_up(xin, gamma, self.eps, wg, wu, self.layout, h=self.h,
+                                           variant=self.gu_variant)
         else:
             dfk.dfk_rmsnorm(xin, gamma, self.eps, out=self.xn)
             dfk.dfk_gemv(self.xn, wg, out=self.a)
             dfk.dfk_gemv(self.xn, wu, out=self.u)
             dfk.dfk_silu(self.a, out=self.s)
             dfk.dfk_mul(self.s, self.u, out=self.h)
-        dfk.dfk_down_proj(self.h, wd, y=y)
+        dfk.dfk_down_proj(self.h, wd, y=y, variant=self.dn_variant)
 
     def _launch_step(self):
         for l in range(len(self.layers)):
@@ -152,6 +167,73 @@ class DecodeStack:
 
     def release(self):
         self.graph = None
+
+    def _candidates(self, gate_up):
+        """Variant ids worth timing in context for one of the two calls: the
+        library's own choice (0) and every tensor-core variant of the call's
+        class (the CUDA-core variants are many; the library's choice stands
+        for that family)."""
+        out = [0]
+        for i in range(1, dfk.dfk_variant_count() + 1):
+            v = dfk.dfk_variant_info(i)
+            if v["family"] != 1:
+                continue
+            is_gu = v["op"] in (dfk.DFK_OP_GATE_UP, dfk.DFK_OP_GATE_UP_FP8)
+            if is_gu != gate_up:
+                continue
+            if v["e4m3_mma"] and not self.fp8:
+                continue
+            out.append(i)
+        return out
+
+    def _time_step(self, steps):
+        """Mean device time of one captured step (ms), or None when a forced
+        variant does not fit the shape."""
+        self.release()
+        try:
+            self.step_eager()
+        except dfk.DfkError:
+            torch.cuda.synchronize(self.stream.device)
+            return None
+        torch.cuda.synchronize(self.stream.device)
+        self.capture()
+        for _ in range(2):
+            self.step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cur = torch.cuda.current_stream(self.stream.device)
+        a.record(cur)
+        for _ in range(steps):
+            self.step()
+        b.record(cur)
+        b.synchronize()
+        self.release()
+        return a.elapsed_time(b) / steps
+
+    def tune_variants(self, steps=10):
+        """Pick the gate/up and down-projection variants by timing the whole
+        captured step: each candidate of the gate/up call with the down
+        projection at its current choice, then each candidate of the down
+        projection.  Changes the stack's state (x advances by the timed steps);
+        returns {"gate_up": id, "down": id, "ms_per_step": best, "library_ms":
+        time with the library's own choices}.  Forced ids count as 0 = the
+        library's choice."""
+        if not self.fused:
+            raise ValueError("in-context tuning covers the fused stacks")
+        self.gu_variant = self.dn_variant = 0
+        base = self._time_step(steps)
+        best = base
+        for attr, gate_up in (("gu_variant", True), ("dn_variant", False)):
+            keep = getattr(self, attr)
+            for vid in self._candidates(gate_up):
+                if vid == keep:
+                    continue
+                setattr(self, attr, vid)
+                t = self._time_step(steps)
+                if t is not None and t < best:
+                    best, keep = t, vid
+            setattr(self, attr, keep)
+        return {"gate_up": self.gu_variant, "down": self.dn_variant, "ms_per_step": best,
+                "library_ms": base}
 
     def kernels_per_step(self):
         """Library calls per step (one kernel each, except the FP8 tensor-core

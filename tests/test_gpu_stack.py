@@ -238,3 +238,41 @@ def test_llama3_8b_stack_teacher_forced_at_steps_0_1_511(layout):
         ok, err = close(y[:, idx].contiguous(), y_ref)
         assert ok, "layout %s step %d layer %d down: max err %g" % (st.layout, step, l, err)
     assert len(got) == 9
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_in_context_tuning_picks_valid_variants_and_stays_within_tolerance(fp8):
+    # the tuner times the captured step with forced variants of each call and
+    # keeps the fastest; the tuned stack must still match the oracle layer by
+    # layer (teacher-forced on the GPU's own layer inputs)
+    x0, params = I.make_stack(3, 4, 1024, 2048, seed=12, w_std=0.02, device="cuda")
+    st = DecodeStack(params, x0, fp8=fp8)
+    res = st.tune_variants(steps=3)
+    assert res["gate_up"] in st._candidates(True)
+    assert res["down"] in st._candidates(False)
+    assert res["ms_per_step"] <= res["library_ms"]
+    assert (st.gu_variant, st.dn_variant) == (res["gate_up"], res["down"])
+    for l in range(len(params)):
+        xin = st.layer_input(l).clone()
+        st._layer(l)
+        torch.cuda.synchronize()
+        host = lambda t: t.detach().cpu().numpy()
+        if fp8:
+            gamma, qg, sg, qu, su, qd, sd = st.layers[l]
+            h_ref = oracle.gate_up_fp8(I.to_bits(xin), host(qg), host(sg), host(qu), host(su),
+                                       gamma=I.to_bits(gamma), eps=1e-5)
+            y_ref = oracle.down_fp8(h_ref, host(qd), host(sd))
+        else:
+            gamma, wg, wu, wd = params[l]
+            _, y_ref = oracle.mlp(I.to_bits(xin), I.to_bits(wg), I.to_bits(wu), I.to_bits(wd),
+                                  gamma=I.to_bits(gamma), eps=1e-5)
+        ok, err = close(st.acts[l % 2], y_ref)
+        assert ok, "tuned (%d, %d) layer %d: max err %g" % (res["gate_up"], res["down"], l, err)
+    st.step()
+    torch.cuda.synchronize()
+
+
+def test_in_context_tuning_refuses_the_unfused_stack():
+    st, _ = small_stack(layers=2, fused=False)
+    with pytest.raises(ValueError):
+        st.tune_variants()
