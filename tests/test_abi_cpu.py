@@ -178,3 +178,23 @@ def test_python_binding_rejects_host_tensors():
     with pytest.raises(dfk.DfkError):
         dfk.dfk_swiglu_gate_up(x, torch.zeros(64, 64, dtype=torch.bfloat16),
                                torch.zeros(64, 64, dtype=torch.bfloat16))
+
+
+def test_stack_tuning_candidates(L):
+    # the in-context tuner's candidate lists (host logic only): the library's
+    # own choice first, then the tensor-core variants of the call's class;
+    # E4M3-MMA variants only for the FP8 stack
+    import types
+    from swiglu_mlp_dfk_b200.stack import DecodeStack
+    for fp8 in (False, True):
+        fake = types.SimpleNamespace(fp8=fp8)
+        for gate_up in (True, False):
+            c = DecodeStack._candidates(fake, gate_up)
+            assert c[0] == 0 and len(c) == len(set(c)) > 1
+            for i in c[1:]:
+                v = dfk.dfk_variant_info(i)
+                assert v["family"] == 1
+                assert (v["op"] in (dfk.DFK_OP_GATE_UP, dfk.DFK_OP_GATE_UP_FP8)) == gate_up
+                assert fp8 or v["e4m3_mma"] == 0
+            has_e4m3 = any(dfk.dfk_variant_info(i)["e4m3_mma"] for i in c[1:])
+            assert has_e4m3 == fp8
