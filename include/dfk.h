@@ -123,10 +123,13 @@ DFK_API int dfk_swiglu_gate_up(const void *x, const void *w_gate, const void *w_
 /*
  * Same, with the RMSNorm fused in front (GPULlama3.java PR #78, the
  * `rms_ffn_gate_up` task):
- *   xn[b][k] = bf16( x[b][k] * r_b * gamma[k] ),
+ *   xn[b][k] = x[b][k] * r_b * gamma[k],
  *   r_b = 1 / sqrt( (1/d_model) * sum_k x[b][k]^2 + eps ),
- * then h = SiLU(xn . W_gate^T) (*) (xn . W_up^T).  xn lives in shared memory
- * only.  gamma [d_model] bf16, device.  eps >= 0.
+ * then h = SiLU(xn . W_gate^T) (*) (xn . W_up^T).  xn is not rounded to
+ * bf16: the CUDA-core kernels keep (x * r_b) * gamma in fp32 in shared
+ * memory; the tensor-core kernels split the exact x * gamma into bf16
+ * hi + lo MMA operands and apply r_b to the fp32 sums.  xn never reaches
+ * HBM.  gamma [d_model] bf16, device.  eps >= 0.
  */
 DFK_API int dfk_rmsnorm_swiglu_gate_up(const void *x, const void *gamma, float eps,
                                const void *w_gate, const void *w_up, int layout,
