@@ -33,7 +33,7 @@
 // at 64 tokens; the host uses NORM = 2 above 32 tokens).
 //
 // Warp roles (192 threads): warp 0 issues TMA copies into an S-stage ring;
-// warp 1 owns TMEM and issues the MMAs (one thread) with tcgen05.commit
+// warp 1 owns TMEM and issues the MMAs (one elected lane) with tcgen05.commit
 // releasing ring stages; warps 2-5 run the x*gamma transform (NORM) and the
 // epilogue (tcgen05.ld -> SiLU * up -> one bf16 store per output).
 #pragma once

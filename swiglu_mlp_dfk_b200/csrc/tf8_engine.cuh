@@ -24,7 +24,7 @@
 // activations as two 64-wide bf16 sub-tiles (TMA, 128-byte swizzle).
 //
 // Warp roles (576 threads): warp 0 issues TMA copies; warp 1 owns TMEM and
-// issues the MMAs (one thread); warps 2-17 dequantise -- the four warps of a
+// issues the MMAs (one elected lane); warps 2-17 dequantise -- the four warps of a
 // TMEM lane quarter split a tile's 128 codes per row into parts of 32, each
 // thread converts its row's 32 codes and stores 16 columns with tcgen05.st
 // into one of two A buffers -- and with the RMSNorm prologue also split x *

@@ -27,7 +27,7 @@
 // Main kernel: one CTA per SM owns r <= 128 weight rows (the MMA's M) over its
 // reduction range (split-K slices for the down projection); a TMA ring
 // carries 128-wide k tiles of codes (128-byte swizzle) and of the activation
-// terms; one thread issues 4 MMAs (K = 32) per matrix per tile; warps 2-5
+// terms; one elected lane issues 4 MMAs (K = 32) per matrix per tile; warps 2-5
 // read the accumulators, combine the terms, apply f_b, s[j], SiLU(gate) * up
 // and store bf16.  Rows of the 128-row MMA beyond r read neighbouring shared
 // memory and give ignored accumulator rows.
