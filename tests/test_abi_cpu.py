@@ -198,3 +198,35 @@ def test_stack_tuning_candidates(L):
                 assert fp8 or v["e4m3_mma"] == 0
             has_e4m3 = any(dfk.dfk_variant_info(i)["e4m3_mma"] for i in c[1:])
             assert has_e4m3 == fp8
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    # a C program (no C++, no torch) includes dfk.h, links against libdfk.so and
+    # the CUDA runtime, and runs: without a device the entry points return a
+    # status (here: invalid argument for the null buffers), never crash
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if gcc is None or not os.path.exists(os.path.join(cuda, "include", "cuda_runtime.h")):
+        pytest.skip("needs gcc and the CUDA headers")
+    src = tmp_path / "app.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "dfk.h"
+int main(void) {
+  int st = dfk_rmsnorm_swiglu_gate_up(0, 0, 1e-5f, 0, 0, DFK_W_ROW_MAJOR, 0, 1, 4096, 14336,
+                                      0, 0);
+  printf("%d %s\n", st, dfk_status_string(st));
+  return st == DFK_ERR_INVALID_ARG ? 0 : 1;
+}
+''')
+    exe = tmp_path / "app"
+    pkg = os.path.dirname(dfk.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", pkg, "-ldfk", "-Wl,-rpath," + pkg, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.split()[0] == str(dfk.DFK_ERR_INVALID_ARG)
