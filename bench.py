@@ -378,6 +378,15 @@ def gpu_arm(args):
     line.update(extra)
     if world == 1:
         line["cpu_baseline"] = cpu_baseline()
+    if "batch_sweep" in line:
+        # last key, so that a reader keeping only the end of the line still
+        # has the B = 1..64 gate/up figures (fraction of the measured peak)
+        sw = line["batch_sweep"]
+        line["batch_sweep_compact"] = {
+            "B": [r["B"] for r in sw],
+            "row_us": [r["row"]["us"] for r in sw], "col_us": [r["col"]["us"] for r in sw],
+            "row_frac": [r["row"]["frac"] for r in sw], "col_frac": [r["col"]["frac"] for r in sw],
+            "family": ["%s/%s" % (r["row"]["family"], r["col"]["family"]) for r in sw]}
     return line
 
 

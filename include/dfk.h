@@ -57,7 +57,9 @@ typedef enum dfk_status {
   DFK_ERR_CUDA = 5,               /* a CUDA runtime call failed; see dfk_last_error() */
   DFK_ERR_ARCH = 6,               /* no sm_100 device current */
   DFK_ERR_TIMEOUT = 7,            /* a kernel's pipeline wait gave up (dfk_device_error) */
-  DFK_ERR_NO_VARIANT = 8          /* no variant fits this shape (shared memory / threads) */
+  DFK_ERR_NO_VARIANT = 8,         /* no variant fits this shape (shared memory / threads) */
+  DFK_ERR_BOUNDS = 9              /* checked build: a kernel's bounds check failed
+                                     (dfk_device_error; the access was skipped)      */
 } dfk_status;
 
 /* Storage of W_gate / W_up (as stated in the pages: W_gate, W_up are [d_ff, d_model]). */
@@ -189,7 +191,10 @@ DFK_API int dfk_down_proj_static_scratch(const void *h, const void *w_down, void
  * with fp32 accumulation); and the E4M3-MMA kernel (ids with e4m3_mma >= 1:
  * the codes feed the E4M3 tensor-core MMA directly, each token's activations
  * are written as E4M3 terms -- two for bf16 x, four for x * gamma, after a
- * power-of-two scale -- either (e4m3_mma = 1) by a small kernel launched
+ * power-of-two scale; exact for elements within 2^14 of the token's largest
+ * magnitude, smaller ones carried to about 2^-21 of it, so a token spanning
+ * more than 2^14 can land outside the bf16 path's accuracy and should use
+ * the CUDA-core or widening ids -- either (e4m3_mma = 1) by a small kernel launched
  * before it, into a library-owned buffer per (device, stream) allocated at
  * first use outside stream capture, or (e4m3_mma = 2, B <= 16) inside the
  * kernel from each ring stage's raw activations; with a k split the latter
@@ -330,9 +335,38 @@ DFK_API const char *dfk_status_string(int status);
  * description of the rejected argument); "" when none. */
 DFK_API const char *dfk_last_error(void);
 
-/* Reads the current device's error word (0 = none; bit 0 = a pipeline wait
- * timed out) into *code and clears it.  Synchronises the device. */
+/* Reads the current device's error word into *code and clears it
+ * (0 = none; bit 0 = a pipeline wait gave up; bit 1 = a bounds check of the
+ * checked build failed).  Synchronises the device.  Returns DFK_OK when the
+ * word was 0, DFK_ERR_BOUNDS when bit 1 was set (dfk_last_error names the
+ * first failing check), else DFK_ERR_TIMEOUT. */
 DFK_API int dfk_device_error(int *code);
+
+/*
+ * Failure detection (no counterpart in the pages): every wait of a kernel's
+ * pipeline on an mbarrier is bounded.  When a wait gives up the kernel sets
+ * bit 0 of the device error word, stops issuing work, waits (with the
+ * default limit) for its own copies and MMAs in flight, releases its tensor
+ * memory and returns; the context stays usable and dfk_device_error reports
+ * DFK_ERR_TIMEOUT.
+ *
+ * dfk_set_wait_limit sets the limit of the pipeline waits for kernels
+ * launched afterwards on the current device: ns > 0, or 0 for the default
+ * of 4 s.  A limit shorter than a call's own duration makes healthy calls
+ * give up; it exists so that tests and health checks need not wait 4 s.
+ * The waits at a kernel's exit for its own copies always allow the default.
+ */
+DFK_API int dfk_set_wait_limit(unsigned long long ns);
+
+/*
+ * Self-test of the bounded wait: launches one warp on `stream` that waits
+ * on an mbarrier no one ever completes.  The wait gives up after the current
+ * limit, sets bit 0 of the device error word, stores the time it waited (ns)
+ * in *elapsed_ns (device memory, 8-byte aligned, caller-owned) and the
+ * kernel returns.  A health check: afterwards dfk_device_error must report
+ * DFK_ERR_TIMEOUT and the device must still run the MLP kernels.
+ */
+DFK_API int dfk_selftest_bounded_wait(void *elapsed_ns, void *stream);
 
 /* Library version, e.g. "dfk 0.1.0 sm_100a". */
 DFK_API const char *dfk_version(void);

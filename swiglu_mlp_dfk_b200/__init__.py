@@ -47,6 +47,7 @@ DFK_ERR_CUDA = 5
 DFK_ERR_ARCH = 6
 DFK_ERR_TIMEOUT = 7
 DFK_ERR_NO_VARIANT = 8
+DFK_ERR_BOUNDS = 9
 
 _LAYOUTS = {"row": DFK_W_ROW_MAJOR, "col": DFK_W_COL_MAJOR, "interleaved": DFK_W_GU_INTERLEAVED,
             "any": DFK_W_ANY}
@@ -60,6 +61,7 @@ EXPORTED = (
     "dfk_variant_info", "dfk_clear_variant_cache", "dfk_rmsnorm",
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
     "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
+    "dfk_set_wait_limit", "dfk_selftest_bounded_wait",
 )
 
 
@@ -122,6 +124,8 @@ def lib():
                 "dfk_rms_rescale": [vp, f, vp, i, i, vp],
                 "dfk_mlp_forward_host": [vp, vp, f, vp, vp, i, vp, vp, vp, vp, vp, i, i, i, vp],
                 "dfk_device_error": [ctypes.POINTER(i)],
+                "dfk_set_wait_limit": [ctypes.c_ulonglong],
+                "dfk_selftest_bounded_wait": [vp, vp],
                 "dfk_status_string": [i],
                 "dfk_last_error": [],
                 "dfk_version": [],
@@ -445,9 +449,30 @@ def dfk_device_error():
     """Read and clear the device error word; returns the code (0 = none)."""
     code = ctypes.c_int(0)
     st = lib().dfk_device_error(ctypes.byref(code))
-    if st not in (DFK_OK, DFK_ERR_TIMEOUT):
+    if st not in (DFK_OK, DFK_ERR_TIMEOUT, DFK_ERR_BOUNDS):
         _check(st)
     return code.value
+
+
+def dfk_device_status():
+    """Read and clear the device error word; returns (dfk_status, code, text)."""
+    code = ctypes.c_int(0)
+    st = lib().dfk_device_error(ctypes.byref(code))
+    return st, code.value, lib().dfk_last_error().decode() if st else ""
+
+
+def dfk_set_wait_limit(ns):
+    """Limit of the kernels' pipeline waits on the current device (0 = default 4 s)."""
+    _check(lib().dfk_set_wait_limit(int(ns)))
+
+
+def dfk_selftest_bounded_wait(elapsed_ns=None, stream=None):
+    """Launch the bounded-wait self-test; returns the int64 device tensor that
+    receives the time the wait took before giving up (ns)."""
+    if elapsed_ns is None:
+        elapsed_ns = torch.zeros(1, dtype=torch.int64, device="cuda")
+    _check(lib().dfk_selftest_bounded_wait(_ptr(elapsed_ns), _stream(stream)))
+    return elapsed_ns
 
 
 def dfk_version():

@@ -37,8 +37,11 @@
 #include "tf8_key.h"
 #include "tf8mma_engine.cuh"
 
-// Device error word: bit 0 = a pipeline wait in some kernel gave up.
-__device__ unsigned g_dfk_err;
+// Device status block: word 0 = error bits (bit 0 = a pipeline wait in some
+// kernel gave up, bit 1 = a bounds check of the checked build failed),
+// word 1 = the site of the first failed bounds check, words 2-3 = the
+// pipeline-wait limit in ns (0 = default).
+__device__ __align__(16) unsigned g_dfk_err[dfk::STATUS_WORDS];
 
 namespace dfk {
 
@@ -844,10 +847,13 @@ static int check_gemv(const void *x, const void *w, const void *out, int B, int 
 
 // The split-K tensor-core down projection on caller-provided scratch: a
 // fixed configuration (no timing), no workspace of its own.  Used by the
-// entry point for callers that cannot allocate (noalloc.cu).
+// entry point for callers that cannot allocate (noalloc.cu).  With
+// clear_counters the row-block counters are zeroed on the stream right
+// before the launch, after every argument has been checked (an invalid call
+// enqueues nothing).
 int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, int d_model,
                            int d_ff, float *part, size_t part_capacity, unsigned *counters,
-                           size_t counter_capacity, cudaStream_t s) {
+                           size_t counter_capacity, bool clear_counters, cudaStream_t s) {
   int rc = check_gemv(h, w_down, y, B, d_ff, d_model, 0);
   if (rc || B == 0) return rc;
   DeviceState *ds;
@@ -900,6 +906,13 @@ int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, in
   p.eps = 0.f;
   p.part = part;
   p.counters = counters;
+  if (clear_counters) {
+    cudaError_t e = cudaMemsetAsync(counters, 0, counter_bytes, s);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "zeroing the split-K counters");
+    }
+  }
   void *args[] = {&maps, &p};
   cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid), dim3(TC_THREADS), pl.smem, s,
                                 pdl_enabled(), args);
@@ -1626,14 +1639,46 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
       return DFK_OK;
     }
   }
+  // Layouts of one gate/up shape agree bit for bit within a variant family
+  // (the same k order reaches the same accumulators), not across families.
+  // Once one layout of this shape has a decision, the other layouts are
+  // chosen within its family, so the row- and column-major results a caller
+  // gets from the scheduler are identical.
+  int lock_family = -1;
+  if (op_class(op) == CLS_GATE_UP) {
+    std::lock_guard<std::mutex> lk(g_tune_mu);
+    for (int l : {LAYOUT_ROW, LAYOUT_COL, LAYOUT_IL}) {
+      TuneKey k2 = key;
+      k2.layout = l;
+      auto it = g_tuned.find(k2);
+      if (l != c.layout && it != g_tuned.end()) {
+        lock_family = it->second.family;
+        break;
+      }
+    }
+  }
+  std::vector<const VDef *> cands = candidates(op, c.B, c);
   const VDef *h = heuristic(op, c.B, c, *ds);
+  if (lock_family >= 0) {
+    cands.erase(std::remove_if(cands.begin(), cands.end(),
+                               [&](const VDef *d) { return d->family != lock_family; }),
+                cands.end());
+    if (h && h->family != lock_family) {
+      h = nullptr;
+      for (const VDef *d : cands)
+        if (feasible(*d, c, *ds)) {
+          h = d;
+          break;
+        }
+    }
+  }
   if (!h) return fail(DFK_ERR_NO_VARIANT, "no variant fits B=%d K=%d N=%d", c.B, c.K, c.N);
   const bool tune = env_flag("DFK_TUNE", true) && !stream_capturing(s);
   const VDef *win = h;
   float us = -1.f;
   int stages = 0;
   if (tune) {
-    const VDef *t = time_candidates(op, c, candidates(op, c.B, c), s, *ds, &us, &stages);
+    const VDef *t = time_candidates(op, c, cands, s, *ds, &us, &stages);
     if (t) win = t;
     else us = -1.f;
   }
@@ -2275,16 +2320,50 @@ int dfk_device_error(int *code) {
   int rc = current_device(&ds);
   if (rc) return rc;
   cudaError_t e = cudaDeviceSynchronize();
-  unsigned v = 0;
-  if (!e) e = cudaMemcpyFromSymbol(&v, g_dfk_err, sizeof v);
-  const unsigned zero = 0;
-  if (!e) e = cudaMemcpyToSymbol(g_dfk_err, &zero, sizeof zero);
+  unsigned v[2] = {0u, 0u};
+  if (!e) e = cudaMemcpyFromSymbol(v, g_dfk_err, sizeof v);
+  const unsigned zero[2] = {0u, 0u};
+  if (!e) e = cudaMemcpyToSymbol(g_dfk_err, zero, sizeof zero);
   if (e) {
     cudaGetLastError();
     return cuda_fail(e, "reading the device error word");
   }
-  *code = static_cast<int>(v);
-  return v ? DFK_ERR_TIMEOUT : DFK_OK;
+  *code = static_cast<int>(v[0]);
+  if (v[0] & dfk::ERR_BOUNDS)
+    return fail(DFK_ERR_BOUNDS, "bounds check failed (first at site %u, source line %u)",
+                v[1] >> 16, v[1] & 0xffffu);
+  if (v[0]) return fail(DFK_ERR_TIMEOUT, "a kernel's pipeline wait gave up");
+  return DFK_OK;
+}
+
+int dfk_set_wait_limit(unsigned long long ns) {
+  DeviceState *ds;
+  int rc = current_device(&ds);
+  if (rc) return rc;
+  // words 2-3 of the status block; a plain copy, ordered after work already
+  // queued on the legacy default stream
+  cudaError_t e = cudaMemcpyToSymbol(g_dfk_err, &ns, sizeof ns, 2 * sizeof(unsigned));
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "setting the wait limit");
+  }
+  return DFK_OK;
+}
+
+int dfk_selftest_bounded_wait(void *elapsed_ns, void *stream) {
+  if (!elapsed_ns) return fail(DFK_ERR_INVALID_ARG, "elapsed_ns is NULL");
+  if (reinterpret_cast<uintptr_t>(elapsed_ns) & 7u)
+    return fail(DFK_ERR_MISALIGNED, "elapsed_ns must be 8-byte aligned");
+  DeviceState *ds;
+  int rc = current_device(&ds);
+  if (rc) return rc;
+  cudaError_t e = dfk::launch_wait_selftest(ds->err, static_cast<unsigned long long *>(elapsed_ns),
+                                            static_cast<cudaStream_t>(stream));
+  if (e) {
+    cudaGetLastError();
+    return cuda_fail(e, "wait self-test launch");
+  }
+  return DFK_OK;
 }
 
 const char *dfk_version(void) { return "dfk 0.1.0 sm_100a"; }

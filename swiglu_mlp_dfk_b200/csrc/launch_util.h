@@ -45,5 +45,7 @@ cudaError_t launch_mul(const void *a, const void *b, void *out, long long n, cud
                        bool pdl);
 cudaError_t launch_copy16(const void *src, void *dst, size_t bytes, bool wait_first,
                           cudaStream_t s, bool pdl);
+// selftest.cu
+cudaError_t launch_wait_selftest(unsigned *err, unsigned long long *elapsed_ns, cudaStream_t s);
 
 }  // namespace dfk

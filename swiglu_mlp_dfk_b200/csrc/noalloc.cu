@@ -23,7 +23,7 @@
 namespace dfk {
 int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, int d_model,
                            int d_ff, float *part, size_t part_capacity, unsigned *counters,
-                           size_t counter_capacity, cudaStream_t s);
+                           size_t counter_capacity, bool clear_counters, cudaStream_t s);
 }  // namespace dfk
 
 namespace {
@@ -79,13 +79,9 @@ extern "C" int dfk_down_proj_static_scratch(const void *h, const void *w_down, v
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned *counters = reinterpret_cast<unsigned *>(base + kPartBytes);
-  // the arrival counters must start at zero (the array keeps the last call's contents)
-  cudaError_t e = cudaMemsetAsync(counters, 0, kCounterBytes, s);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return DFK_ERR_CUDA;
-  }
+  // the arrival counters must start at zero (the array keeps the last call's
+  // contents): cleared on the stream once the arguments have been accepted
   return dfk::down_proj_with_scratch(h, w_down, y, B, d_model, d_ff,
                                      reinterpret_cast<float *>(base), kPartBytes, counters,
-                                     kCounterBytes, s);
+                                     kCounterBytes, /*clear_counters=*/true, s);
 }

@@ -6,12 +6,26 @@
 
 namespace dfk {
 
-// Device error word bits (read by dfk_device_error).
+// Device status block (one per device, read by dfk_device_error): word 0
+// holds the error bits, word 1 the site of the first failed bounds check
+// (checked builds), words 2-3 the pipeline-wait limit in ns as a 64-bit
+// value (0 = the default), set by dfk_set_wait_limit.  Every kernel gets a
+// pointer to word 0 (`err`).
 constexpr unsigned ERR_WAIT_TIMEOUT = 1u;
+constexpr unsigned ERR_BOUNDS = 2u;
+constexpr int STATUS_WORDS = 4;
 
-// A pipeline wait gives up after this long (the data it waits for arrives
-// in microseconds in a healthy run).
+// A pipeline wait gives up after this long by default (the data it waits
+// for arrives in microseconds in a healthy run).
 constexpr unsigned long long WAIT_TIMEOUT_NS = 4000000000ull;
+
+// The wait limit in force for kernels given the status block `err`.
+__device__ __forceinline__ unsigned long long wait_limit_ns(const unsigned *err) {
+  if (!err) return WAIT_TIMEOUT_NS;
+  const unsigned long long v =
+      *reinterpret_cast<const volatile unsigned long long *>(err + 2);
+  return v ? v : WAIT_TIMEOUT_NS;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -55,18 +69,23 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up
-// (returns false) when *abort_flag becomes non-zero, or after
-// WAIT_TIMEOUT_NS, in which case it sets *abort_flag and the device error
-// word.  Never spins unboundedly.
+// (returns false) when *abort_flag becomes non-zero, or after the wait
+// limit, in which case it sets *abort_flag and the device error word.
+// Pipeline waits (abort_flag given) use the limit set for the device
+// (dfk_set_wait_limit, default WAIT_TIMEOUT_NS); the waits at exit for
+// copies and MMAs still in flight (abort_flag == nullptr) always allow the
+// default, so a short limit never lets a CTA leave while its shared memory
+// is still being written.  Never spins unboundedly.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag, unsigned *err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
+  const unsigned long long limit = abort_flag ? wait_limit_ns(err) : WAIT_TIMEOUT_NS;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (global_timer_ns() - t0 > WAIT_TIMEOUT_NS || it > (1u << 30)) {
+      if (global_timer_ns() - t0 > limit || it > (1u << 30)) {
         if (abort_flag) *abort_flag = 1;
         if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
         return false;

@@ -509,3 +509,114 @@ def test_fp8_in_kernel_terms_capture_on_a_fresh_stream(B):
     assert bits_equal(h, h_ref)
     assert bits_equal(y, y_ref)
     del g
+
+
+# ------------------------------------------------------------------ E4M3 terms: wide dynamic range
+
+def _wide_range_tokens(B, D, seed, spread_log2):
+    """Activations whose tokens span a wide dynamic range: token 0 has two
+    elements at 2^10 and -2^9 and the rest near 2^(10 - spread); token 1 lies
+    entirely near 2^-30; token 2 mixes 2^8-sized and 2^(8 - spread)-sized
+    halves; the others are N(0, 1)."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(B, D, generator=g)
+    sign = torch.where(torch.rand(B, D, generator=g) < 0.5, -1.0, 1.0)
+    mag = 1.0 + torch.rand(B, D, generator=g)
+    x[0] = sign[0] * mag[0] * 2.0 ** (10 - spread_log2)
+    x[0, 17] = 1024.0
+    x[0, D // 2] = -512.0
+    x[1] = sign[1] * mag[1] * 2.0 ** -30
+    x[2, : D // 2] = sign[2, : D // 2] * mag[2, : D // 2] * 2.0 ** 8
+    x[2, D // 2:] = sign[2, D // 2:] * mag[2, D // 2:] * 2.0 ** (8 - spread_log2)
+    return x.to(torch.bfloat16).cuda()
+
+
+def _fp8_exact_ids():
+    """FP8 gate/up variants that multiply by the exact activations: a
+    CUDA-core one and the widening tensor-core one."""
+    cc = next(w["variant_id"] for w in cc_ids(dfk.DFK_OP_GATE_UP_FP8)
+              if w["j_per_thread"] == 4 and w["token_tile"] == 4)
+    return [cc] + [v["variant_id"] for v in tc_fp8_ids(False)][:1]
+
+
+@pytest.mark.parametrize("norm", [False, True])
+def test_e4m3_mma_wide_range_within_the_exact_domain(norm):
+    # Tokens spanning 2^13 (inside the 2^14 the two / four E4M3 terms carry
+    # exactly), with gamma near the small end of bf16's normal range on a
+    # quarter of the channels (x * gamma there is an fp32 subnormal whose
+    # contribution is far below any rounding): every E4M3-MMA variant
+    # (prep-kernel and in-kernel terms) and the exact-activation kernels
+    # match the oracle within the contract tolerance.
+    B, D, F = 4, 1024, 1496
+    L = Fp8Layer(B, D, F, seed=530 + norm, norm=True, with_down=False)
+    L.inp.x.copy_(_wide_range_tokens(B, D, 531, 13))
+    gam = L.inp.gamma.clone()
+    gam[: D // 4] = (torch.rand(D // 4, device="cuda") + 1.0).to(torch.bfloat16) * 2.0 ** -125
+    L.inp.gamma.copy_(gam)
+    want = L.oracle_gate_up(norm)
+    ran = 0
+    for vid in [v["variant_id"] for v in e4m3_mma_ids(False)] + _fp8_exact_ids():
+        h = try_variant(lambda v: L.gate_up(norm, variant=v), vid)
+        if h is None:
+            continue
+        torch.cuda.synchronize()
+        assert_close(h, want, "wide-range fp8 gate/up variant %d norm=%d" % (vid, norm))
+        ran += 1
+    assert ran >= 5
+
+
+@pytest.mark.parametrize("norm", [False, True])
+def test_fp8_exact_activation_kernels_beyond_the_e4m3_domain(norm):
+    # Tokens spanning 2^22: the kernels that multiply by the exact
+    # activations (CUDA-core, widening tensor-core) still meet the contract
+    # tolerance.  (The E4M3-MMA variants carry elements more than 2^14 below
+    # their token's largest only to about 2^-21 of it; the down-projection
+    # test below checks that bound.)
+    B, D, F = 4, 1024, 1496
+    L = Fp8Layer(B, D, F, seed=532 + norm, norm=True, with_down=False)
+    L.inp.x.copy_(_wide_range_tokens(B, D, 533, 22))
+    want = L.oracle_gate_up(norm)
+    for vid in _fp8_exact_ids():
+        h = L.gate_up(norm, variant=vid)
+        torch.cuda.synchronize()
+        assert_close(h, want, "wide-range fp8 gate/up variant %d norm=%d" % (vid, norm))
+
+
+def test_e4m3_mma_wide_dynamic_range_down_error_bound():
+    # The activation terms carry each element exactly when it lies within
+    # 2^14 of its token's largest |value| (two terms for bf16 h: 8 significant
+    # bits, the second term's last bit at 2^-13 after the scale that puts the
+    # largest in [128, 256)); a smaller element is carried to within 2^-21 of
+    # the largest.  Rows whose code at the large elements is zero see only the
+    # small elements, so their error shows that bound directly:
+    #   |y - oracle| <= 2^-8 |oracle| + 2^-21 max_k|h_k| sum_k |W_jk|
+    #                   + 2^-12 sum_k |W_jk h_k|
+    # (output rounding, the term representation, and a generous allowance for
+    # the MMA's fp32 accumulation over K).
+    B, D, F = 4, 512, 2048
+    L = Fp8Layer(B, D, F, seed=540, norm=False)
+    h = _wide_range_tokens(B, F, 541, 22)
+    qd = L.qd.clone()
+    qd[0::2, 17] = 0            # even rows: blind to the two large elements of token 0
+    qd[0::2, F // 2] = 0
+    want = oracle.down_fp8(I.bf16_values(h), L.host(qd), L.host(L.sd))
+    hv = np.abs(I.bf16_values(h))
+    qv = np.abs(I.fp8_values(qd)) * L.host(L.sd)[:, None]          # |W| per element
+    hmax = hv.max(axis=1, keepdims=True)
+    bound = (2.0 ** -8 * np.abs(want) + (2.0 ** -21 * hmax) * qv.sum(1)[None, :]
+             + 2.0 ** -12 * (hv @ qv.T) + 1e-30)
+    ran = 0
+    for v in e4m3_mma_ids(True):
+        y = try_variant(lambda vid: dfk.dfk_down_proj_fp8(h, qd, L.sd, variant=vid),
+                        v["variant_id"])
+        if y is None:
+            continue
+        torch.cuda.synchronize()
+        got = I.bf16_values(y)
+        assert_close(y, want, "wide-range fp8 down variant %d" % v["variant_id"])
+        excess = np.abs(got - want) - bound
+        assert (excess <= 0).all(), ("variant %d: error beyond the term bound at %s"
+                                     % (v["variant_id"], np.unravel_index(np.argmax(excess),
+                                                                         excess.shape)))
+        ran += 1
+    assert ran >= 4

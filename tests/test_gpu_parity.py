@@ -507,3 +507,72 @@ def test_tensor_core_rmsnorm_captured_on_a_fresh_stream():
     torch.cuda.synchronize()
     assert_close(h2, ref, "prepared RMSNorm activations")
     del g
+
+
+# ------------------------------------------------------------------ tensor-core bitwise layouts
+
+def _tc_bitwise_all(inp, B, norm, rows=None, ref=None, what=""):
+    """Runs every tensor-core gate/up variant in every layout; all results must
+    be bit-identical (and, when given, match the oracle on `rows`)."""
+    layouts = {}
+    for layout in (I.LAYOUT_ROW, I.LAYOUT_COL, I.LAYOUT_INTERLEAVED):
+        layouts[layout] = I.to_layout(inp.w_gate, inp.w_up, layout)
+    base = None
+    for vid in tc_variants(dfk.DFK_OP_GATE_UP):
+        for layout, (wg, wu) in layouts.items():
+            if norm:
+                h = dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu, layout,
+                                                   variant=vid)
+            else:
+                h = dfk.dfk_swiglu_gate_up(inp.x, wg, wu, layout, variant=vid)
+            torch.cuda.synchronize()
+            if base is None:
+                base = h
+                if ref is not None:
+                    assert_close(h[:, rows] if rows is not None else h, ref, what)
+            else:
+                assert bits_equal(base, h), "%s: variant %d layout %d differs bitwise" % (
+                    what, vid, layout)
+    return base
+
+
+@pytest.mark.parametrize("B", [4, 8, 16, 32, 64])
+@pytest.mark.parametrize("norm", [False, True])
+def test_tensor_core_layouts_bitwise_llama3_8b(B, norm):
+    # The row- and column-major variants must agree bit for bit on identical
+    # input.  In the tensor-core family every layout feeds the same 16-wide
+    # MMA k-slices in the same order into one TMEM accumulator per output, and
+    # the RMSNorm r_b (in-kernel up to 32 tokens, prep kernel above) does not
+    # depend on the layout either; every variant (rows over the SMs or full
+    # 128-row tiles, one or two k-tiles per stage) gives the same bits.
+    inp = I.make_workload("llama3_8b_sweep", B=B, device="cuda", with_down=False)
+    rows = sample_rows(inp.w_gate.shape[0], 256, 40 + B)
+    ref = oracle.gate_up(I.to_bits(inp.x), I.to_bits(inp.w_gate), I.to_bits(inp.w_up),
+                         gamma=I.to_bits(inp.gamma) if norm else None, eps=inp.eps, rows=rows)
+    _tc_bitwise_all(inp, B, norm, rows=rows, ref=ref, what="8B B=%d norm=%d" % (B, norm))
+
+
+@pytest.mark.parametrize("B,D,F", [s for s in TC_SHAPES if s[0] >= 4])
+def test_tensor_core_layouts_bitwise_ragged(B, D, F):
+    inp = I.make_inputs(B, D, F, seed=500 + B, w_std=0.05, with_down=False, device="cuda")
+    for norm in (False, True):
+        _tc_bitwise_all(inp, B, norm, ref=oracle_gate_up(inp, norm),
+                        what="B=%d D=%d F=%d norm=%d" % (B, D, F, norm))
+
+
+@pytest.mark.parametrize("B", [4, 16, 64])
+def test_scheduler_row_and_col_agree_bitwise(B):
+    # what a caller sees with variant = 0: the scheduler's pick for row-major
+    # weights and its pick for column-major weights give the same bits
+    inp = I.make_inputs(B, 1024, 2048, seed=600 + B, w_std=0.03, with_down=False, device="cuda")
+    wg_c, wu_c = I.to_layout(inp.w_gate, inp.w_up, I.LAYOUT_COL)
+    a = dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, inp.w_gate, inp.w_up, "row")
+    b = dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg_c, wu_c, "col")
+    torch.cuda.synchronize()
+    fa = dfk.dfk_cached_variant(dfk.DFK_OP_RMSNORM_GATE_UP, B, 1024, 2048, "row")["family"]
+    fb = dfk.dfk_cached_variant(dfk.DFK_OP_RMSNORM_GATE_UP, B, 1024, 2048, "col")["family"]
+    ref = oracle_gate_up(inp, True)
+    assert_close(a, ref, "row pick")
+    assert_close(b, ref, "col pick")
+    if fa == fb:
+        assert bits_equal(a, b), "B=%d: the scheduler's row and col picks differ bitwise" % B

@@ -103,6 +103,10 @@ def test_capture_on_fresh_stream_without_workspace():
         dfk.dfk_down_proj(h, wd, y=y)
     graph.replay()
     torch.cuda.synchronize()
+    # the unsplit launch taken during capture, against the fp64 oracle (all
+    # 4096 outputs of the 8 tokens) and against the eager split-K result
+    ok, err = close(y, oracle.down(I.to_bits(h), I.to_bits(wd)))
+    assert ok, err
     ok, err = close(y, I.bf16_values(eager))
     assert ok, err
     del graph
