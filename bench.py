@@ -886,6 +886,83 @@ def profile_arm(args):
     return None
 
 
+def tp_arm(args):
+    """Tensor-parallel layer: the same 8B-shaped layer with d_ff sharded over
+    the torchrun ranks (one GPU each), the all-reduce fused into the down
+    projection.  Strong scaling: the layer is fixed, every rank streams its
+    1/N of the weights; value = the layer's algorithmic bytes per step /
+    max-over-ranks step time."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local if world > 1 else 0)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import swiglu_mlp_dfk_b200 as dfk
+    from swiglu_mlp_dfk_b200 import build as kbuild
+    from swiglu_mlp_dfk_b200 import inputs as I
+    from swiglu_mlp_dfk_b200 import tp
+
+    if rank == 0 or not os.path.exists(kbuild.LIB):
+        kbuild.build()
+    if world > 1:
+        dist.barrier()
+    dfk.dfk_device_error()
+    inp = I.make_inputs(B1, D, F, seed=SEED, w_std=0.02, norm=True, with_down=True,
+                        device="cuda")
+    # two shard copies in rotation (inputs larger than L2)
+    shards = [tp.shard_weights(inp.w_gate, inp.w_up, inp.w_down, I.LAYOUT_ROW, world, rank)]
+    shards.append(tuple(t.clone() if torch.is_tensor(t) else t for t in shards[0]))
+    group = tp.TPGroup(world, rank, 64, D)
+    h = torch.empty(B1, shards[0][2].shape[1], dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(B1, D, dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        wg, wu, wd, _ = shards[i % 2]
+        dfk.dfk_rmsnorm_swiglu_gate_up(inp.x, inp.gamma, inp.eps, wg, wu, "row", h=h)
+        group.down_proj_allreduce(h, wd, y=y)
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.phase = "timed"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks.phase = "extra"
+    clocks.stop()
+    t_max = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, "cuda")
+    err = dfk.dfk_device_error()
+    group.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    value = step_bytes(B1, D, F) * args.steps / (t_max / 1e3) / 1e9
+    return {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(config_dict("tp%d" % world),
+                           step="per rank: fused RMSNorm+gate/up on its d_ff shard, then the "
+                                "down projection with the all-reduce fused in"),
+            "gpu_launches": 2 * args.steps, "clocks": clocks.summary("timed"),
+            "device_error_word": err}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -903,12 +980,18 @@ def main():
     ap.add_argument("--layout", default="row", help="weight layout for --profile")
     ap.add_argument("--variant", type=int, default=0,
                     help="variant id for --profile (0 = the scheduler's choice)")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor-parallel layer over the torchrun ranks (d_ff sharded, the "
+                         "all-reduce fused into the down projection) instead of replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.profile:
         return profile_arm(args)
-    line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
+    if args.tp and args.impl != "reference":
+        line = tp_arm(args)
+    else:
+        line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

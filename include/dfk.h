@@ -287,6 +287,67 @@ DFK_API int dfk_variant_info(int variant_id, dfk_variant *out);
 /* Forget every cached scheduler decision (all devices). */
 DFK_API void dfk_clear_variant_cache(void);
 
+/* ---- tensor-parallel MLP ---------------------------------------------------
+ * "Deep Kernel Fusion for Transformers" (abstract) keeps the fused kernel
+ * adaptable to inference configurations; on several GPUs the MLP shards
+ * d_ff: rank r holds rows [f0_r, f1_r) of W_gate and W_up (whole gate/up
+ * pairs, so the fused gate/up kernel runs unchanged on the shard and needs
+ * no communication) and columns [f0_r, f1_r) of W_down, stored as its own
+ * contiguous [d_model][f1_r - f0_r] matrix.  Each rank computes a partial
+ * y_r = h_r . W_down_r^T; the full y is the sum over ranks.  The down
+ * projection below does that sum inside the kernel: each CTA writes its
+ * fp32 partial rows into every rank's receive buffer with plain stores to
+ * peer memory (NVLink), raises a flag there, waits (bounded by the device's
+ * wait limit) for every rank's flag of its rows, and adds the ranks'
+ * partials in rank order 0, 1, ... -- so every rank computes the same bits
+ * of bf16 y.  No library collective and no multicast load is involved.
+ *
+ * One process per GPU.  Setup, on every rank with its device current:
+ *   dfk_tp_group_create(world, rank, max_B, d_model, &g, handle)
+ *       allocates this rank's buffer (2 x world x max_B x d_model fp32 plus
+ *       flags; zeroed) and writes its CUDA IPC handle into `handle`
+ *       (DFK_TP_HANDLE_BYTES bytes, host memory);
+ *   exchange the handles (e.g. an all-gather over torch.distributed);
+ *   dfk_tp_group_connect(g, handles)  -- `handles` = world handles in rank
+ *       order (host memory); maps every peer's buffer.
+ * Then dfk_tp_down_proj_allreduce on every rank, in the same order of calls
+ * on all ranks (a call waits for the same call on the other ranks; each
+ * rank counts its calls on the device, so the call can be captured in a
+ * CUDA graph).  h [B][d_ff_shard] and w_down_shard [d_model][d_ff_shard]
+ * are this rank's, y [B][d_model] receives the full result; B <= max_B,
+ * d_ff_shard % 8 == 0 (may differ between ranks), d_model as created.  If a
+ * peer never arrives the wait gives up after the wait limit, y is not
+ * written and dfk_device_error reports DFK_ERR_TIMEOUT.
+ * dfk_tp_group_destroy synchronises the device and frees the buffer.
+ * world = 1 is valid (no peers).
+ */
+#define DFK_TP_HANDLE_BYTES 64
+typedef struct dfk_tp_group dfk_tp_group;
+
+DFK_API int dfk_tp_group_create(int world, int rank, int max_B, int d_model,
+                                dfk_tp_group **group, void *handle);
+DFK_API int dfk_tp_group_connect(dfk_tp_group *group, const void *handles);
+DFK_API int dfk_tp_down_proj_allreduce(dfk_tp_group *group, const void *h,
+                                       const void *w_down_shard, void *y, int B, int d_model,
+                                       int d_ff_shard, void *stream);
+DFK_API int dfk_tp_group_destroy(dfk_tp_group *group);
+
+/*
+ * The same fused down projection and all-reduce for a group of `world`
+ * ranks emulated on the current device: one cooperative grid computes every
+ * rank's shard (its CTAs wait on one another's flags, so all of them must be
+ * resident at once; shapes needing more CTAs than that are rejected with
+ * DFK_ERR_UNSUPPORTED_SHAPE).  Runs the kernel code of the multi-GPU call on
+ * one GPU.  h_all [world][B][d_ff_shard], w_all [world][d_model][d_ff_shard]
+ * (rank r's shard at index r; equal shard sizes), y_all [world][B][d_model]
+ * (every rank's copy of y).  The buffers for the emulated ranks are
+ * allocated by the library on the first call per (device, world, d_model),
+ * which must not be made during stream capture.
+ */
+DFK_API int dfk_tp_down_proj_allreduce_emulated(int world, const void *h_all,
+                                                const void *w_all, void *y_all, int B,
+                                                int d_model, int d_ff_shard, void *stream);
+
 /* ---- building blocks of the unfused baseline and of the decode stack -------
  * These exist to measure what the fusion saves (separate RMSNorm, GEMV,
  * SiLU and multiply kernels with bf16 intermediates in HBM) and to run a

@@ -62,6 +62,8 @@ EXPORTED = (
     "dfk_gemv", "dfk_silu", "dfk_mul", "dfk_rms_rescale", "dfk_mlp_forward_host",
     "dfk_status_string", "dfk_last_error", "dfk_device_error", "dfk_version",
     "dfk_set_wait_limit", "dfk_selftest_bounded_wait",
+    "dfk_tp_group_create", "dfk_tp_group_connect", "dfk_tp_down_proj_allreduce",
+    "dfk_tp_group_destroy", "dfk_tp_down_proj_allreduce_emulated",
 )
 
 
@@ -126,6 +128,11 @@ def lib():
                 "dfk_device_error": [ctypes.POINTER(i)],
                 "dfk_set_wait_limit": [ctypes.c_ulonglong],
                 "dfk_selftest_bounded_wait": [vp, vp],
+                "dfk_tp_group_create": [i, i, i, i, ctypes.POINTER(vp), vp],
+                "dfk_tp_group_connect": [vp, vp],
+                "dfk_tp_down_proj_allreduce": [vp, vp, vp, vp, i, i, i, vp],
+                "dfk_tp_group_destroy": [vp],
+                "dfk_tp_down_proj_allreduce_emulated": [i, vp, vp, vp, i, i, i, vp],
                 "dfk_status_string": [i],
                 "dfk_last_error": [],
                 "dfk_version": [],
@@ -477,3 +484,48 @@ def dfk_selftest_bounded_wait(elapsed_ns=None, stream=None):
 
 def dfk_version():
     return lib().dfk_version().decode()
+
+
+# ---- tensor-parallel down projection (see swiglu_mlp_dfk_b200.tp for the MLP)
+
+DFK_TP_HANDLE_BYTES = 64
+
+
+def dfk_tp_group_create(world, rank, max_B, d_model):
+    """Returns (group handle, this rank's IPC handle as bytes)."""
+    g = ctypes.c_void_p()
+    hb = ctypes.create_string_buffer(DFK_TP_HANDLE_BYTES)
+    _check(lib().dfk_tp_group_create(int(world), int(rank), int(max_B), int(d_model),
+                                     ctypes.byref(g), hb))
+    return g, hb.raw
+
+
+def dfk_tp_group_connect(group, handles):
+    """handles: every rank's IPC handle (bytes), in rank order."""
+    blob = b"".join(handles)
+    _check(lib().dfk_tp_group_connect(group, ctypes.create_string_buffer(blob, len(blob))))
+
+
+def dfk_tp_down_proj_allreduce(group, h, w_down_shard, y=None, stream=None):
+    B, F = h.shape
+    D = w_down_shard.shape[0]
+    if y is None:
+        y = torch.empty(B, D, dtype=torch.bfloat16, device=h.device)
+    _check(lib().dfk_tp_down_proj_allreduce(group, _ptr(h), _ptr(w_down_shard), _ptr(y), B, D,
+                                            F, _stream(stream)))
+    return y
+
+
+def dfk_tp_group_destroy(group):
+    _check(lib().dfk_tp_group_destroy(group))
+
+
+def dfk_tp_down_proj_allreduce_emulated(h_all, w_all, y_all=None, stream=None):
+    """h_all [world][B][F_shard], w_all [world][D][F_shard] -> y_all [world][B][D]."""
+    P, B, F = h_all.shape
+    D = w_all.shape[1]
+    if y_all is None:
+        y_all = torch.empty(P, B, D, dtype=torch.bfloat16, device=h_all.device)
+    _check(lib().dfk_tp_down_proj_allreduce_emulated(P, _ptr(h_all), _ptr(w_all), _ptr(y_all),
+                                                     B, D, F, _stream(stream)))
+    return y_all

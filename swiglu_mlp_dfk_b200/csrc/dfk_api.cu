@@ -36,6 +36,7 @@
 #include "tf8_engine.cuh"
 #include "tf8_key.h"
 #include "tf8mma_engine.cuh"
+#include "tp_internal.h"
 
 // Device status block: word 0 = error bits (bit 0 = a pipeline wait in some
 // kernel gave up, bit 1 = a bounds check of the checked build failed),
@@ -919,6 +920,90 @@ int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, in
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_fail(e, "tensor-core kernel launch");
+  }
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- tensor parallel
+
+int report_error(int status, const char *msg) { return fail(status, "%s", msg); }
+
+TpLayout tp_layout(int world, int bmax, int d_model) {
+  TpLayout l;
+  l.recv_bytes = static_cast<size_t>(2) * world * bmax * d_model * sizeof(float);
+  l.flags_off = (l.recv_bytes + 255) & ~static_cast<size_t>(255);
+  l.seq_off = l.flags_off + static_cast<size_t>(TP_MAX_BLOCKS) * world * 8;
+  l.exit_off = l.seq_off + 8;
+  l.total = (l.exit_off + 8 + 255) & ~static_cast<size_t>(255);
+  return l;
+}
+
+// The tensor-parallel down projection with the all-reduce fused in: the
+// tensor-core GEMV (no split-K, one CTA per SM over this rank's rows) whose
+// epilogue exchanges the fp32 partial sums (tc_engine.cuh, tp_* fields).
+int launch_tp_down(const TpLaunch &a, cudaStream_t s) {
+  if (a.world < 1 || a.world > TP_MAX_RANKS || a.ranks_here < 1 || a.rank0 < 0 ||
+      a.rank0 + a.ranks_here > a.world)
+    return fail(DFK_ERR_INVALID_ARG, "bad tensor-parallel group (world %d)", a.world);
+  int rc = check_gemv(a.h, a.w, a.y, a.B, a.d_ff_shard, a.d_model, 0);
+  if (rc || a.B == 0) return rc;
+  if (a.B > a.bmax)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "B=%d exceeds the group's capacity %d", a.B, a.bmax);
+  DeviceState *ds;
+  int dev;
+  if ((rc = current_device(&ds, &dev))) return rc;
+  DeviceState sub = *ds;
+  sub.sms = ds->sms / a.ranks_here;
+  const VDef *v = nullptr;
+  for (const VDef &d : variants())
+    if (d.cls == CLS_GEMV && d.family == DFK_FAMILY_TENSOR_CORE && bf16_capable(d) &&
+        d.ksplit == 1 && d.nt == 2 && d.full == 0)
+      v = &d;
+  TcPlan pl;
+  std::string why;
+  if (!v || !plan_tc(LAYOUT_ROW, 1, false, *v, a.B, a.d_ff_shard, a.d_model, sub, &pl, &why))
+    return fail(DFK_ERR_NO_VARIANT, "no tensor-parallel plan for B=%d d_model=%d shard=%d: %s",
+                a.B, a.d_model, a.d_ff_shard, why.c_str());
+  if (pl.grid > sub.sms || pl.grid > TP_MAX_BLOCKS || pl.p.kslices != 1)
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "d_model=%d needs %d row blocks per rank; at most %d "
+                "fit (one co-resident CTA per block)", a.d_model, pl.grid,
+                std::min(sub.sms, TP_MAX_BLOCKS));
+  if ((rc = ensure_smem_attr(dev, pl.fn))) return rc;
+  TcMaps maps;
+  memset(&maps, 0, sizeof maps);
+  const uint64_t rows = static_cast<uint64_t>(a.ranks_here) * a.d_model;
+  for (int lo = 0; lo < 2; ++lo) {
+    const uint32_t hgt = static_cast<uint32_t>(std::max(1, pl.p.hmax - lo));
+    if ((rc = tensor_map_2d(a.w, a.d_ff_shard, rows, static_cast<uint64_t>(a.d_ff_shard) * 2,
+                            TC_TILE_K, hgt, &maps.wg[lo], true)))
+      return rc;
+  }
+  if ((rc = tensor_map_2d(a.h, a.d_ff_shard, static_cast<uint64_t>(a.ranks_here) * a.B,
+                          static_cast<uint64_t>(a.d_ff_shard) * 2, TC_TILE_K, pl.p.bn, &maps.x,
+                          true)))
+    return rc;
+  TcParams p = pl.p;
+  p.out = static_cast<uint16_t *>(a.y);
+  p.err = ds->err;
+  p.tp_world = a.world;
+  p.tp_rank0 = a.rank0;
+  p.tp_blocks = pl.grid;
+  p.tp_bmax = a.bmax;
+  const TpLayout L = tp_layout(a.world, a.bmax, a.d_model);
+  for (int r = 0; r < a.world; ++r) {
+    char *b = static_cast<char *>(a.buf[r]);
+    if (!b) return fail(DFK_ERR_INVALID_ARG, "rank %d's buffer is not connected", r);
+    p.tp_recv[r] = reinterpret_cast<float *>(b);
+    p.tp_flags[r] = reinterpret_cast<unsigned long long *>(b + L.flags_off);
+  }
+  p.tp_seq = reinterpret_cast<unsigned long long *>(static_cast<char *>(a.ctl) + L.seq_off);
+  p.tp_exit = reinterpret_cast<unsigned *>(static_cast<char *>(a.ctl) + L.exit_off);
+  void *args[] = {&maps, &p};
+  cudaError_t e = launch_kernel(pl.fn, dim3(pl.grid * a.ranks_here), dim3(TC_THREADS), pl.smem,
+                                s, pdl_enabled() && !a.cooperative, args, 1, a.cooperative);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "tensor-parallel down projection launch");
   }
   return DFK_OK;
 }

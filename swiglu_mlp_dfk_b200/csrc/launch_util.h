@@ -10,16 +10,23 @@ namespace dfk {
 // previous kernel writes, so this only overlaps their prologues.
 // `cluster_x` > 1 groups that many consecutive blocks along x into a
 // thread-block cluster (portable sizes: at most 8).
+// `cooperative`: every block of the grid is resident at once (the launch
+// fails otherwise); for grids whose blocks wait on one another.
 inline cudaError_t launch_kernel(const void *fn, dim3 grid, dim3 block, size_t smem,
                                  cudaStream_t stream, bool pdl, void **args,
-                                 unsigned cluster_x = 1) {
+                                 unsigned cluster_x = 1, bool cooperative = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   unsigned n = 0;
+  if (cooperative) {
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
   if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;

@@ -94,6 +94,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// System-scope release store / acquire load of a 64-bit flag (peer memory
+// over NVLink included).
+__device__ __forceinline__ void st_release_sys_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_sys_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until each of the n flags fl[0 .. n) holds a value >= want.  Bounded
+// like mbar_wait_bounded: gives up when *abort_flag becomes non-zero or after
+// the device's wait limit (then sets *abort_flag and the error word).
+__device__ __forceinline__ bool flags_wait_bounded(const unsigned long long *fl, int n,
+                                                   unsigned long long want,
+                                                   volatile int *abort_flag, unsigned *err) {
+  const unsigned long long t0 = global_timer_ns();
+  const unsigned long long limit = wait_limit_ns(err);
+  for (int s = 0; s < n; ++s) {
+    for (uint32_t it = 1; ld_acquire_sys_u64(fl + s) < want; ++it) {
+      if ((it & 15u) == 0) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit || it > (1u << 30)) {
+          *abort_flag = 1;
+          if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
+          return false;
+        }
+      }
+      __nanosleep(32);
+    }
+  }
+  return true;
+}
+
 // Bulk tensor copy global -> shared, 2-D tile, completion counted on `bar`.
 // The innermost coordinate c0 times the element size must be a multiple of
 // 16 bytes (callers pass multiples of 8 bf16 elements).

@@ -48,6 +48,7 @@ namespace dfk {
 constexpr int TC_THREADS = 192;
 constexpr int TC_TILE_K = 64;       // reduction elements per k-tile (one 128-byte swizzle row)
 constexpr int TC_ATOM = 1024;       // bytes of an 8-row swizzle atom
+constexpr int TP_MAX = 8;           // ranks of a tensor-parallel group
 
 struct TcParams {
   uint16_t *out;          // [B][N] bf16
@@ -82,6 +83,24 @@ struct TcParams {
   int full;               // 1: every CTA owns 128 rows (the last one fewer); boxes of 128 rows
   int pf_steps;           // ring steps after the first fill whose weight boxes are prefetched
                           // into L2 before the wait on the previous kernel
+  // Tensor-parallel down projection with the all-reduce fused in (GEMV,
+  // no split-K; tp_world = 0: off).  The reduction dimension is sharded over
+  // tp_world ranks; this grid computes the shards of ranks tp_rank0 ..
+  // tp_rank0 + (grid / tp_blocks) - 1 (one rank on a multi-GPU run; all of
+  // them when the ranks are emulated on one device), tp_blocks row blocks
+  // each.  Rank r's weights are rows r * N .. of the weight map and its
+  // activations rows r * B .. of the activation map.  Each CTA writes its
+  // fp32 partial rows into every rank's receive buffer, raises its flag
+  // there, waits (bounded) for every rank's flag of its row block, adds the
+  // ranks' partials in rank order and stores bf16 y of its own rank.
+  int tp_world;
+  int tp_rank0;
+  int tp_blocks;
+  float *tp_recv[TP_MAX];               // per rank: [2][tp_world][tp_bmax][N] fp32
+  unsigned long long *tp_flags[TP_MAX]; // per rank: [row blocks][tp_world]
+  unsigned long long *tp_seq;           // this grid's call counter (calls completed)
+  unsigned *tp_exit;                    // CTAs of this grid that finished (0 between calls)
+  int tp_bmax;                          // token capacity of the receive buffers
 };
 
 // wg/wu: [0] box height hmax, [1] box height hmax - 1; x: activations box {64, bn}.
@@ -170,7 +189,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // ---- this CTA's rows [j0, j0 + r), cut into MT sub-tiles, and its
   // reduction range: k-tiles [tile0, tile1)
   const int cta = blockIdx.x;
-  const int blk = cta / p.kslices, slc = cta - blk * p.kslices;
+  int blk = cta / p.kslices;
+  const int slc = cta - blk * p.kslices;
+  // tensor-parallel: this CTA computes rank tp_rank0 + tpl's shard; its rows
+  // and activations sit at these offsets of the (stacked) maps
+  const int tpl = (NMAT == 1 && p.tp_world) ? blk / p.tp_blocks : 0;
+  blk -= tpl * p.tp_blocks;
+  const int wrow = tpl * p.N, xrow = tpl * p.B;
   const int j0 = blk * p.rbase + min(blk, p.rextra);
   const bool full = COLM || p.full;  // 128-row boxes, zero-filled past the last row
   const int r = full ? min(p.rbase, p.N - j0) : p.rbase + (blk < p.rextra ? 1 : 0);
@@ -239,7 +264,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (i >= S0) {
             const int tl = tile0 + i * NT + kt;
             tma_load_2d(sb + p.a_bytes + kt * p.xt_bytes, &maps.x, xbar,
-                        NORM == 2 ? 0 : k0, NORM == 2 ? tl * 2 * BN : 0, pol_x);
+                        NORM == 2 ? 0 : k0, NORM == 2 ? tl * 2 * BN : xrow, pol_x);
           }
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
@@ -255,7 +280,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 tma_load_2d(dst, wm, &fullb[st], j0, k0, pol_w);
                 tma_load_2d(dst + 8192, wm, &fullb[st], j0 + 64, k0, pol_w);
               } else {
-                tma_load_2d(dst, wm, &fullb[st], k0, j0 + rs[t], pol_w);
+                tma_load_2d(dst, wm, &fullb[st], k0, wrow + j0 + rs[t], pol_w);
               }
             }
           }
@@ -280,7 +305,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     tma_prefetch_2d(wm, j0, k0);
                     tma_prefetch_2d(wm, j0 + 64, k0);
                   } else {
-                    tma_prefetch_2d(wm, k0, j0 + rs[t]);
+                    tma_prefetch_2d(wm, k0, wrow + j0 + rs[t]);
                   }
                 }
               }
@@ -295,7 +320,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                               kt * p.xt_bytes,
                           &maps.x, NORM == 1 ? &xfull[ii] : &fullb[ii],
                           NORM == 2 ? 0 : tl * TC_TILE_K,
-                          NORM == 2 ? tl * 2 * BN : 0, pol_x);
+                          NORM == 2 ? tl * 2 * BN : xrow, pol_x);
             }
           }
         }
@@ -447,6 +472,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const bool go = __all_sync(0xffffffffu, ok && !*s_abort);
     const int q = warp & 3;               // TMEM lanes 32q .. 32q + 31 belong to this warp
     const int row = 32 * q + lane;
+    const bool tp = NMAT == 1 && p.tp_world > 0;
+    const int tp_src = p.tp_rank0 + tpl;  // this CTA's rank
+    unsigned long long tp_seq = 0;
+    int tp_set = 0;
+    if (tp) {
+      // the previous call's counter update is visible once the grids before
+      // this one have completed
+      pdl_wait();
+      tp_seq = *reinterpret_cast<volatile unsigned long long *>(p.tp_seq) + 1;
+      tp_set = static_cast<int>(tp_seq & 1);
+    }
     if (go) {
       const int NB = p.nbank;
 #pragma unroll
@@ -464,6 +500,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             float *mine = p.part + (static_cast<size_t>(slc) * p.nblocks + blk) * BN * 128;
 #pragma unroll
             for (int e = 0; e < 16; ++e) mine[(c + e) * 128 + row] = g[e];
+          } else if (tp) {
+            // tensor-parallel: this rank's fp32 partial rows into slot tp_src
+            // of every rank's receive buffer (peer stores over NVLink)
+            if (row < h[t]) {
+              const int j = j0 + rs[t] + row;
+              for (int d = 0; d < p.tp_world; ++d) {
+                float *dst = p.tp_recv[d] +
+                             (static_cast<size_t>(tp_set * p.tp_world + tp_src) * p.tp_bmax) * p.N +
+                             j;
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  if (c + e < p.B) dst[static_cast<size_t>(c + e) * p.N] = g[e];
+              }
+            }
           } else if (row < h[t]) {
             const int j = j0 + rs[t] + row;
 #pragma unroll
@@ -506,6 +556,52 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             });
         named_barrier(2, 128);
         if (et == 0) p.counters[blk] = 0u;
+      }
+    }
+    if (tp) {
+      // publish: every thread's partial rows are visible system-wide before
+      // this CTA's flag is raised in each rank's flag array
+      __threadfence_system();
+      named_barrier(2, 128);
+      if (et == 0 && go) {
+        for (int d = 0; d < p.tp_world; ++d)
+          st_release_sys_u64(p.tp_flags[d] + static_cast<size_t>(blk) * p.tp_world + tp_src,
+                             tp_seq);
+        // every rank's partial of this row block has arrived (bounded wait)
+        flags_wait_bounded(p.tp_flags[tp_src] + static_cast<size_t>(blk) * p.tp_world,
+                           p.tp_world, tp_seq, s_abort, p.err);
+      }
+      named_barrier(2, 128);
+      if (go && !*s_abort) {
+        // y = the ranks' partial sums added in rank order 0, 1, ..., the same
+        // order (and so the same bits) on every rank
+        const float *src = p.tp_recv[tp_src] +
+                           static_cast<size_t>(tp_set) * p.tp_world * p.tp_bmax * p.N;
+        uint16_t *y = p.out + static_cast<size_t>(tpl) * p.B * p.N;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (row < h[t]) {
+            const int j = j0 + rs[t] + row;
+            for (int n = 0; n < p.B; ++n) {
+              const float *v = src + static_cast<size_t>(n) * p.N + j;
+              float acc = __ldcg(v);
+              for (int r = 1; r < p.tp_world; ++r)
+                acc = acc + __ldcg(v + static_cast<size_t>(r) * p.tp_bmax * p.N);
+              y[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(acc);
+            }
+          }
+        }
+      }
+      // the grid's last CTA to get here advances the call counter (every CTA
+      // has read it above) and re-arms the exit count
+      named_barrier(2, 128);
+      if (et == 0) {
+        __threadfence();
+        if (atomicAdd(p.tp_exit, 1u) == gridDim.x - 1) {
+          *reinterpret_cast<volatile unsigned long long *>(p.tp_seq) = tp_seq;
+          *reinterpret_cast<volatile unsigned *>(p.tp_exit) = 0u;
+          __threadfence();
+        }
       }
     }
     tc_fence_before();
