@@ -287,6 +287,45 @@ DFK_API int dfk_variant_info(int variant_id, dfk_variant *out);
 /* Forget every cached scheduler decision (all devices). */
 DFK_API void dfk_clear_variant_cache(void);
 
+/* ---- one decode step of a layer stack in one launch ------------------------
+ * The FlashFormer abstract (paper-listing page) puts a whole model's decode
+ * step into one kernel for low-batch inference; here that is applied to a
+ * stack of the fused MLP layers.  dfk_mlp_stack_step runs, in ONE persistent
+ * kernel (one CTA per SM, a cooperative launch), for l = 0 .. layers-1:
+ *   h_l = SiLU(xn_l . W_gate_l^T) (*) (xn_l . W_up_l^T),
+ *         xn_l = RMSNorm(x_l; gamma_l, eps)      (as dfk_rmsnorm_swiglu_gate_up)
+ *   y_l = h_l . W_down_l^T                       (as dfk_down_proj)
+ *   x_{l+1} = y_l,   x_0 = x
+ * and then x := y_{L-1} / sqrt(mean(y_{L-1}^2) + eps) per row (as
+ * dfk_rms_rescale), in place, ready for the next step.  The weight stream
+ * never stops at a layer boundary: each SM's producer streams the next
+ * phase's weights while the previous phase finishes on the other SMs.
+ *   gammas    [layers][d_model] bf16
+ *   w_gate    [layers][d_ff][d_model] bf16 row-major (one allocation)
+ *   w_up      [layers][d_ff][d_model]
+ *   w_down    [layers][d_model][d_ff]
+ *   x         [B][d_model] bf16, read and overwritten with the next input
+ *   h_all     [layers][B][d_ff] bf16, every layer's h (written)
+ *   y_all     [layers][B][d_model] bf16, every layer's y (written)
+ *   workspace dfk_mlp_stack_workspace_bytes(...) bytes of device memory,
+ *             zeroed by the caller once before the first call and then
+ *             left to the library (it holds the grid's phase counters);
+ *             after a call that reported DFK_ERR_TIMEOUT, zero it again
+ * The arithmetic is that of the separate kernels with the tensor-core
+ * gate/up (in-kernel RMSNorm, 16 token slots) and the four-slice split-K
+ * tensor-core down projection, so one call gives the same bits as those
+ * 2 x layers + 1 launches.  Constraints: 1 <= B <= 16; d_model, d_ff
+ * multiples of 8; d_ff <= 128 rows per SM, d_model <= 128 rows per four
+ * SMs (the Llama-3-8B shape fits); DFK_ERR_UNSUPPORTED_SHAPE otherwise.
+ * Calls on one workspace must not overlap on the GPU.  No allocation, so
+ * the call can be captured in a CUDA graph.
+ */
+DFK_API long long dfk_mlp_stack_workspace_bytes(int layers, int B, int d_model, int d_ff);
+DFK_API int dfk_mlp_stack_step(const void *gammas, float eps, const void *w_gate,
+                               const void *w_up, const void *w_down, void *x, void *h_all,
+                               void *y_all, void *workspace, long long workspace_bytes,
+                               int layers, int B, int d_model, int d_ff, void *stream);
+
 /* ---- tensor-parallel MLP ---------------------------------------------------
  * "Deep Kernel Fusion for Transformers" (abstract) keeps the fused kernel
  * adaptable to inference configurations; on several GPUs the MLP shards

@@ -64,6 +64,7 @@ EXPORTED = (
     "dfk_set_wait_limit", "dfk_selftest_bounded_wait",
     "dfk_tp_group_create", "dfk_tp_group_connect", "dfk_tp_down_proj_allreduce",
     "dfk_tp_group_destroy", "dfk_tp_down_proj_allreduce_emulated",
+    "dfk_mlp_stack_workspace_bytes", "dfk_mlp_stack_step",
 )
 
 
@@ -133,6 +134,7 @@ def lib():
                 "dfk_tp_down_proj_allreduce": [vp, vp, vp, vp, i, i, i, vp],
                 "dfk_tp_group_destroy": [vp],
                 "dfk_tp_down_proj_allreduce_emulated": [i, vp, vp, vp, i, i, i, vp],
+                "dfk_mlp_stack_step": [vp, f, vp, vp, vp, vp, vp, vp, vp, ll, i, i, i, i, vp],
                 "dfk_status_string": [i],
                 "dfk_last_error": [],
                 "dfk_version": [],
@@ -143,6 +145,8 @@ def lib():
                 fn.restype = i
             for name in ("dfk_status_string", "dfk_last_error", "dfk_version"):
                 getattr(L, name).restype = ctypes.c_char_p
+            L.dfk_mlp_stack_workspace_bytes.argtypes = [i, i, i, i]
+            L.dfk_mlp_stack_workspace_bytes.restype = ll
             L.dfk_clear_variant_cache.argtypes = []
             L.dfk_clear_variant_cache.restype = None
             _lib = L
@@ -529,3 +533,24 @@ def dfk_tp_down_proj_allreduce_emulated(h_all, w_all, y_all=None, stream=None):
     _check(lib().dfk_tp_down_proj_allreduce_emulated(P, _ptr(h_all), _ptr(w_all), _ptr(y_all),
                                                      B, D, F, _stream(stream)))
     return y_all
+
+
+# ---- one decode step of a layer stack in one persistent kernel
+
+def dfk_mlp_stack_workspace_bytes(layers, B, d_model, d_ff):
+    n = lib().dfk_mlp_stack_workspace_bytes(int(layers), int(B), int(d_model), int(d_ff))
+    if n < 0:
+        _check(DFK_ERR_UNSUPPORTED_SHAPE)
+    return n
+
+
+def dfk_mlp_stack_step(gammas, eps, w_gate, w_up, w_down, x, h_all, y_all, workspace,
+                       stream=None):
+    """gammas [L, D], w_gate / w_up [L, F, D], w_down [L, D, F], x [B, D] (updated in
+    place), h_all [L, B, F], y_all [L, B, D], workspace: uint8 device tensor."""
+    L, F, D = w_gate.shape
+    B = x.shape[0]
+    _check(lib().dfk_mlp_stack_step(_ptr(gammas), float(eps), _ptr(w_gate), _ptr(w_up),
+                                    _ptr(w_down), _ptr(x), _ptr(h_all), _ptr(y_all),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    L, B, D, F, _stream(stream)))

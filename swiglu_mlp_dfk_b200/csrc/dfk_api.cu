@@ -37,6 +37,7 @@
 #include "tf8_key.h"
 #include "tf8mma_engine.cuh"
 #include "tp_internal.h"
+#include "pstack_engine.cuh"
 
 // Device status block: word 0 = error bits (bit 0 = a pipeline wait in some
 // kernel gave up, bit 1 = a bounds check of the checked build failed),
@@ -924,6 +925,8 @@ int down_proj_with_scratch(const void *h, const void *w_down, void *y, int B, in
   return DFK_OK;
 }
 
+static bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
 // ---------------------------------------------------------------- tensor parallel
 
 int report_error(int status, const char *msg) { return fail(status, "%s", msg); }
@@ -1004,6 +1007,122 @@ int launch_tp_down(const TpLaunch &a, cudaStream_t s) {
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_fail(e, "tensor-parallel down projection launch");
+  }
+  return DFK_OK;
+}
+
+// ---------------------------------------------------------------- persistent decode step
+
+const void *pstack_fn();
+
+struct PsPlan {
+  PsParams p{};
+  size_t smem = 0;
+  size_t ws_ctl = 0, ws_part = 0;  // workspace: control words, then partial sums
+};
+
+// Partition and shared-memory plan of the persistent decode step
+// (pstack_engine.cuh) for an L-layer stack on a device with `sms` SMs.
+static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPlan *pl,
+                        std::string *why) {
+  auto no = [&](const char *m) {
+    if (why) *why = m;
+    return false;
+  };
+  if (L < 1 || B < 1 || B > PS_BN) return no("need L >= 1 and 1 <= B <= 16");
+  if (D % 8 || F % 8) return no("d_model and d_ff must be multiples of 8");
+  const int G = sms - sms % PS_KSPLIT;
+  if (G < PS_KSPLIT) return no("too few SMs");
+  PsParams &p = pl->p;
+  p = PsParams{};
+  p.L = L;
+  p.B = B;
+  p.D = D;
+  p.F = F;
+  p.gu_rbase = F / G;
+  p.gu_rextra = F % G;
+  p.gu_hmax = p.gu_rbase + (p.gu_rextra ? 1 : 0);
+  if (p.gu_rbase < 1 || p.gu_hmax > 128) return no("d_ff needs 1 .. 128 rows per SM");
+  p.gu_rc = round_up(p.gu_hmax, 8);
+  p.gu_tiles = ceil_div(D, PS_TILE_K);
+  p.dn_nblk = G / PS_KSPLIT;
+  p.dn_rbase = D / p.dn_nblk;
+  p.dn_rextra = D % p.dn_nblk;
+  p.dn_hmax = p.dn_rbase + (p.dn_rextra ? 1 : 0);
+  if (p.dn_rbase < 1 || p.dn_hmax > 128) return no("d_model needs 1 .. 128 rows per row block");
+  p.dn_rc = round_up(p.dn_hmax, 8);
+  p.dn_tiles = ceil_div(F, PS_TILE_K);
+  if (p.dn_tiles < PS_KSPLIT) return no("d_ff too short for four reduction slices");
+  p.slot_bytes = round_up(std::max(2 * p.gu_rc * 128, 2 * p.dn_rc * 128), 1024);
+  // an MMA reads 128 rows from each A tile start: keep the over-read of the
+  // last slot inside shared memory
+  const int slack = round_up(std::max(0, 16384 - std::min(p.gu_rc, p.dn_rc) * 128), 1024);
+  p.A = 8;
+  const int bar_bytes = (2 * 8 + 2 * p.A + 5) * 8 + 32 + PS_BN * 4;
+  const int fixed = 1024 /* alignment */ + slack + p.A * PS_ASTAGE + round_up(bar_bytes, 128);
+  p.S = std::min(8, (smem_cap - fixed) / p.slot_bytes);
+  if (p.S < 2) return no("the weight ring does not fit shared memory");
+  p.a_off = p.S * p.slot_bytes + slack;
+  p.bar_off = p.a_off + p.A * PS_ASTAGE;
+  pl->smem = 1024 + static_cast<size_t>(p.bar_off) + round_up(bar_bytes, 128);
+  pl->ws_ctl = round_up((2 + 2 * L + p.dn_nblk) * 4, 256);
+  pl->ws_part = static_cast<size_t>(PS_KSPLIT) * p.dn_nblk * PS_BN * 128 * sizeof(float);
+  return true;
+}
+
+static int pstack_step(const void *gamma, float eps, const void *wg, const void *wu,
+                       const void *wd, void *x, void *h_all, void *y_all, void *ws,
+                       size_t ws_bytes, int L, int B, int D, int F, cudaStream_t s) {
+  if (L < 1 || B < 0 || D <= 0 || F <= 0) return fail(DFK_ERR_INVALID_ARG, "bad sizes");
+  if (!(eps >= 0.f && std::isfinite(eps))) return fail(DFK_ERR_INVALID_ARG, "bad eps");
+  if (B == 0) return DFK_OK;
+  if (!gamma || !wg || !wu || !wd || !x || !h_all || !y_all || !ws)
+    return fail(DFK_ERR_INVALID_ARG, "null pointer argument");
+  if (misaligned(gamma) || misaligned(wg) || misaligned(wu) || misaligned(wd) ||
+      misaligned(x) || misaligned(h_all) || misaligned(y_all) || misaligned(ws))
+    return fail(DFK_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  DeviceState *ds;
+  int dev;
+  int rc = current_device(&ds, &dev);
+  if (rc) return rc;
+  PsPlan pl;
+  std::string why;
+  if (!plan_pstack(L, B, D, F, ds->sms, std::min(ds->smem_optin, 232448), &pl, &why))
+    return fail(DFK_ERR_UNSUPPORTED_SHAPE, "persistent decode step: %s", why.c_str());
+  if (ws_bytes < pl.ws_ctl + pl.ws_part)
+    return fail(DFK_ERR_INVALID_ARG, "workspace of %zu bytes; %zu needed", ws_bytes,
+                pl.ws_ctl + pl.ws_part);
+  const void *fn = pstack_fn();
+  if ((rc = ensure_smem_attr(dev, fn))) return rc;
+  PsMaps maps;
+  memset(&maps, 0, sizeof maps);
+  PsParams &p = pl.p;
+  for (int lo = 0; lo < 2; ++lo) {
+    const uint32_t gh = static_cast<uint32_t>(std::max(1, p.gu_hmax - lo));
+    const uint32_t dh = static_cast<uint32_t>(std::max(1, p.dn_hmax - lo));
+    if ((rc = tensor_map_2d(wg, D, static_cast<uint64_t>(L) * F, static_cast<uint64_t>(D) * 2,
+                            PS_TILE_K, gh, &maps.wg[lo], true)) ||
+        (rc = tensor_map_2d(wu, D, static_cast<uint64_t>(L) * F, static_cast<uint64_t>(D) * 2,
+                            PS_TILE_K, gh, &maps.wu[lo], true)) ||
+        (rc = tensor_map_2d(wd, F, static_cast<uint64_t>(L) * D, static_cast<uint64_t>(F) * 2,
+                            PS_TILE_K, dh, &maps.wd[lo], true)))
+      return rc;
+  }
+  p.gamma = static_cast<const uint16_t *>(gamma);
+  p.x = static_cast<uint16_t *>(x);
+  p.h = static_cast<uint16_t *>(h_all);
+  p.y = static_cast<uint16_t *>(y_all);
+  p.ctl = static_cast<unsigned *>(ws);
+  p.part = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.ws_ctl);
+  p.err = ds->err;
+  p.eps = eps;
+  void *args[] = {&maps, &p};
+  const int G = ds->sms - ds->sms % PS_KSPLIT;
+  cudaError_t e = launch_kernel(fn, dim3(G), dim3(PS_THREADS), pl.smem, s, false, args, 1,
+                                /*cooperative=*/true);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "persistent decode-step launch");
   }
   return DFK_OK;
 }
@@ -1782,7 +1901,6 @@ static int resolve(int op, int variant, const CcCall &c, cudaStream_t s, const V
 
 // ---------------------------------------------------------------- validation
 
-static bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 static int check_gate_up(const void *x, const void *gamma, bool norm, float eps, const void *wg,
                          const void *wu, int layout, const void *h, int B, int D, int F,
@@ -2125,6 +2243,29 @@ int dfk_cached_variant(int op, int B, int d_model, int d_ff, int layout, dfk_var
   if (it == g_tuned.end()) return fail(DFK_ERR_NO_VARIANT, "no cached decision for this shape");
   *out = it->second;
   return DFK_OK;
+}
+
+long long dfk_mlp_stack_workspace_bytes(int layers, int B, int d_model, int d_ff) {
+  DeviceState *ds;
+  if (dfk::current_device(&ds)) return -1;
+  dfk::PsPlan pl;
+  std::string why;
+  if (!dfk::plan_pstack(layers, B, d_model, d_ff, ds->sms, std::min(ds->smem_optin, 232448),
+                        &pl, &why)) {
+    dfk::fail(DFK_ERR_UNSUPPORTED_SHAPE, "persistent decode step: %s", why.c_str());
+    return -1;
+  }
+  return static_cast<long long>(pl.ws_ctl + pl.ws_part);
+}
+
+int dfk_mlp_stack_step(const void *gammas, float eps, const void *w_gate, const void *w_up,
+                       const void *w_down, void *x, void *h_all, void *y_all, void *workspace,
+                       long long workspace_bytes, int layers, int B, int d_model, int d_ff,
+                       void *stream) {
+  if (workspace_bytes < 0) return dfk::fail(DFK_ERR_INVALID_ARG, "negative workspace size");
+  return dfk::pstack_step(gammas, eps, w_gate, w_up, w_down, x, h_all, y_all, workspace,
+                          static_cast<size_t>(workspace_bytes), layers, B, d_model, d_ff,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int dfk_variant_count(void) { return static_cast<int>(variants().size()); }

@@ -250,3 +250,78 @@ class DecodeStack:
         per_layer = (2 * F * D * 2 + B * D * 2 + D * 2 + B * F * 2      # fused gate/up
                      + D * F * 2 + B * F * 2 + B * D * 2)               # down projection
         return len(self.layers) * per_layer + 2 * B * D * 2             # + rescale
+
+
+class PersistentDecodeStack:
+    """The fused bf16 decode step of ``DecodeStack`` (row-major weights) as
+    ONE kernel launch per step (``dfk_mlp_stack_step``): a persistent kernel
+    whose per-SM producers stream the weights of every layer's gate/up and
+    down projection back to back, with grid-wide counters between the
+    phases instead of kernel boundaries.
+
+    layers: list of (gamma [D], W_gate [F, D], W_up [F, D], W_down [D, F]) bf16,
+            or ``stacked=(gammas [L, D], W_gate [L, F, D], W_up [L, F, D],
+            W_down [L, D, F])`` to use existing stacked tensors without a copy
+    x0:     [B, D] bf16 first-step input
+
+    After a step, ``h_all[l]`` and ``y_all[l]`` hold every layer's h and y and
+    ``x`` the next step's input.
+    """
+
+    def __init__(self, layers=None, x0=None, eps=1e-5, stacked=None):
+        if stacked is None:
+            stacked = tuple(torch.stack([lay[i] for lay in layers]).contiguous()
+                            for i in range(4))
+        self.gammas, self.wg, self.wu, self.wd = stacked
+        self.L, self.F, self.D = self.wg.shape
+        self.B = x0.shape[0]
+        self.eps = float(eps)
+        dev = x0.device
+        self.stream = torch.cuda.Stream(device=dev)
+        self.x = x0.clone()
+        self.h_all = torch.empty(self.L, self.B, self.F, dtype=torch.bfloat16, device=dev)
+        self.y_all = torch.empty(self.L, self.B, self.D, dtype=torch.bfloat16, device=dev)
+        n = dfk.dfk_mlp_stack_workspace_bytes(self.L, self.B, self.D, self.F)
+        self.workspace = torch.zeros(n, dtype=torch.uint8, device=dev)
+        self.graph = None
+
+    def _launch_step(self):
+        dfk.dfk_mlp_stack_step(self.gammas, self.eps, self.wg, self.wu, self.wd, self.x,
+                               self.h_all, self.y_all, self.workspace)
+
+    def step_eager(self):
+        cur = torch.cuda.current_stream(self.stream.device)
+        self.stream.wait_stream(cur)
+        with torch.cuda.stream(self.stream):
+            self._launch_step()
+        cur.wait_stream(self.stream)
+
+    def capture(self):
+        torch.cuda.synchronize(self.stream.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self._launch_step()
+        self.graph = g
+        return g
+
+    def step(self):
+        if self.graph is not None:
+            cur = torch.cuda.current_stream(self.stream.device)
+            self.stream.wait_stream(cur)
+            with torch.cuda.stream(self.stream):
+                self.graph.replay()
+            cur.wait_stream(self.stream)
+        else:
+            self.step_eager()
+
+    def release(self):
+        self.graph = None
+
+    def kernels_per_step(self):
+        return 1
+
+    def bytes_per_step(self):
+        B, D, F = self.B, self.D, self.F
+        per_layer = (2 * F * D * 2 + B * D * 2 + D * 2 + B * F * 2
+                     + D * F * 2 + B * F * 2 + B * D * 2)
+        return self.L * per_layer + 2 * B * D * 2
