@@ -21,7 +21,11 @@ import threading
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdfk.so")
+# DFK_CHECKED=1 selects the bounds-checked build of the same library (every
+# result store and activation load tests its index; failures are recorded in
+# the device status word, read by dfk_device_error)
+LIB_PATH = os.path.join(_PKG, "libdfk_checked.so" if os.environ.get("DFK_CHECKED") == "1"
+                        else "libdfk.so")
 
 # dfk_wlayout
 DFK_W_ROW_MAJOR = 0

@@ -8,6 +8,12 @@ SiLU uses the accurate expf and IEEE division), objects go to ``_build/`` and
 the shared library to ``swiglu_mlp_dfk_b200/libdfk.so``.  The CUDA runtime is
 linked statically and only the ``dfk_*`` C symbols are exported, so the
 library loads with or without PyTorch in the process.
+
+A second, checked build (``-DDFK_CHECKED``: every global store of a result
+and the activation loads test their index against the tensor's extent and
+record the first failure in the device status word instead of accessing
+memory) goes to ``_build/checked/`` and ``swiglu_mlp_dfk_b200/libdfk_checked.so``;
+the binding loads it when ``DFK_CHECKED=1`` is set.
 """
 import concurrent.futures as cf
 import os
@@ -20,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdfk.so")
+LIB_CHECKED = os.path.join(PKG, "libdfk_checked.so")
 
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -40,44 +47,54 @@ def _newest(paths):
     return max(os.path.getmtime(p) for p in paths)
 
 
-def _compile(src, force, hdr_time):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src, force, hdr_time, outdir, extra):
+    obj = os.path.join(outdir, os.path.basename(src)[:-3] + ".o")
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(
             os.path.getmtime(src), hdr_time):
         return obj, None
-    cmd = [NVCC] + CFLAGS + ["-c", src, "-o", obj]
+    cmd = [NVCC] + CFLAGS + extra + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         return obj, "%s\n%s%s" % (" ".join(cmd), r.stdout, r.stderr)
     return obj, None
 
 
-def build(force: bool = False, jobs: int = 0, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ and link libdfk.so; returns its path."""
-    os.makedirs(BUILD, exist_ok=True)
+def _build_one(lib, outdir, extra, force, jobs, verbose):
+    os.makedirs(outdir, exist_ok=True)
     srcs = sources()
     hdr_time = _newest(headers())
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(_newest(srcs), hdr_time)):
-        return LIB
+    if (not force and os.path.exists(lib)
+            and os.path.getmtime(lib) >= max(_newest(srcs), hdr_time)):
+        return lib
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     objs, errors = [], []
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        for obj, err in ex.map(lambda s: _compile(s, force, hdr_time), srcs):
+        for obj, err in ex.map(lambda s: _compile(s, force, hdr_time, outdir, extra), srcs):
             objs.append(obj)
             if err:
                 errors.append(err)
     if errors:
         raise RuntimeError("nvcc failed:\n" + "\n".join(errors))
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     cmd = [NVCC] + ARCH + ["-shared", "-Xcompiler", "-fvisibility=hidden", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s\n%s%s" % (" ".join(cmd), r.stdout, r.stderr))
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     if verbose:
-        print(LIB)
-    return LIB
+        print(lib)
+    return lib
+
+
+def build(force: bool = False, jobs: int = 0, verbose: bool = False,
+          checked: bool = True) -> str:
+    """Compile every .cu under csrc/ and link libdfk.so (and, with `checked`,
+    the bounds-checked libdfk_checked.so); returns the path of libdfk.so."""
+    lib = _build_one(LIB, BUILD, [], force, jobs, verbose)
+    if checked:
+        _build_one(LIB_CHECKED, os.path.join(BUILD, "checked"), ["-DDFK_CHECKED"], force, jobs,
+                   verbose)
+    return lib
 
 
 if __name__ == "__main__":

@@ -243,10 +243,11 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
             if (idx < nx) {
               const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
               if (b0 + bb < p.B && k < p.K)
-                v[u] = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
+                if (DFK_IN_BOUNDS(b0 + bb < p.B && k + 8 <= p.K, 2, p.err))
+                  v[u] = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
             } else if (idx < ntot) {
               const int k = (idx - nx) * 8;
-              if (k < p.K) v[u] = ld_nc_v4(p.gamma + k);
+              if (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 3, p.err)) v[u] = ld_nc_v4(p.gamma + k);
             }
           }
 #pragma unroll

@@ -824,6 +824,7 @@ static int launch_tc(const CcCall &c, const VDef &v, cudaStream_t s, int *stages
     pp.bn = p.bn;
     pp.ntiles = p.ntiles;
     pp.eps = c.eps;
+    pp.err = ds->err;
     void *pargs[] = {&pp};
     // one CTA per token slot
     cudaError_t e = launch_kernel(tc_norm_prep_fn(), dim3(p.bn), dim3(TC_PREP_THREADS), 0, s,
@@ -1053,17 +1054,23 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   p.dn_rc = round_up(p.dn_hmax, 8);
   p.dn_tiles = ceil_div(F, PS_TILE_K);
   if (p.dn_tiles < PS_KSPLIT) return no("d_ff too short for four reduction slices");
-  p.slot_bytes = round_up(std::max(2 * p.gu_rc * 128, 2 * p.dn_rc * 128), 1024);
+  // k tiles per ring step: 256 / 512 contiguous bytes of each weight row per
+  // step (the tensor-core kernels' tuned stage sizes for these phases)
+  p.gu_nt = 2;
+  p.dn_nt = 4;
+  p.slot_bytes = round_up(std::max(p.gu_nt * 2 * p.gu_rc * 128, p.dn_nt * p.dn_rc * 128), 1024);
   // an MMA reads 128 rows from each A tile start: keep the over-read of the
   // last slot inside shared memory
   const int slack = round_up(std::max(0, 16384 - std::min(p.gu_rc, p.dn_rc) * 128), 1024);
   p.A = 8;
-  const int bar_bytes = (2 * 8 + 2 * p.A + 5) * 8 + 32 + PS_BN * 4;
-  const int fixed = 1024 /* alignment */ + slack + p.A * PS_ASTAGE + round_up(bar_bytes, 128);
+  const int bar_bytes = (2 * 8 + 3 * p.A + 5) * 8 + 32 + PS_BN * 4;
+  const int fixed = 1024 /* alignment */ + slack + p.A * (PS_ASTAGE + 128) +
+                    round_up(bar_bytes, 128);
   p.S = std::min(8, (smem_cap - fixed) / p.slot_bytes);
   if (p.S < 2) return no("the weight ring does not fit shared memory");
   p.a_off = p.S * p.slot_bytes + slack;
-  p.bar_off = p.a_off + p.A * PS_ASTAGE;
+  p.g_off = p.a_off + p.A * PS_ASTAGE;
+  p.bar_off = p.g_off + p.A * 128;
   pl->smem = 1024 + static_cast<size_t>(p.bar_off) + round_up(bar_bytes, 128);
   pl->ws_ctl = round_up((2 + 2 * L + p.dn_nblk) * 4, 256);
   pl->ws_part = static_cast<size_t>(PS_KSPLIT) * p.dn_nblk * PS_BN * 128 * sizeof(float);
@@ -1108,6 +1115,17 @@ static int pstack_step(const void *gamma, float eps, const void *wg, const void 
                             PS_TILE_K, dh, &maps.wd[lo], true)))
       return rc;
   }
+  // activations (16-row boxes: rows past a layer's B tokens feed ignored MMA
+  // columns) and the gammas
+  if ((rc = tensor_map_2d(x, D, B, static_cast<uint64_t>(D) * 2, PS_TILE_K, PS_BN, &maps.x,
+                          true)) ||
+      (rc = tensor_map_2d(y_all, D, static_cast<uint64_t>(L) * B, static_cast<uint64_t>(D) * 2,
+                          PS_TILE_K, PS_BN, &maps.y, true)) ||
+      (rc = tensor_map_2d(h_all, F, static_cast<uint64_t>(L) * B, static_cast<uint64_t>(F) * 2,
+                          PS_TILE_K, PS_BN, &maps.h, true)) ||
+      (rc = tensor_map_2d(gamma, D, L, static_cast<uint64_t>(D) * 2, PS_TILE_K, 1, &maps.gam,
+                          false)))
+    return rc;
   p.gamma = static_cast<const uint16_t *>(gamma);
   p.x = static_cast<uint16_t *>(x);
   p.h = static_cast<uint16_t *>(h_all);
@@ -1479,6 +1497,7 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
     pp.T = p.T;
     pp.ntiles = p.ntiles;
     pp.eps = c.eps;
+    pp.err = ds->err;
     void *pargs[] = {&pp};
     // one CTA per token slot
     e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
@@ -2534,6 +2553,7 @@ const char *dfk_status_string(int status) {
     case DFK_ERR_ARCH: return "no sm_100 device";
     case DFK_ERR_TIMEOUT: return "device pipeline wait timed out";
     case DFK_ERR_NO_VARIANT: return "no variant fits this shape";
+    case DFK_ERR_BOUNDS: return "a kernel's bounds check failed";
     default: return "unknown status";
   }
 }

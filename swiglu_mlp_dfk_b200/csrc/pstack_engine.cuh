@@ -35,18 +35,24 @@
 // slices, the rescale kernel), so a step gives the same bits as the 2L + 1
 // kernel launches with those variants.
 //
-// Warp roles (192 threads):
+// Warp roles (224 threads):
 //   warp 0     weight producer (one lane): TMA tiles of phase after phase
 //              into an S-slot ring (128-byte swizzle);
 //   warp 1     MMA issuer (one elected lane): for each k tile, waits for its
 //              weight slot and its activation stage, issues the MMAs into
 //              the phase's TMEM buffer (two buffers, alternating phases);
-//   warps 2-5  activations and epilogue: wait for the previous phase grid-
-//              wide, write each k tile's activations into an A-stage ring
-//              (gate/up: x * gamma split into bf16 hi and lo rows, the sum
-//              of squares on the way; down: h), then read the accumulators
-//              and store h (SiLU(a) * u) or the down projection's partial
-//              sums, and count the phase as done.
+//   warp 2     activation producer (one lane): waits for the previous phase
+//              grid-wide, then TMA-loads the phase's activation tiles (x or
+//              y of the previous layer, or h) into an A-stage ring, as far
+//              ahead as the ring allows;
+//   warps 3-6  transform and epilogue: turn each gate/up activation tile into
+//              x * gamma split into bf16 hi and lo rows in place (the sum of
+//              squares on the way), then read the accumulators and store h
+//              (SiLU(a) * u) or the down projection's partial sums, and
+//              count the phase as done.
+// Outputs that a later phase loads with TMA are written by ordinary stores:
+// the writer fences them toward the async proxy before counting its phase,
+// and the activation producer fences after seeing the count.
 // Every wait is bounded; a wait that gives up sets the abort flag and the
 // device error word, and the CTA winds down without issuing more work.
 #pragma once
@@ -59,7 +65,7 @@
 
 namespace dfk {
 
-constexpr int PS_THREADS = 192;
+constexpr int PS_THREADS = 224;
 constexpr int PS_BN = 16;       // token slots on the MMA's N (x hi rows; + 16 lo rows)
 constexpr int PS_KSPLIT = 4;    // reduction slices of the down projection
 constexpr int PS_TILE_K = 64;   // reduction elements per k tile (one 128-byte row)
@@ -70,7 +76,17 @@ struct PsMaps {
   CUtensorMap wg[2];  // stacked W_gate [L * F][D]: box {64, gu_hmax}, {64, gu_hmax - 1}
   CUtensorMap wu[2];  // stacked W_up, same boxes
   CUtensorMap wd[2];  // stacked W_down [L * D][F]: box {64, dn_hmax}, {64, dn_hmax - 1}
+  CUtensorMap x;      // step input [B][D]: box {64, 16}
+  CUtensorMap y;      // every layer's y [L * B][D]: box {64, 16}
+  CUtensorMap h;      // every layer's h [L * B][F]: box {64, 16}
+  CUtensorMap gam;    // gammas [L][D]: box {64, 1}, no swizzle
 };
+
+// Orders this thread's generic-proxy global writes before later async-proxy
+// (TMA) accesses, and the reverse.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 struct PsParams {
   const uint16_t *gamma;  // [L][D] bf16
@@ -83,11 +99,14 @@ struct PsParams {
   unsigned *err;          // device status block
   int L, B, D, F;
   float eps;
-  int gu_rbase, gu_rextra, gu_hmax, gu_rc, gu_tiles;
-  int dn_nblk, dn_rbase, dn_rextra, dn_hmax, dn_rc, dn_tiles;
+  int gu_rbase, gu_rextra, gu_hmax, gu_rc, gu_tiles, gu_nt;
+  int dn_nblk, dn_rbase, dn_rextra, dn_hmax, dn_rc, dn_tiles, dn_nt;
+  // (nt: k tiles per weight-ring step -- consecutive 128-byte pieces of each
+  // weight row in one step, for DRAM locality)
   int S, slot_bytes;      // weight ring
   int A;                  // activation stages
-  int a_off, bar_off;     // shared-memory offsets from the 1024-byte aligned base
+  int a_off, g_off, bar_off;  // shared-memory offsets from the 1024-byte aligned base
+                              // (activation stages, their gamma slices, barriers)
 };
 
 #ifdef DFK_PSTACK_KERNELS
@@ -128,8 +147,9 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
 
   uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   uint64_t *wempty = wfull + S;
-  uint64_t *afull = wempty + S;
-  uint64_t *aempty = afull + A;
+  uint64_t *afull = wempty + S;      // activation tile landed (TMA)
+  uint64_t *xready = afull + A;       // activation tile ready for the MMA
+  uint64_t *aempty = xready + A;      // activation stage read by the MMA
   uint64_t *accfull = aempty + A;     // [2]
   uint64_t *tmempty = accfull + 2;    // [2]
   uint64_t *mmadone = tmempty + 2;
@@ -138,8 +158,10 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mmadone + 1) + 2;
   volatile int *s_last = reinterpret_cast<volatile int *>(mmadone + 1) + 3;
   unsigned *s_epoch = reinterpret_cast<unsigned *>(mmadone + 1) + 4;
+  int *s_aissued = reinterpret_cast<int *>(mmadone + 1) + 5;
   float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(mmadone + 1) + 32);
   uint8_t *astage0 = smem + p.a_off;
+  uint8_t *gslot0 = smem + p.g_off;   // [A][128 bytes]: gamma of a gate/up tile
 
   // ---- partitions
   const int gu_j0 = cta * p.gu_rbase + min(cta, p.gu_rextra);
@@ -156,7 +178,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
       mbar_init(&wempty[s], 1);
     }
     for (int s = 0; s < A; ++s) {
-      mbar_init(&afull[s], 128);
+      mbar_init(&afull[s], 1);
+      mbar_init(&xready[s], 128);
       mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -166,13 +189,10 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
     mbar_init(mmadone, 1);
     *s_abort = 0;
     *s_issued = 0;
+    *s_aissued = 0;
     *s_epoch = *reinterpret_cast<volatile unsigned *>(p.ctl);
     fence_mbar_init();
   }
-  // activation stages start at zero: the token slots >= B are never written
-  for (int i = tid; i < A * PS_ASTAGE / 16; i += PS_THREADS)
-    reinterpret_cast<uint4 *>(astage0)[i] = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(s_tmem, PS_TMEM_COLS);
     tmem_relinquish();
@@ -194,7 +214,9 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
       for (int ph = 0; ph < nphase && ok; ++ph) {
         const int l = ph >> 1;
         const bool gu = (ph & 1) == 0;
-        const int nsteps = gu ? p.gu_tiles : (dn_t1 - dn_t0 + 1) / 2;
+        const int nt = gu ? p.gu_nt : p.dn_nt;
+        const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+        const int nsteps = (ntl + nt - 1) / nt;
         for (int i = 0; i < nsteps; ++i, ++q) {
           const int st = q % S;
           if (q >= S && !mbar_wait_bounded(&wempty[st], ((q / S) - 1) & 1, s_abort, p.err)) {
@@ -202,19 +224,25 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             break;
           }
           uint8_t *slot = smem + static_cast<size_t>(st) * p.slot_bytes;
+          const int nv = min(nt, ntl - nt * i);  // k tiles of this step
           if (gu) {
+            // tiles [kt][gate | up], gu_rc rows each
             const int mi = gu_r == p.gu_hmax ? 0 : 1;
-            mbar_arrive_expect_tx(&wfull[st], 2u * gu_r * 128u);
-            const int k0 = i * PS_TILE_K, row = l * p.F + gu_j0;
-            tma_load_2d(slot, &maps.wg[mi], &wfull[st], k0, row, pol);
-            tma_load_2d(slot + p.gu_rc * 128, &maps.wu[mi], &wfull[st], k0, row, pol);
+            mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * 2u * gu_r * 128u);
+            const int row = l * p.F + gu_j0;
+            for (int kt = 0; kt < nv; ++kt) {
+              const int k0 = (nt * i + kt) * PS_TILE_K;
+              tma_load_2d(slot + (2 * kt) * p.gu_rc * 128, &maps.wg[mi], &wfull[st], k0, row,
+                          pol);
+              tma_load_2d(slot + (2 * kt + 1) * p.gu_rc * 128, &maps.wu[mi], &wfull[st], k0,
+                          row, pol);
+            }
           } else {
             const int mi = dn_r == p.dn_hmax ? 0 : 1;
-            const int nv = min(2, dn_t1 - dn_t0 - 2 * i);
             mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * dn_r * 128u);
             for (int kt = 0; kt < nv; ++kt)
               tma_load_2d(slot + kt * p.dn_rc * 128, &maps.wd[mi], &wfull[st],
-                          (dn_t0 + 2 * i + kt) * PS_TILE_K, l * p.D + dn_j0, pol);
+                          (dn_t0 + nt * i + kt) * PS_TILE_K, l * p.D + dn_j0, pol);
           }
         }
         *s_issued = q;
@@ -236,17 +264,19 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
       if (ph >= 2) ok = mbar_wait_bounded(&tmempty[buf], ((ph >> 1) - 1) & 1, s_abort, p.err);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int nsteps = gu ? p.gu_tiles : (dn_t1 - dn_t0 + 1) / 2;
+      const int nt = gu ? p.gu_nt : p.dn_nt;
+      const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+      const int nsteps = (ntl + nt - 1) / nt;
       int tin = 0;  // k tiles of this phase issued
       for (int i = 0; i < nsteps && ok; ++i, ++q) {
         const int st = q % S;
         ok = mbar_wait_bounded(&wfull[st], (q / S) & 1, s_abort, p.err);
         if (!__all_sync(0xffffffffu, ok)) break;
         const uint64_t ws = desc0 + (static_cast<uint32_t>(st * p.slot_bytes) >> 4);
-        const int nv = gu ? 1 : min(2, dn_t1 - dn_t0 - 2 * i);
+        const int nv = min(nt, ntl - nt * i);
         for (int kt = 0; kt < nv; ++kt, ++g, ++tin) {
           const int as = g % A;
-          ok = mbar_wait_bounded(&afull[as], (g / A) & 1, s_abort, p.err);
+          ok = mbar_wait_bounded(&xready[as], (g / A) & 1, s_abort, p.err);
           if (!__all_sync(0xffffffffu, ok)) break;
           tc_fence_after();
           const uint64_t bx = desc0 + a_enc0 + (static_cast<uint32_t>(as * PS_ASTAGE) >> 4);
@@ -256,7 +286,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             if (gu) {
 #pragma unroll
               for (int m = 0; m < 2; ++m) {
-                const uint64_t a = ws + (static_cast<uint32_t>(m * p.gu_rc * 128) >> 4) + 2 * kk;
+                const uint64_t a =
+                    ws + (static_cast<uint32_t>((2 * kt + m) * p.gu_rc * 128) >> 4) + 2 * kk;
                 if (leader)
                   umma_bf16(tmem + buf * 64 + m * 2 * PS_BN, a, bx + 2 * kk, idesc_gu, acc);
               }
@@ -276,84 +307,85 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
     }
     if (leader) umma_commit(mmadone);  // every MMA issued above has completed
     __syncwarp();
+  } else if (warp == 2) {
+    // ================= activation producer (one lane)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_normal();
+      int g = 0;  // activation tiles issued over all phases
+      bool ok = true;
+      for (int ph = 0; ph < nphase && ok; ++ph) {
+        const int l = ph >> 1;
+        const bool gu = (ph & 1) == 0;
+        if (ph > 0) {
+          // every CTA has finished the previous phase (its outputs are in memory)
+          ok = ps_grid_wait(done + ph - 1, target, s_abort, p.err);
+          fence_proxy_async_global();
+          if (!ok) break;
+        }
+        const CUtensorMap *map = gu ? (l == 0 ? &maps.x : &maps.y) : &maps.h;
+        const int row0 = gu ? (l == 0 ? 0 : (l - 1) * p.B) : l * p.B;
+        const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+        for (int i = 0; i < ntl; ++i, ++g) {
+          const int as = g % A;
+          if (g >= A && !mbar_wait_bounded(&aempty[as], ((g / A) - 1) & 1, s_abort, p.err)) {
+            ok = false;
+            break;
+          }
+          const int k0 = ((gu ? 0 : dn_t0) + i) * PS_TILE_K;
+          mbar_arrive_expect_tx(&afull[as], PS_BN * 128u + (gu ? 128u : 0u));
+          tma_load_2d(astage0 + as * PS_ASTAGE, map, &afull[as], k0, row0, pol);
+          if (gu) tma_load_2d(gslot0 + as * 128, &maps.gam, &afull[as], k0, l, pol);
+          *s_aissued = g + 1;
+        }
+      }
+    }
   } else {
-    // ================= activations and epilogue: warps 2..5 (128 threads)
-    const int et = tid - 64;
+    // ================= transform and epilogue: warps 3..6 (128 threads)
+    const int et = tid - 96;
     const int q4 = warp & 3;            // TMEM lanes 32 q4 .. 32 q4 + 31
     const int row = 32 * q4 + lane;     // accumulator row (output row of the CTA)
-    const int n = et >> 3;              // token slot this thread writes (0 .. 15)
+    const int n = et >> 3;              // token slot this thread converts (0 .. 15)
     const int pc = et & 7;              // physical 16-byte chunk of the 128-byte row
     const int lc = pc ^ (n & 7);        // its logical chunk (128-byte swizzle)
-    const bool real = n < p.B;
-    int g = 0;                          // activation tiles written over all phases
+    int g = 0;                          // activation tiles seen over all phases
     for (int ph = 0; ph < nphase; ++ph) {
       const int l = ph >> 1;
       const bool gu = (ph & 1) == 0;
       const int buf = ph & 1;
-      if (ph > 0) {
-        // every CTA has finished the previous phase (its outputs are in memory)
-        if (et == 0) ps_grid_wait(done + ph - 1, target, s_abort, p.err);
-        named_barrier(1, 128);
-      }
-      const bool live = !*s_abort;
       const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
-      const int K = gu ? p.D : p.F;
-      // the source row of this thread's token slot
-      const uint16_t *src = nullptr;
-      if (real)
-        src = gu ? (l == 0 ? p.x : p.y + (static_cast<size_t>(l - 1) * p.B) * p.D) +
-                       static_cast<size_t>(n) * p.D
-                 : p.h + (static_cast<size_t>(l) * p.B + n) * p.F;
-      const uint16_t *gam = p.gamma + static_cast<size_t>(l) * p.D;
       float ss = 0.f;
-      // k tiles in groups of 4: the loads of a group are issued together
-      for (int i0 = 0; i0 < ntl && live && !*s_abort; i0 += 4) {
-        uint4 xv[4], gv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          xv[u] = gv[u] = make_uint4(0u, 0u, 0u, 0u);
-          const int kt = (gu ? 0 : dn_t0) + i0 + u;
-          const int k = kt * PS_TILE_K + 8 * lc;
-          if (i0 + u < ntl && real && k < K) {
-            xv[u] = __ldcg(reinterpret_cast<const uint4 *>(src + k));
-            if (gu) gv[u] = __ldcg(reinterpret_cast<const uint4 *>(gam + k));
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (i0 + u >= ntl) break;
-          const int gi = g + i0 + u, as = gi % A;
-          if (gi >= A && !mbar_wait_bounded(&aempty[as], ((gi / A) - 1) & 1, s_abort, p.err))
-            break;
+      for (int i = 0; i < ntl; ++i) {
+        const int gi = g + i, as = gi % A;
+        if (!mbar_wait_bounded(&afull[as], (gi / A) & 1, s_abort, p.err)) break;
+        if (gu) {
+          // x * gamma (exact in fp32) split into bf16 hi + lo; sum of x^2
           uint8_t *xt = astage0 + as * PS_ASTAGE;
-          if (gu) {
-            // x * gamma (exact in fp32) split into bf16 hi + lo; sum of x^2
-            const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-            const uint32_t gw[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
-            uint32_t hw[4], lw[4];
+          // gamma of this tile (zeros past d_model: the copy's fill value)
+          const uint4 gv = *reinterpret_cast<const uint4 *>(gslot0 + as * 128 + 16 * lc);
+          const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+          uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const float x0 = bf16_lo(xw[qq]), x1 = bf16_hi(xw[qq]);
-              ss = fmaf(x0, x0, ss);
-              ss = fmaf(x1, x1, ss);
-              const float p0 = x0 * bf16_lo(gw[qq]), p1 = x1 * bf16_hi(gw[qq]);
-              const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
-              const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
-              const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
-              hw[qq] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-              lw[qq] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
-                       (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
-            }
-            *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) =
-                make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4 *>(xt + (PS_BN + n) * 128 + pc * 16) =
-                make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          } else {
-            *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) = xv[u];
+          for (int qq = 0; qq < 4; ++qq) {
+            const float x0 = bf16_lo(xw[qq]), x1 = bf16_hi(xw[qq]);
+            ss = fmaf(x0, x0, ss);
+            ss = fmaf(x1, x1, ss);
+            const float p0 = x0 * bf16_lo(gw[qq]), p1 = x1 * bf16_hi(gw[qq]);
+            const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
+            const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+            const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+            hw[qq] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+            lw[qq] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
+                     (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
           }
+          *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) =
+              make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4 *>(xt + (PS_BN + n) * 128 + pc * 16) =
+              make_uint4(lw[0], lw[1], lw[2], lw[3]);
           fence_proxy_async_smem();
-          mbar_arrive(&afull[as]);
         }
+        mbar_arrive(&xready[as]);
       }
       g += ntl;
       if (gu) {
@@ -362,7 +394,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
         v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (pc == 0) s_rinv[n] = real ? 1.0f / sqrtf(v / static_cast<float>(p.D) + p.eps) : 0.f;
+        if (pc == 0)
+          s_rinv[n] = n < p.B ? 1.0f / sqrtf(v / static_cast<float>(p.D) + p.eps) : 0.f;
         named_barrier(1, 128);
       }
 
@@ -384,8 +417,9 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
               if (e < p.B) {
                 const float sc = s_rinv[e];
                 const float aa = a[e] * sc, uu = u[e] * sc;
-                p.h[(static_cast<size_t>(l) * p.B + e) * p.F + j] =
-                    f32_to_bf16_bits((aa / (1.0f + expf(-aa))) * uu);
+                if (DFK_IN_BOUNDS(j < p.F, 16, p.err))
+                  p.h[(static_cast<size_t>(l) * p.B + e) * p.F + j] =
+                      f32_to_bf16_bits((aa / (1.0f + expf(-aa))) * uu);
               }
             }
           }
@@ -416,6 +450,7 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
           if (row < dn_r && !*s_abort)
             splitk_reduce_row(p.part, PS_KSPLIT, p.dn_nblk, dn_blk, PS_BN, p.B, row,
                               [&](int nn, float acc) {
+                                if (DFK_IN_BOUNDS(nn < p.B && dn_j0 + row < p.D, 17, p.err))
                                 p.y[(static_cast<size_t>(l) * p.B + nn) * p.D + dn_j0 + row] =
                                     f32_to_bf16_bits(acc);
                               });
@@ -423,7 +458,9 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
           if (et == 0) blkctr[dn_blk] = 0u;
         }
       }
-      // this CTA's share of the phase is in memory: count it
+      // this CTA's share of the phase is in memory: count it (the next phase
+      // reads it with TMA, through the async proxy)
+      fence_proxy_async_global();
       __threadfence();
       named_barrier(2, 128);
       if (et == 0) atomicAdd(&done[ph], 1u);
@@ -463,7 +500,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             const uint32_t hi = f32_to_bf16_bits((bf16_hi(w[i]) * r) * 1.0f);
             o[i] = lo | (hi << 16);
           }
-          *reinterpret_cast<uint4 *>(xr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+          if (DFK_IN_BOUNDS(k + 8 <= p.D, 18, p.err))
+            *reinterpret_cast<uint4 *>(xr + k) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
     }
@@ -480,10 +518,13 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   }
   if (tid == 0) {
     if (*s_abort) {
-      // after an aborted pipeline, wait (bounded) for weight copies in flight
+      // after an aborted pipeline, wait (bounded) for copies in flight
       const int issued = *s_issued;
       for (int q = issued - 1; q >= 0 && q >= issued - S; --q)
         mbar_wait_bounded(&wfull[q % S], (q / S) & 1, nullptr, p.err);
+      const int aissued = *s_aissued;
+      for (int q = aissued - 1; q >= 0 && q >= aissued - A; --q)
+        mbar_wait_bounded(&afull[q % A], (q / A) & 1, nullptr, p.err);
     }
     // the grid's last CTA starts the next launch's epoch
     __threadfence();

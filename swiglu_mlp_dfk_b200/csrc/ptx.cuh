@@ -15,6 +15,26 @@ constexpr unsigned ERR_WAIT_TIMEOUT = 1u;
 constexpr unsigned ERR_BOUNDS = 2u;
 constexpr int STATUS_WORDS = 4;
 
+// Checked builds (-DDFK_CHECKED): the kernels test the index of every global
+// store of a result and of the activation loads against the tensor's extent
+// first; a failed test skips the access, records the first failing check in
+// word 1 of the status block (site number << 16 | source line) and sets
+// ERR_BOUNDS -- never a trap.  In ordinary builds the test compiles away.
+#ifdef DFK_CHECKED
+static __device__ __noinline__ void bounds_failed(unsigned *err, unsigned site_line) {
+  if (err) {
+    atomicCAS(err + 1, 0u, site_line);
+    atomicOr(err, 2u);
+  }
+}
+#define DFK_IN_BOUNDS(cond, site, err)                                                  \
+  ((cond) || (::dfk::bounds_failed((err), (static_cast<unsigned>(site) << 16) |          \
+                                              (static_cast<unsigned>(__LINE__) & 0xffffu)), \
+              false))
+#else
+#define DFK_IN_BOUNDS(cond, site, err) true
+#endif
+
 // A pipeline wait gives up after this long by default (the data it waits
 // for arrives in microseconds in a healthy run).
 constexpr unsigned long long WAIT_TIMEOUT_NS = 4000000000ull;
@@ -268,6 +288,7 @@ __device__ __forceinline__ float round_bf16(float f) {
 // Output element (b, j): row j of the one output, or of its q / k / v part.
 template <typename P>
 __device__ __forceinline__ void store_out(const P &p, int b, int j, uint16_t v) {
+  if (!DFK_IN_BOUNDS(b >= 0 && b < p.B && j >= 0 && j < p.N, 1, p.err)) return;
   if (p.outs[0] == nullptr) {
     p.out[static_cast<size_t>(b) * p.N + j] = v;
   } else if (j < p.split[0]) {

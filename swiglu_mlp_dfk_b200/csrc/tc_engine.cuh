@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int idx = et; idx < kpad / 8; idx += 128) {
         const int k = idx * 8;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (k < p.K) v = ld_nc_v4(p.gamma + k);
+        if (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 4, p.err)) v = ld_nc_v4(p.gamma + k);
         *reinterpret_cast<uint4 *>(gs + k) = v;
       }
       named_barrier(1, 128);
@@ -511,7 +511,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                              j;
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                  if (c + e < p.B) dst[static_cast<size_t>(c + e) * p.N] = g[e];
+                  if (c + e < p.B &&
+                      DFK_IN_BOUNDS(j < p.N && c + e < p.tp_bmax && d < p.tp_world, 5, p.err))
+                    dst[static_cast<size_t>(c + e) * p.N] = g[e];
               }
             }
           } else if (row < h[t]) {
@@ -587,7 +589,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               float acc = __ldcg(v);
               for (int r = 1; r < p.tp_world; ++r)
                 acc = acc + __ldcg(v + static_cast<size_t>(r) * p.tp_bmax * p.N);
-              y[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(acc);
+              if (DFK_IN_BOUNDS(j < p.N && n < p.B, 6, p.err))
+                y[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(acc);
             }
           }
         }
@@ -645,6 +648,7 @@ struct TcPrepParams {
   float *rinv;            // [bn]
   int B, K, bn, ntiles;
   float eps;
+  unsigned *err;          // device status block (checked builds)
 };
 
 constexpr int TC_PREP_THREADS = 512;
@@ -664,7 +668,7 @@ __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcP
     for (int i = 0; i < 4; ++i) {  // up to four chunks' loads in flight per thread
       const int c = c0 + i * TC_PREP_THREADS;
       xv[i] = gv[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (real && c < kchunks) {
+      if (real && c < kchunks && DFK_IN_BOUNDS(8 * c + 8 <= p.K, 7, p.err)) {
         xv[i] = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
         gv[i] = ld_nc_v4(p.gamma + 8 * c);
       }
@@ -691,6 +695,7 @@ __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcP
                 (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
       }
       const int k = 8 * c, tile = k / TC_TILE_K, kk = k % TC_TILE_K;
+      if (!DFK_IN_BOUNDS(tile < p.ntiles && b < p.bn, 8, p.err)) continue;
       uint16_t *hrow = p.xg + (static_cast<size_t>(tile) * 2 * p.bn + b) * TC_TILE_K;
       *reinterpret_cast<uint4 *>(hrow + kk) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4 *>(hrow + static_cast<size_t>(p.bn) * TC_TILE_K + kk) =

@@ -354,7 +354,8 @@ __global__ void __launch_bounds__(TF8_THREADS, 1)
                 } else {
                   res = g[e] * sg;
                 }
-                p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
+                if (DFK_IN_BOUNDS(j < p.N, 9, p.err))
+                  p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
               }
             }
           }
@@ -376,6 +377,7 @@ __global__ void __launch_bounds__(TF8_THREADS, 1)
             const float sd = __ldg(p.scale[0] + j0 + row);
             splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, BN, p.B, row,
                               [&](int n, float acc) {
+                                if (DFK_IN_BOUNDS(n < p.B && j0 + row < p.N, 10, p.err))
                                 p.out[static_cast<size_t>(n) * p.N + j0 + row] =
                                     f32_to_bf16_bits(acc * sd);
                               });

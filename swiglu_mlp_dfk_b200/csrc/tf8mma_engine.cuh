@@ -116,6 +116,7 @@ struct Tm8PrepParams {
   float *fac;             // [bnp]: f_b (0 for padding tokens)
   int B, K, bnp, T, ntiles;
   float eps;
+  unsigned *err;          // device status block (checked builds)
 };
 
 // One CTA per token slot b = blockIdx.x, one pass over x: thread t holds
@@ -128,6 +129,8 @@ struct Tm8PrepParams {
 #ifdef DFK_TF8MMA_KERNELS
 __device__ __forceinline__ void tm8_load_chunk(const Tm8PrepParams &p, int b, int c, uint4 &xv,
                                                uint4 &gv) {
+  xv = gv = make_uint4(0u, 0u, 0u, 0u);
+  if (!DFK_IN_BOUNDS(b < p.B && 8 * c + 8 <= p.K, 13, p.err)) return;
   xv = ld_nc_v4(p.x + static_cast<size_t>(b) * p.K + 8 * c);
   gv = p.gamma ? ld_nc_v4(p.gamma + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
 }
@@ -169,6 +172,7 @@ __device__ __forceinline__ void tm8_write_terms(const Tm8PrepParams &p, int b, i
       w0 = f32x2_to_e4m3x2(u[0], u[1]) | (f32x2_to_e4m3x2(u[2], u[3]) << 16);
       w1 = f32x2_to_e4m3x2(u[4], u[5]) | (f32x2_to_e4m3x2(u[6], u[7]) << 16);
     }
+    if (!DFK_IN_BOUNDS(tile < p.ntiles && b < p.bnp, 14, p.err)) return;
     uint8_t *dst = p.terms + (static_cast<size_t>(tile) * rows + t * p.bnp + b) * TM8_TILE_K + kk;
     *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
   }
@@ -528,7 +532,8 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
               } else {
                 res = (g[e] * f) * sg;
               }
-              p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
+              if (DFK_IN_BOUNDS(j < p.N, 11, p.err))
+                p.out[static_cast<size_t>(n) * p.N + j] = f32_to_bf16_bits(res);
             }
           }
         }
@@ -550,6 +555,7 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
           const float sd = __ldg(p.scale[0] + j0 + row);
           splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, p.bnp, p.B, row,
                             [&](int n, float acc) {
+                              if (DFK_IN_BOUNDS(n < p.B && j0 + row < p.N, 12, p.err))
                               p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(
                                   INK ? acc * sd : (acc * __ldg(p.fac + n)) * sd);
                             });

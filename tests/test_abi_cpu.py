@@ -43,8 +43,16 @@ def test_library_exports_every_declared_symbol(L):
     assert dfk.dfk_version().startswith("dfk ")
 
 
+def test_checked_library_exports_every_declared_symbol(L):
+    # the bounds-checked build of the same sources (-DDFK_CHECKED)
+    from swiglu_mlp_dfk_b200 import build
+    C = ctypes.CDLL(build.LIB_CHECKED)
+    for n in header_functions():
+        assert hasattr(C, n), n
+
+
 def test_status_strings(L):
-    for s in range(9):
+    for s in range(10):
         assert L.dfk_status_string(s).decode()
     assert L.dfk_status_string(99).decode() == "unknown status"
 
@@ -110,6 +118,31 @@ MIS = ctypes.c_void_p(0x10008)
     (lambda L: L.dfk_down_proj(P, P2, P3, 1, 64, 64, 1, None),   # id 1 is a gate/up variant
      dfk.DFK_ERR_INVALID_ARG),
     (lambda L: L.dfk_silu(P, P2, -5, None), dfk.DFK_ERR_INVALID_ARG),
+    # tensor-parallel group and the emulated call
+    (lambda L: L.dfk_tp_group_create(0, 0, 4, 64, ctypes.byref(ctypes.c_void_p()),
+                                     ctypes.create_string_buffer(64)), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_tp_group_create(2, 2, 4, 64, ctypes.byref(ctypes.c_void_p()),
+                                     ctypes.create_string_buffer(64)), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_tp_group_create(2, 0, 65, 64, ctypes.byref(ctypes.c_void_p()),
+                                     ctypes.create_string_buffer(64)),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    (lambda L: L.dfk_tp_down_proj_allreduce(None, P, P2, P3, 1, 64, 64, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_tp_down_proj_allreduce_emulated(9, P, P2, P3, 1, 64, 64, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_tp_down_proj_allreduce_emulated(2, P, P2, P3, 65, 64, 64, None),
+     dfk.DFK_ERR_UNSUPPORTED_SHAPE),
+    # one-launch decode step
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, P, P, P, None, 1 << 20, 2, 4, 64, 64,
+                                    None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, MIS, P, P, P, 1 << 20, 2, 4, 64, 64,
+                                    None), dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_mlp_stack_step(P, -1.0, P2, P3, P2, P, P, P, P, 1 << 20, 2, 4, 64, 64,
+                                    None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, P, P, P, P, -1, 2, 4, 64, 64, None),
+     dfk.DFK_ERR_INVALID_ARG),
+    # the bounded-wait self-test
+    (lambda L: L.dfk_selftest_bounded_wait(None, None), dfk.DFK_ERR_INVALID_ARG),
     # FP8 weights: reduction length % 16, null scales, misaligned scales, tensor-core ids
     (lambda L: L.dfk_swiglu_gate_up_fp8(P, P2, P3, P2, P3, P, 1, 72, 64, 0, None),
      dfk.DFK_ERR_UNSUPPORTED_SHAPE),
