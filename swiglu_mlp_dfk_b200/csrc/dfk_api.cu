@@ -1058,19 +1058,23 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   // step (the tensor-core kernels' tuned stage sizes for these phases)
   p.gu_nt = 2;
   p.dn_nt = 4;
-  p.slot_bytes = round_up(std::max(p.gu_nt * 2 * p.gu_rc * 128, p.dn_nt * p.dn_rc * 128), 1024);
-  // an MMA reads 128 rows from each A tile start: keep the over-read of the
-  // last slot inside shared memory
-  const int slack = round_up(std::max(0, 16384 - std::min(p.gu_rc, p.dn_rc) * 128), 1024);
-  p.A = 8;
-  const int bar_bytes = (2 * 8 + 3 * p.A + 5) * 8 + 32 + PS_BN * 4;
-  const int fixed = 1024 /* alignment */ + slack + p.A * (PS_ASTAGE + 128) +
-                    round_up(bar_bytes, 128);
+  p.nt_max = std::max(p.gu_nt, p.dn_nt);
+  p.pf_ahead = env_int("DFK_PS_PREFETCH", 0);
+  // a slot: the step's weight tiles, then its activation tiles (hi + lo rows
+  // each), then the gamma slices of a gate/up step.  An MMA reads 128 rows
+  // from each weight tile start; the over-read past the weights stays
+  // inside the slot's activation area.
+  const int w_bytes = std::max(p.gu_nt * 2 * p.gu_rc * 128, p.dn_nt * p.dn_rc * 128);
+  p.x_off = round_up(w_bytes, 1024);
+  if (p.x_off + p.nt_max * PS_ATILE < std::max((2 * p.gu_nt - 1) * p.gu_rc * 128,
+                                               (p.dn_nt - 1) * p.dn_rc * 128) + 16384)
+    return no("slot layout");
+  p.slot_bytes = round_up(p.x_off + p.nt_max * PS_ATILE + p.nt_max * 128, 1024);
+  const int bar_bytes = (4 * 8 + 5) * 8 + 32 + PS_BN * 4;
+  const int fixed = 1024 /* alignment */ + round_up(bar_bytes, 128);
   p.S = std::min(8, (smem_cap - fixed) / p.slot_bytes);
-  if (p.S < 2) return no("the weight ring does not fit shared memory");
-  p.a_off = p.S * p.slot_bytes + slack;
-  p.g_off = p.a_off + p.A * PS_ASTAGE;
-  p.bar_off = p.g_off + p.A * 128;
+  if (p.S < 2) return no("the ring does not fit shared memory");
+  p.bar_off = p.S * p.slot_bytes;
   pl->smem = 1024 + static_cast<size_t>(p.bar_off) + round_up(bar_bytes, 128);
   pl->ws_ctl = round_up((2 + 2 * L + p.dn_nblk) * 4, 256);
   pl->ws_part = static_cast<size_t>(PS_KSPLIT) * p.dn_nblk * PS_BN * 128 * sizeof(float);

@@ -35,26 +35,26 @@
 // slices, the rescale kernel), so a step gives the same bits as the 2L + 1
 // kernel launches with those variants.
 //
-// Warp roles (224 threads):
-//   warp 0     weight producer (one lane): TMA tiles of phase after phase
-//              into an S-slot ring (128-byte swizzle);
-//   warp 1     MMA issuer (one elected lane): for each k tile, waits for its
-//              weight slot and its activation stage, issues the MMAs into
-//              the phase's TMEM buffer (two buffers, alternating phases);
-//   warp 2     activation producer (one lane): waits for the previous phase
-//              grid-wide, then TMA-loads the phase's activation tiles (x or
-//              y of the previous layer, or h) into an A-stage ring, as far
-//              ahead as the ring allows;
-//   warps 3-6  transform and epilogue: turn each gate/up activation tile into
-//              x * gamma split into bf16 hi and lo rows in place (the sum of
-//              squares on the way), then read the accumulators and store h
-//              (SiLU(a) * u) or the down projection's partial sums, and
-//              count the phase as done.
+// Warp roles (192 threads):
+//   warp 0     producer (one lane): for every ring step of every phase it
+//              issues the weight tiles at once -- weights never depend on
+//              the activations -- and the step's activation tiles (x or the
+//              previous layer's y, and gamma, for gate/up; h for the down
+//              projection) as soon as the phase's grid-wide count shows the
+//              previous phase done; steps issued before that get their
+//              activation tiles back-filled when it does;
+//   warp 1     MMA issuer (one elected lane): per step, waits for the
+//              weights and for the activation tiles to be ready, issues the
+//              MMAs into the phase's TMEM buffer (two buffers, alternating
+//              phases) and frees the slot with a commit;
+//   warps 2-5  transform and epilogue: turn each gate/up activation tile
+//              into x * gamma split into bf16 hi and lo rows in place (the
+//              sum of squares on the way), then read the accumulators and
+//              store h (SiLU(a) * u) or the down projection's partial sums,
+//              and count the phase as done.
 // Outputs that a later phase loads with TMA are written by ordinary stores:
 // the writer fences them toward the async proxy before counting its phase,
-// and the activation producer fences after seeing the count.
-// Every wait is bounded; a wait that gives up sets the abort flag and the
-// device error word, and the CTA winds down without issuing more work.
+// and the producer fences after seeing the count.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -65,11 +65,11 @@
 
 namespace dfk {
 
-constexpr int PS_THREADS = 224;
+constexpr int PS_THREADS = 192;
 constexpr int PS_BN = 16;       // token slots on the MMA's N (x hi rows; + 16 lo rows)
 constexpr int PS_KSPLIT = 4;    // reduction slices of the down projection
 constexpr int PS_TILE_K = 64;   // reduction elements per k tile (one 128-byte row)
-constexpr int PS_ASTAGE = 2 * PS_BN * 128;  // activation stage: hi rows then lo rows
+constexpr int PS_ATILE = 2 * PS_BN * 128;   // activation tile: hi rows then lo rows
 constexpr int PS_TMEM_COLS = 128;           // two buffers of 64 columns
 
 struct PsMaps {
@@ -101,12 +101,13 @@ struct PsParams {
   float eps;
   int gu_rbase, gu_rextra, gu_hmax, gu_rc, gu_tiles, gu_nt;
   int dn_nblk, dn_rbase, dn_rextra, dn_hmax, dn_rc, dn_tiles, dn_nt;
-  // (nt: k tiles per weight-ring step -- consecutive 128-byte pieces of each
-  // weight row in one step, for DRAM locality)
-  int S, slot_bytes;      // weight ring
-  int A;                  // activation stages
-  int a_off, g_off, bar_off;  // shared-memory offsets from the 1024-byte aligned base
-                              // (activation stages, their gamma slices, barriers)
+  // (nt: k tiles per ring step -- consecutive 128-byte pieces of each weight
+  // row in one step, for DRAM locality)
+  int S, slot_bytes;      // ring: S slots of slot_bytes
+  int x_off;              // offset of a slot's activation tiles (then gamma slices)
+  int nt_max;             // max(gu_nt, dn_nt): activation tiles a slot holds
+  int pf_ahead;           // weight steps beyond the ring prefetched into L2 (0: none)
+  int bar_off;            // barriers, from the 1024-byte aligned base
 };
 
 #ifdef DFK_PSTACK_KERNELS
@@ -141,16 +142,15 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   const uint32_t sbase = smem_addr(smem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = p.S, A = p.A;
+  const int S = p.S;
   const int G = gridDim.x, cta = blockIdx.x;
   const int nphase = 2 * p.L;
 
-  uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-  uint64_t *wempty = wfull + S;
-  uint64_t *afull = wempty + S;      // activation tile landed (TMA)
-  uint64_t *xready = afull + A;       // activation tile ready for the MMA
-  uint64_t *aempty = xready + A;      // activation stage read by the MMA
-  uint64_t *accfull = aempty + A;     // [2]
+  uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + p.bar_off);  // weights landed
+  uint64_t *afull = wfull + S;        // activation tiles (and gamma) landed
+  uint64_t *xready = afull + S;       // activation tiles ready for the MMA
+  uint64_t *wempty = xready + S;      // slot read by the MMAs
+  uint64_t *accfull = wempty + S;     // [2]
   uint64_t *tmempty = accfull + 2;    // [2]
   uint64_t *mmadone = tmempty + 2;
   volatile int *s_abort = reinterpret_cast<volatile int *>(mmadone + 1);
@@ -160,8 +160,6 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   unsigned *s_epoch = reinterpret_cast<unsigned *>(mmadone + 1) + 4;
   int *s_aissued = reinterpret_cast<int *>(mmadone + 1) + 5;
   float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(mmadone + 1) + 32);
-  uint8_t *astage0 = smem + p.a_off;
-  uint8_t *gslot0 = smem + p.g_off;   // [A][128 bytes]: gamma of a gate/up tile
 
   // ---- partitions
   const int gu_j0 = cta * p.gu_rbase + min(cta, p.gu_rextra);
@@ -171,16 +169,16 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   const int dn_r = p.dn_rbase + (dn_blk < p.dn_rextra ? 1 : 0);
   const int dn_t0 = (dn_slc * p.dn_tiles) / PS_KSPLIT;
   const int dn_t1 = ((dn_slc + 1) * p.dn_tiles) / PS_KSPLIT;
+  // k tiles and ring steps of a phase
+  auto phase_tiles = [&](bool gu) { return gu ? p.gu_tiles : dn_t1 - dn_t0; };
+  auto phase_nt = [&](bool gu) { return gu ? p.gu_nt : p.dn_nt; };
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 1);
-    }
-    for (int s = 0; s < A; ++s) {
       mbar_init(&afull[s], 1);
       mbar_init(&xready[s], 128);
-      mbar_init(&aempty[s], 1);
+      mbar_init(&wempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -206,57 +204,161 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   unsigned *blkctr = p.ctl + 2 + nphase;
 
   if (warp == 0) {
-    // ================= weight producer (one lane): never waits on activations
+    // ================= producer (one lane)
     if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      int q = 0;  // weight steps issued over all phases
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_normal();
+      // activation tiles of step (phase ph, step i) into ring slot st
+      auto issue_act = [&](int ph, int i, int st) {
+        const int l = ph >> 1;
+        const bool gu = (ph & 1) == 0;
+        const int nt = phase_nt(gu), ntl = phase_tiles(gu);
+        const int nv = min(nt, ntl - nt * i);
+        uint8_t *xa = smem + static_cast<size_t>(st) * p.slot_bytes + p.x_off;
+        const CUtensorMap *map = gu ? (l == 0 ? &maps.x : &maps.y) : &maps.h;
+        const int row0 = gu ? (l == 0 ? 0 : (l - 1) * p.B) : l * p.B;
+        mbar_arrive_expect_tx(&afull[st],
+                              static_cast<uint32_t>(nv) * (PS_BN * 128u + (gu ? 128u : 0u)));
+        for (int kt = 0; kt < nv; ++kt) {
+          const int k0 = ((gu ? 0 : dn_t0) + nt * i + kt) * PS_TILE_K;
+          tma_load_2d(xa + kt * PS_ATILE, map, &afull[st], k0, row0, pol_x);
+          if (gu)
+            tma_load_2d(xa + p.nt_max * PS_ATILE + kt * 128, &maps.gam, &afull[st], k0, l, pol_x);
+        }
+      };
+      // the previous phase is done grid-wide (checked without waiting); its
+      // outputs are then visible to this thread's TMA loads
+      auto phase_open = [&](int ph) {
+        if (ph == 0) return true;
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(done + ph - 1)
+                     : "memory");
+        if (static_cast<int>(v - target) < 0) return false;
+        fence_proxy_async_global();
+        return true;
+      };
+      int open_ph = 0;              // phases up to this one have their activations open
+      int pend_q[8], pend_ph[8], pend_i[8];
+      int npend = 0, head = 0;      // steps issued without activation tiles (FIFO)
+      int q = 0;
       bool ok = true;
+      const unsigned long long limit = wait_limit_ns(p.err);
+      // L2 prefetch cursor: the weights of the step pf_ahead steps past the
+      // ring are pulled into L2 as each step is issued, so the stream keeps
+      // HBM busy across a phase boundary, where the ring alone (a few µs of
+      // streaming) cannot cover the epilogue, the count and the stragglers
+      int pph = 0, pi = 0;
+      auto prefetch_next = [&](bool issue) {
+        if (pph >= nphase) return;
+        const bool pgu = (pph & 1) == 0;
+        const int pnt = phase_nt(pgu), pntl = phase_tiles(pgu);
+        const int pl = pph >> 1;
+        const int pnv = issue ? min(pnt, pntl - pnt * pi) : 0;
+        for (int kt = 0; kt < pnv; ++kt) {
+          if (pgu) {
+            const int mi = gu_r == p.gu_hmax ? 0 : 1;
+            tma_prefetch_2d(&maps.wg[mi], (pnt * pi + kt) * PS_TILE_K, pl * p.F + gu_j0);
+            tma_prefetch_2d(&maps.wu[mi], (pnt * pi + kt) * PS_TILE_K, pl * p.F + gu_j0);
+          } else {
+            const int mi = dn_r == p.dn_hmax ? 0 : 1;
+            tma_prefetch_2d(&maps.wd[mi], (dn_t0 + pnt * pi + kt) * PS_TILE_K,
+                            pl * p.D + dn_j0);
+          }
+        }
+        if (++pi == (pntl + pnt - 1) / pnt) {
+          pi = 0;
+          ++pph;
+        }
+      };
+      if (p.pf_ahead > 0)  // steps S .. S + pf_ahead - 1 (the first S go to the ring now)
+        for (int k = 0; k < S + p.pf_ahead; ++k) prefetch_next(k >= S);
+      // issue the pending activation tiles once their phase opens
+      auto flush = [&]() {
+        while (npend > 0) {
+          const int ph = pend_ph[head];
+          if (ph > open_ph) {
+            if (!phase_open(ph)) return;
+            open_ph = ph;
+          }
+          issue_act(ph, pend_i[head], pend_q[head] % S);
+          *s_aissued = pend_q[head] + 1;
+          head = (head + 1) & 7;
+          --npend;
+        }
+      };
       for (int ph = 0; ph < nphase && ok; ++ph) {
         const int l = ph >> 1;
         const bool gu = (ph & 1) == 0;
-        const int nt = gu ? p.gu_nt : p.dn_nt;
-        const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+        const int nt = phase_nt(gu), ntl = phase_tiles(gu);
         const int nsteps = (ntl + nt - 1) / nt;
         for (int i = 0; i < nsteps; ++i, ++q) {
           const int st = q % S;
-          if (q >= S && !mbar_wait_bounded(&wempty[st], ((q / S) - 1) & 1, s_abort, p.err)) {
-            ok = false;
-            break;
+          if (q >= S) {
+            // wait for the slot, opening pending activations meanwhile
+            const unsigned long long t0 = global_timer_ns();
+            for (uint32_t it = 1; !mbar_try_wait(&wempty[st], ((q / S) - 1) & 1); ++it) {
+              if (npend) flush();
+              if ((it & 15u) == 0) {
+                if (*s_abort || global_timer_ns() - t0 > limit) {
+                  if (!*s_abort) atomicOr(p.err, ERR_WAIT_TIMEOUT);
+                  *s_abort = 1;
+                  ok = false;
+                  break;
+                }
+              }
+            }
+            if (!ok) break;
           }
           uint8_t *slot = smem + static_cast<size_t>(st) * p.slot_bytes;
           const int nv = min(nt, ntl - nt * i);  // k tiles of this step
           if (gu) {
-            // tiles [kt][gate | up], gu_rc rows each
+            // weight tiles [kt][gate | up], gu_rc rows each
             const int mi = gu_r == p.gu_hmax ? 0 : 1;
             mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * 2u * gu_r * 128u);
             const int row = l * p.F + gu_j0;
             for (int kt = 0; kt < nv; ++kt) {
               const int k0 = (nt * i + kt) * PS_TILE_K;
               tma_load_2d(slot + (2 * kt) * p.gu_rc * 128, &maps.wg[mi], &wfull[st], k0, row,
-                          pol);
+                          pol_w);
               tma_load_2d(slot + (2 * kt + 1) * p.gu_rc * 128, &maps.wu[mi], &wfull[st], k0,
-                          row, pol);
+                          row, pol_w);
             }
           } else {
             const int mi = dn_r == p.dn_hmax ? 0 : 1;
             mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * dn_r * 128u);
             for (int kt = 0; kt < nv; ++kt)
               tma_load_2d(slot + kt * p.dn_rc * 128, &maps.wd[mi], &wfull[st],
-                          (dn_t0 + nt * i + kt) * PS_TILE_K, l * p.D + dn_j0, pol);
+                          (dn_t0 + nt * i + kt) * PS_TILE_K, l * p.D + dn_j0, pol_w);
           }
+          *s_issued = q + 1;
+          if (p.pf_ahead > 0) prefetch_next(true);  // step q + S + pf_ahead
+          // the activation tiles now, or when the phase opens
+          pend_q[(head + npend) & 7] = q;
+          pend_ph[(head + npend) & 7] = ph;
+          pend_i[(head + npend) & 7] = i;
+          ++npend;
+          flush();
         }
-        *s_issued = q;
+      }
+      // the last steps' activations (bounded wait for their phase)
+      const unsigned long long t0 = global_timer_ns();
+      for (uint32_t it = 1; ok && npend > 0; ++it) {
+        flush();
+        if (npend && (it & 15u) == 0 && (*s_abort || global_timer_ns() - t0 > limit)) {
+          if (!*s_abort) atomicOr(p.err, ERR_WAIT_TIMEOUT);
+          *s_abort = 1;
+          break;
+        }
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer: the warp walks the rings, one lane issues
+    // ================= MMA issuer: the warp walks the ring, one lane issues
     __syncwarp();
     const uint32_t leader = elect_one_sync();
     const uint32_t idesc_gu = umma_idesc_bf16_f32(128, 2 * PS_BN);
     const uint32_t idesc_dn = umma_idesc_bf16_f32(128, PS_BN);
     const uint64_t desc0 = umma_desc_sw128(sbase);
-    const uint32_t a_enc0 = static_cast<uint32_t>(p.a_off) >> 4;
-    int q = 0, g = 0;  // weight steps and activation tiles consumed over all phases
+    int q = 0;  // ring steps consumed over all phases
     bool ok = true;
     for (int ph = 0; ph < nphase && ok; ++ph) {
       const bool gu = (ph & 1) == 0;
@@ -264,25 +366,22 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
       if (ph >= 2) ok = mbar_wait_bounded(&tmempty[buf], ((ph >> 1) - 1) & 1, s_abort, p.err);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int nt = gu ? p.gu_nt : p.dn_nt;
-      const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+      const int nt = phase_nt(gu), ntl = phase_tiles(gu);
       const int nsteps = (ntl + nt - 1) / nt;
-      int tin = 0;  // k tiles of this phase issued
       for (int i = 0; i < nsteps && ok; ++i, ++q) {
         const int st = q % S;
         ok = mbar_wait_bounded(&wfull[st], (q / S) & 1, s_abort, p.err);
+        if (ok) ok = mbar_wait_bounded(&xready[st], (q / S) & 1, s_abort, p.err);
         if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
         const uint64_t ws = desc0 + (static_cast<uint32_t>(st * p.slot_bytes) >> 4);
+        const uint64_t xs = ws + (static_cast<uint32_t>(p.x_off) >> 4);
         const int nv = min(nt, ntl - nt * i);
-        for (int kt = 0; kt < nv; ++kt, ++g, ++tin) {
-          const int as = g % A;
-          ok = mbar_wait_bounded(&xready[as], (g / A) & 1, s_abort, p.err);
-          if (!__all_sync(0xffffffffu, ok)) break;
-          tc_fence_after();
-          const uint64_t bx = desc0 + a_enc0 + (static_cast<uint32_t>(as * PS_ASTAGE) >> 4);
+        for (int kt = 0; kt < nv; ++kt) {
+          const uint64_t bx = xs + (static_cast<uint32_t>(kt * PS_ATILE) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (tin > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (i > 0 || kt > 0 || kk > 0) ? 1u : 0u;
             if (gu) {
 #pragma unroll
               for (int m = 0; m < 2; ++m) {
@@ -296,10 +395,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
               if (leader) umma_bf16(tmem + buf * 64, a, bx + 2 * kk, idesc_dn, acc);
             }
           }
-          if (leader) umma_commit(&aempty[as]);  // the stage is free once these MMAs read it
-          __syncwarp();
         }
-        if (ok && leader) umma_commit(&wempty[st]);
+        if (leader) umma_commit(&wempty[st]);  // the slot is free once these MMAs read it
         __syncwarp();
       }
       if (ok && leader) umma_commit(&accfull[buf]);
@@ -307,87 +404,61 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
     }
     if (leader) umma_commit(mmadone);  // every MMA issued above has completed
     __syncwarp();
-  } else if (warp == 2) {
-    // ================= activation producer (one lane)
-    if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_normal();
-      int g = 0;  // activation tiles issued over all phases
-      bool ok = true;
-      for (int ph = 0; ph < nphase && ok; ++ph) {
-        const int l = ph >> 1;
-        const bool gu = (ph & 1) == 0;
-        if (ph > 0) {
-          // every CTA has finished the previous phase (its outputs are in memory)
-          ok = ps_grid_wait(done + ph - 1, target, s_abort, p.err);
-          fence_proxy_async_global();
-          if (!ok) break;
-        }
-        const CUtensorMap *map = gu ? (l == 0 ? &maps.x : &maps.y) : &maps.h;
-        const int row0 = gu ? (l == 0 ? 0 : (l - 1) * p.B) : l * p.B;
-        const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
-        for (int i = 0; i < ntl; ++i, ++g) {
-          const int as = g % A;
-          if (g >= A && !mbar_wait_bounded(&aempty[as], ((g / A) - 1) & 1, s_abort, p.err)) {
-            ok = false;
-            break;
-          }
-          const int k0 = ((gu ? 0 : dn_t0) + i) * PS_TILE_K;
-          mbar_arrive_expect_tx(&afull[as], PS_BN * 128u + (gu ? 128u : 0u));
-          tma_load_2d(astage0 + as * PS_ASTAGE, map, &afull[as], k0, row0, pol);
-          if (gu) tma_load_2d(gslot0 + as * 128, &maps.gam, &afull[as], k0, l, pol);
-          *s_aissued = g + 1;
-        }
-      }
-    }
   } else {
-    // ================= transform and epilogue: warps 3..6 (128 threads)
-    const int et = tid - 96;
+    // ================= transform and epilogue: warps 2..5 (128 threads)
+    const int et = tid - 64;
     const int q4 = warp & 3;            // TMEM lanes 32 q4 .. 32 q4 + 31
     const int row = 32 * q4 + lane;     // accumulator row (output row of the CTA)
     const int n = et >> 3;              // token slot this thread converts (0 .. 15)
     const int pc = et & 7;              // physical 16-byte chunk of the 128-byte row
-    const int lc = pc ^ (n & 7);        // its logical chunk (128-byte swizzle)
-    int g = 0;                          // activation tiles seen over all phases
+    int q = 0;                          // ring steps seen over all phases
     for (int ph = 0; ph < nphase; ++ph) {
       const int l = ph >> 1;
       const bool gu = (ph & 1) == 0;
       const int buf = ph & 1;
-      const int ntl = gu ? p.gu_tiles : dn_t1 - dn_t0;
+      const int nt = phase_nt(gu), ntl = phase_tiles(gu);
+      const int nsteps = (ntl + nt - 1) / nt;
       float ss = 0.f;
-      for (int i = 0; i < ntl; ++i) {
-        const int gi = g + i, as = gi % A;
-        if (!mbar_wait_bounded(&afull[as], (gi / A) & 1, s_abort, p.err)) break;
+      for (int i = 0; i < nsteps; ++i, ++q) {
+        const int st = q % S;
+        // every step's activations pass through here, so each slot's barrier
+        // phases are waited for in order
+        if (!mbar_wait_bounded(&afull[st], (q / S) & 1, s_abort, p.err)) break;
         if (gu) {
-          // x * gamma (exact in fp32) split into bf16 hi + lo; sum of x^2
-          uint8_t *xt = astage0 + as * PS_ASTAGE;
-          // gamma of this tile (zeros past d_model: the copy's fill value)
-          const uint4 gv = *reinterpret_cast<const uint4 *>(gslot0 + as * 128 + 16 * lc);
-          const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-          uint32_t hw[4], lw[4];
+          uint8_t *xa = smem + static_cast<size_t>(st) * p.slot_bytes + p.x_off;
+          const int nv = min(nt, ntl - nt * i);
+          for (int kt = 0; kt < nv; ++kt) {
+            // x * gamma (exact in fp32) split into bf16 hi + lo; sum of x^2
+            uint8_t *xt = xa + kt * PS_ATILE;
+            const int lc = pc ^ (n & 7);  // logical chunk (128-byte swizzle)
+            const uint4 gv =
+                *reinterpret_cast<const uint4 *>(xa + p.nt_max * PS_ATILE + kt * 128 + 16 * lc);
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t hw[4], lw[4];
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const float x0 = bf16_lo(xw[qq]), x1 = bf16_hi(xw[qq]);
-            ss = fmaf(x0, x0, ss);
-            ss = fmaf(x1, x1, ss);
-            const float p0 = x0 * bf16_lo(gw[qq]), p1 = x1 * bf16_hi(gw[qq]);
-            const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
-            const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
-            const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
-            hw[qq] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-            lw[qq] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
-                     (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
+            for (int qq = 0; qq < 4; ++qq) {
+              const float x0 = bf16_lo(xw[qq]), x1 = bf16_hi(xw[qq]);
+              ss = fmaf(x0, x0, ss);
+              ss = fmaf(x1, x1, ss);
+              const float p0 = x0 * bf16_lo(gw[qq]), p1 = x1 * bf16_hi(gw[qq]);
+              const uint16_t h0 = f32_to_bf16_bits(p0), h1 = f32_to_bf16_bits(p1);
+              const float r0 = p0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+              const float r1 = p1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+              hw[qq] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+              lw[qq] = static_cast<uint32_t>(f32_to_bf16_bits(r0)) |
+                       (static_cast<uint32_t>(f32_to_bf16_bits(r1)) << 16);
+            }
+            *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) =
+                make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4 *>(xt + (PS_BN + n) * 128 + pc * 16) =
+                make_uint4(lw[0], lw[1], lw[2], lw[3]);
           }
-          *reinterpret_cast<uint4 *>(xt + n * 128 + pc * 16) =
-              make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4 *>(xt + (PS_BN + n) * 128 + pc * 16) =
-              make_uint4(lw[0], lw[1], lw[2], lw[3]);
           fence_proxy_async_smem();
         }
-        mbar_arrive(&xready[as]);
+        mbar_arrive(&xready[st]);
       }
-      g += ntl;
       if (gu) {
         // r_b: each token row's 8 chunks sit in 8 adjacent lanes
         float v = ss;
@@ -451,8 +522,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             splitk_reduce_row(p.part, PS_KSPLIT, p.dn_nblk, dn_blk, PS_BN, p.B, row,
                               [&](int nn, float acc) {
                                 if (DFK_IN_BOUNDS(nn < p.B && dn_j0 + row < p.D, 17, p.err))
-                                p.y[(static_cast<size_t>(l) * p.B + nn) * p.D + dn_j0 + row] =
-                                    f32_to_bf16_bits(acc);
+                                  p.y[(static_cast<size_t>(l) * p.B + nn) * p.D + dn_j0 +
+                                      row] = f32_to_bf16_bits(acc);
                               });
           named_barrier(2, 128);
           if (et == 0) blkctr[dn_blk] = 0u;
@@ -519,12 +590,11 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   if (tid == 0) {
     if (*s_abort) {
       // after an aborted pipeline, wait (bounded) for copies in flight
-      const int issued = *s_issued;
+      const int issued = *s_issued, aissued = *s_aissued;
       for (int q = issued - 1; q >= 0 && q >= issued - S; --q)
         mbar_wait_bounded(&wfull[q % S], (q / S) & 1, nullptr, p.err);
-      const int aissued = *s_aissued;
-      for (int q = aissued - 1; q >= 0 && q >= aissued - A; --q)
-        mbar_wait_bounded(&afull[q % A], (q / A) & 1, nullptr, p.err);
+      for (int q = aissued - 1; q >= 0 && q >= aissued - S; --q)
+        mbar_wait_bounded(&afull[q % S], (q / S) & 1, nullptr, p.err);
     }
     // the grid's last CTA starts the next launch's epoch
     __threadfence();
