@@ -1056,20 +1056,21 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   if (p.dn_tiles < PS_KSPLIT) return no("d_ff too short for four reduction slices");
   // k tiles per ring step: 256 / 512 contiguous bytes of each weight row per
   // step (the tensor-core kernels' tuned stage sizes for these phases)
-  p.gu_nt = 2;
-  p.dn_nt = 4;
-  p.nt_max = std::max(p.gu_nt, p.dn_nt);
-  p.pf_ahead = env_int("DFK_PS_PREFETCH", 0);
-  // a slot: the step's weight tiles, then its activation tiles (hi + lo rows
-  // each), then the gamma slices of a gate/up step.  An MMA reads 128 rows
-  // from each weight tile start; the over-read past the weights stays
-  // inside the slot's activation area.
+  p.gu_nt = env_int("DFK_PS_GU_NT", 2);
+  p.dn_nt = env_int("DFK_PS_DN_NT", 4);
+  if (p.gu_nt < 1 || p.dn_nt < 1 || p.gu_nt > 8 || p.dn_nt > 8) return no("tiles per step");
+  // a slot: the step's weight tiles, then its activation tiles (gate/up: hi
+  // + lo rows each; down: h rows), then the gamma slices of a gate/up step.
+  // An MMA reads 128 rows from each weight tile start; the over-read past
+  // the weights stays inside the slot.
   const int w_bytes = std::max(p.gu_nt * 2 * p.gu_rc * 128, p.dn_nt * p.dn_rc * 128);
   p.x_off = round_up(w_bytes, 1024);
-  if (p.x_off + p.nt_max * PS_ATILE < std::max((2 * p.gu_nt - 1) * p.gu_rc * 128,
-                                               (p.dn_nt - 1) * p.dn_rc * 128) + 16384)
-    return no("slot layout");
-  p.slot_bytes = round_up(p.x_off + p.nt_max * PS_ATILE + p.nt_max * 128, 1024);
+  p.g_off = p.x_off + std::max(p.gu_nt * PS_ATILE, p.dn_nt * PS_DTILE);
+  p.slot_bytes = round_up(p.g_off + p.gu_nt * 128, 1024);
+  if (p.slot_bytes < std::max((2 * p.gu_nt - 1) * p.gu_rc * 128, (p.dn_nt - 1) * p.dn_rc * 128) +
+                         16384)
+    p.slot_bytes = round_up(std::max((2 * p.gu_nt - 1) * p.gu_rc * 128,
+                                     (p.dn_nt - 1) * p.dn_rc * 128) + 16384, 1024);
   const int bar_bytes = (4 * 8 + 5) * 8 + 32 + PS_BN * 4;
   const int fixed = 1024 /* alignment */ + round_up(bar_bytes, 128);
   p.S = std::min(8, (smem_cap - fixed) / p.slot_bytes);

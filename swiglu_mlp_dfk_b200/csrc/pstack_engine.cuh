@@ -69,7 +69,8 @@ constexpr int PS_THREADS = 192;
 constexpr int PS_BN = 16;       // token slots on the MMA's N (x hi rows; + 16 lo rows)
 constexpr int PS_KSPLIT = 4;    // reduction slices of the down projection
 constexpr int PS_TILE_K = 64;   // reduction elements per k tile (one 128-byte row)
-constexpr int PS_ATILE = 2 * PS_BN * 128;   // activation tile: hi rows then lo rows
+constexpr int PS_ATILE = 2 * PS_BN * 128;   // gate/up activation tile: hi rows then lo rows
+constexpr int PS_DTILE = PS_BN * 128;       // down activation tile (h rows)
 constexpr int PS_TMEM_COLS = 128;           // two buffers of 64 columns
 
 struct PsMaps {
@@ -104,9 +105,8 @@ struct PsParams {
   // (nt: k tiles per ring step -- consecutive 128-byte pieces of each weight
   // row in one step, for DRAM locality)
   int S, slot_bytes;      // ring: S slots of slot_bytes
-  int x_off;              // offset of a slot's activation tiles (then gamma slices)
-  int nt_max;             // max(gu_nt, dn_nt): activation tiles a slot holds
-  int pf_ahead;           // weight steps beyond the ring prefetched into L2 (0: none)
+  int x_off;              // offset of a slot's activation tiles
+  int g_off;              // offset of a slot's gamma slices (gate/up steps)
   int bar_off;            // barriers, from the 1024-byte aligned base
 };
 
@@ -221,9 +221,10 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
                               static_cast<uint32_t>(nv) * (PS_BN * 128u + (gu ? 128u : 0u)));
         for (int kt = 0; kt < nv; ++kt) {
           const int k0 = ((gu ? 0 : dn_t0) + nt * i + kt) * PS_TILE_K;
-          tma_load_2d(xa + kt * PS_ATILE, map, &afull[st], k0, row0, pol_x);
+          tma_load_2d(xa + kt * (gu ? PS_ATILE : PS_DTILE), map, &afull[st], k0, row0, pol_x);
           if (gu)
-            tma_load_2d(xa + p.nt_max * PS_ATILE + kt * 128, &maps.gam, &afull[st], k0, l, pol_x);
+            tma_load_2d(smem + static_cast<size_t>(st) * p.slot_bytes + p.g_off + kt * 128,
+                        &maps.gam, &afull[st], k0, l, pol_x);
         }
       };
       // the previous phase is done grid-wide (checked without waiting); its
@@ -243,35 +244,6 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
       int q = 0;
       bool ok = true;
       const unsigned long long limit = wait_limit_ns(p.err);
-      // L2 prefetch cursor: the weights of the step pf_ahead steps past the
-      // ring are pulled into L2 as each step is issued, so the stream keeps
-      // HBM busy across a phase boundary, where the ring alone (a few µs of
-      // streaming) cannot cover the epilogue, the count and the stragglers
-      int pph = 0, pi = 0;
-      auto prefetch_next = [&](bool issue) {
-        if (pph >= nphase) return;
-        const bool pgu = (pph & 1) == 0;
-        const int pnt = phase_nt(pgu), pntl = phase_tiles(pgu);
-        const int pl = pph >> 1;
-        const int pnv = issue ? min(pnt, pntl - pnt * pi) : 0;
-        for (int kt = 0; kt < pnv; ++kt) {
-          if (pgu) {
-            const int mi = gu_r == p.gu_hmax ? 0 : 1;
-            tma_prefetch_2d(&maps.wg[mi], (pnt * pi + kt) * PS_TILE_K, pl * p.F + gu_j0);
-            tma_prefetch_2d(&maps.wu[mi], (pnt * pi + kt) * PS_TILE_K, pl * p.F + gu_j0);
-          } else {
-            const int mi = dn_r == p.dn_hmax ? 0 : 1;
-            tma_prefetch_2d(&maps.wd[mi], (dn_t0 + pnt * pi + kt) * PS_TILE_K,
-                            pl * p.D + dn_j0);
-          }
-        }
-        if (++pi == (pntl + pnt - 1) / pnt) {
-          pi = 0;
-          ++pph;
-        }
-      };
-      if (p.pf_ahead > 0)  // steps S .. S + pf_ahead - 1 (the first S go to the ring now)
-        for (int k = 0; k < S + p.pf_ahead; ++k) prefetch_next(k >= S);
       // issue the pending activation tiles once their phase opens
       auto flush = [&]() {
         while (npend > 0) {
@@ -331,7 +303,6 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
                           (dn_t0 + nt * i + kt) * PS_TILE_K, l * p.D + dn_j0, pol_w);
           }
           *s_issued = q + 1;
-          if (p.pf_ahead > 0) prefetch_next(true);  // step q + S + pf_ahead
           // the activation tiles now, or when the phase opens
           pend_q[(head + npend) & 7] = q;
           pend_ph[(head + npend) & 7] = ph;
@@ -378,7 +349,7 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
         const uint64_t xs = ws + (static_cast<uint32_t>(p.x_off) >> 4);
         const int nv = min(nt, ntl - nt * i);
         for (int kt = 0; kt < nv; ++kt) {
-          const uint64_t bx = xs + (static_cast<uint32_t>(kt * PS_ATILE) >> 4);
+          const uint64_t bx = xs + (static_cast<uint32_t>(kt * (gu ? PS_ATILE : PS_DTILE)) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (i > 0 || kt > 0 || kk > 0) ? 1u : 0u;
@@ -431,8 +402,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             // x * gamma (exact in fp32) split into bf16 hi + lo; sum of x^2
             uint8_t *xt = xa + kt * PS_ATILE;
             const int lc = pc ^ (n & 7);  // logical chunk (128-byte swizzle)
-            const uint4 gv =
-                *reinterpret_cast<const uint4 *>(xa + p.nt_max * PS_ATILE + kt * 128 + 16 * lc);
+            const uint4 gv = *reinterpret_cast<const uint4 *>(
+                smem + static_cast<size_t>(st) * p.slot_bytes + p.g_off + kt * 128 + 16 * lc);
             const uint4 xv = *reinterpret_cast<const uint4 *>(xt + n * 128 + pc * 16);
             const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
             const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};

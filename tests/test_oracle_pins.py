@@ -13,6 +13,7 @@ RMSNorm prologue of GPULlama3.java PR #78 (the ``rms_ffn_gate_up`` task).
 import math
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -263,6 +264,35 @@ def test_thread_count_does_not_change_result(oracle_mod):
     finally:
         oracle.set_threads(n0)
     assert np.array_equal(one, many)
+
+
+def _torch_bf16(v):
+    # torch's own cast (float64 -> bfloat16, round to nearest even) as the
+    # independent rounding routine
+    return torch.tensor(np.asarray(v, dtype=np.float64)).to(torch.bfloat16).to(
+        torch.float64).numpy()
+
+
+def test_mirror_mode_rounds_at_the_stated_points(oracle_mod):
+    # mirror mode = the pure computation with a bf16 rounding (RNE) of xn, of
+    # h and of y: each stage checked against torch's rounding of the pure
+    # stage fed the previous stage's rounded values
+    rng = np.random.default_rng(18)
+    B, D, F = 3, 48, 40
+    x = oracle.f64_to_bf16(rng.standard_normal((B, D)))
+    g = oracle.f64_to_bf16(1.0 + 0.1 * rng.standard_normal(D))
+    wg = oracle.f64_to_bf16(0.2 * rng.standard_normal((F, D)))
+    wu = oracle.f64_to_bf16(0.2 * rng.standard_normal((F, D)))
+    wd = oracle.f64_to_bf16(0.2 * rng.standard_normal((D, F)))
+    xn_m = oracle.rmsnorm(x, g, 1e-5, mirror=True)
+    assert np.array_equal(xn_m, _torch_bf16(oracle.rmsnorm(x, g, 1e-5)))
+    h_m = oracle.gate_up(x, wg, wu, gamma=g, eps=1e-5, mirror=True)
+    h_from_rounded_xn = oracle.gate_up(oracle.f64_to_bf16(xn_m), wg, wu)
+    assert np.array_equal(h_m, _torch_bf16(h_from_rounded_xn))
+    y_m = oracle.down(h_m, wd, mirror=True)
+    assert np.array_equal(y_m, _torch_bf16(oracle.down(h_m, wd)))
+    # and mirror mode differs from the pure one (it does round)
+    assert not np.array_equal(y_m, oracle.down(h_m, wd))
 
 
 def test_mirror_mode_outputs_are_bf16(oracle_mod):
