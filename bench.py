@@ -872,8 +872,32 @@ def profile_arm(args):
 
     torch.cuda.set_device(0)
     B = args.batch
-    inp = I.make_inputs(B, D, F, seed=SEED, w_std=0.02, norm=True,
-                        with_down=args.profile.startswith("down"), device="cuda")
+    if args.profile == "pstack":
+        # the one-launch decode step on a 2-layer Llama-3-8B-shaped stack
+        # (0.7 GB of weights: small enough for a full ncu capture)
+        from swiglu_mlp_dfk_b200.stack import PersistentDecodeStack
+        x0, params = I.make_stack(2, B, D, F, seed=4, w_std=0.02, device="cuda")
+        ps = PersistentDecodeStack(params, x0)
+        fn = ps.step_eager
+    else:
+        inp = I.make_inputs(B, D, F, seed=SEED, w_std=0.02, norm=True,
+                            with_down=args.profile.startswith("down"), device="cuda")
+        return _profile_one(args, dfk, I, inp, B)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("dfk_profile")
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    print(json.dumps({"profile": args.profile, "B": B, "layers": 2, "calls": args.steps,
+                      "device_error_word": dfk.dfk_device_error()}))
+    return None
+
+
+def _profile_one(args, dfk, I, inp, B):
+    import torch
     h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
     y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
     lay = {"row": I.LAYOUT_ROW, "col": I.LAYOUT_COL, "interleaved": I.LAYOUT_INTERLEAVED}
@@ -996,7 +1020,8 @@ def main():
                     help="skip the sweep / unfused / interleaved / decode-stack measurements")
     ap.add_argument("--stack-steps", type=int, default=512,
                     help="decode steps of the 32-layer stack measurement")
-    ap.add_argument("--profile", choices=["gate_up", "down", "gate_up_fp8", "down_fp8", "qkv"],
+    ap.add_argument("--profile",
+                    choices=["gate_up", "down", "gate_up_fp8", "down_fp8", "qkv", "pstack"],
                     default=None,
                     help="run only this kernel (inside an NVTX range) for ncu")
     ap.add_argument("--batch", type=int, default=1, help="batch for --profile")
