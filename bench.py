@@ -762,28 +762,32 @@ def decode_stack_measure(steps, layers=32, B=4):
         st.release()
         del st
     # one persistent kernel per step (dfk_mlp_stack_step): the same layers,
-    # stacked into [L][...] tensors
+    # stacked into [L][...] tensors, with row- and column-major gate/up weights
     from swiglu_mlp_dfk_b200.stack import PersistentDecodeStack
     stacked = tuple(torch.stack([p[i] for p in params]) for i in range(4))
-    ps = PersistentDecodeStack(x0=x0, stacked=stacked)
-    ps.step_eager()
-    torch.cuda.synchronize()
-    ps.capture()
-    for _ in range(3):
-        ps.step()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        ps.step()
-    b.record()
-    torch.cuda.synchronize()
-    pms = a.elapsed_time(b) / steps
-    res["persistent_ms_per_step"] = round(pms, 4)
-    res["persistent_kernels_per_step"] = ps.kernels_per_step()
-    res["persistent_frac_of_peak"] = round(ps.bytes_per_step() / (pms * 1e-3) / 1e9 / peak, 4)
-    res["persistent_speedup_over_fused"] = round(res["fused_ms_per_step"] / pms, 3)
-    ps.release()
-    del ps, stacked
+    for lay in ("row", "col"):
+        ps = PersistentDecodeStack(x0=x0, stacked=stacked, layout=lay)
+        ps.step_eager()
+        torch.cuda.synchronize()
+        ps.capture()
+        for _ in range(3):
+            ps.step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            ps.step()
+        b.record()
+        torch.cuda.synchronize()
+        pms = a.elapsed_time(b) / steps
+        key = "persistent" if lay == "row" else "persistent_col"
+        res[key + "_ms_per_step"] = round(pms, 4)
+        res[key + "_frac_of_peak"] = round(ps.bytes_per_step() / (pms * 1e-3) / 1e9 / peak, 4)
+        res[key + "_speedup_over_fused"] = round(res["fused_ms_per_step"] / pms, 3)
+        res["persistent_kernels_per_step"] = ps.kernels_per_step()
+        ps.release()
+        del ps
+        torch.cuda.empty_cache()
+    del stacked
     res["fused_speedup"] = round(res["unfused_ms_per_step"] / res["fused_ms_per_step"], 3)
     res["fused_auto_speedup_over_row"] = round(res["fused_ms_per_step"] /
                                                res["fused_auto_ms_per_step"], 3)

@@ -301,8 +301,11 @@ DFK_API void dfk_clear_variant_cache(void);
  * never stops at a layer boundary: each SM's producer streams the next
  * phase's weights while the previous phase finishes on the other SMs.
  *   gammas    [layers][d_model] bf16
- *   w_gate    [layers][d_ff][d_model] bf16 row-major (one allocation)
- *   w_up      [layers][d_ff][d_model]
+ *   w_gate    [layers][d_ff][d_model] bf16 (layout DFK_W_ROW_MAJOR), or
+ *             [layers][d_model][d_ff] (DFK_W_COL_MAJOR: the gate/up phases
+ *             then take 128 columns per SM, as the column-major tensor-core
+ *             kernel does); one allocation
+ *   w_up      the same shape as w_gate
  *   w_down    [layers][d_model][d_ff]
  *   x         [B][d_model] bf16, read and overwritten with the next input
  *   h_all     [layers][B][d_ff] bf16, every layer's h (written)
@@ -314,17 +317,19 @@ DFK_API void dfk_clear_variant_cache(void);
  * The arithmetic is that of the separate kernels with the tensor-core
  * gate/up (in-kernel RMSNorm, 16 token slots) and the four-slice split-K
  * tensor-core down projection, so one call gives the same bits as those
- * 2 x layers + 1 launches.  Constraints: 1 <= B <= 16; d_model, d_ff
- * multiples of 8; d_ff <= 128 rows per SM, d_model <= 128 rows per four
- * SMs (the Llama-3-8B shape fits); DFK_ERR_UNSUPPORTED_SHAPE otherwise.
+ * 2 x layers + 1 launches (with the same weight layout).  Constraints: 1 <= B <= 16; d_model, d_ff
+ * multiples of 8; d_ff <= 128 rows (or columns) per SM, d_model <= 128 rows
+ * per four SMs (the Llama-3-8B shape fits); DFK_ERR_UNSUPPORTED_SHAPE
+ * otherwise.  Any other layout: DFK_ERR_UNSUPPORTED_LAYOUT.
  * Calls on one workspace must not overlap on the GPU.  No allocation, so
  * the call can be captured in a CUDA graph.
  */
 DFK_API long long dfk_mlp_stack_workspace_bytes(int layers, int B, int d_model, int d_ff);
 DFK_API int dfk_mlp_stack_step(const void *gammas, float eps, const void *w_gate,
-                               const void *w_up, const void *w_down, void *x, void *h_all,
-                               void *y_all, void *workspace, long long workspace_bytes,
-                               int layers, int B, int d_model, int d_ff, void *stream);
+                               const void *w_up, int layout, const void *w_down, void *x,
+                               void *h_all, void *y_all, void *workspace,
+                               long long workspace_bytes, int layers, int B, int d_model,
+                               int d_ff, void *stream);
 
 /* ---- tensor-parallel MLP ---------------------------------------------------
  * "Deep Kernel Fusion for Transformers" (abstract) keeps the fused kernel

@@ -138,7 +138,7 @@ def lib():
                 "dfk_tp_down_proj_allreduce": [vp, vp, vp, vp, i, i, i, vp],
                 "dfk_tp_group_destroy": [vp],
                 "dfk_tp_down_proj_allreduce_emulated": [i, vp, vp, vp, i, i, i, vp],
-                "dfk_mlp_stack_step": [vp, f, vp, vp, vp, vp, vp, vp, vp, ll, i, i, i, i, vp],
+                "dfk_mlp_stack_step": [vp, f, vp, vp, i, vp, vp, vp, vp, vp, ll, i, i, i, i, vp],
                 "dfk_status_string": [i],
                 "dfk_last_error": [],
                 "dfk_version": [],
@@ -549,12 +549,14 @@ def dfk_mlp_stack_workspace_bytes(layers, B, d_model, d_ff):
 
 
 def dfk_mlp_stack_step(gammas, eps, w_gate, w_up, w_down, x, h_all, y_all, workspace,
-                       stream=None):
-    """gammas [L, D], w_gate / w_up [L, F, D], w_down [L, D, F], x [B, D] (updated in
-    place), h_all [L, B, F], y_all [L, B, D], workspace: uint8 device tensor."""
-    L, F, D = w_gate.shape
+                       layout=DFK_W_ROW_MAJOR, stream=None):
+    """gammas [L, D], w_gate / w_up [L, F, D] (row-major) or [L, D, F] (layout "col"),
+    w_down [L, D, F], x [B, D] (updated in place), h_all [L, B, F], y_all [L, B, D],
+    workspace: uint8 device tensor."""
+    layout = _layout(layout)
+    L, D, F = w_down.shape
     B = x.shape[0]
-    _check(lib().dfk_mlp_stack_step(_ptr(gammas), float(eps), _ptr(w_gate), _ptr(w_up),
+    _check(lib().dfk_mlp_stack_step(_ptr(gammas), float(eps), _ptr(w_gate), _ptr(w_up), layout,
                                     _ptr(w_down), _ptr(x), _ptr(h_all), _ptr(y_all),
                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
                                     L, B, D, F, _stream(stream)))

@@ -1025,7 +1025,7 @@ struct PsPlan {
 // Partition and shared-memory plan of the persistent decode step
 // (pstack_engine.cuh) for an L-layer stack on a device with `sms` SMs.
 static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPlan *pl,
-                        std::string *why) {
+                        std::string *why, bool col = false) {
   auto no = [&](const char *m) {
     if (why) *why = m;
     return false;
@@ -1040,11 +1040,17 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   p.B = B;
   p.D = D;
   p.F = F;
+  p.gu_col = col ? 1 : 0;
   p.gu_rbase = F / G;
   p.gu_rextra = F % G;
   p.gu_hmax = p.gu_rbase + (p.gu_rextra ? 1 : 0);
-  if (p.gu_rbase < 1 || p.gu_hmax > 128) return no("d_ff needs 1 .. 128 rows per SM");
-  p.gu_rc = round_up(p.gu_hmax, 8);
+  if (col) {
+    if (ceil_div(F, 128) > G) return no("column-major d_ff needs at most 128 columns per SM");
+    p.gu_rc = 128;  // two 64-column boxes per matrix and k tile
+  } else {
+    if (p.gu_rbase < 1 || p.gu_hmax > 128) return no("d_ff needs 1 .. 128 rows per SM");
+    p.gu_rc = round_up(p.gu_hmax, 8);
+  }
   p.gu_tiles = ceil_div(D, PS_TILE_K);
   p.dn_nblk = G / PS_KSPLIT;
   p.dn_rbase = D / p.dn_nblk;
@@ -1082,10 +1088,14 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   return true;
 }
 
-static int pstack_step(const void *gamma, float eps, const void *wg, const void *wu,
+static int pstack_step(const void *gamma, float eps, const void *wg, const void *wu, int layout,
                        const void *wd, void *x, void *h_all, void *y_all, void *ws,
                        size_t ws_bytes, int L, int B, int D, int F, cudaStream_t s) {
   if (L < 1 || B < 0 || D <= 0 || F <= 0) return fail(DFK_ERR_INVALID_ARG, "bad sizes");
+  if (layout != DFK_W_ROW_MAJOR && layout != DFK_W_COL_MAJOR)
+    return fail(DFK_ERR_UNSUPPORTED_LAYOUT, "the decode step takes row- or column-major "
+                "gate/up weights");
+  const bool col = layout == DFK_W_COL_MAJOR;
   if (!(eps >= 0.f && std::isfinite(eps))) return fail(DFK_ERR_INVALID_ARG, "bad eps");
   if (B == 0) return DFK_OK;
   if (!gamma || !wg || !wu || !wd || !x || !h_all || !y_all || !ws)
@@ -1099,7 +1109,7 @@ static int pstack_step(const void *gamma, float eps, const void *wg, const void 
   if (rc) return rc;
   PsPlan pl;
   std::string why;
-  if (!plan_pstack(L, B, D, F, ds->sms, std::min(ds->smem_optin, 232448), &pl, &why))
+  if (!plan_pstack(L, B, D, F, ds->sms, std::min(ds->smem_optin, 232448), &pl, &why, col))
     return fail(DFK_ERR_UNSUPPORTED_SHAPE, "persistent decode step: %s", why.c_str());
   if (ws_bytes < pl.ws_ctl + pl.ws_part)
     return fail(DFK_ERR_INVALID_ARG, "workspace of %zu bytes; %zu needed", ws_bytes,
@@ -1112,11 +1122,22 @@ static int pstack_step(const void *gamma, float eps, const void *wg, const void 
   for (int lo = 0; lo < 2; ++lo) {
     const uint32_t gh = static_cast<uint32_t>(std::max(1, p.gu_hmax - lo));
     const uint32_t dh = static_cast<uint32_t>(std::max(1, p.dn_hmax - lo));
-    if ((rc = tensor_map_2d(wg, D, static_cast<uint64_t>(L) * F, static_cast<uint64_t>(D) * 2,
-                            PS_TILE_K, gh, &maps.wg[lo], true)) ||
-        (rc = tensor_map_2d(wu, D, static_cast<uint64_t>(L) * F, static_cast<uint64_t>(D) * 2,
-                            PS_TILE_K, gh, &maps.wu[lo], true)) ||
-        (rc = tensor_map_2d(wd, F, static_cast<uint64_t>(L) * D, static_cast<uint64_t>(F) * 2,
+    if (col) {
+      // [L * D][F]: boxes of 64 columns x 64 k rows
+      if ((rc = tensor_map_2d(wg, F, static_cast<uint64_t>(L) * D, static_cast<uint64_t>(F) * 2,
+                              64, PS_TILE_K, &maps.wg[lo], true)) ||
+          (rc = tensor_map_2d(wu, F, static_cast<uint64_t>(L) * D, static_cast<uint64_t>(F) * 2,
+                              64, PS_TILE_K, &maps.wu[lo], true)))
+        return rc;
+    } else if ((rc = tensor_map_2d(wg, D, static_cast<uint64_t>(L) * F,
+                                   static_cast<uint64_t>(D) * 2, PS_TILE_K, gh, &maps.wg[lo],
+                                   true)) ||
+               (rc = tensor_map_2d(wu, D, static_cast<uint64_t>(L) * F,
+                                   static_cast<uint64_t>(D) * 2, PS_TILE_K, gh, &maps.wu[lo],
+                                   true))) {
+      return rc;
+    }
+    if ((rc = tensor_map_2d(wd, F, static_cast<uint64_t>(L) * D, static_cast<uint64_t>(F) * 2,
                             PS_TILE_K, dh, &maps.wd[lo], true)))
       return rc;
   }
@@ -2283,11 +2304,11 @@ long long dfk_mlp_stack_workspace_bytes(int layers, int B, int d_model, int d_ff
 }
 
 int dfk_mlp_stack_step(const void *gammas, float eps, const void *w_gate, const void *w_up,
-                       const void *w_down, void *x, void *h_all, void *y_all, void *workspace,
-                       long long workspace_bytes, int layers, int B, int d_model, int d_ff,
-                       void *stream) {
+                       int layout, const void *w_down, void *x, void *h_all, void *y_all,
+                       void *workspace, long long workspace_bytes, int layers, int B,
+                       int d_model, int d_ff, void *stream) {
   if (workspace_bytes < 0) return dfk::fail(DFK_ERR_INVALID_ARG, "negative workspace size");
-  return dfk::pstack_step(gammas, eps, w_gate, w_up, w_down, x, h_all, y_all, workspace,
+  return dfk::pstack_step(gammas, eps, w_gate, w_up, layout, w_down, x, h_all, y_all, workspace,
                           static_cast<size_t>(workspace_bytes), layers, B, d_model, d_ff,
                           static_cast<cudaStream_t>(stream));
 }

@@ -74,7 +74,8 @@ constexpr int PS_DTILE = PS_BN * 128;       // down activation tile (h rows)
 constexpr int PS_TMEM_COLS = 128;           // two buffers of 64 columns
 
 struct PsMaps {
-  CUtensorMap wg[2];  // stacked W_gate [L * F][D]: box {64, gu_hmax}, {64, gu_hmax - 1}
+  CUtensorMap wg[2];  // stacked W_gate [L * F][D]: box {64, gu_hmax}, {64, gu_hmax - 1};
+                      // column-major [L * D][F]: box {64 columns, 64 k rows} in wg[0]
   CUtensorMap wu[2];  // stacked W_up, same boxes
   CUtensorMap wd[2];  // stacked W_down [L * D][F]: box {64, dn_hmax}, {64, dn_hmax - 1}
   CUtensorMap x;      // step input [B][D]: box {64, 16}
@@ -101,6 +102,7 @@ struct PsParams {
   int L, B, D, F;
   float eps;
   int gu_rbase, gu_rextra, gu_hmax, gu_rc, gu_tiles, gu_nt;
+  int gu_col;             // 1: W_gate / W_up column-major, 128 columns per CTA (MN-major A)
   int dn_nblk, dn_rbase, dn_rextra, dn_hmax, dn_rc, dn_tiles, dn_nt;
   // (nt: k tiles per ring step -- consecutive 128-byte pieces of each weight
   // row in one step, for DRAM locality)
@@ -162,15 +164,18 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
   float *s_rinv = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(mmadone + 1) + 32);
 
   // ---- partitions
-  const int gu_j0 = cta * p.gu_rbase + min(cta, p.gu_rextra);
-  const int gu_r = p.gu_rbase + (cta < p.gu_rextra ? 1 : 0);
+  // gate/up rows: row-major ~F / G rows per CTA; column-major 128 columns per
+  // CTA (the CTAs past the last column have no gate/up work)
+  const int gu_j0 = p.gu_col ? cta * 128 : cta * p.gu_rbase + min(cta, p.gu_rextra);
+  const int gu_r = p.gu_col ? max(0, min(128, p.F - gu_j0))
+                            : p.gu_rbase + (cta < p.gu_rextra ? 1 : 0);
   const int dn_blk = cta / PS_KSPLIT, dn_slc = cta - dn_blk * PS_KSPLIT;
   const int dn_j0 = dn_blk * p.dn_rbase + min(dn_blk, p.dn_rextra);
   const int dn_r = p.dn_rbase + (dn_blk < p.dn_rextra ? 1 : 0);
   const int dn_t0 = (dn_slc * p.dn_tiles) / PS_KSPLIT;
   const int dn_t1 = ((dn_slc + 1) * p.dn_tiles) / PS_KSPLIT;
   // k tiles and ring steps of a phase
-  auto phase_tiles = [&](bool gu) { return gu ? p.gu_tiles : dn_t1 - dn_t0; };
+  auto phase_tiles = [&](bool gu) { return gu ? (gu_r > 0 ? p.gu_tiles : 0) : dn_t1 - dn_t0; };
   auto phase_nt = [&](bool gu) { return gu ? p.gu_nt : p.dn_nt; };
 
   if (tid == 0) {
@@ -283,7 +288,20 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
           }
           uint8_t *slot = smem + static_cast<size_t>(st) * p.slot_bytes;
           const int nv = min(nt, ntl - nt * i);  // k tiles of this step
-          if (gu) {
+          if (gu && p.gu_col) {
+            // weight tiles [kt][gate | up], each two boxes of 64 columns x 64 k rows
+            mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * 2u * 16384u);
+            for (int kt = 0; kt < nv; ++kt) {
+              const int krow = l * p.D + (nt * i + kt) * PS_TILE_K;
+#pragma unroll
+              for (int m = 0; m < 2; ++m) {
+                uint8_t *tile = slot + (2 * kt + m) * 16384;
+                const CUtensorMap *wm = m == 0 ? &maps.wg[0] : &maps.wu[0];
+                tma_load_2d(tile, wm, &wfull[st], gu_j0, krow, pol_w);
+                tma_load_2d(tile + 8192, wm, &wfull[st], gu_j0 + 64, krow, pol_w);
+              }
+            }
+          } else if (gu) {
             // weight tiles [kt][gate | up], gu_rc rows each
             const int mi = gu_r == p.gu_hmax ? 0 : 1;
             mbar_arrive_expect_tx(&wfull[st], static_cast<uint32_t>(nv) * 2u * gu_r * 128u);
@@ -326,7 +344,7 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
     // ================= MMA issuer: the warp walks the ring, one lane issues
     __syncwarp();
     const uint32_t leader = elect_one_sync();
-    const uint32_t idesc_gu = umma_idesc_bf16_f32(128, 2 * PS_BN);
+    const uint32_t idesc_gu = umma_idesc_bf16_f32(128, 2 * PS_BN, p.gu_col != 0);
     const uint32_t idesc_dn = umma_idesc_bf16_f32(128, PS_BN);
     const uint64_t desc0 = umma_desc_sw128(sbase);
     int q = 0;  // ring steps consumed over all phases
@@ -356,8 +374,18 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
             if (gu) {
 #pragma unroll
               for (int m = 0; m < 2; ++m) {
+                // K-major rows: the 16-element k slice kk starts 32 bytes into
+                // each swizzled row; MN-major (column-major weights): it is the
+                // atom pair 2 kk, 2 kk + 1 (2048 bytes per slice), atoms 8 KB
+                // apart along M
                 const uint64_t a =
-                    ws + (static_cast<uint32_t>((2 * kt + m) * p.gu_rc * 128) >> 4) + 2 * kk;
+                    p.gu_col
+                        ? umma_desc_sw128_mn(0u, 8192u, 1024u) +
+                              ((((ws + (static_cast<uint32_t>((2 * kt + m) * 16384) >> 4)) &
+                                 0x3FFFull)) +
+                               (2048u >> 4) * kk)
+                        : ws + (static_cast<uint32_t>((2 * kt + m) * p.gu_rc * 128) >> 4) +
+                              2 * kk;
                 if (leader)
                   umma_bf16(tmem + buf * 64 + m * 2 * PS_BN, a, bx + 2 * kk, idesc_gu, acc);
               }

@@ -263,17 +263,26 @@ class PersistentDecodeStack:
             or ``stacked=(gammas [L, D], W_gate [L, F, D], W_up [L, F, D],
             W_down [L, D, F])`` to use existing stacked tensors without a copy
     x0:     [B, D] bf16 first-step input
+    layout: "row" or "col" -- how the step reads W_gate / W_up ("col" stores
+            a transposed copy [L, D, F] once)
 
     After a step, ``h_all[l]`` and ``y_all[l]`` hold every layer's h and y and
     ``x`` the next step's input.
     """
 
-    def __init__(self, layers=None, x0=None, eps=1e-5, stacked=None):
+    def __init__(self, layers=None, x0=None, eps=1e-5, stacked=None, layout="row"):
+        if layout not in ("row", "col"):
+            raise ValueError("layout must be row or col")
         if stacked is None:
             stacked = tuple(torch.stack([lay[i] for lay in layers]).contiguous()
                             for i in range(4))
         self.gammas, self.wg, self.wu, self.wd = stacked
-        self.L, self.F, self.D = self.wg.shape
+        self.L, self.D, self.F = self.wd.shape
+        self.layout = layout
+        if layout == "col" and self.wg.shape[1] != self.D:
+            # stored once as [L][D][F] (the column-major gate/up phases)
+            self.wg = self.wg.transpose(1, 2).contiguous()
+            self.wu = self.wu.transpose(1, 2).contiguous()
         self.B = x0.shape[0]
         self.eps = float(eps)
         dev = x0.device
@@ -287,7 +296,7 @@ class PersistentDecodeStack:
 
     def _launch_step(self):
         dfk.dfk_mlp_stack_step(self.gammas, self.eps, self.wg, self.wu, self.wd, self.x,
-                               self.h_all, self.y_all, self.workspace)
+                               self.h_all, self.y_all, self.workspace, layout=self.layout)
 
     def step_eager(self):
         cur = torch.cuda.current_stream(self.stream.device)

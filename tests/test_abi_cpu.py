@@ -133,14 +133,16 @@ MIS = ctypes.c_void_p(0x10008)
     (lambda L: L.dfk_tp_down_proj_allreduce_emulated(2, P, P2, P3, 65, 64, 64, None),
      dfk.DFK_ERR_UNSUPPORTED_SHAPE),
     # one-launch decode step
-    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, P, P, P, None, 1 << 20, 2, 4, 64, 64,
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, 0, P2, P, P, P, None, 1 << 20, 2, 4, 64,
+                                    64, None), dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, 0, P2, MIS, P, P, P, 1 << 20, 2, 4, 64,
+                                    64, None), dfk.DFK_ERR_MISALIGNED),
+    (lambda L: L.dfk_mlp_stack_step(P, -1.0, P2, P3, 0, P2, P, P, P, P, 1 << 20, 2, 4, 64, 64,
                                     None), dfk.DFK_ERR_INVALID_ARG),
-    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, MIS, P, P, P, 1 << 20, 2, 4, 64, 64,
-                                    None), dfk.DFK_ERR_MISALIGNED),
-    (lambda L: L.dfk_mlp_stack_step(P, -1.0, P2, P3, P2, P, P, P, P, 1 << 20, 2, 4, 64, 64,
-                                    None), dfk.DFK_ERR_INVALID_ARG),
-    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, P2, P, P, P, P, -1, 2, 4, 64, 64, None),
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, 0, P2, P, P, P, P, -1, 2, 4, 64, 64, None),
      dfk.DFK_ERR_INVALID_ARG),
+    (lambda L: L.dfk_mlp_stack_step(P, 1e-5, P2, P3, 2, P2, P, P, P, P, 1 << 20, 2, 4, 64, 64,
+                                    None), dfk.DFK_ERR_UNSUPPORTED_LAYOUT),
     # the bounded-wait self-test
     (lambda L: L.dfk_selftest_bounded_wait(None, None), dfk.DFK_ERR_INVALID_ARG),
     # FP8 weights: reduction length % 16, null scales, misaligned scales, tensor-core ids

@@ -42,7 +42,9 @@ def bits_equal(a, b):
 
 
 def matching_variants():
-    """A tensor-core gate/up id and the four-slice split-K tensor-core GEMV id."""
+    """A tensor-core gate/up id and the four-slice split-K tensor-core GEMV id
+    (the column-major gate/up kernel always takes 128 columns per CTA, like
+    the one-launch step's column-major phases)."""
     gu = dn = None
     for i in range(1, dfk.dfk_variant_count() + 1):
         v = dfk.dfk_variant_info(i)
@@ -59,6 +61,8 @@ def matching_variants():
 def teacher_forced(ps, x_in, layers, rows=None, drows=None):
     """Check every listed layer of the step just run against the oracle."""
     gam, wg, wu, wd = (t for t in (ps.gammas, ps.wg, ps.wu, ps.wd))
+    if ps.layout == "col":
+        wg, wu = wg.transpose(1, 2).contiguous(), wu.transpose(1, 2).contiguous()
     for l in layers:
         xin = x_in if l == 0 else ps.y_all[l - 1]
         ref_h = oracle.gate_up(I.to_bits(xin), I.to_bits(wg[l]), I.to_bits(wu[l]),
@@ -73,11 +77,12 @@ def teacher_forced(ps, x_in, layers, rows=None, drows=None):
 
 
 @pytest.mark.parametrize("B", [1, 4, 13, 16])
-def test_persistent_step_equals_separate_kernels_and_oracle(B):
+@pytest.mark.parametrize("layout", ["row", "col"])
+def test_persistent_step_equals_separate_kernels_and_oracle(B, layout):
     L, D, F = 3, 512, 1024
     x0, params = I.make_stack(L, B, D, F, seed=40 + B, w_std=0.03, device="cuda")
-    ps = PersistentDecodeStack(params, x0)
-    ref = DecodeStack(params, x0)
+    ps = PersistentDecodeStack(params, x0, layout=layout)
+    ref = DecodeStack(params, x0, layout=layout)
     ref.gu_variant, ref.dn_variant = matching_variants()
     for step in range(3):
         x_in = ps.x.clone()
@@ -112,7 +117,8 @@ def test_persistent_step_graph_replay():
     ps.release()
 
 
-def test_persistent_step_llama3_8b_stack():
+@pytest.mark.parametrize("layout", ["row", "col"])
+def test_persistent_step_llama3_8b_stack(layout):
     # the 32-layer Llama-3-8B-shaped stack (B = 4): bit-identical to the
     # separate kernels over two steps, teacher-forced against the oracle on
     # layers 0, 15 and 31 (sampled output rows)
@@ -121,8 +127,8 @@ def test_persistent_step_llama3_8b_stack():
     stacked = tuple(torch.stack([p[i] for p in params]) for i in range(4))
     del params
     layers = [tuple(t[l] for t in stacked) for l in range(L)]
-    ps = PersistentDecodeStack(x0=x0, stacked=stacked)
-    ref = DecodeStack(layers, x0)
+    ps = PersistentDecodeStack(x0=x0, stacked=stacked, layout=layout)
+    ref = DecodeStack(layers, x0, layout=layout)
     ref.gu_variant, ref.dn_variant = matching_variants()
     rng = np.random.default_rng(9)
     rows = np.unique(np.concatenate([[0, F - 1], rng.integers(0, F, 192)])).astype(np.int32)
