@@ -1062,9 +1062,10 @@ static bool plan_pstack(int L, int B, int D, int F, int sms, int smem_cap, PsPla
   if (p.dn_tiles < PS_KSPLIT) return no("d_ff too short for four reduction slices");
   // k tiles per ring step: 256 / 512 contiguous bytes of each weight row per
   // step (the tensor-core kernels' tuned stage sizes for these phases)
-  p.gu_nt = env_int("DFK_PS_GU_NT", 2);
-  p.dn_nt = env_int("DFK_PS_DN_NT", 4);
-  if (p.gu_nt < 1 || p.dn_nt < 1 || p.gu_nt > 8 || p.dn_nt > 8) return no("tiles per step");
+  // (measured: 1 / 2 / 3 gate/up tiles and 1 - 6 down tiles per step, with
+  // the ring depth that fits; two and four are the fastest mix)
+  p.gu_nt = 2;
+  p.dn_nt = 4;
   // a slot: the step's weight tiles, then its activation tiles (gate/up: hi
   // + lo rows each; down: h rows), then the gamma slices of a gate/up step.
   // An MMA reads 128 rows from each weight tile start; the over-read past
