@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(PS_THREADS, 1)
         if (*s_last) {
           __threadfence();
           if (row < dn_r && !*s_abort)
-            splitk_reduce_row(p.part, PS_KSPLIT, p.dn_nblk, dn_blk, PS_BN, p.B, row,
+            splitk_reduce_row_n<PS_KSPLIT>(p.part, PS_KSPLIT, p.dn_nblk, dn_blk, PS_BN, p.B, row,
                               [&](int nn, float acc) {
                                 if (DFK_IN_BOUNDS(nn < p.B && dn_j0 + row < p.D, 17, p.err))
                                   p.y[(static_cast<size_t>(l) * p.B + nn) * p.D + dn_j0 +

@@ -302,21 +302,23 @@ __device__ __forceinline__ void store_out(const P &p, int b, int j, uint16_t v) 
 
 // Split-K tail for output row `row` of row block `blk`: adds the kslices
 // (<= 8) fp32 partial sums of tokens 0 .. B-1 in slice order (slice 0
-// first) and hands each total to emit(n, total).  The loads of 8 tokens x
-// all slices are issued before any add, so the tail costs a few L2 round
-// trips rather than one per token.  part: [kslices][nblocks][bnp][128].
+// first) and hands each total to emit(n, total).  The loads of a batch of
+// tokens x all slices (64 values: 16 tokens at up to 4 slices, 8 at up to 8)
+// are issued before any add, so the tail costs a few L2 round trips rather
+// than one per token.  part: [kslices][nblocks][bnp][128].
 constexpr int SPLITK_MAX = 8;
 
-template <typename Emit>
-__device__ __forceinline__ void splitk_reduce_row(const float *part, int kslices, int nblocks,
-                                                  int blk, int bnp, int B, int row, Emit emit) {
-  constexpr int TB = 8;
+template <int KSM, typename Emit>
+__device__ __forceinline__ void splitk_reduce_row_n(const float *part, int kslices, int nblocks,
+                                                    int blk, int bnp, int B, int row,
+                                                    Emit emit) {
+  constexpr int TB = 64 / KSM;
   for (int n0 = 0; n0 < B; n0 += TB) {
-    float v[TB][SPLITK_MAX];
+    float v[TB][KSM];
 #pragma unroll
     for (int i = 0; i < TB; ++i)
 #pragma unroll
-      for (int sl = 0; sl < SPLITK_MAX; ++sl)
+      for (int sl = 0; sl < KSM; ++sl)
         v[i][sl] = (n0 + i < B && sl < kslices)
                        ? __ldcg(part + ((static_cast<size_t>(sl) * nblocks + blk) * bnp + n0 + i) *
                                            128 + row)
@@ -326,12 +328,18 @@ __device__ __forceinline__ void splitk_reduce_row(const float *part, int kslices
       if (n0 + i < B) {
         float acc = v[i][0];
 #pragma unroll
-        for (int sl = 1; sl < SPLITK_MAX; ++sl)
+        for (int sl = 1; sl < KSM; ++sl)
           if (sl < kslices) acc = acc + v[i][sl];
         emit(n0 + i, acc);
       }
     }
   }
+}
+
+template <typename Emit>
+__device__ __forceinline__ void splitk_reduce_row(const float *part, int kslices, int nblocks,
+                                                  int blk, int bnp, int B, int row, Emit emit) {
+  splitk_reduce_row_n<SPLITK_MAX>(part, kslices, nblocks, blk, bnp, B, row, emit);
 }
 
 }  // namespace dfk

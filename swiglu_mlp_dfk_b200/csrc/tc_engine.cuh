@@ -549,13 +549,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       named_barrier(2, 128);
       if (*s_last) {
         __threadfence();
-        if (row < r && !*s_abort)
-          splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, BN, p.B, row,
-                            [&](int n, float acc) {
-                              // RMSNorm with split-K only in mode 2 (r_b over all of K)
-                              if (NORM == 2) acc *= p.rinv[n];
-                              store_out(p, n, j0 + row, f32_to_bf16_bits(acc));
-                            });
+        if (row < r && !*s_abort) {
+          auto emit = [&](int n, float acc) {
+            // RMSNorm with split-K only in mode 2 (r_b over all of K)
+            if (NORM == 2) acc *= p.rinv[n];
+            store_out(p, n, j0 + row, f32_to_bf16_bits(acc));
+          };
+          // up to four slices: 16 tokens per batch of loads, else 8
+          if (p.kslices <= 4)
+            splitk_reduce_row_n<4>(p.part, p.kslices, p.nblocks, blk, BN, p.B, row, emit);
+          else
+            splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, BN, p.B, row, emit);
+        }
         named_barrier(2, 128);
         if (et == 0) p.counters[blk] = 0u;
       }
