@@ -541,6 +541,17 @@ static int pow2_ceil(int v) {
   return p;
 }
 
+// Dynamic shared memory of a kernel that follows its prep kernel (RMSNorm
+// hi/lo rows, FP8 activation terms) in the stream.  The prep kernel's CTAs
+// (one per token slot) become resident while the previous kernel runs and
+// stay until their results are written; an SM holding one must still take a
+// CTA of the main kernel, or that CTA starts its weight stream only after the
+// prep CTA has left (up to 64 SMs late, one per token slot).  228 KB per SM,
+// less 1 KB per resident CTA and the prep kernel's 1 KB static array, leaves
+// 230,400 bytes.  (The prep kernels' register budgets are capped for the same
+// reason.)
+constexpr int SMEM_BESIDE_PREP = 233472 - 2 * 1024 - 1024;
+
 // One CTA per SM over rows [j0, j0 + r) for the whole reduction; each
 // 128-row MMA tile reads 128 rows from shared memory starting at its A
 // tile, so the space behind the last A tile of the ring is kept readable.
@@ -567,7 +578,7 @@ static bool plan_tc(int layout, int nmat, bool norm, const VDef &v, int B, int K
     return false;
   }
   const int bn = B <= 16 ? 16 : (B <= 32 ? 32 : 64);
-  const int cap = std::min(ds.smem_optin, 232448);
+  const int cap = std::min(ds.smem_optin, (norm && prepped) ? SMEM_BESIDE_PREP : 232448);
   const int nt = v.nt;
   const int ntiles = ceil_div(K, TC_TILE_K);
   // GEMV in full tiles: k slices = SMs per row block (k split 0 = automatic)
@@ -1380,7 +1391,7 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   const int over = (v.nt * nmat - 1) * r8 * 128 + 128 * 128;
   const int slack = std::max(0, over - stage - tarea);
   const int bar_bytes = 512;  // 2 S + 2 barriers, flags, per-token factors and scales
-  const int smem_cap = std::min(ds.smem_optin, 232448);
+  const int smem_cap = std::min(ds.smem_optin, ink ? 232448 : SMEM_BESIDE_PREP);
   const int S = std::min(8, (smem_cap - 1024 - bar_bytes - slack - tarea) / stage);
   if (S < 2) {
     if (why) *why = "shared memory too small for two ring stages";

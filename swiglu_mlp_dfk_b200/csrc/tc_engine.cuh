@@ -659,7 +659,10 @@ struct TcPrepParams {
 constexpr int TC_PREP_THREADS = 512;
 
 #ifdef DFK_TC_KERNELS
-__global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcPrepParams p) {
+// At most 40 registers a thread (three CTAs' worth per SM): a prep CTA must
+// fit in the register file beside one CTA of the main kernel (192 threads,
+// up to 216 registers).
+__global__ void __launch_bounds__(TC_PREP_THREADS, 3) tc_norm_prep_kernel(const TcPrepParams p) {
   __shared__ float s_wss[TC_PREP_THREADS / 32];
   pdl_launch_dependents();
   pdl_wait();  // x comes from the previous kernel
@@ -667,10 +670,10 @@ __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcP
   const bool real = b < p.B;
   const int nchunk = p.ntiles * TC_TILE_K / 8, kchunks = p.K / 8;
   float ss = 0.f;
-  for (int c0 = tid; c0 < nchunk; c0 += 4 * TC_PREP_THREADS) {
-    uint4 xv[4], gv[4];
+  for (int c0 = tid; c0 < nchunk; c0 += 2 * TC_PREP_THREADS) {
+    uint4 xv[2], gv[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // up to four chunks' loads in flight per thread
+    for (int i = 0; i < 2; ++i) {  // two chunks' loads in flight per thread
       const int c = c0 + i * TC_PREP_THREADS;
       xv[i] = gv[i] = make_uint4(0u, 0u, 0u, 0u);
       if (real && c < kchunks && DFK_IN_BOUNDS(8 * c + 8 <= p.K, 7, p.err)) {
@@ -679,7 +682,7 @@ __global__ void __launch_bounds__(TC_PREP_THREADS) tc_norm_prep_kernel(const TcP
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       const int c = c0 + i * TC_PREP_THREADS;
       if (c >= nchunk) continue;
       const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};

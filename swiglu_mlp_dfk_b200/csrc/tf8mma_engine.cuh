@@ -178,7 +178,9 @@ __device__ __forceinline__ void tm8_write_terms(const Tm8PrepParams &p, int b, i
   }
 }
 
-__global__ void __launch_bounds__(TM8_PREP_THREADS) tf8mma_prep_kernel(const Tm8PrepParams p) {
+// At most 64 registers a thread: a prep CTA must fit in the register file
+// beside one CTA of the main kernel (192 threads x 128 registers).
+__global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const Tm8PrepParams p) {
   __shared__ float s_wmax[TM8_PREP_THREADS / 32], s_wss[TM8_PREP_THREADS / 32];
   __shared__ float s_scale;
   pdl_launch_dependents();
@@ -699,10 +701,30 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
     // fit in one window)
     if (real) {
       if (one) {
+        // term by term over the thread's chunks: the loop over the terms stays
+        // rolled, so the conversion is one short stretch of code
+        float uu[W][8];
 #pragma unroll
         for (int u = 0; u < W; ++u) {
-          const int c = c_lo + sub + tpt * u;
-          if (c < c_end) emit(c, xv[u], gv[u], scb);
+          values(xv[u], gv[u], uu[u]);
+#pragma unroll
+          for (int h = 0; h < 8; ++h) uu[u][h] *= scb;
+        }
+#pragma unroll 1
+        for (int t = 0; t < IT; ++t) {
+          const int rw = t * IBP + tok;
+#pragma unroll
+          for (int u = 0; u < W; ++u) {
+            const int c = c_lo + sub + tpt * u;
+            if (c < c_end) {
+              uint32_t w0, w1;
+              tm8_encode_term(uu[u], w0, w1);  // (the last term's residual is not used)
+              const int kl = 8 * (c - c_lo), jc = (kl & (TM8_TILE_K - 1)) >> 3;
+              *reinterpret_cast<uint2 *>(tarea + (kl / TM8_TILE_K) * IR * 128 + rw * 128 +
+                                         (((jc >> 1) ^ (rw & 7)) << 4) + ((jc & 1) << 3)) =
+                  make_uint2(w0, w1);
+            }
+          }
         }
       } else {
         for (int c0 = c_lo + sub; c0 < c_end; c0 += tpt * W) {

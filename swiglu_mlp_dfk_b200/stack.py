@@ -28,8 +28,12 @@ In-context tuning (``tune_variants``): the library's scheduler times each
 operation on its own, in bursts of back-to-back launches of that one
 operation.  Inside the stack every gate/up call follows a down projection and
 every down projection follows a gate/up call, and a variant that wins in a
-burst can lose there (with FP8 weights the in-kernel-term E4M3 variants win
-the bursts at B = 4 but cost ~5 us per layer in the stack).  The tuner
+burst can lose there.  With FP8 weights the in-kernel-term E4M3 variants
+win the bursts at B = 4 but lose inside the stack: every CTA converts the
+whole activation into E4M3 terms before its first MMA, and in the stack, where
+the two kernels alternate on every SM, that code runs from a cold
+instruction cache at half the speed it has in a burst, so the variants with
+a prep kernel (which converts once per token) win there.  The tuner
 times the captured step itself with each candidate variant of one
 operation while the other keeps its current choice, first for the gate/up
 call, then for the down projection, and keeps the fastest.
