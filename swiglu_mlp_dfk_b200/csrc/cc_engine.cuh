@@ -24,12 +24,15 @@
 //   with KSPLIT teams, team c owns the tiles t with floor(t / nt) = c
 //   (mod KSPLIT), nt = tiles per ring stage (KSPLIT = 1: one team, all tiles).
 //   p[c][s] = fp32 chain from +0 over its tiles t ascending, then e
-//             ascending:  p = fma(xn[b][k], W[j][k], p);
+//             ascending:  p = fma(a[b][k], W[j][k], p);
 //   q[c]    = ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7));
 //   total   = left fold q[0] + q[1] + ... + q[KSPLIT-1].
-// With the RMSNorm prologue, xn = (x * r) * gamma stays in fp32 (it is not
-// rounded to bf16), so the products are fused multiply-adds of an fp32 and a
-// bf16 value; without it, x is bf16 and every product is exact in fp32.
+// Without the RMSNorm a = x (bf16, every product exact in fp32).  With it
+// a = x * gamma, the product of two bf16 values and so exact in fp32, and the
+// epilogue multiplies total by r_b = 1 / sqrt(mean_k x[b][k]^2 + eps) (the
+// sum of squares in the order of the standalone RMSNorm): RMSNorm(x) * W
+// = r_b * sum_k (x gamma)[k] W[k], with r_b out of the dot product as in the
+// tensor-core family, so the first FMA does not wait for the reduction.
 // Either way the result is fixed by the order above.
 //
 // FP8 weights (W8, row-major only): W[j][k] = s[j] * Q[j][k] with Q in FP8
@@ -76,7 +79,7 @@ struct CcParams {
   int npass;        // ceil(B / BT)
   int tpt;          // consumer threads per K team (multiple of 32)
   int xs_off;       // shared-memory offset of the activation / reduction area
-  int g_off;        // shared-memory offset of gamma (bf16 bits, NORM only)
+  int g_off;        // (unused)
   int bar_off;      // shared-memory offset of the barrier area
   int pf_steps;     // ring steps after the first fill whose weight boxes are prefetched into L2
 };
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
 
   const int tid = threadIdx.x;
   const int nthr = blockDim.x;
-  const int ncons = nthr - 32;
+  const int ncons = nthr - 32 - (NORM ? 32 : 0);  // consumer threads (then [norm warp], producer)
   const int warp = tid >> 5, lane = tid & 31;
   const int S = p.stages;
 
@@ -201,6 +204,48 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
       }
       *s_issued = issued;
     }
+  } else if (NORM && warp == (nthr >> 5) - 2) {
+    // ================= norm warp: r_b = 1 / sqrt(mean(x^2) + eps) of each token
+    // of each pass, beside the consumers (r_b multiplies the row sums in the
+    // epilogue, so no FMA waits for it).  Fixed order: lane l chains k = 8 l + e
+    // + 256 c (c, then e ascending), then a xor butterfly over the 32 lanes (the
+    // order of the standalone RMSNorm).  x comes from global memory (L2), eight
+    // chunks a lane in flight; s_rinv alternates between two halves by pass.
+    pdl_wait();  // x comes from the previous kernel in the stream
+    for (int pass = 0; pass < p.npass; ++pass) {
+      const int b0 = pass * BT;
+      for (int bb = 0; bb < BT; ++bb) {
+        float ss = 0.f;
+        const bool real = b0 + bb < p.B;
+        const uint16_t *xr = p.x + static_cast<size_t>(real ? b0 + bb : 0) * p.K;
+        for (int k0 = 8 * lane; real && k0 < p.K; k0 += 8 * 256) {
+          uint4 xv[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int k = k0 + 256 * c;
+            xv[c] = (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 3, p.err))
+                        ? ld_nc_v4(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (k0 + 256 * c >= p.K) break;
+            const uint32_t w4[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float e0 = bf16_lo(w4[h]), e1 = bf16_hi(w4[h]);
+              ss = fmaf(e0, e0, ss);
+              ss = fmaf(e1, e1, ss);
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        if (lane == 0)
+          s_rinv[(pass & 1) * BT + bb] =
+              real ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 0.f;
+      }
+      named_barrier(2, ncons + 32);  // the consumers read this pass's r_b after it
+    }
   } else {
     // ================= consumer warps
     const int team = tid / p.tpt;
@@ -220,98 +265,60 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
     float *xs_f = reinterpret_cast<float *>(smem + p.xs_off);
     uint16_t *xs_h = reinterpret_cast<uint16_t *>(smem + p.xs_off);
     float *red = reinterpret_cast<float *>(smem + p.xs_off);  // reused after the K loop
-    uint16_t *gs = reinterpret_cast<uint16_t *>(smem + p.g_off);  // gamma (NORM only)
 
     pdl_wait();  // activations come from the previous kernel in the stream
 
     for (int pass = 0; pass < p.npass; ++pass) {
       const int b0 = pass * BT;
 
-      // ---- prologue 1: raw activations (and gamma) into shared memory.  Every
-      // consumer thread issues its 16-byte loads back to back, so the whole
-      // prologue costs one L2 round trip; x is read only after pdl_wait().
+      // ---- prologue: the activations into shared memory -- x, or with the
+      // RMSNorm xg = x * gamma (the product of two bf16 values, exact in fp32;
+      // r_b multiplies the row sums in the epilogue).  Every consumer thread
+      // issues its 16-byte loads back to back, so the prologue costs one L2
+      // round trip; x is read only after pdl_wait().
       {
-        const int c8n = p.kpad >> 3;               // 8-element chunks per activation row
-        const int nx = BT * c8n;                   // activation chunks
-        const int ntot = nx + (NORM ? c8n : 0);    // + gamma chunks
-        for (int base = tid; base < ntot; base += 4 * ncons) {
-          uint4 v[4];
+        const int c8n = p.kpad >> 3;  // 8-element chunks per activation row
+        const int nx = BT * c8n;      // activation chunks
+        for (int base = tid; base < nx; base += 4 * ncons) {
+          uint4 v[4], g[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int idx = base + u * ncons;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            v[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
             if (idx < nx) {
               const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
               if (b0 + bb < p.B && k < p.K)
-                if (DFK_IN_BOUNDS(b0 + bb < p.B && k + 8 <= p.K, 2, p.err))
+                if (DFK_IN_BOUNDS(b0 + bb < p.B && k + 8 <= p.K, 2, p.err)) {
                   v[u] = ld_nc_v4(p.x + static_cast<size_t>(b0 + bb) * p.K + k);
-            } else if (idx < ntot) {
-              const int k = (idx - nx) * 8;
-              if (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 3, p.err)) v[u] = ld_nc_v4(p.gamma + k);
+                  if (NORM) g[u] = ld_nc_v4(p.gamma + k);
+                }
             }
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int idx = base + u * ncons;
-            if (idx >= ntot) continue;
-            if (idx >= nx) {  // gamma, kept as bf16 bits
-              *reinterpret_cast<uint4 *>(gs + (idx - nx) * 8) = v[u];
-              continue;
-            }
+            if (idx >= nx) continue;
             const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
             if (XF32) {
               // within a 64-wide tile, element 8s + 4h + i sits at 32h + 4s + i
               float *row = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63);
               const int s8 = (k >> 3) & 7;
-              *reinterpret_cast<float4 *>(row + 4 * s8) =
-                  make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y));
-              *reinterpret_cast<float4 *>(row + 32 + 4 * s8) =
-                  make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w));
+              float4 lo = make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y),
+                                      bf16_hi(v[u].y));
+              float4 hi = make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w),
+                                      bf16_hi(v[u].w));
+              if (NORM) {
+                lo.x *= bf16_lo(g[u].x); lo.y *= bf16_hi(g[u].x);
+                lo.z *= bf16_lo(g[u].y); lo.w *= bf16_hi(g[u].y);
+                hi.x *= bf16_lo(g[u].z); hi.y *= bf16_hi(g[u].z);
+                hi.z *= bf16_lo(g[u].w); hi.w *= bf16_hi(g[u].w);
+              }
+              *reinterpret_cast<float4 *>(row + 4 * s8) = lo;
+              *reinterpret_cast<float4 *>(row + 32 + 4 * s8) = hi;
             } else {
               *reinterpret_cast<uint4 *>(xs_h + static_cast<size_t>(bb) * p.kpad + k) = v[u];
             }
           }
-        }
-        named_barrier(1, ncons);
-      }
-
-      if (NORM) {
-        // ---- prologue 2: r_b = 1/sqrt(mean(x^2) + eps), one warp per token.  Fixed
-        // order: lane l chains k = 8 l + e + 256 c (c, then e ascending), then a xor
-        // butterfly over the 32 lanes (the same order as the standalone RMSNorm).
-        for (int bb = cw; bb < BT; bb += ncw) {
-          float ss = 0.f;
-          const float *row = xs_f + static_cast<size_t>(bb) * p.kpad;
-          for (int k = 8 * lane; k < p.K; k += 256) {
-            const float *tp = row + (k & ~63) + 4 * ((k >> 3) & 7);
-            const float4 lo = *reinterpret_cast<const float4 *>(tp);
-            const float4 hi = *reinterpret_cast<const float4 *>(tp + 32);
-            ss = fmaf(lo.x, lo.x, ss); ss = fmaf(lo.y, lo.y, ss);
-            ss = fmaf(lo.z, lo.z, ss); ss = fmaf(lo.w, lo.w, ss);
-            ss = fmaf(hi.x, hi.x, ss); ss = fmaf(hi.y, hi.y, ss);
-            ss = fmaf(hi.z, hi.z, ss); ss = fmaf(hi.w, hi.w, ss);
-          }
-#pragma unroll
-          for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-          if (lane == 0)
-            s_rinv[bb] = (b0 + bb < p.B) ? 1.0f / sqrtf(ss / static_cast<float>(p.K) + p.eps) : 0.f;
-        }
-        named_barrier(1, ncons);
-        // ---- prologue 3: xn = (x * r) * gamma in place, kept in fp32
-        const int c8n = p.kpad >> 3;
-        for (int idx = tid; idx < BT * c8n; idx += ncons) {
-          const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
-          float *tp = xs_f + static_cast<size_t>(bb) * p.kpad + (k & ~63) + 4 * ((k >> 3) & 7);
-          const uint4 g = *reinterpret_cast<const uint4 *>(gs + k);
-          const float rr = s_rinv[bb];
-          float4 lo = *reinterpret_cast<float4 *>(tp);
-          float4 hi = *reinterpret_cast<float4 *>(tp + 32);
-          lo.x = (lo.x * rr) * bf16_lo(g.x); lo.y = (lo.y * rr) * bf16_hi(g.x);
-          lo.z = (lo.z * rr) * bf16_lo(g.y); lo.w = (lo.w * rr) * bf16_hi(g.y);
-          hi.x = (hi.x * rr) * bf16_lo(g.z); hi.y = (hi.y * rr) * bf16_hi(g.z);
-          hi.z = (hi.z * rr) * bf16_lo(g.w); hi.w = (hi.w * rr) * bf16_hi(g.w);
-          *reinterpret_cast<float4 *>(tp) = lo;
-          *reinterpret_cast<float4 *>(tp + 32) = hi;
         }
         named_barrier(1, ncons);
       }
@@ -557,6 +564,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
               acc.v[m][jj][bb] = v;
             }
       }
+      if (NORM) named_barrier(2, ncons + 32);  // this pass's r_b from the norm warp
       named_barrier(1, ncons);  // activation reads done: `red` aliases them
       const int rh = p.r_hi;
       if (active) {
@@ -607,6 +615,10 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
           v[m] = tot;
         }
         if (!aborted && b < p.B && j < p.N) {
+          if constexpr (NORM) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) v[m] *= s_rinv[(pass & 1) * BT + bb];
+          }
           if constexpr (W8) {
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) v[m] *= __ldg(p.scale[m] + j);

@@ -369,7 +369,9 @@ static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int
     const int nq = r_hi / v.jpt;
     const int tpt = (layout == LAYOUT_COL) ? 256 * ceil_div(nq, 32) : round_up(8 * nq, 32);
     const int ncons = v.ksplit * tpt;
-    if (ncons + 32 > CC_MAX_THREADS) continue;
+    // consumers, the producer warp and (RMSNorm) the warp that computes r_b
+    const int nthreads = ncons + 32 + (norm ? 32 : 0);
+    if (nthreads > CC_MAX_THREADS) continue;
     const int nT = ceil_div(K, tk);
     const int nsteps = ceil_div(nT, v.ksplit * v.nt);
     const int kpad = nsteps * v.ksplit * v.nt * tk;
@@ -381,7 +383,7 @@ static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int
     // normalised activations are kept in fp32: only the fp32 store is allowed then
     for (int xf = 1; xf >= (norm ? 1 : 0); --xf) {
       const int xs_bytes = v.bt * kpad * (xf ? 4 : 2);
-      const int g_bytes = norm ? kpad * 2 : 0;  // gamma, prologue only (aliases `red`)
+      const int g_bytes = 0;  // (gamma is multiplied in as x is loaded)
       const int region = round_up(std::max(xs_bytes + g_bytes, red_bytes), 128);
       const int avail = smem_cap - region - bar_bytes;
       const int S = avail > 0 ? std::min(8, avail / stage_bytes) : 0;
@@ -401,7 +403,7 @@ static bool plan_cc(int layout, int nmat, bool norm, bool w8, const VDef &v, int
     }
     pl->fn = fn;
     pl->grid = P;
-    pl->block = ncons + 32;
+    pl->block = nthreads;
     pl->r_lo = r_lo;
     pl->xf32 = best_xf32;
     CcParams &p = pl->p;
