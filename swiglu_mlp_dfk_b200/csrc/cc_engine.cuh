@@ -279,10 +279,13 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
       {
         const int c8n = p.kpad >> 3;  // 8-element chunks per activation row
         const int nx = BT * c8n;      // activation chunks
-        for (int base = tid; base < nx; base += 4 * ncons) {
-          uint4 v[4], g[4];
+        // chunks a thread has in flight: 8 without the RMSNorm (one round trip
+        // for the 1792 chunks of a 14336-long row), 4 with it (x and gamma)
+        constexpr int PB = NORM ? 4 : 8;
+        for (int base = tid; base < nx; base += PB * ncons) {
+          uint4 v[PB], g[PB];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < PB; ++u) {
             const int idx = base + u * ncons;
             v[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
             if (idx < nx) {
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(CC_MAX_THREADS, 1)
             }
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < PB; ++u) {
             const int idx = base + u * ncons;
             if (idx >= nx) continue;
             const int bb = idx / c8n, k = (idx - bb * c8n) * 8;
