@@ -73,7 +73,9 @@ def test_corrupted_tune_cache_is_ignored(tmp_path):
     assert "malformed" in err
 
 
-def test_fault_injection_falls_back_to_heuristic():
-    res, _ = run_child({"DFK_FAULT": "tune"})
+def test_fault_injection_falls_back_to_heuristic(tmp_path):
+    # a cache of its own: a cache file named by the environment may already
+    # hold a timed decision for this shape
+    res, _ = run_child({"DFK_FAULT": "tune", "DFK_TUNE_CACHE": str(tmp_path / "tune.txt")})
     assert res["ok"] and res["dev_err"] == 0
     assert res["us"] < 0            # chosen without timing
