@@ -33,6 +33,13 @@
  *     for every batch size (row b of the output depends on row b of x only).
  *   - There is no CPU fallback: without an sm_100 device every compute call
  *     returns DFK_ERR_ARCH (or DFK_ERR_CUDA).
+ *   - Kernels start while the previous kernel in the stream finishes
+ *     (programmatic dependent launch): they read the weights -- W_gate,
+ *     W_up, W_down, FP8 codes and scales, gamma -- as soon as they start,
+ *     and the activations (x, h) and their outputs only once the previous
+ *     kernel's results are visible.  A weight must not be written by work
+ *     still running in the same stream (order such writes with an event or
+ *     a synchronisation, as loading weights normally does).
  *   - Thread-safe: the variant cache and descriptor cache are locked.
  */
 #ifndef DFK_H

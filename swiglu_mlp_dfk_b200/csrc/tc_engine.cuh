@@ -394,14 +394,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int et = tid - 64;
     if (NORM == 2) pdl_wait();  // r_b comes from the prep kernel
     if (NORM == 1) {
-      pdl_wait();
+      // gamma is a weight: read before the dependency on the previous kernel
+      // resolves, every thread's loads in flight together
       const int kpad = ((p.ntiles + NT - 1) / NT) * NT * TC_TILE_K;
-      for (int idx = et; idx < kpad / 8; idx += 128) {
-        const int k = idx * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 4, p.err)) v = ld_nc_v4(p.gamma + k);
-        *reinterpret_cast<uint4 *>(gs + k) = v;
+      for (int base = et; base < kpad / 8; base += 4 * 128) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = (base + 128 * u) * 8;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (k < p.K && DFK_IN_BOUNDS(k + 8 <= p.K, 4, p.err)) v[u] = ld_nc_v4(p.gamma + k);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (base + 128 * u < kpad / 8)
+            *reinterpret_cast<uint4 *>(gs + (base + 128 * u) * 8) = v[u];
       }
+      pdl_wait();
       named_barrier(1, 128);
       // task t = et + 128 c (c < BN / 16) is 16-byte chunk (t & 7) of token row
       // t >> 3: the 8 lanes of a shared-memory phase cover the 8 chunks of one
