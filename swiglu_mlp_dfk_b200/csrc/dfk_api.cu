@@ -1368,6 +1368,10 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   }
   const int ks = nmat == 1 ? v.ksplit : 1;
   const int ntiles = ceil_div(K, TM8_TILE_K);
+  if (norm && ks > 1) {  // r_b needs all of K in one prep CTA per token
+    if (why) *why = "RMSNorm with a k split";
+    return false;
+  }
   if (ks > ntiles) {
     if (why) *why = "more k slices than k tiles";
     return false;
@@ -1430,7 +1434,8 @@ static bool plan_tm8(int nmat, bool norm, const VDef &v, int B, int K, int N,
   pl->grid = nblocks * ks;
   pl->threads = ink ? TM8_INK_THREADS : TM8_THREADS;
   pl->smem = 1024 + static_cast<size_t>(p.bar_off) + bar_bytes;
-  pl->term_bytes = ink ? 0 : static_cast<size_t>(ntiles) * np * 128 + 64 * sizeof(float);
+  // codes, then the factors [kslices][bnp] (at most 8 x 64)
+  pl->term_bytes = ink ? 0 : static_cast<size_t>(ntiles) * np * 128 + 8 * 64 * sizeof(float);
   return true;
 }
 
@@ -1536,11 +1541,12 @@ static int launch_tm8(const CcCall &c, const VDef &v, cudaStream_t s, int *stage
     pp.bnp = p.bnp;
     pp.T = p.T;
     pp.ntiles = p.ntiles;
+    pp.kslices = p.kslices;
     pp.eps = c.eps;
     pp.err = ds->err;
     void *pargs[] = {&pp};
-    // one CTA per token slot
-    e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp), dim3(TM8_PREP_THREADS), 0, s,
+    // one CTA per token slot and reduction slice
+    e = launch_kernel(tf8mma_prep_fn(), dim3(p.bnp, p.kslices), dim3(TM8_PREP_THREADS), 0, s,
                       pdl_enabled(), pargs);
     if (e != cudaSuccess) {
       cudaGetLastError();

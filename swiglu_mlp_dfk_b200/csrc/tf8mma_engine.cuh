@@ -18,11 +18,15 @@
 // reads each weight tile once for all terms and tokens, and
 //   sum_k W[j][k] v[k] = s[j] * 2^-e_b * sum_t 16^-t D[j][t * bnp + b],
 // the terms combined smallest first (Horner in 1/16, exact scalings).
-// The prep kernel (one CTA per token, a single pass over x held in
-// registers: the x-dependent chain between the previous kernel and this one
-// is one L2 round trip and one block reduction) also computes r_b = 1 /
-// sqrt(mean x^2 + eps) for the RMSNorm and stores f_b = r_b * 2^-e_b
-// (1 * 2^-e_b without it).
+// The prep kernel (one CTA per token and reduction slice, a single pass
+// over its part of x held in registers: the x-dependent chain between the
+// previous kernel and this one is one L2 round trip and one block
+// reduction) also computes r_b = 1 / sqrt(mean x^2 + eps) for the RMSNorm
+// and stores f_b = r_b * 2^-e_b (1 * 2^-e_b without it).  With a k split
+// (the down projection, no RMSNorm) each slice of each token has its own
+// scale 2^e_b from the slice's largest element, as with the in-kernel
+// terms, and each slice's partial sums are multiplied by its f_b before
+// they are added (exact: a power of two).
 //
 // Main kernel: one CTA per SM owns r <= 128 weight rows (the MMA's M) over its
 // reduction range (split-K slices for the down projection); a TMA ring
@@ -111,17 +115,19 @@ __device__ __forceinline__ void tm8_encode_term(float (&u)[8], uint32_t &w0, uin
 
 struct Tm8PrepParams {
   const uint16_t *x;      // [B][K] bf16
-  const uint16_t *gamma;  // [K] bf16 or nullptr (no RMSNorm)
+  const uint16_t *gamma;  // [K] bf16 or nullptr (no RMSNorm; then kslices may exceed 1)
   uint8_t *terms;         // [ntiles][T * bnp][128] E4M3 codes
-  float *fac;             // [bnp]: f_b (0 for padding tokens)
+  float *fac;             // [kslices][bnp]: f_b of each reduction slice (0 for padding tokens)
   int B, K, bnp, T, ntiles;
+  int kslices;            // the main kernel's reduction slices: one scale per token and slice
   float eps;
   unsigned *err;          // device status block (checked builds)
 };
 
-// One CTA per token slot b = blockIdx.x, one pass over x: thread t holds
-// chunks c = t + TM8_PREP_THREADS * i (8 elements each) in registers for
-// i < TM8_PREP_CPT and re-reads any further ones.  max |v| and sum x^2 in a
+// One CTA per token slot b = blockIdx.x and reduction slice blockIdx.y,
+// one pass over the slice's part of x: thread t holds chunks c = c_lo + t +
+// TM8_PREP_THREADS * i (8 elements each) in registers for i < TM8_PREP_CPT
+// and re-reads any further ones.  max |v| and sum x^2 in a
 // fixed order (each thread chains its chunks, i then e ascending; a xor
 // butterfly per warp; the warps in order), then the T term codes of every
 // chunk (zeros past K and for b >= B).  Defined in the one file that
@@ -186,23 +192,29 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const 
   pdl_launch_dependents();
   pdl_wait();  // x comes from the previous kernel
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nchunk = (p.ntiles * TM8_TILE_K) / 8;  // 8-element chunks incl. padding
-  const int kchunks = p.K / 8;
+  // this CTA's range: the 128-wide k tiles of reduction slice blockIdx.y, as
+  // the main kernel splits them (the whole of K without a split)
+  const int slc = blockIdx.y;
+  const int c_lo = ((slc * p.ntiles) / p.kslices) * (TM8_TILE_K / 8);
+  const int nchunk = (((slc + 1) * p.ntiles) / p.kslices) * (TM8_TILE_K / 8);  // range end,
+                                                                                // padding incl.
+  const int kchunks = min(nchunk, p.K / 8);  // end of the chunks inside K
+  float *fac = p.fac + static_cast<size_t>(slc) * p.bnp + b;
   constexpr int NT = TM8_PREP_THREADS, CPT = TM8_PREP_CPT;
   if (b >= p.B) {  // padding token slot: zero codes, zero factor
     float z[8];
-    for (int c = tid; c < nchunk; c += NT) {
+    for (int c = c_lo + tid; c < nchunk; c += NT) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) z[i] = 0.f;
       tm8_write_terms(p, b, c, z);
     }
-    if (tid == 0) p.fac[b] = 0.f;
+    if (tid == 0) *fac = 0.f;
     return;
   }
   uint4 xr[CPT], gr[CPT];
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {  // every load issued before any use
-    const int c = tid + NT * i;
+    const int c = c_lo + tid + NT * i;
     xr[i] = gr[i] = make_uint4(0u, 0u, 0u, 0u);
     if (c < kchunks) tm8_load_chunk(p, b, c, xr[i], gr[i]);
   }
@@ -213,7 +225,7 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const 
     tm8_chunk_values(p, xr[i], gr[i], v);
     tm8_chunk_stats(xr[i], v, mx, ss);
   }
-  for (int c = tid + NT * CPT; c < kchunks; c += NT) {
+  for (int c = c_lo + tid + NT * CPT; c < kchunks; c += NT) {
     uint4 xv, gv;
     tm8_load_chunk(p, b, c, xv, gv);
     float v[8];
@@ -244,13 +256,13 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const 
     }
     s_scale = ldexpf(1.0f, e);
     const float r = p.gamma ? 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps) : 1.0f;
-    p.fac[b] = r * ldexpf(1.0f, -e);
+    *fac = r * ldexpf(1.0f, -e);
   }
   __syncthreads();
   const float sc = s_scale;
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
-    const int c = tid + NT * i;
+    const int c = c_lo + tid + NT * i;
     if (c < nchunk) {
       float u[8];
       tm8_chunk_values(p, xr[i], gr[i], u);  // zeros past K
@@ -259,7 +271,7 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const 
       tm8_write_terms(p, b, c, u);
     }
   }
-  for (int c = tid + NT * CPT; c < nchunk; c += NT) {
+  for (int c = c_lo + tid + NT * CPT; c < nchunk; c += NT) {
     uint4 xv = make_uint4(0u, 0u, 0u, 0u), gv = make_uint4(0u, 0u, 0u, 0u);
     if (c < kchunks) tm8_load_chunk(p, b, c, xv, gv);
     float u[8];
@@ -274,7 +286,7 @@ __global__ void __launch_bounds__(TM8_PREP_THREADS, 2) tf8mma_prep_kernel(const 
 struct Tm8Params {
   uint16_t *out;          // [B][N] bf16
   const float *scale[2];  // per-row scales [N]
-  const float *fac;       // [bnp] per-token factor f_b (prep kernel)
+  const float *fac;       // [kslices][bnp] factors f_b of each slice (prep kernel)
   unsigned *err;
   int B, K, N;
   int rbase, rextra, hmax, r8;
@@ -520,7 +532,10 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
           float *mine = p.part + (static_cast<size_t>(slc) * p.nblocks + blk) * p.bnp * 128;
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            if (e < cstep) mine[(c + e) * 128 + row] = INK ? g[e] * s_fac[c + e] : g[e];
+            if (e < cstep)
+              mine[(c + e) * 128 + row] =
+                  g[e] * (INK ? s_fac[c + e]
+                              : __ldg(p.fac + static_cast<size_t>(slc) * p.bnp + c + e));
         } else if (row < r) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -558,8 +573,8 @@ __global__ void __launch_bounds__(IBP > 0 ? TM8_INK_THREADS : TM8_THREADS, 1)
           splitk_reduce_row(p.part, p.kslices, p.nblocks, blk, p.bnp, p.B, row,
                             [&](int n, float acc) {
                               if (DFK_IN_BOUNDS(n < p.B && j0 + row < p.N, 12, p.err))
-                              p.out[static_cast<size_t>(n) * p.N + j0 + row] = f32_to_bf16_bits(
-                                  INK ? acc * sd : (acc * __ldg(p.fac + n)) * sd);
+                              p.out[static_cast<size_t>(n) * p.N + j0 + row] =
+                                  f32_to_bf16_bits(acc * sd);
                             });
         }
         named_barrier(2, 128);

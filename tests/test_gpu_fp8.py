@@ -451,6 +451,32 @@ def test_fp8_in_kernel_terms_equal_prep_kernel_terms(B, D, F):
         assert bits_equal(outs[0], outs[1]), "nt=%d" % nt
 
 
+@pytest.mark.parametrize("B,D,F", [(1, 256, 1024), (3, 512, 2208), (8, 384, 4096)])
+def test_fp8_split_k_in_kernel_terms_equal_prep_kernel_terms(B, D, F):
+    # with a k split both kinds take one power of two per token and slice
+    # (from the largest |h| in the slice) and multiply each slice's partial
+    # sums by it before the slices are added in order: the same y bit for bit
+    L = Fp8Layer(B, D, F, seed=540 + B, norm=False)
+    g = torch.Generator(device="cuda").manual_seed(541 + B)
+    h = (0.5 * torch.randn(B, F, device="cuda", generator=g)).to(torch.bfloat16)
+    h[:, : F // 3] *= 64            # slices of different magnitude
+    compared = 0
+    for ks in (2, 4):
+        for nt in (1, 2):
+            pair = {}
+            for v in e4m3_mma_ids(True):
+                if v["k_split"] == ks and v["k_tiles_per_stage"] == nt:
+                    pair[v["e4m3_mma"]] = v["variant_id"]
+            run = lambda vid: dfk.dfk_down_proj_fp8(h, L.qd, L.sd, variant=vid)
+            outs = [try_variant(run, pair[k]) if k in pair else None for k in (1, 2)]
+            if outs[0] is None or outs[1] is None:
+                continue
+            torch.cuda.synchronize()
+            assert bits_equal(outs[0], outs[1]), "k split %d, nt %d" % (ks, nt)
+            compared += 1
+    assert compared >= 2
+
+
 @pytest.mark.parametrize("B", [1, 16, 64])
 def test_fp8_e4m3_mma_llama3_8b_sampled_rows(B):
     w = I.WORKLOADS["llama3_8b"]
