@@ -51,7 +51,7 @@ constexpr int TM8_TILE_K = 128;
 constexpr int TM8_XF_THREADS = 256;
 constexpr int TM8_INK_THREADS = TM8_THREADS + TM8_XF_THREADS;
 constexpr int TM8_PREP_THREADS = 512;
-constexpr int TM8_PREP_CPT = 4;  // chunks per prep thread kept in registers
+constexpr int TM8_PREP_CPT = 2;  // chunks per prep thread kept in registers
 
 // kind::f8f6f4 instruction descriptor: E4M3 A and B (format 0), fp32 D,
 // both K-major, shape M x N.
