@@ -382,11 +382,24 @@ def gpu_arm(args):
         # last key, so that a reader keeping only the end of the line still
         # has the B = 1..64 gate/up figures (fraction of the measured peak)
         sw = line["batch_sweep"]
-        line["batch_sweep_compact"] = {
+        compact = {
             "B": [r["B"] for r in sw],
             "row_us": [r["row"]["us"] for r in sw], "col_us": [r["col"]["us"] for r in sw],
             "row_frac": [r["row"]["frac"] for r in sw], "col_frac": [r["col"]["frac"] for r in sw],
             "family": ["%s/%s" % (r["row"]["family"], r["col"]["family"]) for r in sw]}
+        # the other operations' sweeps, fractions of the measured peak
+        if "down_sweep" in line:
+            compact["down_frac"] = [r["frac"] for r in line["down_sweep"]]
+        if "qkv_projection" in line:
+            q = line["qkv_projection"]["sweep"]
+            compact["qkv_B"] = [r["B"] for r in q]
+            compact["qkv_frac"] = [r["fused_frac"] for r in q]
+        if "fp8_weights" in line:
+            f8 = line["fp8_weights"]["sweep"]
+            compact["fp8_B"] = [r["B"] for r in f8]
+            compact["fp8_gate_up_frac"] = [r["gate_up_frac"] for r in f8]
+            compact["fp8_down_frac"] = [r["down_frac"] for r in f8]
+        line["batch_sweep_compact"] = compact
     return line
 
 
@@ -482,6 +495,19 @@ def extra_measurements(args, inp, copies, h, y, down_ws):
         row["scheduler_pick"] = "row" if row["row"]["us"] <= row["col"]["us"] else "col"
         sweep.append(row)
     out["batch_sweep"] = sweep
+    # down projection B = 1..64 (the scheduler's choice; eight W_down copies)
+    dsweep = []
+    for B in (1, 2, 4, 8, 16, 32, 64):
+        hb = (0.5 * torch.randn(B, F, device="cuda")).to(torch.bfloat16)
+        yb = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+        dfk.dfk_down_proj(hb, down_ws[0], y=yb)  # first call: the scheduler times its variants
+        t = timed_us(lambda i: dfk.dfk_down_proj(hb, down_ws[i % len(down_ws)], y=yb), reps,
+                     flush)
+        gbs = down_bytes(B, D, F) / (t * 1e-6) / 1e9
+        v = dfk.dfk_cached_variant(dfk.DFK_OP_DOWN, B, D, F) or {}
+        dsweep.append({"B": B, "us": round(t, 2), "frac": round(gbs / peak, 4),
+                       "family": {0: "cuda_core", 1: "tensor_core"}.get(v.get("family"))})
+    out["down_sweep"] = dsweep
     del x64, col, row_w, flush
     torch.cuda.empty_cache()
     out["llama3_70b"] = llama70b_measure()
